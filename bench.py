@@ -1,0 +1,408 @@
+"""Benchmark: exact attention forward + backward on B200 through the C ABI.
+
+One step = one pass of the whole hot path over one batch of synthetic input: fa_fwd (O, LSE)
+followed by the backward's three launches (preprocess, main, dQ conversion). The default
+workload is the training configuration B=2, H=16, N=8192, d=128, causal, bf16.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+For N > 1 it is launched with torch.distributed.run, one rank per GPU: every rank runs its
+own copy of the workload (independent problems, no data-path collective: weak scaling);
+the timed region is bracketed by barriers and the max over ranks is reported.
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (rank 0 only).
+
+Prints one JSON line (rank 0).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_attention_116_b200 import binding  # noqa: E402
+from exact_attention_116_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+from exact_attention_116_b200.workload import flops, hbm_bytes, visible_pairs  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOPS (bf16, causal) and % of B200 dense BF16 peak"
+UNIT = "TFLOPS"
+L2_BYTES = 126 * 2**20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_116_b200", "csrc", f)
+                  for f in ("fa_api.cu", "fa_fwd.cuh", "fa_bwd.cuh", "sm100_ptx.cuh")]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it still matches the source."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    with open(PROFILE_TRAFFIC) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    k = d.get("kernels", {}).get(kernel)
+    return None if k is None else k.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons, filtered to a time window."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            gid = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", gid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                    rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+                except (ValueError, IndexError):
+                    continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t0 - 0.15 <= r[0] <= t1 + 0.15]
+        window = "timed"
+        if not inside:
+            inside, window = rows, "warmup+timed"
+        if not inside:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) timing
+
+def oracle_sample(cfg, seconds: float, q=None, k=None, v=None, do=None):
+    """Time the fp64 oracle, as it stands, on blocks of query rows, head after head of batch 0
+    (forward of the rows and their backward contributions) until `seconds` have passed.
+
+    Returns (TFLOPS by the same pair-count convention, seconds, rows done, BLAS threads).
+    """
+    from oracle import attention_fp64 as oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        threads = os.cpu_count()
+    if q is None:
+        q, k, v, do = make_inputs(cfg)
+    n, block = cfg.N, min(512, cfg.N)
+    wr = 0 if cfg.causal else cfg.win_r
+    row_pairs = []
+    for i in range(n):
+        lo = max(0, i - cfg.win_l) if cfg.win_l >= 0 else 0
+        hi = min(n - 1, i + wr) if wr >= 0 else n - 1
+        row_pairs.append(hi - lo + 1)
+    pairs, rows_done = 0, 0
+    t0 = time.perf_counter()
+    for h in range(cfg.H):
+        q4, k4, v4 = (x[:1, :, h:h + 1].to(torch.float64).numpy() for x in (q, k, v))
+        qh, kh, vh, doh = q4[0, :, 0], k4[0, :, 0], v4[0, :, 0], do[0, :, h].to(torch.float64).numpy()
+        dq, dk, dv = np.zeros_like(qh), np.zeros_like(kh), np.zeros_like(vh)
+        dvec = np.zeros(n)
+        r1 = n
+        while r1 > 0:
+            r0 = max(0, r1 - block)
+            oracle.forward_rows(q4, k4, v4, 0, 0, np.arange(r0, r1), cfg.scale, cfg.causal, cfg.win_l, cfg.win_r)
+            oracle.backward_rows(qh, kh, vh, doh, r0, r1, cfg.scale, cfg.causal, cfg.win_l, cfg.win_r,
+                                 dq, dk, dv, dvec)
+            pairs += sum(row_pairs[r0:r1])
+            rows_done += r1 - r0
+            r1 = r0
+            if time.perf_counter() - t0 >= seconds:
+                break
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return 14 * cfg.d * pairs / dt / 1e12, dt, rows_done, threads
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_gpu(args):
+    world, rank, local = dist_setup(args.gpus)
+    cfg = CONFIGS[args.config]
+    if not cfg.backward:
+        raise SystemExit(f"config {cfg.name} has no backward; a step is forward + backward")
+    scale, causal, win = cfg.scale, cfg.causal, (cfg.win_l, cfg.win_r)
+    B, N, H, d = cfg.shape
+    q_h, k_h, v_h, do_h = make_inputs(cfg)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v, do = (x.to(dev) for x in (q_h, k_h, v_h, do_h))
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(binding.workspace_bytes(B, N, H, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    ev = {}
+
+    def mark(name):
+        def rec(i):
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(stream)
+            ev.setdefault(f"{name}{i}", []).append(e)
+        return rec
+
+    def step(record: bool):
+        if record:
+            mark("f")(0)
+        binding.fwd_into(q, k, v, o, lse, scale, causal, win)
+        binding.bwd_stages(q, k, v, o, lse, do, dq, dk, dv, ws, scale, causal, win,
+                           between=mark("b") if record else None)
+
+    for _ in range(args.warmup):
+        step(False)
+    binding.check()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(dev.index) if local == 0 else None
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall1 = time.time()
+    binding.check()
+    clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
+
+    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(world, ms_total)
+    ms_step = ms_total / args.steps
+    f_fwd, f_bwd = flops(B, N, H, d, causal, *win)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["f0"], ev["b0"]))
+    pre_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["b0"], ev["b1"]))
+    main_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["b1"], ev["b2"]))
+    conv_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["b2"], ev["b3"]))
+    bwd_ms = pre_ms + main_ms + conv_ms
+
+    # ---- end to end through the public API with host buffers (pinned), copies inside the timed region
+    pin = [x.pin_memory() for x in (q_h, k_h, v_h, do_h)]
+    out_h = [torch.empty_like(q_h).pin_memory() for _ in range(4)]
+    lse_h = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for src, dst in zip(pin, (q, k, v, do)):
+            dst.copy_(src, non_blocking=True)
+        binding.fwd_into(q, k, v, o, lse, scale, causal, win)
+        binding.bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale, causal, win, workspace=ws)
+        for src, dst in zip((o, dq, dk, dv), out_h):
+            dst.copy_(src, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    binding.check()
+    e2e_ms = max_over_ranks(world, e0.elapsed_time(e1)) / e2e_steps
+
+    peak, peak_src = peaks()
+    tflops_step = (f_fwd + f_bwd) / (ms_step * 1e-3) / 1e12
+    main_tflops = f_bwd / (main_ms * 1e-3) / 1e12
+    fwd_tflops = f_fwd / (fwd_ms * 1e-3) / 1e12
+    bwd_tflops = f_bwd / (bwd_ms * 1e-3) / 1e12
+    dominant = "fa_bwd_kernel" if main_ms >= fwd_ms else "fa_fwd_kernel"
+    dom_ms, dom_flops = (main_ms, f_bwd) if dominant == "fa_bwd_kernel" else (fwd_ms, f_fwd)
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    traffic = recorded_traffic(dominant)
+    t_bytes = B * N * H * d * 2
+    res = {
+        "metric": METRIC, "value": round(tflops_step * world, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": f"{cfg.name}: {cfg.note}", "B": B, "N": N, "H": H, "d": d, "causal": causal,
+                   "window": list(win), "seed": cfg.seed,
+                   "l2": f"inputs larger than L2 (q,k,v,dO = {4 * t_bytes / 2**20:.0f} MiB > 126 MiB); no flush",
+                   "flops": "fwd 4*d*pairs + bwd 10*d*pairs over exactly counted visible pairs",
+                   "per_rank": "each rank runs the whole workload on its own inputs"},
+        "fwd_tflops": round(fwd_tflops, 2), "bwd_tflops": round(bwd_tflops, 2),
+        "bwd_main_tflops": round(main_tflops, 2),
+        "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+        "bwd_stage_ms": {"preprocess": round(pre_ms, 4), "main": round(main_ms, 4), "dq_convert": round(conv_ms, 4)},
+        "frac_of_peak": {"fwd": round(fwd_tflops / peak["bf16_tflops"], 4),
+                         "bwd": round(bwd_tflops / peak["bf16_tflops"], 4),
+                         "denominator": f"bf16_tflops {peak['bf16_tflops']} ({peak_src})",
+                         "fwd_of_datasheet_2250": round(fwd_tflops / 2250.0, 4),
+                         "bwd_of_datasheet_2250": round(bwd_tflops / 2250.0, 4)},
+        "roofline": {"kernel": dominant, "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peak["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peak["bf16_tflops"], 4),
+                     "frac_of_sustained": round(achieved / peak.get("bf16_tflops_sustained", peak["bf16_tflops"]), 4),
+                     "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": traffic,
+                     "algorithmic_bytes": hbm_bytes(B, N, H, d)[1 if dominant == "fa_bwd_kernel" else 0]},
+        "e2e": {"value": round((f_fwd + f_bwd) / (e2e_ms * 1e-3) / 1e12 * world, 3), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": 4 * t_bytes,
+                "d2h_bytes_per_step": 4 * t_bytes + B * H * N * 4},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, dt, rows, threads = oracle_sample(cfg, args.cpu_seconds, q_h, k_h, v_h, do_h)
+        res["cpu_baseline"] = {"value": round(tf, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                               "sample": f"fp64 oracle, forward+backward of {rows} query rows (512-row blocks, heads of "
+                                         f"batch 0 in order) of {cfg.name}, {dt:.1f} s, same pair-count FLOP convention"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm (CPU oracle)
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cfg = CONFIGS[args.config]
+    q, k, v, do = make_inputs(cfg)
+    per_step = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(cfg, per_step, q, k, v, do)
+    vals, threads, rows, secs = [], 1, 0, 0.0
+    for _ in range(args.steps):
+        tf, dt, rows, threads = oracle_sample(cfg, per_step, q, k, v, do)
+        vals.append(tf)
+        secs += dt
+    value = statistics.mean(vals)
+    sample = (f"fp64 oracle, forward+backward of {rows} query rows (512-row blocks, heads of batch 0 in order) of {cfg.name} per step, "
+              f"about {per_step:.1f} s each")
+    res = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / max(1, args.steps) * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded N(0,1) bf16 widened to fp64)",
+           "config": {"workload": f"{cfg.name}: {cfg.note}", "B": cfg.B, "N": cfg.N, "H": cfg.H, "d": cfg.d,
+                      "causal": cfg.causal, "window": [cfg.win_l, cfg.win_r], "seed": cfg.seed},
+           "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="train_fwd_bwd", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

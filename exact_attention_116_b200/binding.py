@@ -1,0 +1,184 @@
+"""ctypes binding of the fa_sm100 C ABI (include/fa_sm100.h): argument marshalling only.
+
+Every step of the computation runs in the CUDA library. There is no CPU or PyTorch
+fallback: if the library is missing or the tensors are not on a CUDA device, the calls
+raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
+
+FA_OK = 0
+STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
+                4: "FA_ERR_TIMEOUT", 5: "FA_ERR_NO_MEMORY", 6: "FA_ERR_DEVICE"}
+EXPORTS = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
+           "fa_bwd_dq_convert", "fa_check", "fa_status_string")
+
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def load() -> ctypes.CDLL:
+    """Load the in-tree CUDA library (built by ``exact_attention_116_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing (run __graft_entry__.build())")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
+    lib.fa_bwd_workspace_bytes.restype = sz
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp, sz, vp]
+    lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
+    lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp, sz, vp]
+    lib.fa_bwd_dq_convert.argtypes = [vp, i, i, i, i, vp, sz, vp]
+    lib.fa_check.argtypes = [vp]
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    for name in ("fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert", "fa_check"):
+        getattr(lib, name).restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load().fa_status_string(int(status)).decode()
+    except RuntimeError:
+        return STATUS_NAMES.get(int(status), "FA_ERR_UNKNOWN")
+
+
+def _raise(status: int, where: str) -> None:
+    if status != FA_OK:
+        raise FaError(status, where)
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check_qkv(*ts: torch.Tensor) -> tuple[int, int, int, int]:
+    shape = ts[0].shape
+    if len(shape) != 4:
+        raise ValueError("tensors must be (batch, seq, heads, head_dim)")
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must be on a CUDA device (there is no CPU path)")
+        if t.dtype != torch.bfloat16:
+            raise ValueError("tensors must be bfloat16")
+        if t.shape != shape or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous and of equal shape")
+    return tuple(int(x) for x in shape)  # type: ignore[return-value]
+
+
+def _scale(scale: float | None, d: int) -> float:
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def fwd_into(q, k, v, o, lse, scale=None, causal=False, window=(-1, -1), stream=None) -> None:
+    """fa_fwd into caller-provided o (B,N,H,d) bf16 and lse (B,H,N) fp32."""
+    B, N, H, d = _check_qkv(q, k, v, o)
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous() or not lse.is_cuda:
+        raise ValueError("lse must be a contiguous (B, H, N) float32 CUDA tensor")
+    st = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, N, H, d,
+                       _scale(scale, d), int(bool(causal)), int(window[0]), int(window[1]), _stream_handle(stream))
+    _raise(st, "fa_fwd")
+
+
+def attention_fwd(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None):
+    """Forward: returns (o, lse) with o (B,N,H,d) bf16 and lse (B,H,N) fp32 (natural log)."""
+    B, N, H, d = _check_qkv(q, k, v)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    fwd_into(q, k, v, o, lse, scale, causal, window, stream)
+    return o, lse
+
+
+def workspace_bytes(B: int, N: int, H: int, d: int) -> int:
+    return int(load().fa_bwd_workspace_bytes(B, N, H, d))
+
+
+def bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale=None, causal=False, window=(-1, -1), workspace=None,
+             stream=None) -> None:
+    """fa_bwd into caller-provided dq, dk, dv. ``workspace``: uint8 CUDA tensor or None."""
+    B, N, H, d = _check_qkv(q, k, v, o, do, dq, dk, dv)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    st = load().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, d, _scale(scale, d),
+                       int(bool(causal)), int(window[0]), int(window[1]), ws_ptr, ws_bytes, _stream_handle(stream))
+    _raise(st, "fa_bwd")
+
+
+def attention_bwd(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1), workspace=None, stream=None):
+    """Backward: returns (dq, dk, dv), the gradients of sum(do * o)."""
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale, causal, window, workspace, stream)
+    return dq, dk, dv
+
+
+def bwd_stages(q, k, v, o, lse, do, dq, dk, dv, workspace, scale=None, causal=False, window=(-1, -1),
+               stream=None, between=None) -> None:
+    """The three launches of the backward issued one by one; ``between(i)`` runs before stage i
+    (i = 0, 1, 2) and once more after the last (i = 3) — e.g. to record CUDA events."""
+    B, N, H, d = _check_qkv(q, k, v, o, do, dq, dk, dv)
+    lib, s = load(), _stream_handle(stream)
+    ws, wb = workspace.data_ptr(), workspace.numel()
+    sc = _scale(scale, d)
+    if between:
+        between(0)
+    _raise(lib.fa_bwd_preprocess(o.data_ptr(), lse.data_ptr(), do.data_ptr(), B, N, H, d, ws, wb, s),
+           "fa_bwd_preprocess")
+    if between:
+        between(1)
+    _raise(lib.fa_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                           B, N, H, d, sc, int(bool(causal)), int(window[0]), int(window[1]), ws, wb, s),
+           "fa_bwd_main")
+    if between:
+        between(2)
+    _raise(lib.fa_bwd_dq_convert(dq.data_ptr(), B, N, H, d, ws, wb, s), "fa_bwd_dq_convert")
+    if between:
+        between(3)
+
+
+def check(stream=None) -> None:
+    """Synchronise and raise if a kernel recorded a device-side error (e.g. a wait timeout)."""
+    _raise(load().fa_check(_stream_handle(stream)), "fa_check")
+
+
+class FlashAttention(torch.autograd.Function):
+    """autograd wrapper: forward saves (q, k, v, o, lse); backward recomputes the scores."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale=None, causal=False, window=(-1, -1)):
+        o, lse = attention_fwd(q, k, v, scale, causal, window)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.args = (scale, causal, window)
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = attention_bwd(q, k, v, o, lse, do.contiguous(), *ctx.args)
+        return dq, dk, dv, None, None, None
+
+
+def flash_attention(q, k, v, scale=None, causal=False, window=(-1, -1)):
+    """Differentiable exact attention on (batch, seq, heads, head_dim) bf16 CUDA tensors."""
+    return FlashAttention.apply(q, k, v, scale, causal, window)

@@ -1,0 +1,405 @@
+// Host side of the fa_sm100 C ABI: argument validation, TMA tensor maps, per-device
+// kernel attributes, launches on the caller's stream and device-side error reporting.
+// The kernels live in fa_fwd.cuh / fa_bwd.cuh and are compiled into this one translation
+// unit (they share the device error word).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "fa_sm100.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+int g_sm_count[kMaxDevices] = {0};
+bool g_attr_done[kMaxDevices] = {false};
+bool g_is_sm100[kMaxDevices] = {false};
+
+EncodeTiledFn encode_fn() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return g_encode;
+}
+
+// Per-device set-up: SM count, sm_100 check, dynamic shared memory opt-in of every kernel.
+int device_setup(int* dev_out, int* sm_count) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_attr_done[dev]) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    g_is_sm100[dev] = (major == 10 && minor == 0);
+    g_sm_count[dev] = sms;
+    if (g_is_sm100[dev]) {
+      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::FwdCfg<64>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::FwdCfg<128>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdCfg<64>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdCfg<128>::kSmemBytes) != cudaSuccess)
+        return FA_ERR_CUDA;
+    }
+    g_attr_done[dev] = true;
+  }
+  if (!g_is_sm100[dev]) return FA_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  *sm_count = g_sm_count[dev];
+  return FA_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Shape {
+  int B, N, H, d;
+  size_t elems() const { return (size_t)B * N * H * d; }
+  size_t tensor_bytes() const { return elems() * 2; }
+  size_t rowvec_bytes() const { return (size_t)B * H * N * 4; }
+  int n_pad() const { return (N + 127) / 128 * 128; }
+};
+
+// Sizes, head dim, windows and scale. Windows are normalised: causal forces win_r = 0,
+// and a bound that reaches the whole sequence becomes -1 (unbounded).
+int check_problem(int B, int N, int H, int d, float scale, int causal, int* win_l, int* win_r) {
+  if (B < 1 || N < 1 || H < 1 || d < 1) return FA_ERR_INVALID_ARG;
+  if (*win_l < -1 || *win_r < -1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  // TMA: strides < 2^40 bytes; item counts and coordinates stay in int.
+  const double row_stride = (double)N * H * d * 2;
+  if (row_stride >= 1099511627776.0) return FA_ERR_INVALID_ARG;
+  if ((double)B * H * ((N + 127) / 128) >= 2147483647.0) return FA_ERR_INVALID_ARG;
+  if (causal) *win_r = 0;
+  if (*win_l >= N - 1) *win_l = -1;
+  if (*win_r >= N - 1) *win_r = -1;
+  return FA_OK;
+}
+
+// 4-D map over a (B, N, H, d) bf16 tensor: dims (d, N, H, B), box (64, 128, 1, 1), 128B swizzle.
+int make_map(CUtensorMap* m, const void* base, const Shape& s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)s.N, (cuuint64_t)s.H, (cuuint64_t)s.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)s.H * s.d * 2, (cuuint64_t)s.d * 2, (cuuint64_t)s.N * s.H * s.d * 2};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID_ARG;
+}
+
+struct Workspace {
+  float* dq_acc;
+  float* lse2;
+  float* dvec;
+};
+
+size_t workspace_bytes(const Shape& s) {
+  return align256(s.elems() * 4) + 2 * align256((size_t)s.B * s.H * s.n_pad() * 4);
+}
+
+Workspace carve(void* ws, const Shape& s) {
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  Workspace w;
+  w.dq_acc = reinterpret_cast<float*>(p);
+  p += align256(s.elems() * 4);
+  w.lse2 = reinterpret_cast<float*>(p);
+  p += align256((size_t)s.B * s.H * s.n_pad() * 4);
+  w.dvec = reinterpret_cast<float*>(p);
+  return w;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+bool log_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = std::getenv("FA_LOG");
+    on = (e && e[0] == '1') ? 1 : 0;
+  }
+  return on == 1;
+}
+
+// ---------------------------------------------------------------- launches (arguments already checked)
+
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& s, float scale,
+               int causal, int win_l, int win_r, int sm_count, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mo;
+  int st;
+  if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
+      (st = make_map(&mo, o, s)))
+    return st;
+  fa::FwdParams p;
+  p.B = s.B;
+  p.N = s.N;
+  p.H = s.H;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.win_l = win_l;
+  p.win_r = win_r;
+  p.causal = causal ? 1 : 0;
+  p.num_pairs = (s.N + 255) / 256;
+  p.num_items = s.B * s.H * p.num_pairs;
+  p.lse = lse;
+  const int grid = p.num_items < sm_count ? p.num_items : sm_count;
+  if (log_enabled())
+    std::fprintf(stderr, "[fa] fwd B=%d N=%d H=%d d=%d causal=%d win=(%d,%d) items=%d grid=%d smem=%d\n", s.B, s.N,
+                 s.H, s.d, p.causal, win_l, win_r, p.num_items, grid,
+                 s.d == 64 ? fa::FwdCfg<64>::kSmemBytes : fa::FwdCfg<128>::kSmemBytes);
+  if (s.d == 64)
+    fa::fa_fwd_kernel<64><<<grid, fa::FwdCfg<64>::kThreads, fa::FwdCfg<64>::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+  else
+    fa::fa_fwd_kernel<128><<<grid, fa::FwdCfg<128>::kThreads, fa::FwdCfg<128>::kSmemBytes, stream>>>(mq, mk, mv, mo,
+                                                                                                     p);
+  return launch_status();
+}
+
+int launch_pre(const void* o, const float* lse, const void* dO, const Shape& s, const Workspace& w,
+               cudaStream_t stream) {
+  const long long warps = (long long)s.B * s.n_pad() * s.H;
+  const long long blocks = (warps + 7) / 8;
+  if (s.d == 64)
+    fa::fa_bwd_pre_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.lse2, w.dvec, w.dq_acc,
+        s.B, s.N, s.H, s.n_pad());
+  else
+    fa::fa_bwd_pre_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.lse2, w.dvec, w.dq_acc,
+        s.B, s.N, s.H, s.n_pad());
+  return launch_status();
+}
+
+int launch_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, const Shape& s,
+                float scale, int causal, int win_l, int win_r, const Workspace& w, int sm_count,
+                cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  int st;
+  if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
+      (st = make_map(&mdo, dO, s)) || (st = make_map(&mdk, dk, s)) || (st = make_map(&mdv, dv, s)))
+    return st;
+  fa::BwdParams p;
+  p.B = s.B;
+  p.N = s.N;
+  p.H = s.H;
+  p.N_pad = s.n_pad();
+  p.scale = scale;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.win_l = win_l;
+  p.win_r = win_r;
+  p.causal = causal ? 1 : 0;
+  p.num_kv_tiles = (s.N + 127) / 128;
+  p.num_items = s.B * s.H * p.num_kv_tiles;
+  p.dq_acc = w.dq_acc;
+  p.lse2 = w.lse2;
+  p.dvec = w.dvec;
+  const int grid = p.num_items < sm_count ? p.num_items : sm_count;
+  if (log_enabled())
+    std::fprintf(stderr, "[fa] bwd B=%d N=%d H=%d d=%d causal=%d win=(%d,%d) items=%d grid=%d smem=%d\n", s.B, s.N,
+                 s.H, s.d, p.causal, win_l, win_r, p.num_items, grid,
+                 s.d == 64 ? fa::BwdCfg<64>::kSmemBytes : fa::BwdCfg<128>::kSmemBytes);
+  if (s.d == 64)
+    fa::fa_bwd_kernel<64><<<grid, fa::BwdCfg<64>::kThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(mq, mk, mv, mdo,
+                                                                                                   mdk, mdv, p);
+  else
+    fa::fa_bwd_kernel<128><<<grid, fa::BwdCfg<128>::kThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdk, mdv, p);
+  return launch_status();
+}
+
+int launch_convert(void* dq, const Shape& s, const Workspace& w, cudaStream_t stream) {
+  const long long n8 = (long long)(s.elems() / 8);
+  const long long blocks = (n8 + 255) / 256;
+  fa::fa_dq_convert_kernel<<<(unsigned)blocks, 256, 0, stream>>>(w.dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+  return launch_status();
+}
+
+// Common checks of the backward calls: problem, pointers, workspace.
+int check_workspace(void* workspace, size_t bytes, const Shape& s) {
+  if (!workspace || !aligned(workspace, 256) || bytes < workspace_bytes(s)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: head dim or device not supported";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA runtime error";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a device-side wait timed out";
+    case FA_ERR_NO_MEMORY: return "FA_ERR_NO_MEMORY: workspace allocation failed";
+    case FA_ERR_DEVICE: return "FA_ERR_DEVICE: a device-side check failed";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+size_t fa_bwd_workspace_bytes(int B, int N, int H, int d) {
+  int wl = -1, wr = -1;
+  if (check_problem(B, N, H, d, 1.0f, 0, &wl, &wr) != FA_OK) return 0;
+  return workspace_bytes(Shape{B, N, H, d});
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N, int H, int d, float scale,
+           int causal, int win_l, int win_r, fa_stream_t stream) {
+  int st = check_problem(B, N, H, d, scale, causal, &win_l, &win_r);
+  if (st) return st;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return FA_ERR_INVALID_ARG;
+  const Shape s{B, N, H, d};
+  const size_t tb = s.tensor_bytes(), lb = s.rowvec_bytes();
+  if (overlap(o, tb, q, tb) || overlap(o, tb, k, tb) || overlap(o, tb, v, tb) || overlap(lse, lb, q, tb) ||
+      overlap(lse, lb, k, tb) || overlap(lse, lb, v, tb) || overlap(lse, lb, o, tb))
+    return FA_ERR_INVALID_ARG;
+  int dev, sms;
+  if ((st = device_setup(&dev, &sms))) return st;
+  return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd_preprocess(const void* o, const float* lse, const void* dO, int B, int N, int H, int d, void* workspace,
+                      size_t workspace_bytes_, fa_stream_t stream) {
+  int wl = -1, wr = -1;
+  int st = check_problem(B, N, H, d, 1.0f, 0, &wl, &wr);
+  if (st) return st;
+  const Shape s{B, N, H, d};
+  if (!o || !lse || !dO || !aligned(o, 16) || !aligned(dO, 16) || !aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  if ((st = check_workspace(workspace, workspace_bytes_, s))) return st;
+  const size_t tb = s.tensor_bytes(), wb = workspace_bytes(s), lb = s.rowvec_bytes();
+  if (overlap(workspace, wb, o, tb) || overlap(workspace, wb, dO, tb) || overlap(workspace, wb, lse, lb))
+    return FA_ERR_INVALID_ARG;
+  int dev, sms;
+  if ((st = device_setup(&dev, &sms))) return st;
+  return launch_pre(o, lse, dO, s, carve(workspace, s), reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, int B, int N, int H,
+                int d, float scale, int causal, int win_l, int win_r, void* workspace, size_t workspace_bytes_,
+                fa_stream_t stream) {
+  int st = check_problem(B, N, H, d, scale, causal, &win_l, &win_r);
+  if (st) return st;
+  const Shape s{B, N, H, d};
+  if (!q || !k || !v || !dO || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(dO, 16) || !aligned(dk, 16) ||
+      !aligned(dv, 16))
+    return FA_ERR_INVALID_ARG;
+  if ((st = check_workspace(workspace, workspace_bytes_, s))) return st;
+  const size_t tb = s.tensor_bytes(), wb = workspace_bytes(s);
+  const void* ins[4] = {q, k, v, dO};
+  for (const void* in : ins)
+    if (overlap(dk, tb, in, tb) || overlap(dv, tb, in, tb) || overlap(workspace, wb, in, tb)) return FA_ERR_INVALID_ARG;
+  if (overlap(dk, tb, dv, tb) || overlap(workspace, wb, dk, tb) || overlap(workspace, wb, dv, tb))
+    return FA_ERR_INVALID_ARG;
+  int dev, sms;
+  if ((st = device_setup(&dev, &sms))) return st;
+  return launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, carve(workspace, s), sms,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd_dq_convert(void* dq, int B, int N, int H, int d, void* workspace, size_t workspace_bytes_,
+                      fa_stream_t stream) {
+  int wl = -1, wr = -1;
+  int st = check_problem(B, N, H, d, 1.0f, 0, &wl, &wr);
+  if (st) return st;
+  const Shape s{B, N, H, d};
+  if (!dq || !aligned(dq, 16)) return FA_ERR_INVALID_ARG;
+  if ((st = check_workspace(workspace, workspace_bytes_, s))) return st;
+  if (overlap(workspace, workspace_bytes(s), dq, s.tensor_bytes())) return FA_ERR_INVALID_ARG;
+  int dev, sms;
+  if ((st = device_setup(&dev, &sms))) return st;
+  return launch_convert(dq, s, carve(workspace, s), reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+           void* dk, void* dv, int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
+           void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_problem(B, N, H, d, scale, causal, &win_l, &win_r);
+  if (st) return st;
+  const Shape s{B, N, H, d};
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  const void* ptrs[8] = {q, k, v, o, dO, dq, dk, dv};
+  for (const void* x : ptrs)
+    if (!aligned(x, 16)) return FA_ERR_INVALID_ARG;
+  if (!aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  const size_t tb = s.tensor_bytes(), lb = s.rowvec_bytes();
+  const void* ins[5] = {q, k, v, o, dO};
+  void* outs[3] = {dq, dk, dv};
+  for (void* out : outs) {
+    for (const void* in : ins)
+      if (overlap(out, tb, in, tb)) return FA_ERR_INVALID_ARG;
+    if (overlap(out, tb, lse, lb)) return FA_ERR_INVALID_ARG;
+  }
+  if (overlap(dq, tb, dk, tb) || overlap(dq, tb, dv, tb) || overlap(dk, tb, dv, tb)) return FA_ERR_INVALID_ARG;
+  if (workspace) {
+    if ((st = check_workspace(workspace, workspace_bytes_, s))) return st;
+    const size_t wb = workspace_bytes(s);
+    for (const void* in : ins)
+      if (overlap(workspace, wb, in, tb)) return FA_ERR_INVALID_ARG;
+    for (void* out : outs)
+      if (overlap(workspace, wb, out, tb)) return FA_ERR_INVALID_ARG;
+    if (overlap(workspace, wb, lse, lb)) return FA_ERR_INVALID_ARG;
+  }
+  int dev, sms;
+  if ((st = device_setup(&dev, &sms))) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  const size_t wbytes = workspace_bytes(s);
+  if (!ws) {
+    if (cudaMallocAsync(&ws, wbytes, cs) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_NO_MEMORY;
+    }
+  }
+  const Workspace w = carve(ws, s);
+  st = launch_pre(o, lse, dO, s, w, cs);
+  if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs);
+  if (!st) st = launch_convert(dq, s, w, cs);
+  if (!workspace && cudaFreeAsync(ws, cs) != cudaSuccess && !st) st = FA_ERR_CUDA;
+  return st;
+}
+
+int fa_check(fa_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int err = 0;
+  if (cudaMemcpyFromSymbol(&err, fa::g_fa_error, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (err == 0) return FA_OK;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(fa::g_fa_error, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  return (err & fa::kErrWaitTimeout) ? FA_ERR_TIMEOUT : FA_ERR_DEVICE;
+}
+
+}  // extern "C"

@@ -1,0 +1,469 @@
+// Forward kernel of exact attention for sm_100a.
+//
+// What it computes ("Flash Attention V2核心网络算子解析" §二.1; "FlashAttention 剖析" §3):
+// for every (b, h) and query row i, O_i = sum_j softmax_j(scale * q_i . k_j) v_j over the
+// keys j visible to i (causal / (left, right) window), and LSE_i = ln sum_j exp(scale * q_i . k_j).
+// Keys are visited in 128-key tiles with a running maximum and running sum per row
+// ("FlashAttention技术解析：加速GPT训练的核心优化" §1 item 3), so the N x N score matrix
+// never leaves the SM.
+//
+// Work decomposition (persistent, one CTA per SM):
+//   work item = (b, h, pair of 128-row Q tiles); the two Q tiles share every K/V tile load.
+//   warp 0      : TMA producer (Q tiles; a ring of K/V tile slots)
+//   warp 1      : tcgen05 MMA issuer (one elected thread) and TMEM owner
+//   warps 2-3   : no role
+//   warps 4-7   : softmax + epilogue for Q tile 0 (one thread per query row / TMEM lane)
+//   warps 8-11  : softmax + epilogue for Q tile 1
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
+// P_t (bf16, two per column) overwrites the first 64 columns of S_t and is the A operand
+// of O_t += P_t V_j, read straight from TMEM.
+//
+// MMA issue order per KV tile j: S0(j), PV1(j-1), S1(j), PV0(j). tcgen05.mma operations
+// issued by one thread execute in order, so S_t(j) never overwrites P_t(j-1) before
+// PV_t(j-1) has read it, and the commit that signals "S_t(j) ready" also covers PV_t(j-1):
+// when a softmax thread sees S_t(j), O_t is quiescent and may be rescaled in place.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  int B, N, H;
+  float scale_log2;  // softmax scale * log2(e)
+  int win_l;         // -1 = unbounded
+  int win_r;         // effective right bound (0 under causal), -1 = unbounded
+  int causal;
+  int num_pairs;     // ceil(N / 256)
+  int num_items;     // B * H * num_pairs
+  float* lse;        // (B, H, N) fp32
+};
+
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kThreads = 384;
+  static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile of Q, K, V or O
+  static constexpr int kBoxes = D / 64;           // 64-column (128-byte) TMA boxes per tile
+  static constexpr int kSlots = (D == 128) ? 4 : 8;
+  static constexpr int kOffQ = 0;                 // Q0, Q1 (also O staging)
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
+  static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+// Barrier block at the end of shared memory.
+template <int D>
+struct FwdBars {
+  uint64_t q_full[2], q_empty[2];
+  uint64_t kv_full[FwdCfg<D>::kSlots], kv_empty[FwdCfg<D>::kSlots];
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Item w -> (b, h, pair). Under causal masking pairs are visited longest first.
+__device__ __forceinline__ void fwd_decode(const FwdParams& p, int w, int& b, int& h, int& pair) {
+  const int bh_count = p.B * p.H;
+  const int r = w / bh_count, bh = w - r * bh_count;
+  pair = p.causal ? (p.num_pairs - 1 - r) : r;
+  b = bh / p.H;
+  h = bh - b * p.H;
+}
+
+// KV tiles visible from Q rows [r0, min(r0+127, N-1)]; empty (hi < lo) if r0 >= N.
+__device__ __forceinline__ void fwd_kv_range(const FwdParams& p, int r0, int& lo, int& hi) {
+  if (r0 >= p.N) { lo = 0; hi = -1; return; }
+  const int r1 = min(r0 + 127, p.N - 1);
+  const int kmin = p.win_l >= 0 ? max(0, r0 - p.win_l) : 0;
+  const int kmax = p.win_r >= 0 ? min(p.N - 1, r1 + p.win_r) : p.N - 1;
+  lo = kmin >> 7;
+  hi = kmax >> 7;
+}
+
+// True when every valid row of the Q tile sees every key of KV tile j (no masking needed).
+__device__ __forceinline__ bool fwd_tile_unmasked(const FwdParams& p, int r0, int j) {
+  const int r1 = min(r0 + 127, p.N - 1);
+  const int k0 = j * 128, k1 = k0 + 127;
+  if (k1 >= p.N) return false;
+  if (p.win_l >= 0 && k0 < r1 - p.win_l) return false;
+  if (p.win_r >= 0 && k1 > r0 + p.win_r) return false;
+  return true;
+}
+
+// ------------------------------------------------------------------ softmax role
+
+template <int D, bool kPosScale>
+__device__ __forceinline__ void fwd_softmax_tile(float (&x)[128], bool masked, int kbase, int kmin, int kmax,
+                                                 float c, float& m_run, float& l_run, uint32_t (&pk)[64],
+                                                 float& alpha, bool& updated) {
+  // 1. mask and tile maximum (in scaled log2 units)
+  float mx[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+  if (masked) {
+#pragma unroll
+    for (int cc = 0; cc < 128; ++cc) {
+      const int key = kbase + cc;
+      const bool vis = (key >= kmin) & (key <= kmax);
+      x[cc] = vis ? (kPosScale ? x[cc] : x[cc] * c) : -INFINITY;
+      mx[cc & 7] = fmaxf(mx[cc & 7], x[cc]);
+    }
+  } else {
+#pragma unroll
+    for (int cc = 0; cc < 128; ++cc) {
+      if (!kPosScale) x[cc] *= c;
+      mx[cc & 7] = fmaxf(mx[cc & 7], x[cc]);
+    }
+  }
+  float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+  if (kPosScale) m_tile *= c;
+
+  // 2. lazy update of the reference maximum
+  const float m_new = fmaxf(m_run, m_tile);
+  updated = m_new > m_run + kRescaleThreshold;
+  alpha = 1.0f;
+  if (updated) {
+    alpha = ex2_approx(m_run - m_new);  // 0 when m_run was -inf
+    m_run = m_new;
+  }
+  const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+
+  // 3. exponentials, row sum, bf16 packing (even column in the low half)
+  float sum[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) sum[u] = 0.0f;
+#pragma unroll
+  for (int cc = 0; cc < 128; cc += 2) {
+    float p0, p1;
+    if (kPosScale) {
+      p0 = ex2_approx(fmaf(x[cc], c, -m_use));
+      p1 = ex2_approx(fmaf(x[cc + 1], c, -m_use));
+    } else {
+      p0 = ex2_approx(x[cc] - m_use);
+      p1 = ex2_approx(x[cc + 1] - m_use);
+    }
+    sum[(cc >> 1) & 7] += p0 + p1;
+    pk[cc >> 1] = pack_bf16x2(p0, p1);
+  }
+  const float s_tile = ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
+  l_run = l_run * alpha + s_tile;
+}
+
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdParams p) {
+  using Cfg = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
+  FwdBars<D>* bars = reinterpret_cast<FwdBars<D>*>(smem_gen + Cfg::kOffBar);
+  auto bar = [&](uint64_t& b) { return smem_u32(&b); };
+
+  const int warp = threadIdx.x >> 5;
+  const Abort ab{&bars->abort_flag};
+
+  if (threadIdx.x == 0) {
+    bars->abort_flag = 0;
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(bars->q_full[t]), 1);
+      mbar_init(bar(bars->q_empty[t]), 1);
+      mbar_init(bar(bars->s_full[t]), 1);
+      mbar_init(bar(bars->p_full[t]), 128);
+      mbar_init(bar(bars->o_full[t]), 1);
+      mbar_init(bar(bars->o_empty[t]), 128);
+    }
+    for (int s = 0; s < Cfg::kSlots; ++s) {
+      mbar_init(bar(bars->kv_full[s]), 1);
+      mbar_init(bar(bars->kv_empty[s]), 1);
+    }
+    mbar_init(bar(bars->mma_done), 1);
+    fence_barrier_init();
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), Cfg::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before_sync();
+  }
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+
+  const uint32_t sQ[2] = {smem_base + Cfg::kOffQ, smem_base + Cfg::kOffQ + Cfg::kTileBytes};
+  const uint32_t sKV = smem_base + Cfg::kOffKV;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane_id() == 0) {
+      uint32_t slot = 0, phase = 0;
+      uint32_t qn[2] = {0, 0};
+      int last_slot_parity[Cfg::kSlots];
+      for (int s = 0; s < Cfg::kSlots; ++s) last_slot_parity[s] = -1;
+      for (int round = 0;; ++round) {
+        const int w = sched_item(round, blockIdx.x, gridDim.x);
+        if (w >= p.num_items || ab.raised()) break;
+        int b, h, pair;
+        fwd_decode(p, w, b, h, pair);
+        int lo_t[2], hi_t[2];
+        fwd_kv_range(p, pair * 256, lo_t[0], hi_t[0]);
+        fwd_kv_range(p, pair * 256 + 128, lo_t[1], hi_t[1]);
+        const bool act1 = hi_t[1] >= lo_t[1];
+        const int lo = act1 ? min(lo_t[0], lo_t[1]) : lo_t[0];
+        const int hi = act1 ? max(hi_t[0], hi_t[1]) : hi_t[0];
+        for (int t = 0; t < 2; ++t) {
+          if (hi_t[t] < lo_t[t]) continue;
+          mbar_wait(bar(bars->q_empty[t]), (qn[t] & 1) ^ 1, ab);
+          mbar_arrive_expect_tx(bar(bars->q_full[t]), Cfg::kTileBytes);
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+            tma_load_4d(sQ[t] + bx * 16384, &tmQ, bar(bars->q_full[t]), bx * 64, pair * 256 + t * 128, h, b);
+          ++qn[t];
+        }
+        for (int j = lo; j <= hi; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            mbar_wait(bar(bars->kv_empty[slot]), phase ^ 1, ab);
+            mbar_arrive_expect_tx(bar(bars->kv_full[slot]), Cfg::kTileBytes);
+            const uint32_t dst = sKV + slot * Cfg::kTileBytes;
+#pragma unroll
+            for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+              tma_load_4d(dst + bx * 16384, kv ? &tmV : &tmK, bar(bars->kv_full[slot]), bx * 64, j * 128, h, b);
+            last_slot_parity[slot] = phase;
+            if (++slot == Cfg::kSlots) { slot = 0; phase ^= 1; }
+          }
+        }
+      }
+      // Drain: every load issued must have landed before the CTA can exit.
+      for (int s = 0; s < Cfg::kSlots; ++s)
+        if (last_slot_parity[s] >= 0) mbar_drain(bar(bars->kv_full[s]), last_slot_parity[s]);
+      for (int t = 0; t < 2; ++t)
+        if (qn[t] > 0) mbar_drain(bar(bars->q_full[t]), (qn[t] - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (elect_one()) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // S = Q K^T, both K-major
+      constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // O += P V, V is MN-major
+      const uint32_t tS[2] = {tmem + Cfg::kColS0, tmem + Cfg::kColS1};
+      const uint32_t tO[2] = {tmem + Cfg::kColO0, tmem + Cfg::kColO1};
+      uint32_t slot = 0, phase = 0;
+      uint32_t qn[2] = {0, 0}, pn[2] = {0, 0};
+
+      auto issue_s = [&](int t, uint32_t k_smem) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tS[t], sdesc_kmajor(sQ[t] + off), sdesc_kmajor(k_smem + off), idS, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, uint32_t v_smem, bool accumulate) {
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts(tO[t], tS[t] + kk * 8, sdesc_mnmajor(v_smem + kk * 2048, 16384), idO, accumulate || kk > 0);
+      };
+
+      for (int round = 0;; ++round) {
+        const int w = sched_item(round, blockIdx.x, gridDim.x);
+        if (w >= p.num_items || ab.raised()) break;
+        int b, h, pair;
+        fwd_decode(p, w, b, h, pair);
+        int lo_t[2], hi_t[2];
+        fwd_kv_range(p, pair * 256, lo_t[0], hi_t[0]);
+        fwd_kv_range(p, pair * 256 + 128, lo_t[1], hi_t[1]);
+        const bool act[2] = {true, hi_t[1] >= lo_t[1]};
+        const int lo = act[1] ? min(lo_t[0], lo_t[1]) : lo_t[0];
+        const int hi = act[1] ? max(hi_t[0], hi_t[1]) : hi_t[0];
+        auto active = [&](int t, int j) { return act[t] && j >= lo_t[t] && j <= hi_t[t]; };
+        bool first_pv[2] = {true, true};
+        for (int t = 0; t < 2; ++t)
+          if (act[t]) mbar_wait(bar(bars->q_full[t]), qn[t] & 1, ab);
+        tc_fence_after_sync();
+
+        uint32_t v_prev_slot = 0;
+        auto wait_p_and_o = [&](int t) {
+          mbar_wait(bar(bars->p_full[t]), pn[t] & 1, ab);
+          ++pn[t];
+          if (first_pv[t]) mbar_wait(bar(bars->o_empty[t]), (qn[t] & 1) ^ 1, ab);
+          tc_fence_after_sync();
+        };
+        for (int j = lo; j <= hi + 1; ++j) {
+          uint32_t k_slot = 0;
+          if (j <= hi) {
+            k_slot = slot;
+            mbar_wait(bar(bars->kv_full[slot]), phase, ab);
+            if (++slot == Cfg::kSlots) { slot = 0; phase ^= 1; }
+            tc_fence_after_sync();
+            if (active(0, j)) {
+              issue_s(0, sKV + k_slot * Cfg::kTileBytes);
+              mma_commit(bar(bars->s_full[0]));
+            }
+          }
+          if (j - 1 >= lo) {
+            if (active(1, j - 1)) {
+              wait_p_and_o(1);
+              issue_pv(1, sKV + v_prev_slot * Cfg::kTileBytes, !first_pv[1]);
+              first_pv[1] = false;
+              if (j - 1 == hi_t[1]) mma_commit(bar(bars->o_full[1]));
+            }
+            mma_commit(bar(bars->kv_empty[v_prev_slot]));
+          }
+          if (j <= hi) {
+            if (active(1, j)) {
+              issue_s(1, sKV + k_slot * Cfg::kTileBytes);
+              mma_commit(bar(bars->s_full[1]));
+            }
+            mma_commit(bar(bars->kv_empty[k_slot]));
+            const uint32_t v_slot = slot;
+            mbar_wait(bar(bars->kv_full[slot]), phase, ab);
+            if (++slot == Cfg::kSlots) { slot = 0; phase ^= 1; }
+            tc_fence_after_sync();
+            if (active(0, j)) {
+              wait_p_and_o(0);
+              issue_pv(0, sKV + v_slot * Cfg::kTileBytes, !first_pv[0]);
+              first_pv[0] = false;
+              if (j == hi_t[0]) mma_commit(bar(bars->o_full[0]));
+            }
+            v_prev_slot = v_slot;
+          }
+        }
+        for (int t = 0; t < 2; ++t)
+          if (act[t]) ++qn[t];
+      }
+      mma_commit(bar(bars->mma_done));
+      mbar_drain(bar(bars->mma_done), 0);
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- softmax + epilogue
+    const int t = (warp - 4) >> 2;           // Q tile of the pair handled by this warpgroup
+    const int row = threadIdx.x - 128 * (1 + t);  // 0..127: TMEM lane and row within the tile
+    const uint32_t lane_field = (uint32_t)((row & ~31) << 16);
+    const uint32_t tS = tmem + lane_field + (t ? Cfg::kColS1 : Cfg::kColS0);
+    const uint32_t tO = tmem + lane_field + (t ? Cfg::kColO1 : Cfg::kColO0);
+    const float c = p.scale_log2;
+    uint32_t sn = 0, on = 0;
+
+    for (int round = 0;; ++round) {
+      const int w = sched_item(round, blockIdx.x, gridDim.x);
+      if (w >= p.num_items || ab.raised()) break;
+      int b, h, pair;
+      fwd_decode(p, w, b, h, pair);
+      const int r0 = pair * 256 + t * 128;
+      int lo, hi;
+      fwd_kv_range(p, r0, lo, hi);
+      if (hi < lo) continue;
+      const int i = r0 + row;
+      const int kmin = p.win_l >= 0 ? i - p.win_l : 0;
+      const int kmax = p.win_r >= 0 ? min(p.N - 1, i + p.win_r) : p.N - 1;
+      float m_run = -INFINITY, l_run = 0.0f;
+
+      for (int j = lo; j <= hi; ++j) {
+        mbar_wait(bar(bars->s_full[t]), sn & 1, ab);
+        ++sn;
+        tc_fence_after_sync();
+        uint32_t r[4][32];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, r[q4]);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tmem_wait_ld(r[q4]);
+        float x[128];
+#pragma unroll
+        for (int cc = 0; cc < 128; ++cc) x[cc] = __uint_as_float(r[cc >> 5][cc & 31]);
+
+        const bool masked = !fwd_tile_unmasked(p, r0, j);
+        uint32_t pk[64];
+        float alpha;
+        bool updated;
+        if (c > 0.0f)
+          fwd_softmax_tile<D, true>(x, masked, j * 128, kmin, kmax, c, m_run, l_run, pk, alpha, updated);
+        else
+          fwd_softmax_tile<D, false>(x, masked, j * 128, kmin, kmax, c, m_run, l_run, pk, alpha, updated);
+
+        // Rescale O_t in TMEM when this warp's reference maximum moved (not on the first tile:
+        // the first PV of an item overwrites O_t).
+        if (__any_sync(0xffffffffu, updated && j > lo)) {
+#pragma unroll 1
+          for (int cc = 0; cc < D; cc += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc, o);
+            tmem_wait_ld(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + cc, o);
+          }
+        }
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t v16[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v16[e] = pk[q4 * 16 + e];
+          tmem_st16(tS + q4 * 16, v16);
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(bar(bars->p_full[t]));
+      }
+
+      // Epilogue: O_t / l -> bf16 -> staging (the Q_t buffer, free once the last PV_t is done) -> TMA store.
+      mbar_wait(bar(bars->o_full[t]), on & 1, ab);
+      ++on;
+      tc_fence_after_sync();
+      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+      const uint32_t stage = sQ[t];
+#pragma unroll 1
+      for (int cc = 0; cc < D; cc += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc, o);
+        tmem_wait_ld(o);
+        const uint32_t box = stage + (cc >> 6) * 16384;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w4[e] = pack_bf16x2(__uint_as_float(o[ch * 8 + 2 * e]) * inv_l, __uint_as_float(o[ch * 8 + 2 * e + 1]) * inv_l);
+          st_shared_v4(box + sw128_offset(row, ((cc & 63) >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(bar(bars->o_empty[t]));
+      fence_proxy_async_smem();
+      named_bar_sync(1 + t, 128);
+      if (row == 0) {
+#pragma unroll
+        for (int bx = 0; bx < Cfg::kBoxes; ++bx) tma_store_4d(&tmO, stage + bx * 16384, bx * 64, r0, h, b);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        mbar_arrive(bar(bars->q_empty[t]));
+      }
+      if (i < p.N) {
+        const float lse = l_run > 0.0f ? (m_run + lg2_approx(l_run)) * kLn2 : -INFINITY;
+        p.lse[((size_t)b * p.H + h) * (size_t)p.N + i] = lse;
+      }
+    }
+    if (row == 0) bulk_wait_group0();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace fa

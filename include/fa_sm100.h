@@ -1,0 +1,116 @@
+/*
+ * fa_sm100 — exact scaled-dot-product attention for NVIDIA B200 (sm_100a), C ABI.
+ *
+ * The operation ("Flash Attention V2核心网络算子解析" §二.1, the attention formula;
+ * "FlashAttention技术解析：加速GPT训练的核心优化" §2.2, the call's causal / window_size /
+ * softmax_scale arguments; "突破大模型训练瓶颈：Flash-Attention编译优化与内存占用解决方案",
+ * 滑动窗口注意力, window_size=(left, right)):
+ *
+ *   S_ij   = scale * q_i . k_j          for keys j visible to query i, else -inf
+ *   O_i    = sum_j softmax_j(S_i.) v_j
+ *   LSE_i  = ln sum_j exp(S_ij)          (natural log)
+ *
+ * Visibility: 0 <= j < N, and (win_l == -1 or j >= i - win_l), and
+ * (win_r' == -1 or j <= i + win_r'), with win_r' = 0 when causal != 0, else win_r.
+ * Window bounds are inclusive; -1 means unbounded. Every query sees at least itself.
+ *
+ * Layout and types (all calls):
+ *   q, k, v, o, dO, dq, dk, dv : contiguous (B, N, H, d) bfloat16 in device memory,
+ *                                 base address 16-byte aligned (a TMA requirement).
+ *   lse                         : contiguous (B, H, N) float32 in device memory.
+ *   d (head dim)                : 64 or 128; anything else returns FA_ERR_UNSUPPORTED.
+ *   B, N, H                     : >= 1. scale: any finite float (0 gives uniform weights).
+ *
+ * Ownership: the caller owns every buffer. The library keeps only per-device caches
+ * (SM count, kernel attributes) and one device-side error word per device.
+ *
+ * Asynchrony and errors: every compute call validates its arguments on the host and
+ * returns an fa_status before launching anything; kernels then run asynchronously on
+ * `stream` (the legacy default stream when NULL). A launch failure returns FA_ERR_CUDA.
+ * Inside the kernels every wait is bounded (about 2 s); a wait that gives up records an
+ * error that fa_check() reports as FA_ERR_TIMEOUT, instead of hanging the GPU.
+ * Outputs must not overlap inputs (FA_ERR_INVALID_ARG).
+ * Thread safety: calls may be made from several host threads.
+ */
+#ifndef FA_SM100_H
+#define FA_SM100_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;                      /* same type as cudaStream_t */
+typedef struct CUstream_st* fa_stream_t;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size or window, non-finite scale, aliasing */
+  FA_ERR_UNSUPPORTED = 2,  /* head dim other than 64 / 128, or no sm_100 device */
+  FA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+  FA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (reported by fa_check) */
+  FA_ERR_NO_MEMORY = 5,    /* workspace allocation failed */
+  FA_ERR_DEVICE = 6        /* another device-side check failed (reported by fa_check) */
+} fa_status;
+
+/*
+ * Forward pass. Writes o (B,N,H,d) bf16 and lse (B,H,N) fp32 (natural log).
+ * One kernel launch on `stream`.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
+           fa_stream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: a float32 dQ accumulator (B,N,H,d) and two
+ * float32 (B,H,ceil(N/128)*128) row vectors (LSE*log2(e) and D = rowsum(dO*O)), each
+ * region 256-byte aligned. Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_bytes(int B, int N, int H, int d);
+
+/*
+ * Backward pass: given the forward's inputs, its outputs o and lse, and the upstream
+ * gradient dO, writes dq, dk, dv (B,N,H,d) bf16 — the gradients of sum(dO * O).
+ * `workspace` (device, 256-byte aligned, at least fa_bwd_workspace_bytes) is scratch
+ * the call overwrites; if it is NULL the call allocates it with cudaMallocAsync on
+ * `stream` and frees it with cudaFreeAsync after its launches.
+ * Three launches on `stream`: fa_bwd_preprocess, fa_bwd_main, fa_bwd_dq_convert.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv,
+           int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
+           void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * The three launches of fa_bwd, exposed so that a caller can time or interleave them.
+ * Same arguments and rules as fa_bwd, except that `workspace` must be non-NULL and must
+ * be the same buffer for the three calls of one backward, issued in this order.
+ *   fa_bwd_preprocess : D = rowsum(dO * O), LSE*log2(e), dQ accumulator := 0
+ *   fa_bwd_main       : dK, dV (written to dk, dv) and the dQ accumulator
+ *   fa_bwd_dq_convert : dq = bf16(dQ accumulator)
+ */
+int fa_bwd_preprocess(const void* o, const float* lse, const void* dO,
+                      int B, int N, int H, int d, void* workspace, size_t workspace_bytes,
+                      fa_stream_t stream);
+int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv,
+                int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
+                void* workspace, size_t workspace_bytes, fa_stream_t stream);
+int fa_bwd_dq_convert(void* dq, int B, int N, int H, int d, void* workspace, size_t workspace_bytes,
+                      fa_stream_t stream);
+
+/*
+ * Synchronises `stream` on the current device and reports what the kernels recorded:
+ * FA_ERR_TIMEOUT if a device wait gave up, FA_ERR_DEVICE for another device-side check,
+ * FA_ERR_CUDA if the synchronisation itself failed, else FA_OK. Clears the record.
+ */
+int fa_check(fa_stream_t stream);
+
+/* Static, human-readable name of a status code. Never NULL. */
+const char* fa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H */

@@ -140,19 +140,26 @@ def head_backward(q, k, v, do, scale, causal=False, win_l=-1, win_r=-1, block_ro
     dv = np.zeros_like(v, dtype=np.float64)
     dvec = np.zeros(n, dtype=np.float64)
     for r0, r1 in _row_blocks(n, block_rows):
-        c0, c1 = visible_key_span(r0, r1, k.shape[0], causal, win_l, win_r)
-        rows = np.arange(r0, r1)
-        s = _head_scores(q, k, rows, slice(c0, c1), scale, causal, win_l, win_r)
-        p, _ = _softmax_rows(s)
-        g = do[r0:r1]
-        dv[c0:c1] += p.T @ g
-        dp = g @ v[c0:c1].T
-        d_i = (p * dp).sum(axis=1)
-        ds = p * (dp - d_i[:, None])
-        dq[r0:r1] = scale * (ds @ k[c0:c1])
-        dk[c0:c1] += scale * (ds.T @ q[r0:r1])
-        dvec[r0:r1] = d_i
+        backward_rows(q, k, v, do, r0, r1, scale, causal, win_l, win_r, dq, dk, dv, dvec)
     return dq, dk, dv, dvec
+
+
+def backward_rows(q, k, v, do, r0, r1, scale, causal, win_l, win_r, dq, dk, dv, dvec):
+    """Contribution of query rows [r0, r1) of one head to the gradients (added into dk, dv;
+    dq and dvec rows [r0, r1) written). Summing it over a partition of the rows gives the
+    whole backward."""
+    c0, c1 = visible_key_span(r0, r1, k.shape[0], causal, win_l, win_r)
+    rows = np.arange(r0, r1)
+    s = _head_scores(q, k, rows, slice(c0, c1), scale, causal, win_l, win_r)
+    p, _ = _softmax_rows(s)
+    g = do[r0:r1]
+    dv[c0:c1] += p.T @ g
+    dp = g @ v[c0:c1].T
+    d_i = (p * dp).sum(axis=1)
+    ds = p * (dp - d_i[:, None])
+    dq[r0:r1] = scale * (ds @ k[c0:c1])
+    dk[c0:c1] += scale * (ds.T @ q[r0:r1])
+    dvec[r0:r1] = d_i
 
 
 def _as_f64(x) -> np.ndarray:

@@ -1,0 +1,126 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol include/fa_sm100.h
+declares, and rejects invalid arguments before launching anything. No GPU is touched:
+every call here fails validation (fake pointers are never dereferenced).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from exact_attention_116_b200 import binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa_sm100.h")
+
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+P = 0x7F0000000000  # a 16-byte aligned fake device address, far from anything real
+T = 1 << 30         # spacing that keeps fake tensors disjoint
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def declared_functions():
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:int|size_t|const char\*)\s+(fa_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_check", "fa_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) == set(binding.EXPORTS)
+
+
+def test_status_strings(lib):
+    for code, name in binding.STATUS_NAMES.items():
+        assert lib.fa_status_string(code).decode().startswith(name)
+    assert lib.fa_status_string(99).decode() == "FA_ERR_UNKNOWN"
+
+
+def test_workspace_bytes(lib):
+    def expect(B, N, H, d):
+        a = lambda x: (x + 255) // 256 * 256  # noqa: E731
+        npad = (N + 127) // 128 * 128
+        return a(B * N * H * d * 4) + 2 * a(B * H * npad * 4)
+
+    for shape in [(1, 1, 1, 64), (2, 8192, 16, 128), (1, 129, 3, 64), (4, 2048, 16, 64)]:
+        assert lib.fa_bwd_workspace_bytes(*shape) == expect(*shape)
+    assert lib.fa_bwd_workspace_bytes(0, 128, 1, 64) == 0
+    assert lib.fa_bwd_workspace_bytes(1, 128, 1, 96) == 0
+
+
+def _fwd(lib, q=P, k=P + T, v=P + 2 * T, o=P + 3 * T, lse=P + 4 * T, B=1, N=128, H=2, d=64, scale=0.125,
+         causal=0, wl=-1, wr=-1):
+    return lib.fa_fwd(q, k, v, o, lse, B, N, H, d, ctypes.c_float(scale), causal, wl, wr, None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(q=0), INVALID), (dict(k=0), INVALID), (dict(v=0), INVALID), (dict(o=0), INVALID), (dict(lse=0), INVALID),
+    (dict(B=0), INVALID), (dict(N=0), INVALID), (dict(H=0), INVALID), (dict(N=-5), INVALID),
+    (dict(d=96), UNSUPPORTED), (dict(d=256), UNSUPPORTED), (dict(d=0), INVALID),
+    (dict(wl=-2), INVALID), (dict(wr=-7), INVALID),
+    (dict(scale=float("nan")), INVALID), (dict(scale=float("inf")), INVALID),
+    (dict(q=P + 8), INVALID), (dict(o=P + 3 * T + 2), INVALID), (dict(lse=P + 4 * T + 2), INVALID),
+    (dict(o=P), INVALID),            # output aliases q
+    (dict(lse=P + T + 64), INVALID),  # lse inside k
+])
+def test_fwd_rejects_invalid_arguments(lib, kw, expected):
+    assert _fwd(lib, **kw) == expected
+
+
+def _bwd(lib, ws=P + 9 * T, ws_bytes=None, dq=P + 6 * T, dk=P + 7 * T, dv=P + 8 * T, B=1, N=128, H=2, d=64,
+         scale=0.125, wl=-1, wr=-1):
+    if ws_bytes is None:
+        ws_bytes = lib.fa_bwd_workspace_bytes(B, N, H, d) if B > 0 and N > 0 and H > 0 else 0
+    return lib.fa_bwd(P, P + T, P + 2 * T, P + 3 * T, P + 4 * T, P + 5 * T, dq, dk, dv, B, N, H, d,
+                      ctypes.c_float(scale), 0, wl, wr, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(dq=0), INVALID), (dict(B=0), INVALID), (dict(d=80), UNSUPPORTED), (dict(wl=-3), INVALID),
+    (dict(scale=float("-inf")), INVALID), (dict(dq=P + 6 * T + 4), INVALID),
+    (dict(dk=P), INVALID),                      # dk aliases q
+    (dict(dv=P + 6 * T + 1024), INVALID),       # dv overlaps dq
+    (dict(ws=P + 9 * T + 16), INVALID),         # workspace not 256-byte aligned
+    (dict(ws_bytes=1024), INVALID),             # workspace too small
+    (dict(ws=P + 5 * T), INVALID),              # workspace overlaps dO
+])
+def test_bwd_rejects_invalid_arguments(lib, kw, expected):
+    assert _bwd(lib, **kw) == expected
+
+
+def test_bwd_stage_calls_reject_invalid_arguments(lib):
+    wsb = lib.fa_bwd_workspace_bytes(1, 128, 2, 64)
+    assert lib.fa_bwd_preprocess(P, P + T, P + 2 * T, 1, 128, 2, 64, 0, wsb, None) == INVALID
+    assert lib.fa_bwd_main(P, P + T, P + 2 * T, P + 3 * T, P + 4 * T, P + 5 * T, 1, 128, 2, 64,
+                           ctypes.c_float(0.1), 0, -1, -1, P + 6 * T, 16, None) == INVALID
+    assert lib.fa_bwd_dq_convert(P + 8, 1, 128, 2, 64, P + 6 * T, wsb, None) == INVALID
+    assert lib.fa_bwd_dq_convert(P, 1, 128, 2, 48, P + 6 * T, wsb, None) == UNSUPPORTED
+
+
+def test_binding_has_no_cpu_path():
+    q = torch.zeros(1, 16, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        binding.attention_fwd(q, q, q)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        binding.load()
