@@ -20,7 +20,7 @@ FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
                 4: "FA_ERR_TIMEOUT", 5: "FA_ERR_NO_MEMORY", 6: "FA_ERR_DEVICE"}
 EXPORTS = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
-           "fa_bwd_dq_convert", "fa_check", "fa_status_string")
+           "fa_bwd_dq_convert", "fa_bwd_static_workspace", "fa_check", "fa_status_string")
 
 _lib = None
 
@@ -155,6 +155,28 @@ def bwd_stages(q, k, v, o, lse, do, dq, dk, dv, workspace, scale=None, causal=Fa
     _raise(lib.fa_bwd_dq_convert(dq.data_ptr(), B, N, H, d, ws, wb, s), "fa_bwd_dq_convert")
     if between:
         between(3)
+
+
+def bwd_into_static_workspace(q, k, v, o, lse, do, dq, dk, dv, scale=None, causal=False, window=(-1, -1),
+                              stream=None) -> None:
+    """fa_bwd_static_workspace: the backward without any device allocation.
+
+    For callers that may not allocate device memory (an allocator they do not own, a fixed
+    memory budget): the scratch is a 32 MiB array inside the library. Larger problems raise
+    FaError(FA_ERR_UNSUPPORTED). Calls that overlap on the GPU share that array and race;
+    issue them one after another. Make the first call on each device outside stream capture.
+    """
+    B, N, H, d = _check_qkv(q, k, v, o, do, dq, dk, dv)
+    lib = load()
+    fn = lib.fa_bwd_static_workspace
+    if fn.argtypes is None:
+        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        fn.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+        fn.restype = i
+    st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, d, _scale(scale, d), int(bool(causal)),
+            int(window[0]), int(window[1]), _stream_handle(stream))
+    _raise(st, "fa_bwd_static_workspace")
 
 
 def check(stream=None) -> None:

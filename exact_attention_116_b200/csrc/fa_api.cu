@@ -253,6 +253,31 @@ int check_workspace(void* workspace, size_t bytes, const Shape& s) {
 
 }  // namespace
 
+// ---------------------------------------------------------------- backward without allocation
+//
+// Scratch for fa_bwd_static_workspace: a fixed array in the library's device image. Host code
+// sees only a stand-in symbol; the device address is looked up once per device (with that
+// device current) and cached. No cudaMalloc, cudaFree or allocating library call is made.
+namespace {
+constexpr size_t kStaticWorkspaceBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+void* g_static_workspace_ptr[kMaxDevices] = {nullptr};
+
+int static_workspace_address(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_workspace_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    g_static_workspace_ptr[dev] = p;
+  }
+  *out = g_static_workspace_ptr[dev];
+  return FA_OK;
+}
+}  // namespace
+
 extern "C" {
 
 const char* fa_status_string(int status) {
@@ -389,6 +414,39 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs);
   if (!st) st = launch_convert(dq, s, w, cs);
   if (!workspace && cudaFreeAsync(ws, cs) != cudaSuccess && !st) st = FA_ERR_CUDA;
+  return st;
+}
+
+int fa_bwd_static_workspace(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dO, void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale,
+                            int causal, int win_l, int win_r, fa_stream_t stream) {
+  int st = check_problem(B, N, H, d, scale, causal, &win_l, &win_r);
+  if (st) return st;
+  const Shape s{B, N, H, d};
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  const void* ptrs[8] = {q, k, v, o, dO, dq, dk, dv};
+  for (const void* x : ptrs)
+    if (!aligned(x, 16)) return FA_ERR_INVALID_ARG;
+  if (!aligned(lse, 4)) return FA_ERR_INVALID_ARG;
+  const size_t tb = s.tensor_bytes(), lb = s.rowvec_bytes();
+  const void* ins[5] = {q, k, v, o, dO};
+  void* outs[3] = {dq, dk, dv};
+  for (void* out : outs) {
+    for (const void* in : ins)
+      if (overlap(out, tb, in, tb)) return FA_ERR_INVALID_ARG;
+    if (overlap(out, tb, lse, lb)) return FA_ERR_INVALID_ARG;
+  }
+  if (overlap(dq, tb, dk, tb) || overlap(dq, tb, dv, tb) || overlap(dk, tb, dv, tb)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes(s) > kStaticWorkspaceBytes) return FA_ERR_UNSUPPORTED;
+  int dev, sms;
+  if ((st = device_setup(&dev, &sms))) return st;
+  void* ws = nullptr;
+  if ((st = static_workspace_address(dev, &ws))) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const Workspace w = carve(ws, s);  // the preprocess launch zeroes dQ and rewrites LSE2 / D
+  st = launch_pre(o, lse, dO, s, w, cs);
+  if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs);
+  if (!st) st = launch_convert(dq, s, w, cs);
   return st;
 }
 

@@ -100,6 +100,26 @@ int fa_bwd_dq_convert(void* dq, int B, int N, int H, int d, void* workspace, siz
                       fa_stream_t stream);
 
 /*
+ * Backward pass that allocates nothing (the pages have no counterpart: this is a deployment
+ * aid). Same arguments, results and rules as fa_bwd, without the workspace: the scratch it
+ * needs lives in a fixed 32 MiB array inside the library's device image, which every GPU
+ * that loads the library keeps until the process exits. It is for callers that may not call
+ * cudaMalloc / cudaMallocAsync at all — code running under an allocator it does not own,
+ * inside a pre-sized memory budget, or on a path where an allocation could fail or stall.
+ *   - Problems whose fa_bwd_workspace_bytes() exceeds 32 MiB return FA_ERR_UNSUPPORTED
+ *     before anything is launched.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     and caches it; make that first call, on every device, before any stream capture.
+ *   - All calls share the one array, and each call rewrites the part it uses (its first
+ *     launch zeroes the dQ accumulator and writes the row statistics). Calls that overlap
+ *     on the GPU — on two streams, or from two host threads — race on it: serialise them.
+ */
+int fa_bwd_static_workspace(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dO, void* dq, void* dk, void* dv,
+                            int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
+                            fa_stream_t stream);
+
+/*
  * Synchronises `stream` on the current device and reports what the kernels recorded:
  * FA_ERR_TIMEOUT if a device wait gave up, FA_ERR_DEVICE for another device-side check,
  * FA_ERR_CUDA if the synchronisation itself failed, else FA_OK. Clears the record.
