@@ -41,6 +41,15 @@ EncodeTiledFn encode_fn() {
   return g_encode;
 }
 
+bool log_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = std::getenv("FA_LOG");
+    on = (e && e[0] == '1') ? 1 : 0;
+  }
+  return on == 1;
+}
+
 // Per-device set-up: SM count, sm_100 check, dynamic shared memory opt-in of every kernel.
 int device_setup(int* dev_out, int* sm_count) {
   int dev = 0;
@@ -121,16 +130,33 @@ int make_map(CUtensorMap* m, const void* base, const Shape& s) {
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID_ARG;
 }
 
+// 4-D map over the (B, N, H, d) fp32 dQ accumulator for TMA reduce-add: box (32, 128, 1, 1)
+// (128 bytes x 128 rows), 128B swizzle.
+int make_map_f32_acc(CUtensorMap* m, const void* base, const Shape& s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)s.N, (cuuint64_t)s.H, (cuuint64_t)s.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)s.H * s.d * 4, (cuuint64_t)s.d * 4, (cuuint64_t)s.N * s.H * s.d * 4};
+  const cuuint32_t box[4] = {32, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID_ARG;
+}
+
 struct Workspace {
   float* dq_acc;
   float* lse2;
   float* dvec;
+  int* next_item;
 };
 
 size_t workspace_bytes(const Shape& s) {
-  return align256(s.elems() * 4) + 2 * align256((size_t)s.B * s.H * s.n_pad() * 4);
+  return align256(s.elems() * 4) + 2 * align256((size_t)s.B * s.H * s.n_pad() * 4) + 256;
 }
 
+// Layout: dQ accumulator | LSE*log2(e) | D | work counter, each 256-byte aligned.
 Workspace carve(void* ws, const Shape& s) {
   uint8_t* p = static_cast<uint8_t*>(ws);
   Workspace w;
@@ -139,19 +165,12 @@ Workspace carve(void* ws, const Shape& s) {
   w.lse2 = reinterpret_cast<float*>(p);
   p += align256((size_t)s.B * s.H * s.n_pad() * 4);
   w.dvec = reinterpret_cast<float*>(p);
+  p += align256((size_t)s.B * s.H * s.n_pad() * 4);
+  w.next_item = reinterpret_cast<int*>(p);
   return w;
 }
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
-
-bool log_enabled() {
-  static int on = -1;
-  if (on < 0) {
-    const char* e = std::getenv("FA_LOG");
-    on = (e && e[0] == '1') ? 1 : 0;
-  }
-  return on == 1;
-}
 
 // ---------------------------------------------------------------- launches (arguments already checked)
 
@@ -193,21 +212,22 @@ int launch_pre(const void* o, const float* lse, const void* dO, const Shape& s, 
   if (s.d == 64)
     fa::fa_bwd_pre_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.lse2, w.dvec, w.dq_acc,
-        s.B, s.N, s.H, s.n_pad());
+        w.next_item, s.B, s.N, s.H, s.n_pad());
   else
     fa::fa_bwd_pre_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.lse2, w.dvec, w.dq_acc,
-        s.B, s.N, s.H, s.n_pad());
+        w.next_item, s.B, s.N, s.H, s.n_pad());
   return launch_status();
 }
 
 int launch_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, const Shape& s,
                 float scale, int causal, int win_l, int win_r, const Workspace& w, int sm_count,
                 cudaStream_t stream) {
-  CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
   int st;
   if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
-      (st = make_map(&mdo, dO, s)) || (st = make_map(&mdk, dk, s)) || (st = make_map(&mdv, dv, s)))
+      (st = make_map(&mdo, dO, s)) || (st = make_map(&mdk, dk, s)) || (st = make_map(&mdv, dv, s)) ||
+      (st = make_map_f32_acc(&mdq, w.dq_acc, s)))
     return st;
   fa::BwdParams p;
   p.B = s.B;
@@ -224,17 +244,18 @@ int launch_main(const void* q, const void* k, const void* v, const void* dO, voi
   p.dq_acc = w.dq_acc;
   p.lse2 = w.lse2;
   p.dvec = w.dvec;
+  p.next_item = w.next_item;
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   if (log_enabled())
     std::fprintf(stderr, "[fa] bwd B=%d N=%d H=%d d=%d causal=%d win=(%d,%d) items=%d grid=%d smem=%d\n", s.B, s.N,
                  s.H, s.d, p.causal, win_l, win_r, p.num_items, grid,
                  s.d == 64 ? fa::BwdCfg<64>::kSmemBytes : fa::BwdCfg<128>::kSmemBytes);
   if (s.d == 64)
-    fa::fa_bwd_kernel<64><<<grid, fa::BwdCfg<64>::kThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(mq, mk, mv, mdo,
-                                                                                                   mdk, mdv, p);
+    fa::fa_bwd_kernel<64><<<grid, fa::BwdCfg<64>::kThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdk, mdv, mdq, p);
   else
     fa::fa_bwd_kernel<128><<<grid, fa::BwdCfg<128>::kThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdk, mdv, p);
+        mq, mk, mv, mdo, mdk, mdv, mdq, p);
   return launch_status();
 }
 

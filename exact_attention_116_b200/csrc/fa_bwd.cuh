@@ -14,15 +14,17 @@
 //   fa_dq_convert_kernel  dQ = bf16(accumulator)
 //
 // fa_bwd_kernel roles (512 threads):
-//   warp 0       TMA producer: K_j, V_j per item; Q_i, dO_i, LSE2_i, D_i in a 2-stage ring
+//   warp 0       work fetch (atomic counter, head-grouped order) and TMA producer: K_j, V_j
+//                per item; Q_i with LSE2_i, D_i in two slots; dO_i in one slot
 //   warp 1       MMA issuer, TMEM owner
-//   warps 4-7    dQ: TMEM -> registers -> red.global.add.v4.f32 into the accumulator
+//   warps 4-7    dQ: TMEM -> registers -> shared staging -> TMA reduce-add into the accumulator
 //   warps 8-11   P/dS for query columns [0, 64) of each tile; dK epilogue
 //   warps 12-15  P/dS for query columns [64, 128); dV epilogue
 // TMEM: dK [0,D), dV [D,2D), dP^T / dQ [2D, 2D+128), S^T / P^T [2D+128, 2D+256).
-// Per Q tile i the MMA warp issues S^T = K Q_i^T, dP^T = V dO_i^T, dV += P^T dO_i (P^T from
-// TMEM), dK += dS^T Q_i and dQ_i = dS K_j (dS^T in shared memory, read K-major for dK and
-// MN-major for dQ).
+// Per Q tile i the MMA warp issues dP^T = V dO_i^T, dV += P^T dO_i (P^T from TMEM), then
+// S^T for tile i+1 (= K Q_{i+1}^T), then dQ_i = dS K_j and dK += dS^T Q_i (dS^T in shared
+// memory, read MN-major for dQ and K-major for dK). Issuing S(i+1) early lets the P of tile
+// i+1 be computed while dQ and dK of tile i run; dQ goes first so its columns free up early.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -43,20 +45,39 @@ struct BwdParams {
   float* dq_acc;       // (B, N, H, d) fp32
   const float* lse2;   // (B, H, N_pad) fp32: LSE * log2(e)
   const float* dvec;   // (B, H, N_pad) fp32: rowsum(dO * O)
+  int* next_item;      // work counter (zeroed by the preprocess kernel)
 };
+
+// Heads per scheduling group: items of a group are handed out before the next group's, so the
+// Q, dO and dQ-accumulator rows of the few heads in flight stay in L2.
+constexpr int kBwdHeadGroup = 4;
+
+// Share of the exponentials computed by exp2_poly on the FMA pipes (pair p of a thread's 32
+// pairs uses the polynomial when p % kPolyDen < kPolyNum).
+#ifndef FA_BWD_POLY_NUM
+#define FA_BWD_POLY_NUM 1
+#endif
+#ifndef FA_BWD_POLY_DEN
+#define FA_BWD_POLY_DEN 4
+#endif
+constexpr int kBwdPolyNum = FA_BWD_POLY_NUM, kBwdPolyDen = FA_BWD_POLY_DEN;
+
 
 // ------------------------------------------------------------------ preprocess
 
 // One warp per (b, n, h) row with n < N_pad: D = sum_c dO*O in fp32 and LSE2 = LSE*log2(e)
-// (0 for padding rows), and the row of the dQ accumulator set to zero.
+// (0 for padding rows), and the row of the dQ accumulator set to zero. Also resets the main
+// kernel's work counter.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
                                                          const float* __restrict__ lse, float* __restrict__ lse2,
                                                          float* __restrict__ dvec, float* __restrict__ dq_acc,
-                                                         int B, int N, int H, int N_pad) {
+                                                         int* __restrict__ next_item, int B, int N, int H,
+                                                         int N_pad) {
   const long long warp_g = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *next_item = 0;
   const long long total = (long long)B * N_pad * H;
   if (warp_g >= total) return;
   const int h = (int)(warp_g % H);
@@ -114,34 +135,57 @@ struct BwdCfg {
   static constexpr int kThreads = 512;
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBoxes = D / 64;
-  static constexpr int kStages = 2;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
-  static constexpr int kOffQ = 2 * kTileBytes;                      // + stage * 2 tiles
-  static constexpr int kOffDS = kOffQ + kStages * 2 * kTileBytes;   // 128 x 128 bf16
-  static constexpr int kOffStat = kOffDS + 32768;                   // + stage * 1024: LSE2[128], D[128]
-  static constexpr int kOffBar = kOffStat + kStages * 1024;
+  static constexpr int kOffQ = 2 * kTileBytes;        // two Q slots
+  static constexpr int kOffDO = 4 * kTileBytes;       // one dO slot
+  static constexpr int kOffDS = 5 * kTileBytes;       // dS^T, 128 x 128 bf16
+  static constexpr int kOffDQ = kOffDS + 32768;       // dQ staging: 128 rows x 64 fp32 (two 32-column boxes)
+  static constexpr int kOffStat = kOffDQ + 32768;     // per Q slot: LSE2[128], D[128]
+  static constexpr int kOffBar = kOffStat + 2 * 1024;
   static constexpr int kSmemBytes = kOffBar + 256;
+  static constexpr int kDqRounds = D / 64;            // staging rounds per dQ tile
   static constexpr uint32_t kColDK = 0, kColDV = D, kColDP = 2 * D, kColS = 2 * D + 128;
   static constexpr uint32_t kTmemCols = 512;
 };
 
 struct BwdBars {
   uint64_t kv_full, kv_empty;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[2], q_empty[2];  // Q_i and its LSE2 / D rows
+  uint64_t do_full, do_empty;
   uint64_t s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_empty, dkv_full, dkv_empty;
   uint64_t mma_done;
+  uint64_t item_full[2], item_empty[2];  // ring of fetched work items, producer -> other roles
+  int item_w[2];
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// Item w -> (b, h, j). Under causal masking low key tiles (more Q tiles to visit) come first.
+// Consumers of a fetched item: the MMA thread, 4 dQ warps and 8 P/dS warps (one arrival each).
+constexpr uint32_t kBwdItemConsumers = 13;
+
+// Item w -> (b, h, j): groups of kBwdHeadGroup heads in order; inside a group, KV tiles in
+// ascending order (under causal masking the low tiles visit the most Q tiles) across its heads.
 __device__ __forceinline__ void bwd_decode(const BwdParams& p, int w, int& b, int& h, int& j) {
-  const int bh_count = p.B * p.H;
-  const int r = w / bh_count, bh = w - r * bh_count;
-  j = r;
+  const int per_group = kBwdHeadGroup * p.num_kv_tiles;
+  const int g = w / per_group;
+  const int pos = w - g * per_group;
+  const int gs = min(kBwdHeadGroup, p.B * p.H - g * kBwdHeadGroup);
+  j = pos / gs;
+  const int bh = g * kBwdHeadGroup + (pos - j * gs);
   b = bh / p.H;
   h = bh - b * p.H;
+}
+
+// Next work item of a consumer role (n counts the items this role has taken). Returns the
+// item index; values >= num_items mean "no more work".
+__device__ __forceinline__ int bwd_take_item(BwdBars* bars, uint32_t n, bool arrive, Abort ab) {
+  const uint32_t slot = n & 1;
+  mbar_wait(smem_u32(&bars->item_full[slot]), (n >> 1) & 1, ab);
+  const int w = *reinterpret_cast<volatile int*>(&bars->item_w[slot]);
+  __syncwarp(__activemask());
+  if (arrive) mbar_arrive(smem_u32(&bars->item_empty[slot]));
+  return ab.raised() ? 0x7fffffff : w;
 }
 
 // Q tiles whose rows see any key of KV tile j.
@@ -167,7 +211,7 @@ __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
   using Cfg = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = smem_u32(smem_raw);
@@ -189,7 +233,11 @@ __global__ void __launch_bounds__(512, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(bars->q_full[s]), 1);
       mbar_init(bar(bars->q_empty[s]), 1);
+      mbar_init(bar(bars->item_full[s]), 1);
+      mbar_init(bar(bars->item_empty[s]), kBwdItemConsumers);
     }
+    mbar_init(bar(bars->do_full), 1);
+    mbar_init(bar(bars->do_empty), 1);
     mbar_init(bar(bars->s_full), 1);
     mbar_init(bar(bars->dp_full), 1);
     mbar_init(bar(bars->p_full), 256);
@@ -207,6 +255,7 @@ __global__ void __launch_bounds__(512, 1)
     prefetch_tmap(&tmdO);
     prefetch_tmap(&tmdK);
     prefetch_tmap(&tmdV);
+    prefetch_tmap(&tmdQacc);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&bars->tmem_base), Cfg::kTmemCols);
@@ -218,19 +267,24 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = bars->tmem_base;
 
   const uint32_t sK = smem_base + Cfg::kOffK, sV = smem_base + Cfg::kOffV;
+  const uint32_t sDO = smem_base + Cfg::kOffDO;
   const uint32_t sDS = smem_base + Cfg::kOffDS;
-  auto sQ = [&](int s) { return smem_base + Cfg::kOffQ + s * 2 * Cfg::kTileBytes; };
-  auto sdO = [&](int s) { return smem_base + Cfg::kOffQ + s * 2 * Cfg::kTileBytes + Cfg::kTileBytes; };
+  const uint32_t sDQ = smem_base + Cfg::kOffDQ;
+  auto sQ = [&](int s) { return smem_base + Cfg::kOffQ + s * Cfg::kTileBytes; };
   auto sStat = [&](int s) { return smem_base + Cfg::kOffStat + s * 1024; };
 
   if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------------- work fetch + TMA producer
     if (lane_id() == 0) {
-      uint32_t items = 0, stage = 0, sphase = 0;
-      int last_stage_parity[2] = {-1, -1};
-      for (int round = 0;; ++round) {
-        const int w = sched_item(round, blockIdx.x, gridDim.x);
-        if (w >= p.num_items || ab.raised()) break;
+      uint32_t items = 0, qs = 0, qphase = 0, dn = 0;
+      int last_q_parity[2] = {-1, -1};
+      for (uint32_t n = 0;; ++n) {
+        const uint32_t slot = n & 1;
+        mbar_wait(bar(bars->item_empty[slot]), ((n >> 1) & 1) ^ 1, ab);
+        const int w = ab.raised() ? p.num_items : atomicAdd(p.next_item, 1);
+        bars->item_w[slot] = w;
+        mbar_arrive(bar(bars->item_full[slot]));
+        if (w >= p.num_items) break;
         int b, h, j;
         bwd_decode(p, w, b, h, j);
         int lo, hi;
@@ -244,62 +298,73 @@ __global__ void __launch_bounds__(512, 1)
         }
         ++items;
         const size_t stat_row = ((size_t)b * p.H + h) * (size_t)p.N_pad;
-        for (int i = lo; i <= hi; ++i) {
-          mbar_wait(bar(bars->q_empty[stage]), sphase ^ 1, ab);
-          const uint32_t fb = bar(bars->q_full[stage]);
-          mbar_arrive_expect_tx(fb, 2 * Cfg::kTileBytes + 1024);
+        for (int i = lo; i <= hi; ++i, ++dn) {
+          // Q_i and its statistics into the next Q slot
+          mbar_wait(bar(bars->q_empty[qs]), qphase ^ 1, ab);
+          const uint32_t fb = bar(bars->q_full[qs]);
+          mbar_arrive_expect_tx(fb, Cfg::kTileBytes + 1024);
 #pragma unroll
-          for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-            tma_load_4d(sQ(stage) + bx * 16384, &tmQ, fb, bx * 64, i * 128, h, b);
-            tma_load_4d(sdO(stage) + bx * 16384, &tmdO, fb, bx * 64, i * 128, h, b);
-          }
-          bulk_load(sStat(stage), p.lse2 + stat_row + i * 128, 512, fb);
-          bulk_load(sStat(stage) + 512, p.dvec + stat_row + i * 128, 512, fb);
-          last_stage_parity[stage] = sphase;
-          if (++stage == 2) { stage = 0; sphase ^= 1; }
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx) tma_load_4d(sQ(qs) + bx * 16384, &tmQ, fb, bx * 64, i * 128, h, b);
+          bulk_load(sStat(qs), p.lse2 + stat_row + i * 128, 512, fb);
+          bulk_load(sStat(qs) + 512, p.dvec + stat_row + i * 128, 512, fb);
+          last_q_parity[qs] = qphase;
+          if (++qs == 2) { qs = 0; qphase ^= 1; }
+          // dO_i into the single dO slot (freed when dV_{i-1} is done)
+          mbar_wait(bar(bars->do_empty), (dn & 1) ^ 1, ab);
+          mbar_arrive_expect_tx(bar(bars->do_full), Cfg::kTileBytes);
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+            tma_load_4d(sDO + bx * 16384, &tmdO, bar(bars->do_full), bx * 64, i * 128, h, b);
         }
       }
       for (int s = 0; s < 2; ++s)
-        if (last_stage_parity[s] >= 0) mbar_drain(bar(bars->q_full[s]), last_stage_parity[s]);
+        if (last_q_parity[s] >= 0) mbar_drain(bar(bars->q_full[s]), last_q_parity[s]);
+      if (dn > 0) mbar_drain(bar(bars->do_full), (dn - 1) & 1);
       if (items > 0) mbar_drain(bar(bars->kv_full), (items - 1) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
+    // Per Q tile i: dP(i), dV(i), then S(i+1) ahead of dQ(i), dK(i), so that the P of tile i+1
+    // is computed while the tensor core works on dQ and dK of tile i.
     if (elect_one()) {
       constexpr uint32_t idSP = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T: K-major A and B
       constexpr uint32_t idKV = idesc_bf16_f32(128, D, false, true);     // dV, dK: B (dO, Q) MN-major
       constexpr uint32_t idQ = idesc_bf16_f32(128, D, true, true);       // dQ: A (dS) and B (K) MN-major
       const uint32_t tDK = tmem + Cfg::kColDK, tDV = tmem + Cfg::kColDV;
       const uint32_t tDP = tmem + Cfg::kColDP, tS = tmem + Cfg::kColS;
-      uint32_t items = 0, n = 0, stage = 0, sphase = 0;
-      for (int round = 0;; ++round) {
-        const int w = sched_item(round, blockIdx.x, gridDim.x);
-        if (w >= p.num_items || ab.raised()) break;
+      uint32_t items = 0, n = 0, qs = 0, qphase = 0;
+      auto issue_s = [&](uint32_t slot, uint32_t phase) {
+        mbar_wait(bar(bars->q_full[slot]), phase, ab);
+        tc_fence_after_sync();
+        const uint32_t q = sQ(slot);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tS, sdesc_kmajor(sK + off), sdesc_kmajor(q + off), idSP, kk > 0);
+        }
+        mma_commit(bar(bars->s_full));
+      };
+      for (uint32_t it = 0;; ++it) {
+        const int w = bwd_take_item(bars, it, true, ab);
+        if (w >= p.num_items) break;
         int b, h, j;
         bwd_decode(p, w, b, h, j);
         int lo, hi;
         bwd_q_range(p, j, lo, hi);
         mbar_wait(bar(bars->kv_full), items & 1, ab);
         tc_fence_after_sync();
-        bool first = true;
+        issue_s(qs, qphase);  // S(lo)
         for (int i = lo; i <= hi; ++i, ++n) {
-          mbar_wait(bar(bars->q_full[stage]), sphase, ab);
-          tc_fence_after_sync();
-          const uint32_t q = sQ(stage), g = sdO(stage);
-          // S^T = K_j Q_i^T
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tS, sdesc_kmajor(sK + off), sdesc_kmajor(q + off), idSP, kk > 0);
-          }
-          mma_commit(bar(bars->s_full));
-          // dP^T = V_j dO_i^T, into the columns dQ_{i-1} occupied
+          const bool first = (i == lo);
+          const uint32_t q = sQ(qs);
+          // dP^T = V_j dO_i^T into the columns dQ_{i-1} occupied
+          mbar_wait(bar(bars->do_full), n & 1, ab);
           mbar_wait(bar(bars->dq_empty), (n & 1) ^ 1, ab);
           tc_fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(tDP, sdesc_kmajor(sV + off), sdesc_kmajor(g + off), idSP, kk > 0);
+            mma_ss(tDP, sdesc_kmajor(sV + off), sdesc_kmajor(sDO + off), idSP, kk > 0);
           }
           mma_commit(bar(bars->dp_full));
           // dV += P^T dO_i (P^T packed in TMEM: queries [0,64) in S columns [0,32), [64,128) in [64,96))
@@ -309,24 +374,28 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t acol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
-            mma_ts(tDV, tS + acol, sdesc_mnmajor(g + kk * 2048, 16384), idKV, !first || kk > 0);
+            mma_ts(tDV, tS + acol, sdesc_mnmajor(sDO + kk * 2048, 16384), idKV, !first || kk > 0);
           }
-          // dK += dS^T Q_i ; dQ_i = dS K_j
+          mma_commit(bar(bars->do_empty));
+          // S(i+1): overwrites P^T(i), which dV(i) (issued before) has read
+          const uint32_t nqs = qs ^ 1, nqphase = qs ? (qphase ^ 1) : qphase;
+          if (i < hi) issue_s(nqs, nqphase);
+          // dQ_i = dS K_j, then dK += dS^T Q_i
           mbar_wait(bar(bars->ds_full), n & 1, ab);
           tc_fence_after_sync();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tDP, sdesc_mnmajor(sDS + kk * 2048, 16384), sdesc_mnmajor(sK + kk * 2048, 16384), idQ, kk > 0);
+          mma_commit(bar(bars->dq_full));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
             mma_ss(tDK, sdesc_kmajor(sDS + off), sdesc_mnmajor(q + kk * 2048, 16384), idKV, !first || kk > 0);
           }
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDP, sdesc_mnmajor(sDS + kk * 2048, 16384), sdesc_mnmajor(sK + kk * 2048, 16384), idQ, kk > 0);
-          mma_commit(bar(bars->dq_full));
           mma_commit(bar(bars->ds_empty));
-          mma_commit(bar(bars->q_empty[stage]));
-          first = false;
-          if (++stage == 2) { stage = 0; sphase ^= 1; }
+          mma_commit(bar(bars->q_empty[qs]));
+          qs = nqs;
+          qphase = nqphase;
         }
         mma_commit(bar(bars->dkv_full));
         ++items;
@@ -336,11 +405,13 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 4 && warp < 8) {
     // ---------------------------------------------------------------- dQ accumulation
+    // dQ_i (fp32, times scale) goes TMEM -> registers -> a 128B-swizzled staging tile in shared
+    // memory, and the TMA unit adds it into the accumulator in global memory, 64 columns per round.
     const int row = threadIdx.x - 128;
     const uint32_t tDQ = tmem + ((uint32_t)(row & ~31) << 16) + Cfg::kColDP;
     uint32_t n = 0;
-    for (int round = 0;; ++round) {
-      const int w = sched_item(round, blockIdx.x, gridDim.x);
+    for (uint32_t it = 0;; ++it) {
+      const int w = bwd_take_item(bars, it, lane_id() == 0, ab);
       if (w >= p.num_items) break;
       int b, h, j;
       bwd_decode(p, w, b, h, j);
@@ -349,37 +420,52 @@ __global__ void __launch_bounds__(512, 1)
       for (int i = lo; i <= hi; ++i, ++n) {
         mbar_wait(bar(bars->dq_full), n & 1, ab);
         tc_fence_after_sync();
-        const int qrow = i * 128 + row;
-        float* dst = p.dq_acc + (((size_t)b * p.N + qrow) * p.H + h) * (size_t)D;
-#pragma unroll 1
-        for (int cc = 0; cc < D; cc += 32) {
-          uint32_t v[32];
-          tmem_ld32(tDQ + cc, v);
-          tmem_wait_ld(v);
-          if (cc + 32 >= D) {
+#pragma unroll
+        for (int r = 0; r < Cfg::kDqRounds; ++r) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tDQ + r * 64, v0);
+          tmem_ld32(tDQ + r * 64 + 32, v1);
+          tmem_wait_ld(v0);
+          tmem_wait_ld(v1);
+          if (r == Cfg::kDqRounds - 1) {
             tc_fence_before_sync();
             mbar_arrive(bar(bars->dq_empty));
           }
-          if (qrow < p.N) {
+          if (row == 0) bulk_wait_group_read0();  // the previous reduction has read the staging tile
+          named_bar_sync(3, 128);
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              red_add_v4_f32(dst + cc + e, __uint_as_float(v[e]) * p.scale, __uint_as_float(v[e + 1]) * p.scale,
-                             __uint_as_float(v[e + 2]) * p.scale, __uint_as_float(v[e + 3]) * p.scale);
+          for (int ch = 0; ch < 8; ++ch) {
+            st_shared_v4(sDQ + sw128_offset(row, ch), __float_as_uint(__uint_as_float(v0[4 * ch]) * p.scale),
+                         __float_as_uint(__uint_as_float(v0[4 * ch + 1]) * p.scale),
+                         __float_as_uint(__uint_as_float(v0[4 * ch + 2]) * p.scale),
+                         __float_as_uint(__uint_as_float(v0[4 * ch + 3]) * p.scale));
+            st_shared_v4(sDQ + 16384 + sw128_offset(row, ch), __float_as_uint(__uint_as_float(v1[4 * ch]) * p.scale),
+                         __float_as_uint(__uint_as_float(v1[4 * ch + 1]) * p.scale),
+                         __float_as_uint(__uint_as_float(v1[4 * ch + 2]) * p.scale),
+                         __float_as_uint(__uint_as_float(v1[4 * ch + 3]) * p.scale));
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(3, 128);
+          if (row == 0) {
+            tma_reduce_add_4d(&tmdQacc, sDQ, r * 64, i * 128, h, b);
+            tma_reduce_add_4d(&tmdQacc, sDQ + 16384, r * 64 + 32, i * 128, h, b);
+            bulk_commit_group();
           }
         }
       }
     }
+    if (row == 0) bulk_wait_group0();
   } else if (warp >= 8) {
     // ---------------------------------------------------------------- P, dS and the dK / dV epilogue
-    const int grp = (warp - 8) >> 2;              // 0: query columns [0,64) and dK; 1: [64,128) and dV
+    const int grp = (warp - 8) >> 2;                // 0: query columns [0,64) and dK; 1: [64,128) and dV
     const int row = threadIdx.x - 256 - 128 * grp;  // key row within the tile == TMEM lane
     const uint32_t lane_field = (uint32_t)((row & ~31) << 16);
     const uint32_t tS = tmem + lane_field + Cfg::kColS + 64 * grp;
     const uint32_t tDP = tmem + lane_field + Cfg::kColDP + 64 * grp;
     const float c = p.scale_log2;
-    uint32_t items = 0, n = 0, stage = 0, sphase = 0;
-    for (int round = 0;; ++round) {
-      const int w = sched_item(round, blockIdx.x, gridDim.x);
+    uint32_t items = 0, n = 0, qs = 0, qphase = 0;
+    for (uint32_t it = 0;; ++it) {
+      const int w = bwd_take_item(bars, it, lane_id() == 0, ab);
       if (w >= p.num_items) break;
       int b, h, j;
       bwd_decode(p, w, b, h, j);
@@ -389,9 +475,9 @@ __global__ void __launch_bounds__(512, 1)
       const int qlo = p.win_r >= 0 ? k - p.win_r : 0;
       const int qhi = (k >= p.N) ? -1 : (p.win_l >= 0 ? min(p.N - 1, k + p.win_l) : p.N - 1);
       for (int i = lo; i <= hi; ++i, ++n) {
-        // wait for the stage's Q_i / dO_i / LSE2_i / D_i (the statistics are read here)
-        mbar_wait(bar(bars->q_full[stage]), sphase, ab);
-        const float* lse2 = reinterpret_cast<const float*>(smem_raw + Cfg::kOffStat + stage * 1024);
+        // the Q slot's LSE2_i / D_i rows are read here
+        mbar_wait(bar(bars->q_full[qs]), qphase, ab);
+        const float* lse2 = reinterpret_cast<const float*>(smem_raw + Cfg::kOffStat + qs * 1024);
         const float* dv = lse2 + 128;
         const bool masked = !bwd_tile_unmasked(p, j, i);
         const int qbase = i * 128 + 64 * grp;
@@ -409,8 +495,16 @@ __global__ void __launch_bounds__(512, 1)
           const float a0 = __uint_as_float(e < 32 ? s0[e] : s1[e - 32]);
           const float a1 = __uint_as_float(e < 32 ? s0[e + 1] : s1[e - 31]);
           const int qc = 64 * grp + e;
-          float p0 = ex2_approx(fmaf(a0, c, -lse2[qc]));
-          float p1 = ex2_approx(fmaf(a1, c, -lse2[qc + 1]));
+          const float x0 = fmaf(a0, c, -lse2[qc]);
+          const float x1 = fmaf(a1, c, -lse2[qc + 1]);
+          float p0, p1;
+          if (((e >> 1) % kBwdPolyDen) < kBwdPolyNum) {
+            p0 = exp2_poly(x0);
+            p1 = exp2_poly(x1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
           if (masked) {
             const int q0 = qbase + e;
             p0 = (q0 >= qlo && q0 <= qhi) ? p0 : 0.0f;
@@ -457,7 +551,7 @@ __global__ void __launch_bounds__(512, 1)
         fence_proxy_async_smem();
         tc_fence_before_sync();
         mbar_arrive(bar(bars->ds_full));
-        if (++stage == 2) { stage = 0; sphase ^= 1; }
+        if (++qs == 2) { qs = 0; qphase ^= 1; }
       }
 
       // Epilogue: dK (group 0, times scale) or dV (group 1) -> bf16 -> the K_j / V_j buffer -> TMA store.

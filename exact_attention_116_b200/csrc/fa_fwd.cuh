@@ -40,6 +40,17 @@ struct FwdParams {
 };
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
+
+// Share of the exponentials computed by exp2_poly on the FMA pipes instead of MUFU: pair p of
+// a row's 64 pairs uses the polynomial when p % kPolyDen < kPolyNum.
+#ifndef FA_FWD_POLY_NUM
+#define FA_FWD_POLY_NUM 1
+#endif
+#ifndef FA_FWD_POLY_DEN
+#define FA_FWD_POLY_DEN 8
+#endif
+constexpr int kFwdPolyNum = FA_FWD_POLY_NUM, kFwdPolyDen = FA_FWD_POLY_DEN;
+
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
@@ -140,13 +151,15 @@ __device__ __forceinline__ void fwd_softmax_tile(float (&x)[128], bool masked, i
   for (int u = 0; u < 8; ++u) sum[u] = 0.0f;
 #pragma unroll
   for (int cc = 0; cc < 128; cc += 2) {
+    const float a0 = kPosScale ? fmaf(x[cc], c, -m_use) : x[cc] - m_use;
+    const float a1 = kPosScale ? fmaf(x[cc + 1], c, -m_use) : x[cc + 1] - m_use;
     float p0, p1;
-    if (kPosScale) {
-      p0 = ex2_approx(fmaf(x[cc], c, -m_use));
-      p1 = ex2_approx(fmaf(x[cc + 1], c, -m_use));
+    if (((cc >> 1) % kFwdPolyDen) < kFwdPolyNum) {
+      p0 = exp2_poly(a0);
+      p1 = exp2_poly(a1);
     } else {
-      p0 = ex2_approx(x[cc] - m_use);
-      p1 = ex2_approx(x[cc + 1] - m_use);
+      p0 = ex2_approx(a0);
+      p1 = ex2_approx(a1);
     }
     sum[(cc >> 1) & 7] += p0 + p1;
     pk[cc >> 1] = pack_bf16x2(p0, p1);

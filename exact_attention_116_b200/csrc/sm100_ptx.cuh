@@ -142,6 +142,17 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* m, uint32_t src,
                : "memory");
 }
 
+// Tiled 4-D reduction shared -> global: the TMA unit adds the box into global memory (the
+// element type and the add come from the tensor map; rows outside the tensor are clipped).
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* m, uint32_t src, int c0, int c1, int c2,
+                                                  int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
 // Untiled bulk copy global -> shared; both addresses 16-byte aligned, size a multiple of 16.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
@@ -291,6 +302,27 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA and integer pipes, to take load off the MUFU unit that ex2.approx uses.
+// Cody-Waite split x = j + f with j = round(x) and |f| <= 1/2 (adding 1.5 * 2^23 rounds x to
+// an integer held in the low mantissa bits), a degree-3 minimax polynomial for 2^f on
+// [-1/2, 1/2] (coefficients fitted by csrc/fit_exp2_poly.py, max relative error 7.5e-5), and
+// j added to the exponent field of the polynomial's value. x is clamped at -125 so the
+// result stays a normal float: for x < -125 (including -inf) it returns about 2^-125.
+constexpr float kExp2C0 = 9.999280572e-01f;
+constexpr float kExp2C1 = 6.932608485e-01f;
+constexpr float kExp2C2 = 2.426111549e-01f;
+constexpr float kExp2C3 = 5.517221987e-02f;
+
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(kExp2C3, f, kExp2C2);
+  p = fmaf(p, f, kExp2C1);
+  p = fmaf(p, f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

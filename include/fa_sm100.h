@@ -63,9 +63,10 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            fa_stream_t stream);
 
 /*
- * Bytes of device workspace fa_bwd needs: a float32 dQ accumulator (B,N,H,d) and two
- * float32 (B,H,ceil(N/128)*128) row vectors (LSE*log2(e) and D = rowsum(dO*O)), each
- * region 256-byte aligned. Returns 0 for invalid sizes.
+ * Bytes of device workspace fa_bwd needs: a float32 dQ accumulator (B,N,H,d), two
+ * float32 (B,H,ceil(N/128)*128) row vectors (LSE*log2(e) and D = rowsum(dO*O)) and a
+ * 256-byte block holding the work counter of the main kernel, each region 256-byte
+ * aligned. Returns 0 for invalid sizes.
  */
 size_t fa_bwd_workspace_bytes(int B, int N, int H, int d);
 
