@@ -156,7 +156,7 @@ size_t workspace_bytes(const Shape& s) {
   return align256(s.elems() * 4) + 2 * align256((size_t)s.B * s.H * s.n_pad() * 4) + 256;
 }
 
-// Layout: dQ accumulator | LSE*log2(e) | D | work counter, each 256-byte aligned.
+// Layout: dQ accumulator | -LSE*log2(e) | -D | work counter, each 256-byte aligned.
 Workspace carve(void* ws, const Shape& s) {
   uint8_t* p = static_cast<uint8_t*>(ws);
   Workspace w;

@@ -7,7 +7,7 @@
 //   dQ = scale * dS K,  dK = scale * dS^T Q.
 //
 // Three launches on the caller's stream:
-//   fa_bwd_pre_kernel   D (fp32), LSE * log2(e) (fp32), zero the fp32 dQ accumulator
+//   fa_bwd_pre_kernel   -D (fp32), -LSE * log2(e) (fp32), zero the fp32 dQ accumulator
 //   fa_bwd_kernel       one work item per (b, h, 128-key tile j): K_j, V_j stay in shared
 //                       memory, dK_j and dV_j accumulate in TMEM over the visible Q tiles i;
 //                       dQ_i partial products are added into the fp32 accumulator in global memory
@@ -43,8 +43,8 @@ struct BwdParams {
   int num_kv_tiles;    // ceil(N / 128)
   int num_items;       // B * H * num_kv_tiles
   float* dq_acc;       // (B, N, H, d) fp32
-  const float* lse2;   // (B, H, N_pad) fp32: LSE * log2(e)
-  const float* dvec;   // (B, H, N_pad) fp32: rowsum(dO * O)
+  const float* lse2;   // (B, H, N_pad) fp32: -LSE * log2(e)
+  const float* dvec;   // (B, H, N_pad) fp32: -rowsum(dO * O)
   int* next_item;      // work counter (zeroed by the preprocess kernel)
 };
 
@@ -65,9 +65,9 @@ constexpr int kBwdPolyNum = FA_BWD_POLY_NUM, kBwdPolyDen = FA_BWD_POLY_DEN;
 
 // ------------------------------------------------------------------ preprocess
 
-// One warp per (b, n, h) row with n < N_pad: D = sum_c dO*O in fp32 and LSE2 = LSE*log2(e)
-// (0 for padding rows), and the row of the dQ accumulator set to zero. Also resets the main
-// kernel's work counter.
+// One warp per (b, n, h) row with n < N_pad: -D = -sum_c dO*O in fp32 and -LSE*log2(e)
+// (0 for padding rows; stored negated so that the main kernel adds them), and the row of the
+// dQ accumulator set to zero. Also resets the main kernel's work counter.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
@@ -107,8 +107,8 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) {
-    dvec[stat] = acc;
-    lse2[stat] = lse[((size_t)b * H + h) * (size_t)N + n] * kLog2e;
+    dvec[stat] = -acc;
+    lse2[stat] = -lse[((size_t)b * H + h) * (size_t)N + n] * kLog2e;
   }
 }
 
@@ -477,8 +477,8 @@ __global__ void __launch_bounds__(512, 1)
       for (int i = lo; i <= hi; ++i, ++n) {
         // the Q slot's LSE2_i / D_i rows are read here
         mbar_wait(bar(bars->q_full[qs]), qphase, ab);
-        const float* lse2 = reinterpret_cast<const float*>(smem_raw + Cfg::kOffStat + qs * 1024);
-        const float* dv = lse2 + 128;
+        const float* nlse2 = reinterpret_cast<const float*>(smem_raw + Cfg::kOffStat + qs * 1024);  // -LSE*log2(e)
+        const float* nd = nlse2 + 128;                                                              // -D
         const bool masked = !bwd_tile_unmasked(p, j, i);
         const int qbase = i * 128 + 64 * grp;
 
@@ -490,27 +490,24 @@ __global__ void __launch_bounds__(512, 1)
         tmem_wait_ld(s0);
         tmem_wait_ld(s1);
         uint32_t pk[32];
+        const float2 c2 = make_float2(c, c);
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
-          const float a0 = __uint_as_float(e < 32 ? s0[e] : s1[e - 32]);
-          const float a1 = __uint_as_float(e < 32 ? s0[e + 1] : s1[e - 31]);
-          const int qc = 64 * grp + e;
-          const float x0 = fmaf(a0, c, -lse2[qc]);
-          const float x1 = fmaf(a1, c, -lse2[qc + 1]);
-          float p0, p1;
+          const float2 sv = make_float2(__uint_as_float(e < 32 ? s0[e] : s1[e - 32]),
+                                        __uint_as_float(e < 32 ? s0[e + 1] : s1[e - 31]));
+          const float2 xv = fma2(sv, c2, *reinterpret_cast<const float2*>(nlse2 + 64 * grp + e));
+          float2 pv;
           if (((e >> 1) % kBwdPolyDen) < kBwdPolyNum) {
-            p0 = exp2_poly(x0);
-            p1 = exp2_poly(x1);
+            pv = exp2_poly2(xv);
           } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
+            pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
           }
           if (masked) {
             const int q0 = qbase + e;
-            p0 = (q0 >= qlo && q0 <= qhi) ? p0 : 0.0f;
-            p1 = (q0 + 1 >= qlo && q0 + 1 <= qhi) ? p1 : 0.0f;
+            pv.x = (q0 >= qlo && q0 <= qhi) ? pv.x : 0.0f;
+            pv.y = (q0 + 1 >= qlo && q0 + 1 <= qhi) ? pv.y : 0.0f;
           }
-          pk[e >> 1] = pack_bf16x2(p0, p1);
+          pk[e >> 1] = pack_bf16x2(pv.x, pv.y);
         }
         {
           uint32_t lo16[16], hi16[16];
@@ -539,12 +536,12 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int col = ch * 8 + 2 * e;  // 0..63 within the group
-            const float g0 = __uint_as_float(col < 32 ? d0[col] : d1[col - 32]);
-            const float g1 = __uint_as_float(col < 32 ? d0[col + 1] : d1[col - 31]);
+            const float2 g = make_float2(__uint_as_float(col < 32 ? d0[col] : d1[col - 32]),
+                                         __uint_as_float(col < 32 ? d0[col + 1] : d1[col - 31]));
             const uint32_t pp = pk[col >> 1];
-            const float ds0 = bf16lo_to_f32(pp) * (g0 - dv[64 * grp + col]);
-            const float ds1 = bf16hi_to_f32(pp) * (g1 - dv[64 * grp + col + 1]);
-            w4[e] = pack_bf16x2(ds0, ds1);
+            const float2 diff = add2(g, *reinterpret_cast<const float2*>(nd + 64 * grp + col));
+            const float2 ds = mul2(make_float2(bf16lo_to_f32(pp), bf16hi_to_f32(pp)), diff);
+            w4[e] = pack_bf16x2(ds.x, ds.y);
           }
           st_shared_v4(box + sw128_offset(row, ch), w4[0], w4[1], w4[2], w4[3]);
         }

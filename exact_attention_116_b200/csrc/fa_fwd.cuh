@@ -109,33 +109,33 @@ __device__ __forceinline__ bool fwd_tile_unmasked(const FwdParams& p, int r0, in
 
 // ------------------------------------------------------------------ softmax role
 
-template <int D, bool kPosScale>
-__device__ __forceinline__ void fwd_softmax_tile(float (&x)[128], bool masked, int kbase, int kmin, int kmax,
-                                                 float c, float& m_run, float& l_run, uint32_t (&pk)[64],
-                                                 float& alpha, bool& updated) {
-  // 1. mask and tile maximum (in scaled log2 units)
-  float mx[8];
+// Row maximum of a 128-key tile (scaled, log2 units) with masking, and the lazy update of
+// the reference maximum. x is scaled in place when the scale is not positive.
+template <bool kPosScale>
+__device__ __forceinline__ void fwd_row_max(float (&x)[128], bool masked, int kbase, int kmin, int kmax, float c,
+                                            float& m_run, float& alpha, bool& updated) {
+  if (!kPosScale) {  // then masking must follow the scaling
 #pragma unroll
-  for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+    for (int cc = 0; cc < 128; cc += 2) {
+      const float2 v = mul2(make_float2(x[cc], x[cc + 1]), make_float2(c, c));
+      x[cc] = v.x;
+      x[cc + 1] = v.y;
+    }
+  }
   if (masked) {
 #pragma unroll
     for (int cc = 0; cc < 128; ++cc) {
       const int key = kbase + cc;
-      const bool vis = (key >= kmin) & (key <= kmax);
-      x[cc] = vis ? (kPosScale ? x[cc] : x[cc] * c) : -INFINITY;
-      mx[cc & 7] = fmaxf(mx[cc & 7], x[cc]);
-    }
-  } else {
-#pragma unroll
-    for (int cc = 0; cc < 128; ++cc) {
-      if (!kPosScale) x[cc] *= c;
-      mx[cc & 7] = fmaxf(mx[cc & 7], x[cc]);
+      x[cc] = ((key >= kmin) & (key <= kmax)) ? x[cc] : -INFINITY;
     }
   }
-  float m_tile = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+  float mx[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < 64; ++k) mx[k & 7] = max3(mx[k & 7], x[2 * k], x[2 * k + 1]);
+  float m_tile = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
   if (kPosScale) m_tile *= c;
-
-  // 2. lazy update of the reference maximum
   const float m_new = fmaxf(m_run, m_tile);
   updated = m_new > m_run + kRescaleThreshold;
   alpha = 1.0f;
@@ -143,29 +143,28 @@ __device__ __forceinline__ void fwd_softmax_tile(float (&x)[128], bool masked, i
     alpha = ex2_approx(m_run - m_new);  // 0 when m_run was -inf
     m_run = m_new;
   }
-  const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+}
 
-  // 3. exponentials, row sum, bf16 packing (even column in the low half)
-  float sum[8];
+// Exponentials of 32 columns (16 pairs starting at pair k0) against the reference maximum,
+// packed to bf16 pairs (even column low) and summed.
+template <bool kPosScale>
+__device__ __forceinline__ void fwd_exp_chunk(const float (&x)[128], int k0, float c, float m_use, uint32_t (&pk)[16],
+                                              float2& sum) {
+  const float2 neg_m = make_float2(-m_use, -m_use);
+  const float2 c2 = make_float2(c, c);
 #pragma unroll
-  for (int u = 0; u < 8; ++u) sum[u] = 0.0f;
-#pragma unroll
-  for (int cc = 0; cc < 128; cc += 2) {
-    const float a0 = kPosScale ? fmaf(x[cc], c, -m_use) : x[cc] - m_use;
-    const float a1 = kPosScale ? fmaf(x[cc + 1], c, -m_use) : x[cc + 1] - m_use;
-    float p0, p1;
-    if (((cc >> 1) % kFwdPolyDen) < kFwdPolyNum) {
-      p0 = exp2_poly(a0);
-      p1 = exp2_poly(a1);
+  for (int k = 0; k < 16; ++k) {
+    const float2 xv = make_float2(x[2 * (k0 + k)], x[2 * (k0 + k) + 1]);
+    const float2 a = kPosScale ? fma2(xv, c2, neg_m) : add2(xv, neg_m);
+    float2 pv;
+    if ((k % kFwdPolyDen) < kFwdPolyNum) {
+      pv = exp2_poly2(a);
     } else {
-      p0 = ex2_approx(a0);
-      p1 = ex2_approx(a1);
+      pv = make_float2(ex2_approx(a.x), ex2_approx(a.y));
     }
-    sum[(cc >> 1) & 7] += p0 + p1;
-    pk[cc >> 1] = pack_bf16x2(p0, p1);
+    sum = add2(sum, pv);
+    pk[k] = pack_bf16x2(pv.x, pv.y);
   }
-  const float s_tile = ((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7]));
-  l_run = l_run * alpha + s_tile;
 }
 
 __device__ __forceinline__ float lg2_approx(float x) {
@@ -399,13 +398,26 @@ __global__ void __launch_bounds__(384, 1)
         for (int cc = 0; cc < 128; ++cc) x[cc] = __uint_as_float(r[cc >> 5][cc & 31]);
 
         const bool masked = !fwd_tile_unmasked(p, r0, j);
-        uint32_t pk[64];
         float alpha;
         bool updated;
         if (c > 0.0f)
-          fwd_softmax_tile<D, true>(x, masked, j * 128, kmin, kmax, c, m_run, l_run, pk, alpha, updated);
+          fwd_row_max<true>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated);
         else
-          fwd_softmax_tile<D, false>(x, masked, j * 128, kmin, kmax, c, m_run, l_run, pk, alpha, updated);
+          fwd_row_max<false>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated);
+        const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
+        // P in 32-column chunks straight into TMEM (over S columns already read into registers)
+        float2 sum0 = make_float2(0.0f, 0.0f), sum1 = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t pk[16];
+          if (c > 0.0f)
+            fwd_exp_chunk<true>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
+          else
+            fwd_exp_chunk<false>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
+          tmem_st16(tS + q4 * 16, pk);
+        }
+        const float2 s01 = add2(sum0, sum1);
+        l_run = l_run * alpha + (s01.x + s01.y);
 
         // Rescale O_t in TMEM when this warp's reference maximum moved (not on the first tile:
         // the first PV of an item overwrites O_t).
@@ -419,13 +431,6 @@ __global__ void __launch_bounds__(384, 1)
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
             tmem_st32(tO + cc, o);
           }
-        }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t v16[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) v16[e] = pk[q4 * 16 + e];
-          tmem_st16(tS + q4 * 16, v16);
         }
         tmem_wait_st();
         tc_fence_before_sync();

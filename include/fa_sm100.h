@@ -64,7 +64,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 
 /*
  * Bytes of device workspace fa_bwd needs: a float32 dQ accumulator (B,N,H,d), two
- * float32 (B,H,ceil(N/128)*128) row vectors (LSE*log2(e) and D = rowsum(dO*O)) and a
+ * float32 (B,H,ceil(N/128)*128) row vectors (-LSE*log2(e) and -D, D = rowsum(dO*O)) and a
  * 256-byte block holding the work counter of the main kernel, each region 256-byte
  * aligned. Returns 0 for invalid sizes.
  */
@@ -87,7 +87,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
  * The three launches of fa_bwd, exposed so that a caller can time or interleave them.
  * Same arguments and rules as fa_bwd, except that `workspace` must be non-NULL and must
  * be the same buffer for the three calls of one backward, issued in this order.
- *   fa_bwd_preprocess : D = rowsum(dO * O), LSE*log2(e), dQ accumulator := 0
+ *   fa_bwd_preprocess : -D = -rowsum(dO * O), -LSE*log2(e), dQ accumulator := 0
  *   fa_bwd_main       : dK, dV (written to dk, dv) and the dQ accumulator
  *   fa_bwd_dq_convert : dq = bf16(dQ accumulator)
  */
