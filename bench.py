@@ -33,6 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_attention_116_b200 import binding  # noqa: E402
+from exact_attention_116_b200 import distributed as mg  # noqa: E402
 from exact_attention_116_b200.inputs import CONFIGS, make_inputs  # noqa: E402
 from exact_attention_116_b200.workload import flops, hbm_bytes, visible_pairs  # noqa: E402
 
@@ -181,38 +182,11 @@ def oracle_sample(cfg, seconds: float, q=None, k=None, v=None, do=None):
 
 # ----------------------------------------------------------------------------- GPU arm
 
-def dist_setup(n_gpus: int):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-
-
-def max_over_ranks(world, x: float) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
 def run_gpu(args):
-    world, rank, local = dist_setup(args.gpus)
+    info = mg.rank_info()
+    world, rank, local = info.world, info.rank, info.local_rank
+    torch.cuda.set_device(local)
+    mg.init(info, "nccl", device=torch.device("cuda", local))
     cfg = CONFIGS[args.config]
     if not cfg.backward:
         raise SystemExit(f"config {cfg.name} has no backward; a step is forward + backward")
@@ -248,7 +222,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
 
     sampler = ClockSampler(dev.index) if local == 0 else None
-    barrier(world)
+    mg.barrier(info)
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -257,13 +231,13 @@ def run_gpu(args):
         step(True)
     end.record(stream)
     torch.cuda.synchronize()
-    barrier(world)
+    mg.barrier(info)
     t_wall1 = time.time()
     binding.check()
     clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
 
     ms_total = start.elapsed_time(end)
-    ms_total = max_over_ranks(world, ms_total)
+    ms_total = mg.max_over_ranks(info, ms_total, dev)
     ms_step = ms_total / args.steps
     f_fwd, f_bwd = flops(B, N, H, d, causal, *win)
     fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["f0"], ev["b0"]))
@@ -290,19 +264,18 @@ def run_gpu(args):
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
-    barrier(world)
+    mg.barrier(info)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    barrier(world)
+    mg.barrier(info)
     binding.check()
-    e2e_ms = max_over_ranks(world, e0.elapsed_time(e1)) / e2e_steps
+    e2e_ms = mg.max_over_ranks(info, e0.elapsed_time(e1), dev) / e2e_steps
 
     peak, peak_src = peaks()
-    tflops_step = (f_fwd + f_bwd) / (ms_step * 1e-3) / 1e12
     main_tflops = f_bwd / (main_ms * 1e-3) / 1e12
     fwd_tflops = f_fwd / (fwd_ms * 1e-3) / 1e12
     bwd_tflops = f_bwd / (bwd_ms * 1e-3) / 1e12
@@ -312,7 +285,8 @@ def run_gpu(args):
     traffic = recorded_traffic(dominant)
     t_bytes = B * N * H * d * 2
     res = {
-        "metric": METRIC, "value": round(tflops_step * world, 3), "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": round(mg.aggregate_rate(f_fwd + f_bwd, world, ms_step * 1e-3) / 1e12, 3),
+        "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16)",
@@ -336,7 +310,7 @@ def run_gpu(args):
                      "frac_of_sustained": round(achieved / peak.get("bf16_tflops_sustained", peak["bf16_tflops"]), 4),
                      "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": traffic,
                      "algorithmic_bytes": hbm_bytes(B, N, H, d)[1 if dominant == "fa_bwd_kernel" else 0]},
-        "e2e": {"value": round((f_fwd + f_bwd) / (e2e_ms * 1e-3) / 1e12 * world, 3), "unit": UNIT,
+        "e2e": {"value": round(mg.aggregate_rate(f_fwd + f_bwd, world, e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": 4 * t_bytes,
                 "d2h_bytes_per_step": 4 * t_bytes + B * H * N * 4},
         "gpu_launches": 4 * args.steps,
@@ -347,9 +321,7 @@ def run_gpu(args):
         res["cpu_baseline"] = {"value": round(tf, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
                                "sample": f"fp64 oracle, forward+backward of {rows} query rows (512-row blocks, heads of "
                                          f"batch 0 in order) of {cfg.name}, {dt:.1f} s, same pair-count FLOP convention"}
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    mg.shutdown(info)
     if rank == 0:
         print(json.dumps(res), flush=True)
 

@@ -192,6 +192,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.num_pairs = (s.N + 255) / 256;
   p.num_items = s.B * s.H * p.num_pairs;
   p.lse = lse;
+  // Test-only fault knob: the forward withholds one internal signal so that a bounded wait in
+  // the kernel runs out (it must report FA_ERR_TIMEOUT through fa_check, not hang).
+  const char* drop = std::getenv("FA_DEBUG_DROP_S_SIGNAL");
+  p.debug_drop_s_signal = (drop && drop[0] == '1') ? 1 : 0;
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   if (log_enabled())
     std::fprintf(stderr, "[fa] fwd B=%d N=%d H=%d d=%d causal=%d win=(%d,%d) items=%d grid=%d smem=%d\n", s.B, s.N,

@@ -37,6 +37,7 @@ struct FwdParams {
   int num_pairs;     // ceil(N / 256)
   int num_items;     // B * H * num_pairs
   float* lse;        // (B, H, N) fp32
+  int debug_drop_s_signal;  // test only: withhold the first "S ready" signal (a wait must time out)
 };
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
@@ -276,6 +277,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t tO[2] = {tmem + Cfg::kColO0, tmem + Cfg::kColO1};
       uint32_t slot = 0, phase = 0;
       uint32_t qn[2] = {0, 0}, pn[2] = {0, 0};
+      bool drop_s_signal = p.debug_drop_s_signal != 0;
 
       auto issue_s = [&](int t, uint32_t k_smem) {
 #pragma unroll
@@ -323,7 +325,8 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_after_sync();
             if (active(0, j)) {
               issue_s(0, sKV + k_slot * Cfg::kTileBytes);
-              mma_commit(bar(bars->s_full[0]));
+              if (drop_s_signal) drop_s_signal = false;
+              else mma_commit(bar(bars->s_full[0]));
             }
           }
           if (j - 1 >= lo) {
