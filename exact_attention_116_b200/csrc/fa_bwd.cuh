@@ -206,6 +206,38 @@ __device__ __forceinline__ bool bwd_tile_unmasked(const BwdParams& p, int j, int
   return true;
 }
 
+// P^T for 64 query columns of this thread's key row: exp2(S^T * c - LSE_q * log2(e)), zero
+// where masked (kMasked), packed to bf16 pairs (even column low). nlse2 holds -LSE * log2(e)
+// of the same 64 queries.
+template <bool kMasked>
+__device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[32], const uint32_t (&s1)[32], float c,
+                                          const float* nlse2, int qbase, int qlo, int qhi, uint32_t (&pk)[32]) {
+  const float2 c2 = make_float2(c, c);
+#pragma unroll
+  for (int e = 0; e < 64; e += 4) {
+    const float4 nl = *reinterpret_cast<const float4*>(nlse2 + e);
+#pragma unroll
+    for (int h2 = 0; h2 < 4; h2 += 2) {
+      const int f = e + h2;
+      const float2 sv = make_float2(__uint_as_float(f < 32 ? s0[f] : s1[f - 32]),
+                                    __uint_as_float(f < 32 ? s0[f + 1] : s1[f - 31]));
+      const float2 xv = fma2(sv, c2, h2 ? make_float2(nl.z, nl.w) : make_float2(nl.x, nl.y));
+      float2 pv;
+      if (((f >> 1) % kBwdPolyDen) < kBwdPolyNum) {
+        pv = exp2_poly2(xv);
+      } else {
+        pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
+      }
+      if (kMasked) {
+        const int q0 = qbase + f;
+        pv.x = (q0 >= qlo && q0 <= qhi) ? pv.x : 0.0f;
+        pv.y = (q0 + 1 >= qlo && q0 + 1 <= qhi) ? pv.y : 0.0f;
+      }
+      pk[f >> 1] = pack_bf16x2(pv.x, pv.y);
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -490,25 +522,10 @@ __global__ void __launch_bounds__(512, 1)
         tmem_wait_ld(s0);
         tmem_wait_ld(s1);
         uint32_t pk[32];
-        const float2 c2 = make_float2(c, c);
-#pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const float2 sv = make_float2(__uint_as_float(e < 32 ? s0[e] : s1[e - 32]),
-                                        __uint_as_float(e < 32 ? s0[e + 1] : s1[e - 31]));
-          const float2 xv = fma2(sv, c2, *reinterpret_cast<const float2*>(nlse2 + 64 * grp + e));
-          float2 pv;
-          if (((e >> 1) % kBwdPolyDen) < kBwdPolyNum) {
-            pv = exp2_poly2(xv);
-          } else {
-            pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
-          }
-          if (masked) {
-            const int q0 = qbase + e;
-            pv.x = (q0 >= qlo && q0 <= qhi) ? pv.x : 0.0f;
-            pv.y = (q0 + 1 >= qlo && q0 + 1 <= qhi) ? pv.y : 0.0f;
-          }
-          pk[e >> 1] = pack_bf16x2(pv.x, pv.y);
-        }
+        if (masked)
+          bwd_probs<true>(s0, s1, c, nlse2 + 64 * grp, qbase, qlo, qhi, pk);
+        else
+          bwd_probs<false>(s0, s1, c, nlse2 + 64 * grp, qbase, qlo, qhi, pk);
         {
           uint32_t lo16[16], hi16[16];
 #pragma unroll
@@ -533,13 +550,17 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t w4[4];
+          const float4 nda = *reinterpret_cast<const float4*>(nd + 64 * grp + ch * 8);
+          const float4 ndb = *reinterpret_cast<const float4*>(nd + 64 * grp + ch * 8 + 4);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int col = ch * 8 + 2 * e;  // 0..63 within the group
             const float2 g = make_float2(__uint_as_float(col < 32 ? d0[col] : d1[col - 32]),
                                          __uint_as_float(col < 32 ? d0[col + 1] : d1[col - 31]));
             const uint32_t pp = pk[col >> 1];
-            const float2 diff = add2(g, *reinterpret_cast<const float2*>(nd + 64 * grp + col));
+            const float2 ndv = e == 0 ? make_float2(nda.x, nda.y) : e == 1 ? make_float2(nda.z, nda.w)
+                             : e == 2 ? make_float2(ndb.x, ndb.y) : make_float2(ndb.z, ndb.w);
+            const float2 diff = add2(g, ndv);
             const float2 ds = mul2(make_float2(bf16lo_to_f32(pp), bf16hi_to_f32(pp)), diff);
             w4[e] = pack_bf16x2(ds.x, ds.y);
           }
