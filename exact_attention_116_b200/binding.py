@@ -19,8 +19,8 @@ LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
                 4: "FA_ERR_TIMEOUT", 5: "FA_ERR_NO_MEMORY", 6: "FA_ERR_DEVICE"}
-EXPORTS = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main",
-           "fa_bwd_dq_convert", "fa_bwd_static_workspace", "fa_check", "fa_status_string")
+EXPORTS = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess",
+           "fa_bwd_main", "fa_bwd_dq_convert", "fa_bwd_static_workspace", "fa_check", "fa_status_string")
 
 _lib = None
 
@@ -44,13 +44,15 @@ def load() -> ctypes.CDLL:
     lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_bytes.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp, sz, vp]
+    lib.fa_bwd_deterministic.argtypes = lib.fa_bwd.argtypes
     lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
     lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp, sz, vp]
     lib.fa_bwd_dq_convert.argtypes = [vp, i, i, i, i, vp, sz, vp]
     lib.fa_check.argtypes = [vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
-    for name in ("fa_fwd", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert", "fa_check"):
+    for name in ("fa_fwd", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
+                 "fa_check"):
         getattr(lib, name).restype = i
     _lib = lib
     return lib
@@ -116,20 +118,25 @@ def workspace_bytes(B: int, N: int, H: int, d: int) -> int:
 
 
 def bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale=None, causal=False, window=(-1, -1), workspace=None,
-             stream=None) -> None:
-    """fa_bwd into caller-provided dq, dk, dv. ``workspace``: uint8 CUDA tensor or None."""
+             stream=None, deterministic=False) -> None:
+    """fa_bwd (or fa_bwd_deterministic) into caller-provided dq, dk, dv.
+    ``workspace``: uint8 CUDA tensor or None."""
     B, N, H, d = _check_qkv(q, k, v, o, do, dq, dk, dv)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
-    st = load().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, d, _scale(scale, d),
-                       int(bool(causal)), int(window[0]), int(window[1]), ws_ptr, ws_bytes, _stream_handle(stream))
-    _raise(st, "fa_bwd")
+    lib = load()
+    fn, name = (lib.fa_bwd_deterministic, "fa_bwd_deterministic") if deterministic else (lib.fa_bwd, "fa_bwd")
+    st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), B, N, H, d, _scale(scale, d), int(bool(causal)), int(window[0]),
+            int(window[1]), ws_ptr, ws_bytes, _stream_handle(stream))
+    _raise(st, name)
 
 
-def attention_bwd(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1), workspace=None, stream=None):
-    """Backward: returns (dq, dk, dv), the gradients of sum(do * o)."""
+def attention_bwd(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1), workspace=None, stream=None,
+                  deterministic=False):
+    """Backward: returns (dq, dk, dv), the gradients of sum(do * o). With deterministic=True the
+    result is bitwise reproducible (dQ accumulated per query tile in a fixed order)."""
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale, causal, window, workspace, stream)
+    bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale, causal, window, workspace, stream, deterministic)
     return dq, dk, dv
 
 

@@ -13,6 +13,7 @@
 
 #include "fa_sm100.h"
 #include "fa_bwd.cuh"
+#include "fa_bwd_dq.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -68,10 +69,18 @@ int device_setup(int* dev_out, int* sm_count) {
                                fa::FwdCfg<64>::kSmemBytes) != cudaSuccess ||
           cudaFuncSetAttribute(fa::fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fa::FwdCfg<128>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+          cudaFuncSetAttribute(fa::fa_bwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fa::BwdCfg<64>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdCfg<128>::kSmemBytes) != cudaSuccess)
+          cudaFuncSetAttribute(fa::fa_bwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdCfg<128>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_bwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdCfg<64>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_bwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdCfg<128>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdDqCfg<64>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::BwdDqCfg<128>::kSmemBytes) != cudaSuccess)
         return FA_ERR_CUDA;
     }
     g_attr_done[dev] = true;
@@ -224,15 +233,7 @@ int launch_pre(const void* o, const float* lse, const void* dO, const Shape& s, 
   return launch_status();
 }
 
-int launch_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, const Shape& s,
-                float scale, int causal, int win_l, int win_r, const Workspace& w, int sm_count,
-                cudaStream_t stream) {
-  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
-  int st;
-  if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
-      (st = make_map(&mdo, dO, s)) || (st = make_map(&mdk, dk, s)) || (st = make_map(&mdv, dv, s)) ||
-      (st = make_map_f32_acc(&mdq, w.dq_acc, s)))
-    return st;
+fa::BwdParams bwd_params(const Shape& s, float scale, int causal, int win_l, int win_r, const Workspace& w) {
   fa::BwdParams p;
   p.B = s.B;
   p.N = s.N;
@@ -249,17 +250,56 @@ int launch_main(const void* q, const void* k, const void* v, const void* dO, voi
   p.lse2 = w.lse2;
   p.dvec = w.dvec;
   p.next_item = w.next_item;
+  return p;
+}
+
+// Main backward kernel; with_dq = false computes dK and dV only (the deterministic backward).
+int launch_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, const Shape& s,
+                float scale, int causal, int win_l, int win_r, const Workspace& w, int sm_count,
+                cudaStream_t stream, bool with_dq = true) {
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
+  int st;
+  if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
+      (st = make_map(&mdo, dO, s)) || (st = make_map(&mdk, dk, s)) || (st = make_map(&mdv, dv, s)) ||
+      (st = make_map_f32_acc(&mdq, w.dq_acc, s)))
+    return st;
+  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w);
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   if (log_enabled())
     std::fprintf(stderr, "[fa] bwd B=%d N=%d H=%d d=%d causal=%d win=(%d,%d) items=%d grid=%d smem=%d\n", s.B, s.N,
                  s.H, s.d, p.causal, win_l, win_r, p.num_items, grid,
                  s.d == 64 ? fa::BwdCfg<64>::kSmemBytes : fa::BwdCfg<128>::kSmemBytes);
-  if (s.d == 64)
-    fa::fa_bwd_kernel<64><<<grid, fa::BwdCfg<64>::kThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(
+  if (s.d == 64 && with_dq)
+    fa::fa_bwd_kernel<64, true><<<grid, fa::BwdCfg<64>::kThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  else if (s.d == 64)
+    fa::fa_bwd_kernel<64, false><<<grid, fa::BwdCfg<64>::kThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  else if (with_dq)
+    fa::fa_bwd_kernel<128, true><<<grid, fa::BwdCfg<128>::kThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(
         mq, mk, mv, mdo, mdk, mdv, mdq, p);
   else
-    fa::fa_bwd_kernel<128><<<grid, fa::BwdCfg<128>::kThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(
+    fa::fa_bwd_kernel<128, false><<<grid, fa::BwdCfg<128>::kThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(
         mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  return launch_status();
+}
+
+// dQ of the deterministic backward: one item per (b, h, Q tile), dQ accumulated in TMEM.
+int launch_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, const Shape& s, float scale,
+              int causal, int win_l, int win_r, const Workspace& w, int sm_count, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mdo, mdq;
+  int st;
+  if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
+      (st = make_map(&mdo, dO, s)) || (st = make_map(&mdq, dq, s)))
+    return st;
+  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w);
+  const int grid = p.num_items < sm_count ? p.num_items : sm_count;
+  if (s.d == 64)
+    fa::fa_bwd_dq_kernel<64><<<grid, fa::BwdDqCfg<64>::kThreads, fa::BwdDqCfg<64>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdq, p);
+  else
+    fa::fa_bwd_dq_kernel<128><<<grid, fa::BwdDqCfg<128>::kThreads, fa::BwdDqCfg<128>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdq, p);
   return launch_status();
 }
 
@@ -394,9 +434,11 @@ int fa_bwd_dq_convert(void* dq, int B, int N, int H, int d, void* workspace, siz
   return launch_convert(dq, s, carve(workspace, s), reinterpret_cast<cudaStream_t>(stream));
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
-           void* dk, void* dv, int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
-           void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+}  // extern "C"
+
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                    void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale, int causal, int win_l,
+                    int win_r, void* workspace, size_t workspace_bytes_, fa_stream_t stream, bool deterministic) {
   int st = check_problem(B, N, H, d, scale, causal, &win_l, &win_r);
   if (st) return st;
   const Shape s{B, N, H, d};
@@ -436,10 +478,32 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   }
   const Workspace w = carve(ws, s);
   st = launch_pre(o, lse, dO, s, w, cs);
-  if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs);
-  if (!st) st = launch_convert(dq, s, w, cs);
+  if (deterministic) {
+    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs, false);
+    if (!st) st = launch_dq(q, k, v, dO, dq, s, scale, causal, win_l, win_r, w, sms, cs);
+  } else {
+    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs);
+    if (!st) st = launch_convert(dq, s, w, cs);
+  }
   if (!workspace && cudaFreeAsync(ws, cs) != cudaSuccess && !st) st = FA_ERR_CUDA;
   return st;
+}
+
+extern "C" {
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, void* dq,
+           void* dk, void* dv, int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
+           void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, N, H, d, scale, causal, win_l, win_r, workspace,
+                  workspace_bytes_, stream, false);
+}
+
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale,
+                         int causal, int win_l, int win_r, void* workspace, size_t workspace_bytes_,
+                         fa_stream_t stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, N, H, d, scale, causal, win_l, win_r, workspace,
+                  workspace_bytes_, stream, true);
 }
 
 int fa_bwd_static_workspace(const void* q, const void* k, const void* v, const void* o, const float* lse,

@@ -45,7 +45,7 @@ struct BwdParams {
   float* dq_acc;       // (B, N, H, d) fp32
   const float* lse2;   // (B, H, N_pad) fp32: -LSE * log2(e)
   const float* dvec;   // (B, H, N_pad) fp32: -rowsum(dO * O)
-  int* next_item;      // work counter (zeroed by the preprocess kernel)
+  int* next_item;      // work counters (zeroed by the preprocess kernel): [0] main kernel, [1] dQ kernel
 };
 
 // Heads per scheduling group: items of a group are handed out before the next group's, so the
@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
                                                          int N_pad) {
   const long long warp_g = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *next_item = 0;
+  if (blockIdx.x == 0 && threadIdx.x < 2) next_item[threadIdx.x] = 0;
   const long long total = (long long)B * N_pad * H;
   if (warp_g >= total) return;
   const int h = (int)(warp_g % H);
@@ -238,7 +238,7 @@ __device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[32], const uint32
   }
 }
 
-template <int D>
+template <int D, bool kDQ>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(512, 1)
           const uint32_t q = sQ(qs);
           // dP^T = V_j dO_i^T into the columns dQ_{i-1} occupied
           mbar_wait(bar(bars->do_full), n & 1, ab);
-          mbar_wait(bar(bars->dq_empty), (n & 1) ^ 1, ab);
+          if (kDQ) mbar_wait(bar(bars->dq_empty), (n & 1) ^ 1, ab);
           tc_fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -415,10 +415,12 @@ __global__ void __launch_bounds__(512, 1)
           // dQ_i = dS K_j, then dK += dS^T Q_i
           mbar_wait(bar(bars->ds_full), n & 1, ab);
           tc_fence_after_sync();
+          if (kDQ) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDP, sdesc_mnmajor(sDS + kk * 2048, 16384), sdesc_mnmajor(sK + kk * 2048, 16384), idQ, kk > 0);
-          mma_commit(bar(bars->dq_full));
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss(tDP, sdesc_mnmajor(sDS + kk * 2048, 16384), sdesc_mnmajor(sK + kk * 2048, 16384), idQ, kk > 0);
+            mma_commit(bar(bars->dq_full));
+          }
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -449,6 +451,7 @@ __global__ void __launch_bounds__(512, 1)
       bwd_decode(p, w, b, h, j);
       int lo, hi;
       bwd_q_range(p, j, lo, hi);
+      if (!kDQ) continue;  // dQ comes from its own kernel: these warps only follow the items
       for (int i = lo; i <= hi; ++i, ++n) {
         mbar_wait(bar(bars->dq_full), n & 1, ab);
         tc_fence_after_sync();

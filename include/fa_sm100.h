@@ -84,6 +84,19 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Deterministic backward ("FlashAttention技术解析：加速GPT训练的核心优化" §2.2, the call's
+ * `deterministic` flag): same arguments, results and workspace as fa_bwd, but dq is
+ * accumulated per query tile in a fixed order instead of by additions into a shared fp32
+ * accumulator, so repeated calls on the same inputs give bitwise identical dq, dk, dv.
+ * Three launches on `stream`: the preprocess, dK/dV, and a dQ kernel that recomputes the
+ * scores per query tile (three more matrix products than fa_bwd's dQ path, no atomics).
+ */
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv,
+                         int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
+                         void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * The three launches of fa_bwd, exposed so that a caller can time or interleave them.
  * Same arguments and rules as fa_bwd, except that `workspace` must be non-NULL and must
  * be the same buffer for the three calls of one backward, issued in this order.

@@ -84,11 +84,11 @@ def test_fwd_rejects_invalid_arguments(lib, kw, expected):
 
 
 def _bwd(lib, ws=P + 9 * T, ws_bytes=None, dq=P + 6 * T, dk=P + 7 * T, dv=P + 8 * T, B=1, N=128, H=2, d=64,
-         scale=0.125, wl=-1, wr=-1):
+         scale=0.125, wl=-1, wr=-1, fn="fa_bwd"):
     if ws_bytes is None:
         ws_bytes = lib.fa_bwd_workspace_bytes(B, N, H, d) if B > 0 and N > 0 and H > 0 else 0
-    return lib.fa_bwd(P, P + T, P + 2 * T, P + 3 * T, P + 4 * T, P + 5 * T, dq, dk, dv, B, N, H, d,
-                      ctypes.c_float(scale), 0, wl, wr, ws, ws_bytes, None)
+    return getattr(lib, fn)(P, P + T, P + 2 * T, P + 3 * T, P + 4 * T, P + 5 * T, dq, dk, dv, B, N, H, d,
+                            ctypes.c_float(scale), 0, wl, wr, ws, ws_bytes, None)
 
 
 @pytest.mark.parametrize("kw,expected", [
@@ -100,8 +100,9 @@ def _bwd(lib, ws=P + 9 * T, ws_bytes=None, dq=P + 6 * T, dk=P + 7 * T, dv=P + 8 
     (dict(ws_bytes=1024), INVALID),             # workspace too small
     (dict(ws=P + 5 * T), INVALID),              # workspace overlaps dO
 ])
-def test_bwd_rejects_invalid_arguments(lib, kw, expected):
-    assert _bwd(lib, **kw) == expected
+@pytest.mark.parametrize("fn", ["fa_bwd", "fa_bwd_deterministic"])
+def test_bwd_rejects_invalid_arguments(lib, kw, expected, fn):
+    assert _bwd(lib, fn=fn, **kw) == expected
 
 
 def test_bwd_stage_calls_reject_invalid_arguments(lib):
