@@ -451,8 +451,8 @@ __global__ void __launch_bounds__(512, 1)
       bwd_decode(p, w, b, h, j);
       int lo, hi;
       bwd_q_range(p, j, lo, hi);
-      if (!kDQ) continue;  // dQ comes from its own kernel: these warps only follow the items
-      for (int i = lo; i <= hi; ++i, ++n) {
+      // Without kDQ, dQ comes from its own kernel: these warps only follow the items.
+      for (int i = lo; kDQ && i <= hi; ++i, ++n) {
         mbar_wait(bar(bars->dq_full), n & 1, ab);
         tc_fence_after_sync();
 #pragma unroll

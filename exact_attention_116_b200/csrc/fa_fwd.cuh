@@ -15,13 +15,21 @@
 //   warps 4-7   : softmax + epilogue for Q tile 0 (one thread per query row / TMEM lane)
 //   warps 8-11  : softmax + epilogue for Q tile 1
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
-// P_t (bf16, two per column) overwrites the first 64 columns of S_t and is the A operand
-// of O_t += P_t V_j, read straight from TMEM.
+// P_t (bf16, two per column) is the A operand of O_t += P_t V_j, read straight from TMEM.
 //
-// MMA issue order per KV tile j: S0(j), PV1(j-1), S1(j), PV0(j). tcgen05.mma operations
-// issued by one thread execute in order, so S_t(j) never overwrites P_t(j-1) before
-// PV_t(j-1) has read it, and the commit that signals "S_t(j) ready" also covers PV_t(j-1):
-// when a softmax thread sees S_t(j), O_t is quiescent and may be rescaled in place.
+// D = 128 (TMEM full): P_t overwrites the first 64 columns of S_t. MMA issue order per KV
+// tile j: S0(j), PV1(j-1), S1(j), PV0(j). tcgen05.mma operations issued by one thread
+// execute in order, so S_t(j) never overwrites P_t(j-1) before PV_t(j-1) has read it, and
+// the commit that signals "S_t(j) ready" also covers PV_t(j-1): when a softmax thread sees
+// S_t(j), O_t is quiescent and may be rescaled in place. The O tile is staged for its TMA
+// store in the Q_t buffer.
+//
+// D = 64 (kSepP): P_t has its own columns P0 [384,448), P1 [448,512), so S_t(j+1) is issued
+// as soon as the softmax threads have read S_t(j) into registers ("S empty"), one tile ahead
+// of PV_t(j): the next scores are ready when a softmax thread finishes a tile. A softmax
+// thread writes P_t(j+1) and rescales O_t only after the commit of PV_t(j) ("PV done"). O is
+// staged in buffers of its own, so Q_t is released by the commit of the item's last S_t and
+// the next item's Q and K/V loads overlap this item's last tiles and epilogue.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -60,11 +68,14 @@ struct FwdCfg {
   static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile of Q, K, V or O
   static constexpr int kBoxes = D / 64;           // 64-column (128-byte) TMA boxes per tile
   static constexpr int kSlots = (D == 128) ? 4 : 8;
-  static constexpr int kOffQ = 0;                 // Q0, Q1 (also O staging)
-  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr bool kSepP = (D == 64);        // P apart from S in TMEM; O staging apart from Q
+  static constexpr int kOffQ = 0;                 // Q0, Q1 (also O staging unless kSepP)
+  static constexpr int kOffO = 2 * kTileBytes;    // O staging 0, 1 (kSepP)
+  static constexpr int kOffKV = (kSepP ? 4 : 2) * kTileBytes;
   static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+  static constexpr uint32_t kColP0 = kSepP ? 384 : kColS0, kColP1 = kSepP ? 448 : kColS1;
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -74,6 +85,7 @@ struct FwdBars {
   uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[FwdCfg<D>::kSlots], kv_empty[FwdCfg<D>::kSlots];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t s_empty[2], pv_done[2];  // kSepP only
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -198,6 +210,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(bars->p_full[t]), 128);
       mbar_init(bar(bars->o_full[t]), 1);
       mbar_init(bar(bars->o_empty[t]), 128);
+      mbar_init(bar(bars->s_empty[t]), 128);
+      mbar_init(bar(bars->pv_done[t]), 1);
     }
     for (int s = 0; s < Cfg::kSlots; ++s) {
       mbar_init(bar(bars->kv_full[s]), 1);
@@ -220,6 +234,8 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = bars->tmem_base;
 
   const uint32_t sQ[2] = {smem_base + Cfg::kOffQ, smem_base + Cfg::kOffQ + Cfg::kTileBytes};
+  const uint32_t sO[2] = {Cfg::kSepP ? smem_base + Cfg::kOffO : sQ[0],
+                          Cfg::kSepP ? smem_base + Cfg::kOffO + Cfg::kTileBytes : sQ[1]};
   const uint32_t sKV = smem_base + Cfg::kOffKV;
 
   if (warp == 0) {
@@ -275,8 +291,10 @@ __global__ void __launch_bounds__(384, 1)
       constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // O += P V, V is MN-major
       const uint32_t tS[2] = {tmem + Cfg::kColS0, tmem + Cfg::kColS1};
       const uint32_t tO[2] = {tmem + Cfg::kColO0, tmem + Cfg::kColO1};
+      const uint32_t tP[2] = {tmem + Cfg::kColP0, tmem + Cfg::kColP1};
       uint32_t slot = 0, phase = 0;
       uint32_t qn[2] = {0, 0}, pn[2] = {0, 0};
+      uint32_t kvn = 0, sq[2] = {0, 0};  // kSepP: K/V stream position, S_t issued
       bool drop_s_signal = p.debug_drop_s_signal != 0;
 
       auto issue_s = [&](int t, uint32_t k_smem) {
@@ -289,7 +307,7 @@ __global__ void __launch_bounds__(384, 1)
       auto issue_pv = [&](int t, uint32_t v_smem, bool accumulate) {
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tO[t], tS[t] + kk * 8, sdesc_mnmajor(v_smem + kk * 2048, 16384), idO, accumulate || kk > 0);
+          mma_ts(tO[t], tP[t] + kk * 8, sdesc_mnmajor(v_smem + kk * 2048, 16384), idO, accumulate || kk > 0);
       };
 
       for (int round = 0;; ++round) {
@@ -308,6 +326,51 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < 2; ++t)
           if (act[t]) mbar_wait(bar(bars->q_full[t]), qn[t] & 1, ab);
         tc_fence_after_sync();
+
+        if constexpr (Cfg::kSepP) {
+          // K(j) is tile n0 + 2(j - lo) of the K/V stream and V(j) the next one; stream tile n
+          // sits in slot n % kSlots, filled for the (n / kSlots)-th time.
+          const uint32_t n0 = kvn;
+          auto kv_wait = [&](uint32_t n) {
+            const uint32_t s = n % Cfg::kSlots;
+            mbar_wait(bar(bars->kv_full[s]), (n / Cfg::kSlots) & 1, ab);
+            tc_fence_after_sync();
+            return s;
+          };
+          auto s_step = [&](int j) {  // S0(j), S1(j), each once the previous S_t has been read
+            const uint32_t ks = kv_wait(n0 + 2 * (j - lo));
+            for (int t = 0; t < 2; ++t) {
+              if (!active(t, j)) continue;
+              mbar_wait(bar(bars->s_empty[t]), (sq[t] & 1) ^ 1, ab);
+              ++sq[t];
+              tc_fence_after_sync();
+              issue_s(t, sKV + ks * Cfg::kTileBytes);
+              if (drop_s_signal) drop_s_signal = false;
+              else mma_commit(bar(bars->s_full[t]));
+              if (j == hi_t[t]) mma_commit(bar(bars->q_empty[t]));  // last read of Q_t in this item
+            }
+            mma_commit(bar(bars->kv_empty[ks]));
+          };
+          s_step(lo);
+          for (int j = lo; j <= hi; ++j) {
+            if (j < hi) s_step(j + 1);
+            const uint32_t vs = kv_wait(n0 + 2 * (j - lo) + 1);
+            for (int t = 0; t < 2; ++t) {
+              if (!active(t, j)) continue;
+              mbar_wait(bar(bars->p_full[t]), pn[t] & 1, ab);
+              ++pn[t];
+              tc_fence_after_sync();
+              issue_pv(t, sKV + vs * Cfg::kTileBytes, !first_pv[t]);
+              first_pv[t] = false;
+              mma_commit(bar(bars->pv_done[t]));
+            }
+            mma_commit(bar(bars->kv_empty[vs]));
+          }
+          kvn = n0 + 2 * (hi - lo + 1);
+          for (int t = 0; t < 2; ++t)
+            if (act[t]) ++qn[t];
+          continue;
+        }
 
         uint32_t v_prev_slot = 0;
         auto wait_p_and_o = [&](int t) {
@@ -370,8 +433,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_field = (uint32_t)((row & ~31) << 16);
     const uint32_t tS = tmem + lane_field + (t ? Cfg::kColS1 : Cfg::kColS0);
     const uint32_t tO = tmem + lane_field + (t ? Cfg::kColO1 : Cfg::kColO0);
+    const uint32_t tP = tmem + lane_field + (t ? Cfg::kColP1 : Cfg::kColP0);
     const float c = p.scale_log2;
-    uint32_t sn = 0, on = 0;
+    uint32_t sn = 0, on = 0, pvn = 0;
 
     for (int round = 0;; ++round) {
       const int w = sched_item(round, blockIdx.x, gridDim.x);
@@ -396,6 +460,10 @@ __global__ void __launch_bounds__(384, 1)
         for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, r[q4]);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) tmem_wait_ld(r[q4]);
+        if constexpr (Cfg::kSepP) {  // S_t may now be overwritten by the next tile's scores
+          tc_fence_before_sync();
+          mbar_arrive(bar(bars->s_empty[t]));
+        }
         float x[128];
 #pragma unroll
         for (int cc = 0; cc < 128; ++cc) x[cc] = __uint_as_float(r[cc >> 5][cc & 31]);
@@ -408,7 +476,12 @@ __global__ void __launch_bounds__(384, 1)
         else
           fwd_row_max<false>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated);
         const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-        // P in 32-column chunks straight into TMEM (over S columns already read into registers)
+        if (Cfg::kSepP && j > lo) {  // PV_t(j-1) has read P_t and O_t is quiescent
+          mbar_wait(bar(bars->pv_done[t]), pvn & 1, ab);
+          ++pvn;
+          tc_fence_after_sync();
+        }
+        // P in 32-column chunks straight into TMEM (D = 128: over S columns already read into registers)
         float2 sum0 = make_float2(0.0f, 0.0f), sum1 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
@@ -417,7 +490,7 @@ __global__ void __launch_bounds__(384, 1)
             fwd_exp_chunk<true>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
           else
             fwd_exp_chunk<false>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
-          tmem_st16(tS + q4 * 16, pk);
+          tmem_st16(tP + q4 * 16, pk);
         }
         const float2 s01 = add2(sum0, sum1);
         l_run = l_run * alpha + (s01.x + s01.y);
@@ -441,11 +514,19 @@ __global__ void __launch_bounds__(384, 1)
       }
 
       // Epilogue: O_t / l -> bf16 -> staging (the Q_t buffer, free once the last PV_t is done) -> TMA store.
-      mbar_wait(bar(bars->o_full[t]), on & 1, ab);
-      ++on;
-      tc_fence_after_sync();
+      if constexpr (Cfg::kSepP) {
+        mbar_wait(bar(bars->pv_done[t]), pvn & 1, ab);  // the item's last PV_t
+        ++pvn;
+        tc_fence_after_sync();
+        if (row == 0) bulk_wait_group_read0();  // the previous store has read the staging tile
+        named_bar_sync(1 + t, 128);
+      } else {
+        mbar_wait(bar(bars->o_full[t]), on & 1, ab);
+        ++on;
+        tc_fence_after_sync();
+      }
       const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-      const uint32_t stage = sQ[t];
+      const uint32_t stage = sO[t];
 #pragma unroll 1
       for (int cc = 0; cc < D; cc += 32) {
         uint32_t o[32];
@@ -461,16 +542,20 @@ __global__ void __launch_bounds__(384, 1)
           st_shared_v4(box + sw128_offset(row, ((cc & 63) >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
         }
       }
-      tc_fence_before_sync();
-      mbar_arrive(bar(bars->o_empty[t]));
+      if constexpr (!Cfg::kSepP) {
+        tc_fence_before_sync();
+        mbar_arrive(bar(bars->o_empty[t]));
+      }
       fence_proxy_async_smem();
       named_bar_sync(1 + t, 128);
       if (row == 0) {
 #pragma unroll
         for (int bx = 0; bx < Cfg::kBoxes; ++bx) tma_store_4d(&tmO, stage + bx * 16384, bx * 64, r0, h, b);
         bulk_commit_group();
-        bulk_wait_group_read0();
-        mbar_arrive(bar(bars->q_empty[t]));
+        if constexpr (!Cfg::kSepP) {  // the Q_t buffer is free again once the store has read it
+          bulk_wait_group_read0();
+          mbar_arrive(bar(bars->q_empty[t]));
+        }
       }
       if (i < p.N) {
         const float lse = l_run > 0.0f ? (m_run + lg2_approx(l_run)) * kLn2 : -INFINITY;

@@ -122,3 +122,15 @@ def test_fwd_autograd_wrapper_matches():
     o1 = fa.flash_attention(qd, kd, vd, None, True)
     o2, _ = fa.attention_fwd(qd, kd, vd, None, True)
     assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("B,N,H", [(2, 777, 48), (3, 200, 64)])
+def test_fwd_many_items_per_cta(d, B, N, H):
+    """More work items than SMs, so each CTA runs several items back to back: the next item's
+    Q and K/V loads and its first scores overlap the previous item's last tiles and epilogue."""
+    q, k, v, _ = make_custom(B, N, H, d, seed=600 + N + d)
+    for causal, win in [(True, (-1, -1)), (False, (64, 200)), (False, (-1, -1))]:
+        o, lse = gpu_fwd(q, k, v, None, causal, win)
+        o_ref, lse_ref = oracle.attention_forward(to_np(q), to_np(k), to_np(v), 1.0 / d ** 0.5, causal, *win)
+        assert_fwd_close(to_np(o), to_np(lse), o_ref, lse_ref, f"B{B} N{N} H{H} d{d} causal={causal} win={win}")
