@@ -55,6 +55,8 @@ def decode_forward(q, k_cache, v_cache, block_table, seqlens, scale, causal=Fals
     lse = np.full((B, H, Sq), -np.inf)
     for b in range(B):
         n = int(seqlens[b])
+        if n == 0:  # no keys: every row keeps O = 0, LSE = -inf
+            continue
         k = gather_sequence(k_cache, block_table, b, n, page_size)
         v = gather_sequence(v_cache, block_table, b, n, page_size)
         pos = np.arange(n - Sq, n, dtype=np.int64)

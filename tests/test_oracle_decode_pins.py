@@ -115,7 +115,26 @@ def pin_page_placement(impl):
         assert np.allclose(out[0], ref[0], atol=1e-12, rtol=0) and np.allclose(out[1], ref[1], atol=1e-12, rtol=0)
 
 
-DECODE_PINS = [pin_window_counts, pin_matches_training_path, pin_page_placement]
+def pin_empty_and_short_sequences(impl):
+    """A sequence without keys gives O = 0 and LSE = -inf; with fewer keys than Sq the rows
+    before its first key see nothing under causal masking."""
+    rng = np.random.default_rng(54)
+    H, d, Sq = 1, 4, 3
+    lens = [0, 2, 5]
+    ks = [rng.standard_normal((max(n, 1), H, d))[:n] for n in lens]
+    vs = [rng.standard_normal((max(n, 1), H, d))[:n] for n in lens]
+    kc, table = paged(np.random.default_rng(6), [k if len(k) else np.zeros((1, H, d)) for k in ks], 4)
+    vc, _ = paged(np.random.default_rng(6), [v if len(v) else np.zeros((1, H, d)) for v in vs], 4)
+    q = rng.standard_normal((3, Sq, H, d))
+    o, lse = impl.decode_forward(q, kc, vc, table, lens, 0.5, True)
+    assert (o[0] == 0).all() and np.isneginf(lse[0]).all()
+    # sequence 1: positions -1, 0, 1 -> row 0 sees nothing, row 1 sees key 0, row 2 keys 0..1
+    assert (o[1, 0] == 0).all() and np.isneginf(lse[1, 0, 0])
+    assert np.allclose(o[1, 1], vs[1][0], atol=1e-12, rtol=0)
+    assert abs(lse[1, 0, 1] - 0.5 * float(q[1, 1, 0] @ ks[1][0, 0])) < 1e-12
+
+
+DECODE_PINS = [pin_window_counts, pin_matches_training_path, pin_page_placement, pin_empty_and_short_sequences]
 
 
 @pytest.mark.parametrize("pin", DECODE_PINS, ids=lambda f: f.__name__)
