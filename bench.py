@@ -3,6 +3,9 @@
 One step = one pass of the whole hot path over one batch of synthetic input: fa_fwd (O, LSE)
 followed by the backward's three launches (preprocess, main, dQ conversion). The default
 workload is the training configuration B=2, H=16, N=8192, d=128, causal, bf16.
+``--config train_fwd_fp8`` instead times the E4M3 forward (fa_fwd_fp8) on the same shape:
+one step = one launch. ``--config decode_paged`` times the paged-KV decode (fa_decode_paged):
+one step = one call (split kernel + merge) over every sequence, reported in GB/s of cache read.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
 
@@ -34,16 +37,20 @@ sys.path.insert(0, ROOT)
 
 from exact_attention_116_b200 import binding  # noqa: E402
 from exact_attention_116_b200 import distributed as mg  # noqa: E402
-from exact_attention_116_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+from exact_attention_116_b200.inputs import (CONFIGS, DECODE_CONFIGS, FP8_CONFIGS, make_decode_inputs,  # noqa: E402
+                                             make_fp8_inputs, make_inputs)
 from exact_attention_116_b200.workload import flops, hbm_bytes, visible_pairs  # noqa: E402
 
 METRIC = "attention fwd/bwd TFLOPS (bf16, causal) and % of B200 dense BF16 peak"
+METRIC_FP8 = "attention fwd TFLOPS (E4M3 inputs, causal) and % of B200 dense FP8 peak"
+FP8_PER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor throughput (4.5 / 2.25 PFLOP/s)
+METRIC_DECODE = "paged-KV decode attention GB/s of KV cache read (bf16) and % of B200 HBM bandwidth"
 UNIT = "TFLOPS"
 L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "ncu_traffic.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_116_b200", "csrc", f)
-                  for f in ("fa_api.cu", "fa_fwd.cuh", "fa_bwd.cuh", "sm100_ptx.cuh")]
+                  for f in ("fa_api.cu", "fa_fwd.cuh", "fa_bwd.cuh", "fa_bwd_dq.cuh", "sm100_ptx.cuh")]
 
 
 def peaks():
@@ -180,7 +187,284 @@ def oracle_sample(cfg, seconds: float, q=None, k=None, v=None, do=None):
     return 14 * cfg.d * pairs / dt / 1e12, dt, rows_done, threads
 
 
+def oracle_sample_fp8(cfg, seconds: float, codes=None, descales=None):
+    """Time the fp64 oracle's E4M3 forward, as it stands, on blocks of 512 query rows, head after
+    head of batch 0, until `seconds` have passed. Returns (TFLOPS by 4*d*pairs, seconds, rows, threads)."""
+    from oracle import fp8_e4m3 as oracle8
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        threads = os.cpu_count()
+    if codes is None:
+        codes, descales = make_fp8_inputs(cfg)
+    cn = [t.numpy() for t in codes]
+    dn = [t.numpy().astype(np.float64) for t in descales]
+    n, block = cfg.N, min(512, cfg.N)
+    wr = 0 if cfg.causal else cfg.win_r
+    pairs, rows_done = 0, 0
+    t0 = time.perf_counter()
+    for h in range(cfg.H):
+        r1 = n
+        while r1 > 0:
+            r0 = max(0, r1 - block)
+            rows = np.arange(r0, r1)
+            oracle8.forward_rows_fp8(*cn, *dn, 0, h, rows, cfg.scale, cfg.causal, cfg.win_l, cfg.win_r)
+            for i in range(r0, r1):
+                lo = max(0, i - cfg.win_l) if cfg.win_l >= 0 else 0
+                hi = min(n - 1, i + wr) if wr >= 0 else n - 1
+                pairs += hi - lo + 1
+            rows_done += r1 - r0
+            r1 = r0
+            if time.perf_counter() - t0 >= seconds:
+                break
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return 4 * cfg.d * pairs / dt / 1e12, dt, rows_done, threads
+
+
 # ----------------------------------------------------------------------------- GPU arm
+
+def decode_cache_bytes(cfg, seqlens) -> int:
+    """Algorithmic bytes of one decode call: the K and V rows every sequence's keys occupy (the
+    whole sequence is visible to its newest rows), plus q, O and LSE."""
+    kv = int(seqlens.sum()) * cfg.H * cfg.d * 2 * 2
+    return kv + 2 * cfg.B * cfg.Sq * cfg.H * cfg.d * 2 + cfg.B * cfg.H * cfg.Sq * 4
+
+
+def oracle_sample_decode(cfg, seconds: float, inputs):
+    """Time the fp64 decode oracle, as it stands, one sequence at a time until `seconds` have passed.
+    Returns (GB/s of cache rows processed, seconds, sequences, threads)."""
+    from oracle import decode_paged_fp64 as oracle_dec
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
+    except Exception:
+        threads = os.cpu_count()
+    q, kc, vc, table, lens = inputs
+    qn, kn, vn, tn, ln_ = q.double().numpy(), kc.float().numpy(), vc.float().numpy(), table.numpy(), lens.numpy()
+    done_bytes, seqs = 0, 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        b = seqs % cfg.B
+        oracle_dec.decode_forward(qn[b:b + 1], kn, vn, tn[b:b + 1], ln_[b:b + 1], cfg.scale, cfg.causal, cfg.win_l,
+                                  cfg.win_r)
+        done_bytes += int(ln_[b]) * cfg.H * cfg.d * 2 * 2
+        seqs += 1
+    dt = time.perf_counter() - t0
+    return done_bytes / dt / 1e9, dt, seqs, threads
+
+
+def run_gpu_decode(args):
+    """Paged-KV decode: one step = one fa_decode_paged call over all sequences."""
+    info = mg.rank_info()
+    world, rank, local = info.world, info.rank, info.local_rank
+    torch.cuda.set_device(local)
+    mg.init(info, "nccl", device=torch.device("cuda", local))
+    cfg = DECODE_CONFIGS[args.config]
+    host = make_decode_inputs(cfg)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, kc, vc, table, lens = (x.to(dev) for x in host)
+    B, Sq, H, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
+    splits = int(args.splits)
+    stream = torch.cuda.current_stream()
+    # the splits the library picks for splits=0 need this workspace at most (128 splits)
+    ws = torch.empty(max(1, binding.decode_workspace_bytes(B, Sq, H, d, 128)), dtype=torch.uint8, device=dev)
+    # L2 flush between steps: the cache is 2x268 MiB > L2 already, q/O are tiny
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        binding.decode_paged_into(q, kc, vc, table, lens, o, lse, cfg.scale, cfg.causal, (cfg.win_l, cfg.win_r),
+                                  splits, ws)
+
+    for _ in range(args.warmup):
+        step()
+    binding.check()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index) if local == 0 else None
+    mg.barrier(info)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    ms = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        b.synchronize()
+        ms += a.elapsed_time(b)
+    torch.cuda.synchronize()
+    mg.barrier(info)
+    t_wall1 = time.time()
+    binding.check()
+    clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
+    ms_step = mg.max_over_ranks(info, ms, dev) / args.steps
+    nbytes = decode_cache_bytes(cfg, host[4])
+    gbs = nbytes / (ms_step * 1e-3) / 1e9
+
+    pin = [x.pin_memory() for x in host]
+    o_h = torch.empty_like(host[0]).pin_memory()
+    lse_h = torch.empty((B, H, Sq), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for src, dst in zip(pin, (q, kc, vc, table, lens)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        o_h.copy_(o, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    mg.barrier(info)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    mg.barrier(info)
+    binding.check()
+    e2e_ms = mg.max_over_ranks(info, e0.elapsed_time(e1), dev) / e2e_steps
+    h2d = sum(x.numel() * x.element_size() for x in host)
+
+    peak, peak_src = peaks()
+    res = {
+        "metric": METRIC_DECODE, "value": round(gbs * world, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 cache, uniform ragged lengths, random page order)",
+        "config": {"workload": f"{cfg.name}: {cfg.note}", "B": B, "Sq": Sq, "H": H, "d": d,
+                   "page_size": cfg.page_size, "lengths": [int(x) for x in host[4]], "causal": cfg.causal,
+                   "splits": splits if splits else "auto", "seed": cfg.seed,
+                   "l2": "L2 flushed (512 MiB write) before every timed step; KV cache > L2",
+                   "bytes": "K and V rows of every visible key + q, O, LSE"},
+        "roofline": {"kernel": "fa_decode_split_kernel<128> + combine", "bound": "hbm", "achieved": round(gbs, 1),
+                     "peak": peak["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peak["hbm_gbs"], 4),
+                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)", "traffic": None,
+                     "algorithmic_bytes": nbytes},
+        "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, seqs, threads = oracle_sample_decode(cfg, args.cpu_seconds, host)
+        res["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                               "sample": f"fp64 decode oracle (page gather + definition) on {seqs} sequences of "
+                                         f"{cfg.name}, {dt:.1f} s, same byte convention"}
+    mg.shutdown(info)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def run_gpu_fp8(args):
+    """E4M3 forward: one step = one fa_fwd_fp8 launch over the whole workload."""
+    info = mg.rank_info()
+    world, rank, local = info.world, info.rank, info.local_rank
+    torch.cuda.set_device(local)
+    mg.init(info, "nccl", device=torch.device("cuda", local))
+    cfg = FP8_CONFIGS[args.config]
+    scale, causal, win = cfg.scale, cfg.causal, (cfg.win_l, cfg.win_r)
+    B, N, H, d = cfg.shape
+    codes_h, desc_h = make_fp8_inputs(cfg)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    codes = [x.to(dev) for x in codes_h]
+    desc = [x.to(dev) for x in desc_h]
+    o = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        binding.fwd_fp8_into(*codes, *desc, o, lse, scale, causal, win)
+
+    for _ in range(args.warmup):
+        step()
+    binding.check()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index) if local == 0 else None
+    mg.barrier(info)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    mg.barrier(info)
+    t_wall1 = time.time()
+    binding.check()
+    clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
+    ms_step = mg.max_over_ranks(info, start.elapsed_time(end), dev) / args.steps
+    f_fwd, _ = flops(B, N, H, d, causal, *win)
+
+    pin = [x.pin_memory() for x in (*codes_h, *desc_h)]
+    o_h = torch.empty((B, N, H, d), dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for src, dst in zip(pin, (*codes, *desc)):
+            dst.copy_(src, non_blocking=True)
+        binding.fwd_fp8_into(*codes, *desc, o, lse, scale, causal, win)
+        o_h.copy_(o, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    mg.barrier(info)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    mg.barrier(info)
+    binding.check()
+    e2e_ms = mg.max_over_ranks(info, e0.elapsed_time(e1), dev) / e2e_steps
+
+    peak, peak_src = peaks()
+    fp8_peak = peak["bf16_tflops"] * FP8_PER_BF16
+    achieved = f_fwd / (ms_step * 1e-3) / 1e12
+    in_bytes = 3 * B * N * H * d + 3 * B * H * 4
+    res = {
+        "metric": METRIC_FP8, "value": round(mg.aggregate_rate(f_fwd, world, ms_step * 1e-3) / 1e12, 3),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic (seeded N(0,1), per-head E4M3 quantisation with descale = amax/448)",
+        "config": {"workload": f"{cfg.name}: {cfg.note}", "B": B, "N": N, "H": H, "d": d, "causal": causal,
+                   "window": list(win), "seed": cfg.seed,
+                   "l2": f"inputs larger than L2 (q,k,v = {in_bytes / 2**20:.0f} MiB > 126 MiB); no flush",
+                   "flops": "4*d*pairs over exactly counted visible pairs",
+                   "per_rank": "each rank runs the whole workload on its own inputs"},
+        "roofline": {"kernel": "fa_fwd_kernel<128, E4M3>", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
+                     "frac_of_bf16_peak": round(achieved / peak["bf16_tflops"], 4),
+                     "peak_source": f"{peak_src} bf16_tflops x {FP8_PER_BF16} (nominal dense FP8/BF16 ratio)",
+                     "traffic": None, "algorithmic_bytes": in_bytes + B * N * H * d * 2 + B * H * N * 4},
+        "e2e": {"value": round(mg.aggregate_rate(f_fwd, world, e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": B * N * H * d * 2 + B * H * N * 4},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, dt, rows, threads = oracle_sample_fp8(cfg, args.cpu_seconds, codes_h, desc_h)
+        res["cpu_baseline"] = {"value": round(tf, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                               "sample": f"fp64 oracle E4M3 forward (decode, descale, definition) of {rows} query rows "
+                                         f"(512-row blocks, heads of batch 0 in order) of {cfg.name}, {dt:.1f} s"}
+    mg.shutdown(info)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
 
 def run_gpu(args):
     info = mg.rank_info()
@@ -333,9 +617,13 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    per_step = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    if args.config in FP8_CONFIGS:
+        return run_reference_fp8(args, FP8_CONFIGS[args.config], per_step, world)
+    if args.config in DECODE_CONFIGS:
+        return run_reference_decode(args, DECODE_CONFIGS[args.config], per_step, world)
     cfg = CONFIGS[args.config]
     q, k, v, do = make_inputs(cfg)
-    per_step = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample(cfg, per_step, q, k, v, do)
     vals, threads, rows, secs = [], 1, 0, 0.0
@@ -358,12 +646,60 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+def run_reference_decode(args, cfg, per_step, world):
+    host = make_decode_inputs(cfg)
+    for _ in range(args.warmup):
+        oracle_sample_decode(cfg, per_step, host)
+    vals, threads, seqs, secs = [], 1, 0, 0.0
+    for _ in range(args.steps):
+        v, dt, seqs, threads = oracle_sample_decode(cfg, per_step, host)
+        vals.append(v)
+        secs += dt
+    value = statistics.mean(vals)
+    res = {"impl": "reference", "metric": METRIC_DECODE, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / max(1, args.steps) * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded N(0,1) bf16 cache widened to fp64)",
+           "config": {"workload": f"{cfg.name}: {cfg.note}", "B": cfg.B, "Sq": cfg.Sq, "H": cfg.H, "d": cfg.d,
+                      "page_size": cfg.page_size, "seed": cfg.seed},
+           "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                            "sample": f"fp64 decode oracle on {seqs} sequences per step, about {per_step:.1f} s each"},
+           "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def run_reference_fp8(args, cfg, per_step, world):
+    codes, descales = make_fp8_inputs(cfg)
+    for _ in range(args.warmup):
+        oracle_sample_fp8(cfg, per_step, codes, descales)
+    vals, threads, rows, secs = [], 1, 0, 0.0
+    for _ in range(args.steps):
+        tf, dt, rows, threads = oracle_sample_fp8(cfg, per_step, codes, descales)
+        vals.append(tf)
+        secs += dt
+    value = statistics.mean(vals)
+    sample = (f"fp64 oracle E4M3 forward of {rows} query rows (512-row blocks, heads of batch 0 in order) of "
+              f"{cfg.name} per step, about {per_step:.1f} s each")
+    res = {"impl": "reference", "metric": METRIC_FP8, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / max(1, args.steps) * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded N(0,1), E4M3 codes decoded to fp64)",
+           "config": {"workload": f"{cfg.name}: {cfg.note}", "B": cfg.B, "N": cfg.N, "H": cfg.H, "d": cfg.d,
+                      "causal": cfg.causal, "window": [cfg.win_l, cfg.win_r], "seed": cfg.seed},
+           "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="train_fwd_bwd", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="train_fwd_bwd",
+                    choices=sorted(CONFIGS) + sorted(FP8_CONFIGS) + sorted(DECODE_CONFIGS))
+    ap.add_argument("--splits", type=int, default=0, help="decode: KV splits per (b, h); 0 = library's choice")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -372,6 +708,10 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.config in FP8_CONFIGS:
+        run_gpu_fp8(args)
+    elif args.config in DECODE_CONFIGS:
+        run_gpu_decode(args)
     else:
         run_gpu(args)
 

@@ -9,11 +9,16 @@ from .binding import (  # noqa: F401
     FaError,
     FlashAttention,
     attention_bwd,
+    attention_decode_paged,
     attention_fwd,
+    attention_fwd_fp8,
     bwd_into,
     bwd_stages,
     check,
+    decode_paged_into,
+    decode_workspace_bytes,
     flash_attention,
+    fwd_fp8_into,
     fwd_into,
     load,
     workspace_bytes,

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
                 4: "FA_ERR_TIMEOUT", 5: "FA_ERR_NO_MEMORY", 6: "FA_ERR_DEVICE"}
-EXPORTS = ("fa_fwd", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess",
+EXPORTS = ("fa_fwd", "fa_fwd_fp8", "fa_decode_workspace_bytes", "fa_decode_paged", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess",
            "fa_bwd_main", "fa_bwd_dq_convert", "fa_bwd_static_workspace", "fa_check", "fa_status_string")
 
 _lib = None
@@ -41,6 +41,10 @@ def load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    lib.fa_decode_workspace_bytes.argtypes = [i, i, i, i, i]
+    lib.fa_decode_workspace_bytes.restype = sz
+    lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, i, vp, sz, vp]
     lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_bytes.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp, sz, vp]
@@ -51,7 +55,7 @@ def load() -> ctypes.CDLL:
     lib.fa_check.argtypes = [vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
-    for name in ("fa_fwd", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
+    for name in ("fa_fwd", "fa_fwd_fp8", "fa_decode_paged", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
                  "fa_check"):
         getattr(lib, name).restype = i
     _lib = lib
@@ -76,15 +80,15 @@ def _stream_handle(stream) -> int | None:
     return stream.cuda_stream
 
 
-def _check_qkv(*ts: torch.Tensor) -> tuple[int, int, int, int]:
+def _check_qkv(*ts: torch.Tensor, dtype=torch.bfloat16) -> tuple[int, int, int, int]:
     shape = ts[0].shape
     if len(shape) != 4:
         raise ValueError("tensors must be (batch, seq, heads, head_dim)")
     for t in ts:
         if not t.is_cuda:
             raise ValueError("tensors must be on a CUDA device (there is no CPU path)")
-        if t.dtype != torch.bfloat16:
-            raise ValueError("tensors must be bfloat16")
+        if t.dtype != dtype:
+            raise ValueError(f"tensors must be {dtype}")
         if t.shape != shape or not t.is_contiguous():
             raise ValueError("tensors must be contiguous and of equal shape")
     return tuple(int(x) for x in shape)  # type: ignore[return-value]
@@ -110,6 +114,41 @@ def attention_fwd(q, k, v, scale=None, causal=False, window=(-1, -1), stream=Non
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     fwd_into(q, k, v, o, lse, scale, causal, window, stream)
+    return o, lse
+
+
+def _as_codes(t: torch.Tensor) -> torch.Tensor:
+    """E4M3 tensors may come as torch.float8_e4m3fn or as their uint8 codes."""
+    return t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t
+
+
+def fwd_fp8_into(q8, k8, v8, q_descale, k_descale, v_descale, o, lse, scale=None, causal=False, window=(-1, -1),
+                 stream=None) -> None:
+    """fa_fwd_fp8: q8, k8, v8 (B,N,H,d) E4M3 codes (uint8 or float8_e4m3fn), descales (B,H) float32,
+    into o (B,N,H,d) bf16 and lse (B,H,N) float32."""
+    q8, k8, v8 = (_as_codes(t) for t in (q8, k8, v8))
+    B, N, H, d = _check_qkv(q8, k8, v8, dtype=torch.uint8)
+    _check_qkv(o)
+    if tuple(o.shape) != (B, N, H, d):
+        raise ValueError("o must have the shape of q")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous() or not lse.is_cuda:
+        raise ValueError("lse must be a contiguous (B, H, N) float32 CUDA tensor")
+    for t in (q_descale, k_descale, v_descale):
+        if t.dtype != torch.float32 or tuple(t.shape) != (B, H) or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("descales must be contiguous (B, H) float32 CUDA tensors")
+    st = load().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_descale.data_ptr(), k_descale.data_ptr(),
+                           v_descale.data_ptr(), o.data_ptr(), lse.data_ptr(), B, N, H, d, _scale(scale, d),
+                           int(bool(causal)), int(window[0]), int(window[1]), _stream_handle(stream))
+    _raise(st, "fa_fwd_fp8")
+
+
+def attention_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal=False, window=(-1, -1),
+                      stream=None):
+    """FP8 forward: returns (o, lse), o (B,N,H,d) bf16 and lse (B,H,N) float32."""
+    B, N, H, d = q8.shape
+    o = torch.empty((B, N, H, d), dtype=torch.bfloat16, device=q8.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    fwd_fp8_into(q8, k8, v8, q_descale, k_descale, v_descale, o, lse, scale, causal, window, stream)
     return o, lse
 
 
@@ -211,3 +250,41 @@ class FlashAttention(torch.autograd.Function):
 def flash_attention(q, k, v, scale=None, causal=False, window=(-1, -1)):
     """Differentiable exact attention on (batch, seq, heads, head_dim) bf16 CUDA tensors."""
     return FlashAttention.apply(q, k, v, scale, causal, window)
+
+
+def decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale=None, causal=False, window=(-1, -1),
+                      splits=0, workspace=None, stream=None) -> None:
+    """fa_decode_paged: q (B,Sq,H,d) bf16 new rows; k_cache, v_cache (num_pages,page_size,H,d) bf16;
+    block_table (B,max_pages) int32; seqlens (B,) int32; into o (B,Sq,H,d) bf16, lse (B,H,Sq) float32."""
+    B, Sq, H, d = _check_qkv(q, o)
+    _check_qkv(k_cache, v_cache)
+    num_pages, page_size, Hc, dc = k_cache.shape
+    if (Hc, dc) != (H, d):
+        raise ValueError("cache heads / head dim must match q")
+    for t, name in ((block_table, "block_table"), (seqlens, "seqlens")):
+        if t.dtype != torch.int32 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(seqlens.shape) != (B,):
+        raise ValueError("block_table must be (B, max_pages) and seqlens (B,)")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Sq) or not lse.is_contiguous() or not lse.is_cuda:
+        raise ValueError("lse must be a contiguous (B, H, Sq) float32 CUDA tensor")
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    st = load().fa_decode_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+                                seqlens.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Sq, H, d, num_pages, page_size,
+                                int(block_table.shape[1]), _scale(scale, d), int(bool(causal)), int(window[0]),
+                                int(window[1]), int(splits), ws_ptr, ws_bytes, _stream_handle(stream))
+    _raise(st, "fa_decode_paged")
+
+
+def decode_workspace_bytes(B: int, Sq: int, H: int, d: int, splits: int) -> int:
+    return int(load().fa_decode_workspace_bytes(B, Sq, H, d, splits))
+
+
+def attention_decode_paged(q, k_cache, v_cache, block_table, seqlens, scale=None, causal=False, window=(-1, -1),
+                           splits=0, stream=None):
+    """Paged-KV decode: returns (o, lse), o (B,Sq,H,d) bf16 and lse (B,H,Sq) float32."""
+    B, Sq, H, d = q.shape
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale, causal, window, splits, None, stream)
+    return o, lse

@@ -14,6 +14,7 @@
 #include "fa_sm100.h"
 #include "fa_bwd.cuh"
 #include "fa_bwd_dq.cuh"
+#include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -69,6 +70,12 @@ int device_setup(int* dev_out, int* sm_count) {
                                fa::FwdCfg<64>::kSmemBytes) != cudaSuccess ||
           cudaFuncSetAttribute(fa::fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fa::FwdCfg<128>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::FwdCfg<128, true>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_decode_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::DecCfg<64>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_decode_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::DecCfg<128>::kSmemBytes) != cudaSuccess ||
           cudaFuncSetAttribute(fa::fa_bwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fa::BwdCfg<64>::kSmemBytes) != cudaSuccess ||
           cudaFuncSetAttribute(fa::fa_bwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -139,6 +146,36 @@ int make_map(CUtensorMap* m, const void* base, const Shape& s) {
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID_ARG;
 }
 
+// 4-D map over a (B, N, H, d) tensor of E4M3 codes: dims (d, N, H, B), box (128, 128, 1, 1)
+// (128 bytes x 128 rows), 128B swizzle.
+int make_map_u8(CUtensorMap* m, const void* base, const Shape& s) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)s.d, (cuuint64_t)s.N, (cuuint64_t)s.H, (cuuint64_t)s.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)s.H * s.d, (cuuint64_t)s.d, (cuuint64_t)s.N * s.H * s.d};
+  const cuuint32_t box[4] = {128, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID_ARG;
+}
+
+// 4-D map over a paged (num_pages, page_size, H, d) bf16 cache: dims (d, H, page_size, num_pages),
+// box (64, 1, 64, 1) (128 bytes x 64 rows of one head and one page), 128B swizzle.
+int make_map_cache(CUtensorMap* m, const void* base, int num_pages, int page_size, int H, int d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)page_size, (cuuint64_t)num_pages};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)page_size * H * d * 2};
+  const cuuint32_t box[4] = {64, 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_INVALID_ARG;
+}
+
 // 4-D map over the (B, N, H, d) fp32 dQ accumulator for TMA reduce-add: box (32, 128, 1, 1)
 // (128 bytes x 128 rows), 128B swizzle.
 int make_map_f32_acc(CUtensorMap* m, const void* base, const Shape& s) {
@@ -183,14 +220,20 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_
 
 // ---------------------------------------------------------------- launches (arguments already checked)
 
+// descales != nullptr: q, k, v hold E4M3 codes (head dim 128) with (B, H) descale factors.
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& s, float scale,
-               int causal, int win_l, int win_r, int sm_count, cudaStream_t stream) {
+               int causal, int win_l, int win_r, int sm_count, cudaStream_t stream,
+               const float* const* descales = nullptr) {
   CUtensorMap mq, mk, mv, mo;
   int st;
-  if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
+  auto in_map = descales ? make_map_u8 : make_map;
+  if ((st = in_map(&mq, q, s)) || (st = in_map(&mk, k, s)) || (st = in_map(&mv, v, s)) ||
       (st = make_map(&mo, o, s)))
     return st;
   fa::FwdParams p;
+  p.q_descale = descales ? descales[0] : nullptr;
+  p.k_descale = descales ? descales[1] : nullptr;
+  p.v_descale = descales ? descales[2] : nullptr;
   p.B = s.B;
   p.N = s.N;
   p.H = s.H;
@@ -210,7 +253,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     std::fprintf(stderr, "[fa] fwd B=%d N=%d H=%d d=%d causal=%d win=(%d,%d) items=%d grid=%d smem=%d\n", s.B, s.N,
                  s.H, s.d, p.causal, win_l, win_r, p.num_items, grid,
                  s.d == 64 ? fa::FwdCfg<64>::kSmemBytes : fa::FwdCfg<128>::kSmemBytes);
-  if (s.d == 64)
+  if (descales)
+    fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128, true>::kThreads, fa::FwdCfg<128, true>::kSmemBytes,
+                                   stream>>>(mq, mk, mv, mo, p);
+  else if (s.d == 64)
     fa::fa_fwd_kernel<64><<<grid, fa::FwdCfg<64>::kThreads, fa::FwdCfg<64>::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
   else
     fa::fa_fwd_kernel<128><<<grid, fa::FwdCfg<128>::kThreads, fa::FwdCfg<128>::kSmemBytes, stream>>>(mq, mk, mv, mo,
@@ -379,6 +425,144 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   int dev, sms;
   if ((st = device_setup(&dev, &sms))) return st;
   return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale, const float* k_descale,
+               const float* v_descale, void* o, float* lse, int B, int N, int H, int d, float scale, int causal,
+               int win_l, int win_r, fa_stream_t stream) {
+  int st = check_problem(B, N, H, d, scale, causal, &win_l, &win_r);
+  if (st) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !q_descale || !k_descale || !v_descale || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(q_descale, 4) || !aligned(k_descale, 4) || !aligned(v_descale, 4))
+    return FA_ERR_INVALID_ARG;
+  const Shape s{B, N, H, d};
+  const size_t ib = s.elems(), ob = s.tensor_bytes(), lb = s.rowvec_bytes(), db = (size_t)B * H * 4;
+  const void* ins[6] = {q, k, v, q_descale, k_descale, v_descale};
+  const size_t in_bytes[6] = {ib, ib, ib, db, db, db};
+  for (int i = 0; i < 6; ++i)
+    if (overlap(o, ob, ins[i], in_bytes[i]) || overlap(lse, lb, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+  if (overlap(o, ob, lse, lb)) return FA_ERR_INVALID_ARG;
+  int dev, sms;
+  if ((st = device_setup(&dev, &sms))) return st;
+  const float* descales[3] = {q_descale, k_descale, v_descale};
+  return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream),
+                    descales);
+}
+
+}  // extern "C"
+
+namespace {
+
+size_t decode_workspace_bytes(int B, int Sq, int H, int d, int splits) {
+  if (splits <= 1) return 0;
+  const size_t rows = (size_t)B * H * Sq * splits;
+  return align256(rows * d * 4) + align256(rows * 4);
+}
+
+// Splits per (b, h) when the caller passes 0: about four CTAs per SM in total (two fit at a
+// time), never more than the 64-key tiles of the longest possible sequence, at most 128.
+int decode_auto_splits(int B, int H, int max_keys, int sm_count) {
+  const long long bh = (long long)B * H;
+  long long s = (4LL * sm_count + bh - 1) / bh;
+  const long long tiles = (max_keys + fa::kDecTile - 1) / fa::kDecTile;
+  if (s > tiles) s = tiles;
+  if (s > 128) s = 128;
+  return s < 1 ? 1 : (int)s;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits) {
+  if (B < 1 || Sq < 1 || H < 1 || (d != 64 && d != 128) || splits < 0) return 0;
+  return decode_workspace_bytes(B, Sq, H, d, splits);
+}
+
+int fa_decode_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                    const int* seqlens, void* o, float* lse, int B, int Sq, int H, int d, int num_pages,
+                    int page_size, int max_pages, float scale, int causal, int win_l, int win_r, int splits,
+                    void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  if (B < 1 || H < 1 || Sq < 1 || num_pages < 1 || max_pages < 1 || page_size < 1 || splits < 0)
+    return FA_ERR_INVALID_ARG;
+  if (win_l < -1 || win_r < -1 || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Sq > fa::kDecMaxSq || page_size % fa::kDecTile != 0) return FA_ERR_UNSUPPORTED;
+  if ((double)num_pages * page_size * H * d * 2 >= 1099511627776.0 ||
+      (double)max_pages * page_size >= 2147483647.0)
+    return FA_ERR_INVALID_ARG;
+  if (!q || !k_cache || !v_cache || !block_table || !seqlens || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(block_table, 4) || !aligned(seqlens, 4))
+    return FA_ERR_INVALID_ARG;
+  if (causal) win_r = 0;
+  const size_t qb = (size_t)B * Sq * H * d * 2, cb = (size_t)num_pages * page_size * H * d * 2;
+  const size_t lb = (size_t)B * H * Sq * 4, tb = (size_t)B * max_pages * 4, sb = (size_t)B * 4;
+  const void* ins[5] = {q, k_cache, v_cache, block_table, seqlens};
+  const size_t in_bytes[5] = {qb, cb, cb, tb, sb};
+  for (int i = 0; i < 5; ++i)
+    if (overlap(o, qb, ins[i], in_bytes[i]) || overlap(lse, lb, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+  if (overlap(o, qb, lse, lb)) return FA_ERR_INVALID_ARG;
+  int dev, sms, st;
+  if ((st = device_setup(&dev, &sms))) return st;
+  if (splits == 0) splits = decode_auto_splits(B, H, max_pages * page_size, sms);
+  const size_t wbytes = decode_workspace_bytes(B, Sq, H, d, splits);
+  if (wbytes > 0 && workspace) {
+    if (!aligned(workspace, 256) || workspace_bytes_ < wbytes) return FA_ERR_INVALID_ARG;
+    for (int i = 0; i < 5; ++i)
+      if (overlap(workspace, wbytes, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+    if (overlap(workspace, wbytes, o, qb) || overlap(workspace, wbytes, lse, lb)) return FA_ERR_INVALID_ARG;
+  }
+  CUtensorMap mk, mv;
+  if ((st = make_map_cache(&mk, k_cache, num_pages, page_size, H, d)) ||
+      (st = make_map_cache(&mv, v_cache, num_pages, page_size, H, d)))
+    return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (wbytes > 0 && !ws) {
+    if (cudaMallocAsync(&ws, wbytes, cs) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_NO_MEMORY;
+    }
+  }
+  fa::DecParams p;
+  p.B = B;
+  p.Sq = Sq;
+  p.H = H;
+  p.page_size = page_size;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.win_l = win_l;
+  p.win_r = win_r;
+  p.splits = splits;
+  p.block_table = block_table;
+  p.seqlens = seqlens;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.o_part = static_cast<float*>(ws);
+  p.lse_part = wbytes ? reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                                 align256((size_t)B * H * Sq * splits * d * 4))
+                      : nullptr;
+  const dim3 grid(splits, H, B);
+  if (d == 64)
+    fa::fa_decode_split_kernel<64><<<grid, fa::kDecThreads, fa::DecCfg<64>::kSmemBytes, cs>>>(mk, mv, p);
+  else
+    fa::fa_decode_split_kernel<128><<<grid, fa::kDecThreads, fa::DecCfg<128>::kSmemBytes, cs>>>(mk, mv, p);
+  st = launch_status();
+  if (!st && splits > 1) {
+    const dim3 cgrid(Sq, H, B);
+    if (d == 64)
+      fa::fa_decode_combine_kernel<64><<<cgrid, 64, 0, cs>>>(p);
+    else
+      fa::fa_decode_combine_kernel<128><<<cgrid, 128, 0, cs>>>(p);
+    st = launch_status();
+  }
+  if (wbytes > 0 && !workspace && cudaFreeAsync(ws, cs) != cudaSuccess && !st) st = FA_ERR_CUDA;
+  return st;
 }
 
 int fa_bwd_preprocess(const void* o, const float* lse, const void* dO, int B, int N, int H, int d, void* workspace,

@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(512, 1)
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
   // 128-byte swizzled tiles need 1024-byte alignment; the kernel reports instead of faulting.
   if (smem_base & 1023u) {
-    if (threadIdx.x == 0) atomicOr(&g_fa_error, 2);
+    if (threadIdx.x == 0) atomicOr(&g_fa_error, kErrSmemAlign);
     return;
   }
 

@@ -46,6 +46,9 @@ struct FwdParams {
   int num_items;     // B * H * num_pairs
   float* lse;        // (B, H, N) fp32
   int debug_drop_s_signal;  // test only: withhold the first "S ready" signal (a wait must time out)
+  const float* q_descale;   // E4M3 inputs only: (B, H) factors, value = descale * code
+  const float* k_descale;
+  const float* v_descale;
 };
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
@@ -62,16 +65,25 @@ constexpr int kFwdPolyNum = FA_FWD_POLY_NUM, kFwdPolyDen = FA_FWD_POLY_DEN;
 
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D>
+// kF8: Q, K, V are E4M3 (one byte per element), S and P·V run as kind::f8f6f4 with P
+// quantised to E4M3 in TMEM (four per column); O is bf16 as for bf16 inputs.
+template <int D, bool kF8 = false>
 struct FwdCfg {
   static constexpr int kThreads = 384;
-  static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile of Q, K, V or O
-  static constexpr int kBoxes = D / 64;           // 64-column (128-byte) TMA boxes per tile
-  static constexpr int kSlots = (D == 128) ? 4 : 8;
-  static constexpr bool kSepP = (D == 64);        // P apart from S in TMEM; O staging apart from Q
-  static constexpr int kOffQ = 0;                 // Q0, Q1 (also O staging unless kSepP)
-  static constexpr int kOffO = 2 * kTileBytes;    // O staging 0, 1 (kSepP)
-  static constexpr int kOffKV = (kSepP ? 4 : 2) * kTileBytes;
+  static constexpr int kElem = kF8 ? 1 : 2;        // bytes per Q/K/V element
+  static constexpr int kTileBytes = 128 * D * kElem;  // one 128-row tile of Q, K or V
+  static constexpr int kOTileBytes = 128 * D * 2;     // one 128-row bf16 tile of O
+  static constexpr int kBoxes = D * kElem / 128;      // 128-byte-wide TMA boxes per Q/K/V tile
+  static constexpr int kBoxElems = 128 / kElem;       // elements per box row
+  static constexpr int kOBoxes = D / 64;              // 64-column boxes per O tile
+  static constexpr int kSlots = (kTileBytes == 32768) ? 4 : 8;
+  static constexpr bool kSepP = (D == 64 && !kF8);    // P apart from S in TMEM
+  static constexpr bool kSepO = kSepP || kF8;         // O staging apart from Q; Q freed by the last S
+  static constexpr int kKSteps = D * kElem / 32;      // MMA steps over d (32 bytes of K each)
+  static constexpr int kPvSteps = kF8 ? 4 : 8;        // MMA steps over the 128 keys of P
+  static constexpr int kOffQ = 0;                     // Q0, Q1 (also O staging unless kSepO)
+  static constexpr int kOffO = 2 * kTileBytes;        // O staging 0, 1 (kSepO)
+  static constexpr int kOffKV = kSepO ? kOffO + 2 * kOTileBytes : 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
@@ -80,10 +92,10 @@ struct FwdCfg {
 };
 
 // Barrier block at the end of shared memory.
-template <int D>
+template <class Cfg>
 struct FwdBars {
   uint64_t q_full[2], q_empty[2];
-  uint64_t kv_full[FwdCfg<D>::kSlots], kv_empty[FwdCfg<D>::kSlots];
+  uint64_t kv_full[Cfg::kSlots], kv_empty[Cfg::kSlots];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t s_empty[2], pv_done[2];  // kSepP only
   uint64_t mma_done;
@@ -180,22 +192,48 @@ __device__ __forceinline__ void fwd_exp_chunk(const float (&x)[128], int k0, flo
   }
 }
 
+// Same for E4M3 P: 32 columns -> 8 words of four E4M3 values (column 4w + i in byte i). The
+// row sum takes the exponentials before quantisation.
+template <bool kPosScale>
+__device__ __forceinline__ void fwd_exp_chunk_e4m3(const float (&x)[128], int k0, float c, float m_use,
+                                                   uint32_t (&pk)[8], float2& sum) {
+  const float2 neg_m = make_float2(-m_use, -m_use);
+  const float2 c2 = make_float2(c, c);
+#pragma unroll
+  for (int k = 0; k < 16; k += 2) {
+    float2 pv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float2 xv = make_float2(x[2 * (k0 + k + u)], x[2 * (k0 + k + u) + 1]);
+      const float2 a = kPosScale ? fma2(xv, c2, neg_m) : add2(xv, neg_m);
+      if (((k + u) % kFwdPolyDen) < kFwdPolyNum)
+        pv[u] = exp2_poly2(a);
+      else
+        pv[u] = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+      sum = add2(sum, pv[u]);
+    }
+    pk[k >> 1] = pack_e4m3x4(pv[0].x, pv[0].y, pv[1].x, pv[1].y);
+  }
+}
+
 __device__ __forceinline__ float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-template <int D>
+template <int D, bool kF8 = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams p) {
-  using Cfg = FwdCfg<D>;
+  using Cfg = FwdCfg<D, kF8>;
+  using Bars = FwdBars<Cfg>;
+  static_assert(!kF8 || D == 128, "E4M3 inputs: head dim 128 (one 128-byte row per TMA box)");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
-  FwdBars<D>* bars = reinterpret_cast<FwdBars<D>*>(smem_gen + Cfg::kOffBar);
+  Bars* bars = reinterpret_cast<Bars*>(smem_gen + Cfg::kOffBar);
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
 
   const int warp = threadIdx.x >> 5;
@@ -234,8 +272,8 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = bars->tmem_base;
 
   const uint32_t sQ[2] = {smem_base + Cfg::kOffQ, smem_base + Cfg::kOffQ + Cfg::kTileBytes};
-  const uint32_t sO[2] = {Cfg::kSepP ? smem_base + Cfg::kOffO : sQ[0],
-                          Cfg::kSepP ? smem_base + Cfg::kOffO + Cfg::kTileBytes : sQ[1]};
+  const uint32_t sO[2] = {Cfg::kSepO ? smem_base + Cfg::kOffO : sQ[0],
+                          Cfg::kSepO ? smem_base + Cfg::kOffO + Cfg::kOTileBytes : sQ[1]};
   const uint32_t sKV = smem_base + Cfg::kOffKV;
 
   if (warp == 0) {
@@ -262,7 +300,8 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(bar(bars->q_full[t]), Cfg::kTileBytes);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_4d(sQ[t] + bx * 16384, &tmQ, bar(bars->q_full[t]), bx * 64, pair * 256 + t * 128, h, b);
+            tma_load_4d(sQ[t] + bx * 16384, &tmQ, bar(bars->q_full[t]), bx * Cfg::kBoxElems, pair * 256 + t * 128, h,
+                        b);
           ++qn[t];
         }
         for (int j = lo; j <= hi; ++j) {
@@ -272,7 +311,8 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t dst = sKV + slot * Cfg::kTileBytes;
 #pragma unroll
             for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-              tma_load_4d(dst + bx * 16384, kv ? &tmV : &tmK, bar(bars->kv_full[slot]), bx * 64, j * 128, h, b);
+              tma_load_4d(dst + bx * 16384, kv ? &tmV : &tmK, bar(bars->kv_full[slot]), bx * Cfg::kBoxElems, j * 128,
+                          h, b);
             last_slot_parity[slot] = phase;
             if (++slot == Cfg::kSlots) { slot = 0; phase ^= 1; }
           }
@@ -287,8 +327,9 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (elect_one()) {
-      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false, false);  // S = Q K^T, both K-major
-      constexpr uint32_t idO = idesc_bf16_f32(128, D, false, true);     // O += P V, V is MN-major
+      // S = Q K^T (both K-major), O += P V (V MN-major)
+      constexpr uint32_t idS = kF8 ? idesc_e4m3_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idO = kF8 ? idesc_e4m3_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
       const uint32_t tS[2] = {tmem + Cfg::kColS0, tmem + Cfg::kColS1};
       const uint32_t tO[2] = {tmem + Cfg::kColO0, tmem + Cfg::kColO1};
       const uint32_t tP[2] = {tmem + Cfg::kColP0, tmem + Cfg::kColP1};
@@ -299,15 +340,24 @@ __global__ void __launch_bounds__(384, 1)
 
       auto issue_s = [&](int t, uint32_t k_smem) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < Cfg::kKSteps; ++kk) {  // 32 bytes of d per step, 4 steps per 128-byte box
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_ss(tS[t], sdesc_kmajor(sQ[t] + off), sdesc_kmajor(k_smem + off), idS, kk > 0);
+          if constexpr (kF8)
+            mma_ss_f8(tS[t], sdesc_kmajor(sQ[t] + off), sdesc_kmajor(k_smem + off), idS, kk > 0);
+          else
+            mma_ss(tS[t], sdesc_kmajor(sQ[t] + off), sdesc_kmajor(k_smem + off), idS, kk > 0);
         }
       };
       auto issue_pv = [&](int t, uint32_t v_smem, bool accumulate) {
+        // 16 (bf16) or 32 (E4M3) keys per step: 8 TMEM columns of P, as many 128-byte rows of V
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tO[t], tP[t] + kk * 8, sdesc_mnmajor(v_smem + kk * 2048, 16384), idO, accumulate || kk > 0);
+        for (int kk = 0; kk < Cfg::kPvSteps; ++kk) {
+          const uint64_t vd = sdesc_mnmajor(v_smem + kk * (kF8 ? 4096 : 2048), 16384);
+          if constexpr (kF8)
+            mma_ts_f8(tO[t], tP[t] + kk * 8, vd, idO, accumulate || kk > 0);
+          else
+            mma_ts(tO[t], tP[t] + kk * 8, vd, idO, accumulate || kk > 0);
+        }
       };
 
       for (int round = 0;; ++round) {
@@ -390,6 +440,7 @@ __global__ void __launch_bounds__(384, 1)
               issue_s(0, sKV + k_slot * Cfg::kTileBytes);
               if (drop_s_signal) drop_s_signal = false;
               else mma_commit(bar(bars->s_full[0]));
+              if (Cfg::kSepO && j == hi_t[0]) mma_commit(bar(bars->q_empty[0]));  // last read of Q_0
             }
           }
           if (j - 1 >= lo) {
@@ -405,6 +456,7 @@ __global__ void __launch_bounds__(384, 1)
             if (active(1, j)) {
               issue_s(1, sKV + k_slot * Cfg::kTileBytes);
               mma_commit(bar(bars->s_full[1]));
+              if (Cfg::kSepO && j == hi_t[1]) mma_commit(bar(bars->q_empty[1]));  // last read of Q_1
             }
             mma_commit(bar(bars->kv_empty[k_slot]));
             const uint32_t v_slot = slot;
@@ -434,7 +486,6 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = tmem + lane_field + (t ? Cfg::kColS1 : Cfg::kColS0);
     const uint32_t tO = tmem + lane_field + (t ? Cfg::kColO1 : Cfg::kColO0);
     const uint32_t tP = tmem + lane_field + (t ? Cfg::kColP1 : Cfg::kColP0);
-    const float c = p.scale_log2;
     uint32_t sn = 0, on = 0, pvn = 0;
 
     for (int round = 0;; ++round) {
@@ -446,6 +497,12 @@ __global__ void __launch_bounds__(384, 1)
       int lo, hi;
       fwd_kv_range(p, r0, lo, hi);
       if (hi < lo) continue;
+      float c = p.scale_log2, o_mul = 1.0f;  // log2-domain score factor; O factor
+      if constexpr (kF8) {
+        const int bh = b * p.H + h;
+        c *= p.q_descale[bh] * p.k_descale[bh];
+        o_mul = p.v_descale[bh];
+      }
       const int i = r0 + row;
       const int kmin = p.win_l >= 0 ? i - p.win_l : 0;
       const int kmax = p.win_r >= 0 ? min(p.N - 1, i + p.win_r) : p.N - 1;
@@ -485,12 +542,21 @@ __global__ void __launch_bounds__(384, 1)
         float2 sum0 = make_float2(0.0f, 0.0f), sum1 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t pk[16];
-          if (c > 0.0f)
-            fwd_exp_chunk<true>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
-          else
-            fwd_exp_chunk<false>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
-          tmem_st16(tP + q4 * 16, pk);
+          if constexpr (kF8) {
+            uint32_t pk[8];
+            if (c > 0.0f)
+              fwd_exp_chunk_e4m3<true>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
+            else
+              fwd_exp_chunk_e4m3<false>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
+            tmem_st8(tP + q4 * 8, pk);
+          } else {
+            uint32_t pk[16];
+            if (c > 0.0f)
+              fwd_exp_chunk<true>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
+            else
+              fwd_exp_chunk<false>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
+            tmem_st16(tP + q4 * 16, pk);
+          }
         }
         const float2 s01 = add2(sum0, sum1);
         l_run = l_run * alpha + (s01.x + s01.y);
@@ -517,15 +583,16 @@ __global__ void __launch_bounds__(384, 1)
       if constexpr (Cfg::kSepP) {
         mbar_wait(bar(bars->pv_done[t]), pvn & 1, ab);  // the item's last PV_t
         ++pvn;
-        tc_fence_after_sync();
-        if (row == 0) bulk_wait_group_read0();  // the previous store has read the staging tile
-        named_bar_sync(1 + t, 128);
       } else {
         mbar_wait(bar(bars->o_full[t]), on & 1, ab);
         ++on;
-        tc_fence_after_sync();
       }
-      const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+      tc_fence_after_sync();
+      if constexpr (Cfg::kSepO) {
+        if (row == 0) bulk_wait_group_read0();  // the previous store has read the staging tile
+        named_bar_sync(1 + t, 128);
+      }
+      const float inv_l = l_run > 0.0f ? o_mul / l_run : 0.0f;
       const uint32_t stage = sO[t];
 #pragma unroll 1
       for (int cc = 0; cc < D; cc += 32) {
@@ -550,9 +617,9 @@ __global__ void __launch_bounds__(384, 1)
       named_bar_sync(1 + t, 128);
       if (row == 0) {
 #pragma unroll
-        for (int bx = 0; bx < Cfg::kBoxes; ++bx) tma_store_4d(&tmO, stage + bx * 16384, bx * 64, r0, h, b);
+        for (int bx = 0; bx < Cfg::kOBoxes; ++bx) tma_store_4d(&tmO, stage + bx * 16384, bx * 64, r0, h, b);
         bulk_commit_group();
-        if constexpr (!Cfg::kSepP) {  // the Q_t buffer is free again once the store has read it
+        if constexpr (!Cfg::kSepO) {  // the Q_t buffer is free again once the store has read it
           bulk_wait_group_read0();
           mbar_arrive(bar(bars->q_empty[t]));
         }

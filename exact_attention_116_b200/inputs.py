@@ -57,6 +57,93 @@ CONFIGS: dict[str, AttnConfig] = {
 }
 
 
+# The E4M3 forward is measured on the training shape.
+FP8_CONFIGS: dict[str, AttnConfig] = {
+    "train_fwd_fp8": AttnConfig("train_fwd_fp8", 2, 8192, 16, 128, True, seed=106, backward=False,
+                                note="B2 H16 N8192 d128 causal, E4M3 Q/K/V with per-head descales, forward only"),
+}
+
+E4M3_MAX = 448.0
+
+
+def make_fp8_inputs(cfg: AttnConfig, *, seed: int | None = None, shape: tuple[int, int, int, int] | None = None):
+    """Return host (q8, k8, v8) uint8 E4M3 codes (B, N, H, d) and float32 (q_descale, k_descale, v_descale) (B, H).
+
+    Q, K, V are drawn as in ``make_inputs`` (float32 N(0, 1), same generator and order, times
+    ``cfg.qk_mult`` for Q and K); each (b, h) slice gets descale = max|x| / 448 and its codes are
+    torch's round-to-nearest-even float8_e4m3fn conversion of x / descale.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(cfg.seed if seed is None else seed)
+    shp = cfg.shape if shape is None else shape
+    codes, descales = [], []
+    for i in range(3):
+        x = torch.randn(shp, generator=g, dtype=torch.float32)
+        if i < 2 and cfg.qk_mult != 1.0:
+            x.mul_(cfg.qk_mult)
+        amax = x.abs().amax(dim=(1, 3))                      # (B, H)
+        ds = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+        y = (x / ds[:, None, :, None]).clamp_(-E4M3_MAX, E4M3_MAX)
+        codes.append(y.to(torch.float8_e4m3fn).view(torch.uint8).contiguous())
+        descales.append(ds.contiguous())
+    return tuple(codes), tuple(descales)
+
+
+@dataclass(frozen=True)
+class DecodeConfig:
+    """A KV-cache decode workload: B sequences of ragged length, Sq new rows each, paged cache."""
+
+    name: str
+    B: int
+    Sq: int
+    H: int
+    d: int
+    len_lo: int
+    len_hi: int
+    page_size: int
+    causal: bool = True
+    win_l: int = -1
+    win_r: int = -1
+    seed: int = 0
+    spare_pages: int = 3
+    note: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / (self.d ** 0.5)
+
+    @property
+    def max_pages(self) -> int:
+        return (self.len_hi + self.page_size - 1) // self.page_size
+
+
+DECODE_CONFIGS: dict[str, DecodeConfig] = {
+    "decode_paged": DecodeConfig("decode_paged", 8, 1, 16, 128, 4096, 8192, 256, True, seed=107,
+                                 note="B8 H16 d128, 1 new row per sequence, context 4096-8192 keys (uniform), "
+                                      "256-key pages in random order"),
+}
+
+
+def make_decode_inputs(cfg: DecodeConfig, *, seed: int | None = None):
+    """Return host tensors (q, k_cache, v_cache, block_table, seqlens).
+
+    Draw order from ``torch.Generator('cpu').manual_seed(seed)``: q (B, Sq, H, d), the K page
+    pool, the V page pool (each (B * max_pages + spare, page_size, H, d)), all float32 N(0, 1)
+    rounded to bf16; then the lengths, uniform integers in [len_lo, len_hi]; then a random
+    permutation of the pages, sequence b taking entries [b * max_pages, (b + 1) * max_pages).
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(cfg.seed if seed is None else seed)
+    num_pages = cfg.B * cfg.max_pages + cfg.spare_pages
+    q = torch.randn((cfg.B, cfg.Sq, cfg.H, cfg.d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    kc = torch.randn((num_pages, cfg.page_size, cfg.H, cfg.d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn((num_pages, cfg.page_size, cfg.H, cfg.d), generator=g, dtype=torch.float32).to(torch.bfloat16)
+    seqlens = torch.randint(cfg.len_lo, cfg.len_hi + 1, (cfg.B,), generator=g, dtype=torch.int64).to(torch.int32)
+    perm = torch.randperm(num_pages, generator=g)[: cfg.B * cfg.max_pages]
+    block_table = perm.reshape(cfg.B, cfg.max_pages).to(torch.int32).contiguous()
+    return q, kc, vc, block_table, seqlens
+
+
 def make_inputs(cfg: AttnConfig, *, seed: int | None = None, shape: tuple[int, int, int, int] | None = None,
                 qk_mult: float | None = None):
     """Return host bf16 tensors (q, k, v, do), each (B, N, H, d), drawn in that order."""

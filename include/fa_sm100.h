@@ -63,6 +63,59 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            fa_stream_t stream);
 
 /*
+ * FP8 forward ("突破大模型训练瓶颈：Flash-Attention编译优化与内存占用解决方案", 混合精度计算:
+ * FP8 inputs with q_descale / k_descale factors). q, k, v are (B,N,H,d) tensors of E4M3
+ * codes (OCP 8-bit format: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits), one byte
+ * per element, 16-byte aligned; q_descale, k_descale, v_descale are device (B,H) float32
+ * arrays: element x of head (b,h) stands for descale[b*H+h] * decode(x). Computes the same
+ * O = softmax(scale * Q K^T) V and LSE as fa_fwd on those values, masks as fa_fwd; o is
+ * (B,N,H,d) bf16, lse (B,H,N) float32. Q K^T and P V run on the tensor cores in E4M3 with
+ * float32 accumulation; P (the unnormalised probabilities, at most 2^8) is rounded to E4M3
+ * for P V, the row sums use the unrounded values. d must be 128 (FA_ERR_UNSUPPORTED
+ * otherwise). One kernel launch on `stream`; errors as fa_fwd.
+ */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale, const float* k_descale,
+               const float* v_descale, void* o, float* lse,
+               int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
+               fa_stream_t stream);
+
+/*
+ * Bytes of device workspace fa_decode_paged needs with `splits` splits per (b, h): the
+ * float32 partial outputs (B,H,Sq,splits,d) and their log-sum-exps (B,H,Sq,splits), each
+ * region 256-byte aligned; 0 when splits <= 1 (nothing to merge) or for invalid sizes.
+ */
+size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits);
+
+/*
+ * Attention of the newest query rows against a paged KV cache ("FlashAttention技术解析：加速
+ * GPT训练的核心优化" §5, FlashDecoding; "突破大模型训练瓶颈：Flash-Attention编译优化与内存占用
+ * 解决方案", Paged KV Cache: the cache in fixed-size pages listed per sequence by a block table).
+ *   q            (B,Sq,H,d) bf16: the new rows, 1 <= Sq <= 8; row i of sequence b sits at
+ *                position seqlens[b] - Sq + i (the new tokens are already in the cache).
+ *   k_cache,
+ *   v_cache      (num_pages,page_size,H,d) bf16 page pools; page_size a multiple of 64.
+ *   block_table  device (B,max_pages) int32: key j of sequence b is row j % page_size of page
+ *                block_table[b*max_pages + j/page_size].
+ *   seqlens      device (B) int32: keys held by sequence b (0 <= seqlens[b] <= max_pages*page_size).
+ *   o, lse       (B,Sq,H,d) bf16 and (B,H,Sq) float32 natural-log LSE; a row that sees no key
+ *                gets O = 0 and LSE = -inf.
+ * Masks as fa_fwd, taken at each row's position (causal keeps keys j <= position). d is 64 or
+ * 128. `splits` cuts every (b, h)'s keys into that many ranges processed in parallel and then
+ * merged by log-sum-exp; 0 chooses a count from B*H and the SM count. With splits > 1 a
+ * workspace of fa_decode_workspace_bytes(B,Sq,H,d,splits) bytes (256-byte aligned) is used; if
+ * `workspace` is NULL the call allocates it with cudaMallocAsync/cudaFreeAsync on `stream`.
+ * One or two launches on `stream`. Sequence lengths or page indices that are out of range are
+ * not read: the sequence counts as empty (or the page as zeros) and fa_check() returns
+ * FA_ERR_DEVICE. Host-visible errors as fa_fwd; Sq > 8 or a page_size that is not a multiple
+ * of 64 give FA_ERR_UNSUPPORTED.
+ */
+int fa_decode_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
+                    const int* seqlens, void* o, float* lse,
+                    int B, int Sq, int H, int d, int num_pages, int page_size, int max_pages,
+                    float scale, int causal, int win_l, int win_r, int splits,
+                    void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * Bytes of device workspace fa_bwd needs: a float32 dQ accumulator (B,N,H,d), two
  * float32 (B,H,ceil(N/128)*128) row vectors (-LSE*log2(e) and -D, D = rowsum(dO*O)) and a
  * 256-byte block holding the work counter of the main kernel, each region 256-byte

@@ -83,6 +83,22 @@ def test_fwd_rejects_invalid_arguments(lib, kw, expected):
     assert _fwd(lib, **kw) == expected
 
 
+def _fwd8(lib, q=P, k=P + T, v=P + 2 * T, qd=P + 3 * T, kd=P + 3 * T + 4096, vd=P + 3 * T + 8192, o=P + 4 * T,
+          lse=P + 5 * T, B=1, N=128, H=2, d=128, scale=0.1):
+    return lib.fa_fwd_fp8(q, k, v, qd, kd, vd, o, lse, B, N, H, d, ctypes.c_float(scale), 0, -1, -1, None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(d=64), UNSUPPORTED), (dict(d=96), UNSUPPORTED), (dict(qd=0), INVALID), (dict(vd=0), INVALID),
+    (dict(q=P + 8), INVALID), (dict(kd=P + 3 * T + 4098), INVALID), (dict(o=P + 4 * T + 4), INVALID),
+    (dict(o=P + 2 * T), INVALID),        # output aliases v
+    (dict(lse=P + 3 * T), INVALID),      # lse overlaps q_descale
+    (dict(scale=float("nan")), INVALID), (dict(N=0), INVALID),
+])
+def test_fwd_fp8_rejects_invalid_arguments(lib, kw, expected):
+    assert _fwd8(lib, **kw) == expected
+
+
 def _bwd(lib, ws=P + 9 * T, ws_bytes=None, dq=P + 6 * T, dk=P + 7 * T, dv=P + 8 * T, B=1, N=128, H=2, d=64,
          scale=0.125, wl=-1, wr=-1, fn="fa_bwd"):
     if ws_bytes is None:

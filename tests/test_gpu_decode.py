@@ -1,0 +1,99 @@
+"""GPU parity of the paged-KV decode (fa_decode_paged, through the C ABI) against the fp64 oracle.
+
+The kernel computes scores, the online softmax and P·V in fp32 on the CUDA cores from the
+exact bf16 inputs (P is not rounded), so the forward's tolerances apply: per row
+max |ΔO| / max(1, |O_ref|) <= 1e-2 and max |ΔLSE| <= 1e-3. Cases cover ragged lengths (empty,
+shorter than Sq, one key, page and tile boundaries), causal / window / full masks, Sq = 1..8,
+page sizes 64..512, split counts 1, automatic and more splits than tiles, and the full decode
+workload compared row by row.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_116_b200 as fa
+from exact_attention_116_b200.inputs import DECODE_CONFIGS, DecodeConfig, make_decode_inputs
+from oracle import decode_paged_fp64 as oracle_dec
+from parity import assert_fwd_close
+
+pytestmark = pytest.mark.gpu
+
+
+def run(q, kc, vc, table, lens, scale, causal, win, splits):
+    dev = [t.cuda() for t in (q, kc, vc, table, lens)]
+    o, lse = fa.attention_decode_paged(*dev, scale, causal, win, splits)
+    fa.check()
+    return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def check(cfg, lens=None, splits=0, causal=None, win=None, what=""):
+    q, kc, vc, table, seqlens = make_decode_inputs(cfg)
+    if lens is not None:
+        seqlens = torch.tensor(lens, dtype=torch.int32)
+    causal = cfg.causal if causal is None else causal
+    win = (cfg.win_l, cfg.win_r) if win is None else win
+    o, lse = run(q, kc, vc, table, seqlens, cfg.scale, causal, win, splits)
+    o_ref, lse_ref = oracle_dec.decode_forward(q.double().numpy(), kc.double().numpy(), vc.double().numpy(),
+                                               table.numpy(), seqlens.numpy(), cfg.scale, causal, *win)
+    dead = ~np.isfinite(lse_ref)
+    assert np.array_equal(dead, ~np.isfinite(lse)), f"{what}: rows without keys differ"
+    assert (o[dead.transpose(0, 2, 1)] == 0).all() if dead.any() else True
+    live = ~dead
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            rows = np.nonzero(live[b, h])[0]
+            if len(rows):
+                assert_fwd_close(o[b, rows, h], lse[b, h, rows], o_ref[b, rows, h], lse_ref[b, h, rows],
+                                 f"{what} b={b} h={h} len={int(seqlens[b])}")
+
+
+SMALL = DecodeConfig("small", 5, 3, 2, 128, 1, 700, 128, True, seed=61)
+
+
+@pytest.mark.parametrize("splits", [1, 0, 3, 40])
+def test_decode_ragged_lengths_and_splits(splits):
+    # empty, fewer keys than Sq, one key, a full 64-key tile, a full page, past a page boundary
+    check(SMALL, lens=[0, 2, 1, 128, 257], splits=splits, what=f"splits={splits}")
+
+
+@pytest.mark.parametrize("causal,win", [(False, (-1, -1)), (True, (-1, -1)), (False, (100, 5)), (True, (70, -1)),
+                                        (False, (0, 0))])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_masks(causal, win, d):
+    cfg = DecodeConfig("masks", 3, 8, 3, d, 300, 900, 64, causal, seed=62 + d)
+    check(cfg, causal=causal, win=win, splits=0, what=f"d={d} causal={causal} win={win}")
+
+
+@pytest.mark.parametrize("Sq,page", [(1, 64), (4, 512), (8, 192)])
+def test_decode_rows_and_page_sizes(Sq, page):
+    cfg = DecodeConfig("pages", 4, Sq, 4, 128, 1, 1500, page, True, seed=63 + Sq)
+    check(cfg, splits=0, what=f"Sq={Sq} page={page}")
+
+
+def test_decode_split_counts_agree():
+    cfg = DecodeConfig("splits", 2, 2, 2, 64, 2000, 3000, 256, True, seed=64)
+    q, kc, vc, table, lens = make_decode_inputs(cfg)
+    outs = [run(q, kc, vc, table, lens, cfg.scale, True, (-1, -1), s) for s in (1, 2, 5, 0)]
+    for o, lse in outs[1:]:
+        assert np.abs(o - outs[0][0]).max() < 1e-2 and np.abs(lse - outs[0][1]).max() < 1e-4
+
+
+def test_decode_workload_all_rows():
+    cfg = DECODE_CONFIGS["decode_paged"]
+    check(cfg, splits=0, what="decode_paged")
+
+
+def test_decode_out_of_range_length_is_reported_not_read():
+    cfg = DecodeConfig("bad", 2, 1, 2, 128, 100, 200, 64, True, seed=65)
+    q, kc, vc, table, lens = make_decode_inputs(cfg)
+    bad = torch.tensor([int(lens[0]), cfg.max_pages * cfg.page_size + 1], dtype=torch.int32)
+    dev = [t.cuda() for t in (q, kc, vc, table, bad)]
+    o, lse = fa.attention_decode_paged(*dev, cfg.scale, True, (-1, -1), 1)
+    with pytest.raises(fa.FaError) as e:
+        fa.check()
+    assert e.value.status == 6  # FA_ERR_DEVICE
+    assert torch.isinf(lse[1]).all() and (o[1] == 0).all()  # the bad sequence counts as empty
+    fa.check()  # the error word was cleared; the context is usable
