@@ -23,6 +23,9 @@ Readings taken where the pages are silent (also listed with the design notes):
   query row i sits at position ``pos = seqlens[b] - Sq + i``.
 * Masks are those of the training path, taken at ``pos``: causal keeps keys j <= pos; a
   (left, right) window keeps pos - left <= j <= pos + right (inclusive, -1 unbounded).
+* New rows' keys and values, when given (``k_new``, ``v_new``: (B, Sq, H, d)), are written
+  into the cache at those positions first, as ``flash_attn_with_kvcache`` updates its cache
+  in place; rows whose position is negative (a sequence shorter than Sq) are not placed.
 * Otherwise the plain definition: O = softmax(scale * q . k) V over the visible keys, and
   LSE the natural-log log-sum-exp of the scaled scores (a row without keys: O = 0,
   LSE = -inf).
@@ -46,11 +49,28 @@ def gather_sequence(cache, block_table, b: int, seqlen: int, page_size: int) -> 
     return np.asarray(rows, dtype=np.float64).reshape(seqlen, *cache.shape[2:])
 
 
-def decode_forward(q, k_cache, v_cache, block_table, seqlens, scale, causal=False, win_l=-1, win_r=-1):
+def append_rows(cache, rows, block_table, seqlens, page_size):
+    """A copy of the cache with rows[b, i] placed at position seqlens[b] - Sq + i of sequence b."""
+    out = np.array(cache, dtype=np.float64, copy=True)
+    rows = np.asarray(rows, dtype=np.float64)
+    Sq = rows.shape[1]
+    for b in range(rows.shape[0]):
+        for i in range(Sq):
+            pos = int(seqlens[b]) - Sq + i
+            if pos >= 0:
+                out[int(block_table[b, pos // page_size]), pos % page_size] = rows[b, i]
+    return out
+
+
+def decode_forward(q, k_cache, v_cache, block_table, seqlens, scale, causal=False, win_l=-1, win_r=-1, k_new=None,
+                   v_new=None):
     """(O, LSE) of the new query rows of every sequence against its cached keys and values."""
     q = np.asarray(q, dtype=np.float64)
     B, Sq, H, d = q.shape
     page_size = np.asarray(k_cache).shape[1]
+    if k_new is not None:
+        k_cache = append_rows(k_cache, k_new, block_table, seqlens, page_size)
+        v_cache = append_rows(v_cache, v_new, block_table, seqlens, page_size)
     o = np.zeros((B, Sq, H, d))
     lse = np.full((B, H, Sq), -np.inf)
     for b in range(B):

@@ -134,7 +134,39 @@ def pin_empty_and_short_sequences(impl):
     assert abs(lse[1, 0, 1] - 0.5 * float(q[1, 1, 0] @ ks[1][0, 0])) < 1e-12
 
 
-DECODE_PINS = [pin_window_counts, pin_matches_training_path, pin_page_placement, pin_empty_and_short_sequences]
+def pin_append_new_rows(impl):
+    """Appending the new tokens' rows gives the training-path result of the sequences that end
+    with them; appending the rows the cache already holds changes nothing."""
+    rng = np.random.default_rng(55)
+    H, d, Sq = 2, 4, 3
+    lens = [11, 6]
+    qs = [rng.standard_normal((n, H, d)) for n in lens]
+    ks = [rng.standard_normal((n, H, d)) for n in lens]
+    vs = [rng.standard_normal((n, H, d)) for n in lens]
+    junk_k = [x.copy() for x in ks]
+    junk_v = [x.copy() for x in vs]
+    for x in junk_k + junk_v:
+        x[-Sq:] = 1e3  # the cache does not yet hold the new rows
+    kc, table = paged(np.random.default_rng(8), junk_k, 4)
+    vc, _ = paged(np.random.default_rng(8), junk_v, 4)
+    q = np.stack([x[-Sq:] for x in qs])
+    k_new = np.stack([x[-Sq:] for x in ks])
+    v_new = np.stack([x[-Sq:] for x in vs])
+    for causal, wl, wr in MASKS:
+        o, lse = impl.decode_forward(q, kc, vc, table, lens, 0.3, causal, wl, wr, k_new=k_new, v_new=v_new)
+        for b, n in enumerate(lens):
+            o_ref, lse_ref = attention_fp64.attention_forward(qs[b][None], ks[b][None], vs[b][None], 0.3, causal, wl, wr)
+            assert np.allclose(o[b], o_ref[0, n - Sq:], atol=1e-12, rtol=0), (causal, wl, wr, b)
+            assert np.allclose(lse[b], lse_ref[0][:, n - Sq:], atol=1e-12, rtol=0)
+    kc2, _ = paged(np.random.default_rng(8), ks, 4)
+    vc2, _ = paged(np.random.default_rng(8), vs, 4)
+    a = impl.decode_forward(q, kc2, vc2, table, lens, 0.3, True)
+    b_ = impl.decode_forward(q, kc2, vc2, table, lens, 0.3, True, k_new=k_new, v_new=v_new)
+    assert np.array_equal(a[0], b_[0]) and np.array_equal(a[1], b_[1])
+
+
+DECODE_PINS = [pin_window_counts, pin_matches_training_path, pin_page_placement, pin_empty_and_short_sequences,
+               pin_append_new_rows]
 
 
 @pytest.mark.parametrize("pin", DECODE_PINS, ids=lambda f: f.__name__)
@@ -150,6 +182,9 @@ MUTANTS = {
     "block_table_ignored": ("cache[int(block_table[b, j // page_size]), j % page_size]",
                             "cache[j // page_size, j % page_size]"),
     "seqlen_ignored": ("n = int(seqlens[b])", "n = int(np.max(seqlens))"),
+    "append_shifted": ("pos = int(seqlens[b]) - Sq + i\n", "pos = int(seqlens[b]) - Sq + i + 1\n"),
+    "append_page_row_swapped": ("out[int(block_table[b, pos // page_size]), pos % page_size] = rows[b, i]",
+                                "out[int(block_table[b, pos % page_size]), pos // page_size] = rows[b, i]"),
     "scale_dropped": ("s = np.where(vis, scale * (q[b, :, h] @ k[:, h].T), -np.inf)",
                       "s = np.where(vis, (q[b, :, h] @ k[:, h].T), -np.inf)"),
 }
