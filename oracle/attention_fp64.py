@@ -27,6 +27,10 @@ Readings taken where the pages are silent (each is also listed with the design n
   always visible) gets O = 0 and LSE = -inf.
 * Backward is the exact derivative of L = sum(dO * O) with respect to Q, K, V;
   there is no upstream gradient into LSE.
+* ALiBi (the call's ``alibi_slopes``, "FlashAttention技术解析" §2.2, which passes None for
+  "no positional bias"): with a slope m for the head, the score of query i and key j gets
+  -m * |i - j| added after scaling, before the mask and the softmax. The slopes are
+  constants of the call (no gradient); the backward uses the biased P.
 
 Layout: q, k, v, dO are (B, N, H, d) arrays (any float dtype; they are widened to
 float64 exactly). LSE and D are (B, H, N).
@@ -70,9 +74,12 @@ def visible_key_span(r0: int, r1: int, n_keys: int, causal: bool, win_l: int, wi
 
 
 def _head_scores(q: np.ndarray, k: np.ndarray, rows: np.ndarray, cols: slice,
-                 scale: float, causal: bool, win_l: int, win_r: int) -> np.ndarray:
-    """Scaled, masked scores S[r, c] = scale * q[rows[r]] . k[c] for keys in cols."""
+                 scale: float, causal: bool, win_l: int, win_r: int, alibi: float = 0.0) -> np.ndarray:
+    """Scaled, masked scores S[r, c] = scale * q[rows[r]] . k[c] - alibi * |rows[r] - c| for keys in cols."""
     s = scale * (q[rows] @ k[cols].T)
+    if alibi != 0.0:
+        keys = np.arange(k.shape[0], dtype=np.int64)[cols]
+        s = s - alibi * np.abs(np.asarray(rows, dtype=np.int64)[:, None] - keys[None, :])
     vis = visible_mask(rows, k.shape[0], causal, win_l, win_r)[:, cols]
     return np.where(vis, s, NEG_INF)
 
@@ -100,7 +107,7 @@ def _row_blocks(n: int, block_rows: int | None):
         yield r0, min(n, r0 + step)
 
 
-def head_forward(q, k, v, scale, causal=False, win_l=-1, win_r=-1, block_rows=None):
+def head_forward(q, k, v, scale, causal=False, win_l=-1, win_r=-1, block_rows=None, alibi=0.0):
     """Forward for one (b, h): q, k, v are (N, d) float64. Returns (O (N,d), LSE (N,)).
 
     ``block_rows`` only bounds memory: each block holds complete score rows, so
@@ -112,20 +119,20 @@ def head_forward(q, k, v, scale, causal=False, win_l=-1, win_r=-1, block_rows=No
     for r0, r1 in _row_blocks(n, block_rows):
         c0, c1 = visible_key_span(r0, r1, k.shape[0], causal, win_l, win_r)
         rows = np.arange(r0, r1)
-        s = _head_scores(q, k, rows, slice(c0, c1), scale, causal, win_l, win_r)
+        s = _head_scores(q, k, rows, slice(c0, c1), scale, causal, win_l, win_r, alibi)
         p, lse[r0:r1] = _softmax_rows(s)
         o[r0:r1] = p @ v[c0:c1]
     return o, lse
 
 
-def head_probs(q, k, scale, causal=False, win_l=-1, win_r=-1):
+def head_probs(q, k, scale, causal=False, win_l=-1, win_r=-1, alibi=0.0):
     """Full softmax matrix P (N, N) of one head (small N only; used by the pins)."""
     n = q.shape[0]
-    s = _head_scores(q, k, np.arange(n), slice(0, k.shape[0]), scale, causal, win_l, win_r)
+    s = _head_scores(q, k, np.arange(n), slice(0, k.shape[0]), scale, causal, win_l, win_r, alibi)
     return _softmax_rows(s)[0]
 
 
-def head_backward(q, k, v, do, scale, causal=False, win_l=-1, win_r=-1, block_rows=None):
+def head_backward(q, k, v, do, scale, causal=False, win_l=-1, win_r=-1, block_rows=None, alibi=0.0):
     """Gradients of L = sum(dO * O) for one head. Returns (dQ, dK, dV, D).
 
     With P the softmax matrix of the forward:
@@ -140,17 +147,17 @@ def head_backward(q, k, v, do, scale, causal=False, win_l=-1, win_r=-1, block_ro
     dv = np.zeros_like(v, dtype=np.float64)
     dvec = np.zeros(n, dtype=np.float64)
     for r0, r1 in _row_blocks(n, block_rows):
-        backward_rows(q, k, v, do, r0, r1, scale, causal, win_l, win_r, dq, dk, dv, dvec)
+        backward_rows(q, k, v, do, r0, r1, scale, causal, win_l, win_r, dq, dk, dv, dvec, alibi)
     return dq, dk, dv, dvec
 
 
-def backward_rows(q, k, v, do, r0, r1, scale, causal, win_l, win_r, dq, dk, dv, dvec):
+def backward_rows(q, k, v, do, r0, r1, scale, causal, win_l, win_r, dq, dk, dv, dvec, alibi=0.0):
     """Contribution of query rows [r0, r1) of one head to the gradients (added into dk, dv;
     dq and dvec rows [r0, r1) written). Summing it over a partition of the rows gives the
     whole backward."""
     c0, c1 = visible_key_span(r0, r1, k.shape[0], causal, win_l, win_r)
     rows = np.arange(r0, r1)
-    s = _head_scores(q, k, rows, slice(c0, c1), scale, causal, win_l, win_r)
+    s = _head_scores(q, k, rows, slice(c0, c1), scale, causal, win_l, win_r, alibi)
     p, _ = _softmax_rows(s)
     g = do[r0:r1]
     dv[c0:c1] += p.T @ g
@@ -166,10 +173,16 @@ def _as_f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def attention_forward(q, k, v, scale, causal=False, win_l=-1, win_r=-1, heads=None, block_rows=None):
+def _slope(alibi_slopes, b: int, h: int) -> float:
+    return 0.0 if alibi_slopes is None else float(np.asarray(alibi_slopes, dtype=np.float64)[b, h])
+
+
+def attention_forward(q, k, v, scale, causal=False, win_l=-1, win_r=-1, heads=None, block_rows=None,
+                      alibi_slopes=None):
     """Forward over (B, N, H, d) inputs. Returns O (B,N,H,d) and LSE (B,H,N), float64.
 
     ``heads``: optional list of (b, h) pairs; heads not listed are left as NaN.
+    ``alibi_slopes``: optional (B, H) slopes (ALiBi bias -m * |i - j|).
     """
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
     b_, n, h_, d = q.shape
@@ -177,11 +190,12 @@ def attention_forward(q, k, v, scale, causal=False, win_l=-1, win_r=-1, heads=No
     lse = np.full((b_, h_, n), np.nan)
     for b, h in (heads if heads is not None else [(b, h) for b in range(b_) for h in range(h_)]):
         o[b, :, h, :], lse[b, h, :] = head_forward(q[b, :, h], k[b, :, h], v[b, :, h], scale,
-                                                   causal, win_l, win_r, block_rows)
+                                                   causal, win_l, win_r, block_rows, _slope(alibi_slopes, b, h))
     return o, lse
 
 
-def attention_backward(q, k, v, do, scale, causal=False, win_l=-1, win_r=-1, heads=None, block_rows=None):
+def attention_backward(q, k, v, do, scale, causal=False, win_l=-1, win_r=-1, heads=None, block_rows=None,
+                       alibi_slopes=None):
     """Backward over (B, N, H, d) inputs. Returns dQ, dK, dV (B,N,H,d) and D (B,H,N), float64."""
     q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(do)
     b_, n, h_, d = q.shape
@@ -191,18 +205,18 @@ def attention_backward(q, k, v, do, scale, causal=False, win_l=-1, win_r=-1, hea
     dvec = np.full((b_, h_, n), np.nan)
     for b, h in (heads if heads is not None else [(b, h) for b in range(b_) for h in range(h_)]):
         g = head_backward(q[b, :, h], k[b, :, h], v[b, :, h], do[b, :, h], scale,
-                          causal, win_l, win_r, block_rows)
+                          causal, win_l, win_r, block_rows, _slope(alibi_slopes, b, h))
         dq[b, :, h], dk[b, :, h], dv[b, :, h], dvec[b, h] = g
     return dq, dk, dv, dvec
 
 
-def forward_rows(q, k, v, b, h, rows, scale, causal=False, win_l=-1, win_r=-1):
+def forward_rows(q, k, v, b, h, rows, scale, causal=False, win_l=-1, win_r=-1, alibi_slopes=None):
     """O and LSE of selected query rows of one head, each computed on its own.
 
     Used to check sampled outputs at sizes where a whole head is too costly.
     """
     q, k, v = _as_f64(q[b, :, h]), _as_f64(k[b, :, h]), _as_f64(v[b, :, h])
     rows = np.asarray(rows, dtype=np.int64)
-    s = _head_scores(q, k, rows, slice(0, k.shape[0]), scale, causal, win_l, win_r)
+    s = _head_scores(q, k, rows, slice(0, k.shape[0]), scale, causal, win_l, win_r, _slope(alibi_slopes, b, h))
     p, lse = _softmax_rows(s)
     return p @ v, lse
