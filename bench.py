@@ -256,8 +256,24 @@ def oracle_sample_decode(cfg, seconds: float, inputs):
     return done_bytes / dt / 1e9, dt, seqs, threads
 
 
+def decode_new_rows(cfg, host):
+    """The new tokens' K and V rows of a decode step: the rows the cache holds at positions
+    len_b - Sq + i (so that writing them back leaves the cache as generated)."""
+    q, kc, vc, table, lens = host
+    k_new = torch.empty_like(q)
+    v_new = torch.empty_like(q)
+    for b in range(cfg.B):
+        for i in range(cfg.Sq):
+            pos = int(lens[b]) - cfg.Sq + i
+            page = int(table[b, pos // cfg.page_size])
+            k_new[b, i] = kc[page, pos % cfg.page_size]
+            v_new[b, i] = vc[page, pos % cfg.page_size]
+    return k_new, v_new
+
+
 def run_gpu_decode(args):
-    """Paged-KV decode: one step = one fa_decode_paged call over all sequences."""
+    """Paged-KV decode: one step = one fa_decode_paged call over all sequences, which writes the
+    new tokens' K/V rows into the resident cache and attends the new rows to the whole cache."""
     info = mg.rank_info()
     world, rank, local = info.world, info.rank, info.local_rank
     torch.cuda.set_device(local)
@@ -266,19 +282,21 @@ def run_gpu_decode(args):
     host = make_decode_inputs(cfg)
     dev = torch.device("cuda", torch.cuda.current_device())
     q, kc, vc, table, lens = (x.to(dev) for x in host)
+    kn_h, vn_h = decode_new_rows(cfg, host)
+    k_new, v_new = kn_h.to(dev), vn_h.to(dev)
     B, Sq, H, d = q.shape
     o = torch.empty_like(q)
     lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
-    splits = int(args.splits)
+    splits = int(args.splits) or binding.decode_splits(B, H, cfg.max_pages * cfg.page_size)
     stream = torch.cuda.current_stream()
-    # the splits the library picks for splits=0 need this workspace at most (128 splits)
-    ws = torch.empty(max(1, binding.decode_workspace_bytes(B, Sq, H, d, 128)), dtype=torch.uint8, device=dev)
+    # workspace of the split count in use (the library's choice unless --splits is given)
+    ws = torch.empty(max(1, binding.decode_workspace_bytes(B, Sq, H, d, splits)), dtype=torch.uint8, device=dev)
     # L2 flush between steps: the cache is 2x268 MiB > L2 already, q/O are tiny
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     def step():
         binding.decode_paged_into(q, kc, vc, table, lens, o, lse, cfg.scale, cfg.causal, (cfg.win_l, cfg.win_r),
-                                  splits, ws)
+                                  splits, ws, k_new=k_new, v_new=v_new)
 
     for _ in range(args.warmup):
         step()
@@ -306,12 +324,15 @@ def run_gpu_decode(args):
     nbytes = decode_cache_bytes(cfg, host[4])
     gbs = nbytes / (ms_step * 1e-3) / 1e9
 
-    pin = [x.pin_memory() for x in host]
+    # a step's host inputs: the new rows' q, K, V, the block table and the lengths (the cache is
+    # device-resident state, as in a serving loop)
+    step_inputs = (host[0], kn_h, vn_h, host[3], host[4])
+    pin = [x.pin_memory() for x in step_inputs]
     o_h = torch.empty_like(host[0]).pin_memory()
     lse_h = torch.empty((B, H, Sq), dtype=torch.float32).pin_memory()
 
     def e2e_step():
-        for src, dst in zip(pin, (q, kc, vc, table, lens)):
+        for src, dst in zip(pin, (q, k_new, v_new, table, lens)):
             dst.copy_(src, non_blocking=True)
         step()
         o_h.copy_(o, non_blocking=True)
@@ -331,7 +352,7 @@ def run_gpu_decode(args):
     mg.barrier(info)
     binding.check()
     e2e_ms = mg.max_over_ranks(info, e0.elapsed_time(e1), dev) / e2e_steps
-    h2d = sum(x.numel() * x.element_size() for x in host)
+    h2d = sum(x.numel() * x.element_size() for x in step_inputs)
 
     peak, peak_src = peaks()
     res = {
@@ -339,9 +360,10 @@ def run_gpu_decode(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 cache, uniform ragged lengths, random page order)",
-        "config": {"workload": f"{cfg.name}: {cfg.note}", "B": B, "Sq": Sq, "H": H, "d": d,
+        "config": {"workload": f"{cfg.name}: {cfg.note}; a step appends the new rows' K/V and attends",
+                   "B": B, "Sq": Sq, "H": H, "d": d,
                    "page_size": cfg.page_size, "lengths": [int(x) for x in host[4]], "causal": cfg.causal,
-                   "splits": splits if splits else "auto", "seed": cfg.seed,
+                   "splits": splits, "seed": cfg.seed,
                    "l2": "L2 flushed (512 MiB write) before every timed step; KV cache > L2",
                    "bytes": "K and V rows of every visible key + q, O, LSE"},
         "roofline": {"kernel": "fa_decode_split_kernel<128> + combine", "bound": "hbm", "achieved": round(gbs, 1),
@@ -351,7 +373,7 @@ def run_gpu_decode(args):
         "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (3 if splits > 1 else 2) * args.steps,  # append, split kernel, merge
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -19,7 +19,8 @@ LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
                 4: "FA_ERR_TIMEOUT", 5: "FA_ERR_NO_MEMORY", 6: "FA_ERR_DEVICE"}
-EXPORTS = ("fa_fwd", "fa_fwd_fp8", "fa_decode_workspace_bytes", "fa_decode_paged", "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess",
+EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_decode_splits", "fa_decode_workspace_bytes", "fa_decode_paged",
+           "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_ex", "fa_bwd_deterministic", "fa_bwd_preprocess",
            "fa_bwd_main", "fa_bwd_dq_convert", "fa_bwd_static_workspace", "fa_check", "fa_status_string")
 
 _lib = None
@@ -42,9 +43,14 @@ def load() -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
     lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, i, vp, sz, vp]
+    lib.fa_decode_splits.argtypes = [i, i, i]
+    lib.fa_decode_splits.restype = i
     lib.fa_decode_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.fa_decode_workspace_bytes.restype = sz
-    lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, i, vp, sz, vp]
+    lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i, i, vp, sz,
+                                    vp]
     lib.fa_bwd_workspace_bytes.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_bytes.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp, sz, vp]
@@ -55,7 +61,7 @@ def load() -> ctypes.CDLL:
     lib.fa_check.argtypes = [vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
-    for name in ("fa_fwd", "fa_fwd_fp8", "fa_decode_paged", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
+    for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_fp8", "fa_decode_paged", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
                  "fa_check"):
         getattr(lib, name).restype = i
     _lib = lib
@@ -98,22 +104,40 @@ def _scale(scale: float | None, d: int) -> float:
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
 
-def fwd_into(q, k, v, o, lse, scale=None, causal=False, window=(-1, -1), stream=None) -> None:
-    """fa_fwd into caller-provided o (B,N,H,d) bf16 and lse (B,H,N) fp32."""
+def _check_slopes(alibi_slopes, B: int, H: int):
+    if alibi_slopes is None:
+        return None
+    t = alibi_slopes
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != (B, H):
+        raise ValueError("alibi_slopes must be a contiguous (B, H) float32 CUDA tensor")
+    return t.data_ptr()
+
+
+def fwd_into(q, k, v, o, lse, scale=None, causal=False, window=(-1, -1), stream=None, alibi_slopes=None) -> None:
+    """fa_fwd (fa_fwd_ex with ALiBi slopes) into caller-provided o (B,N,H,d) bf16 and lse (B,H,N) fp32."""
     B, N, H, d = _check_qkv(q, k, v, o)
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous() or not lse.is_cuda:
         raise ValueError("lse must be a contiguous (B, H, N) float32 CUDA tensor")
-    st = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, N, H, d,
-                       _scale(scale, d), int(bool(causal)), int(window[0]), int(window[1]), _stream_handle(stream))
-    _raise(st, "fa_fwd")
+    slopes = _check_slopes(alibi_slopes, B, H)
+    if slopes is None:
+        st = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, N, H, d,
+                           _scale(scale, d), int(bool(causal)), int(window[0]), int(window[1]),
+                           _stream_handle(stream))
+        _raise(st, "fa_fwd")
+    else:
+        st = load().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), slopes, o.data_ptr(), lse.data_ptr(), B, N,
+                              H, d, _scale(scale, d), int(bool(causal)), int(window[0]), int(window[1]),
+                              _stream_handle(stream))
+        _raise(st, "fa_fwd_ex")
 
 
-def attention_fwd(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None):
-    """Forward: returns (o, lse) with o (B,N,H,d) bf16 and lse (B,H,N) fp32 (natural log)."""
+def attention_fwd(q, k, v, scale=None, causal=False, window=(-1, -1), stream=None, alibi_slopes=None):
+    """Forward: returns (o, lse) with o (B,N,H,d) bf16 and lse (B,H,N) fp32 (natural log).
+    ``alibi_slopes``: optional (B, H) float32 CUDA tensor (bias -m |i - j|)."""
     B, N, H, d = _check_qkv(q, k, v)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    fwd_into(q, k, v, o, lse, scale, causal, window, stream)
+    fwd_into(q, k, v, o, lse, scale, causal, window, stream, alibi_slopes)
     return o, lse
 
 
@@ -157,12 +181,20 @@ def workspace_bytes(B: int, N: int, H: int, d: int) -> int:
 
 
 def bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale=None, causal=False, window=(-1, -1), workspace=None,
-             stream=None, deterministic=False) -> None:
-    """fa_bwd (or fa_bwd_deterministic) into caller-provided dq, dk, dv.
+             stream=None, deterministic=False, alibi_slopes=None) -> None:
+    """fa_bwd (or fa_bwd_deterministic; fa_bwd_ex with ALiBi slopes) into caller-provided dq, dk, dv.
     ``workspace``: uint8 CUDA tensor or None."""
     B, N, H, d = _check_qkv(q, k, v, o, do, dq, dk, dv)
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
     lib = load()
+    slopes = _check_slopes(alibi_slopes, B, H)
+    if slopes is not None:
+        st = lib.fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                           slopes, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, d, _scale(scale, d),
+                           int(bool(causal)), int(window[0]), int(window[1]), int(bool(deterministic)), ws_ptr,
+                           ws_bytes, _stream_handle(stream))
+        _raise(st, "fa_bwd_ex")
+        return
     fn, name = (lib.fa_bwd_deterministic, "fa_bwd_deterministic") if deterministic else (lib.fa_bwd, "fa_bwd")
     st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(), dq.data_ptr(),
             dk.data_ptr(), dv.data_ptr(), B, N, H, d, _scale(scale, d), int(bool(causal)), int(window[0]),
@@ -171,11 +203,11 @@ def bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale=None, causal=False, window=(
 
 
 def attention_bwd(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1), workspace=None, stream=None,
-                  deterministic=False):
+                  deterministic=False, alibi_slopes=None):
     """Backward: returns (dq, dk, dv), the gradients of sum(do * o). With deterministic=True the
     result is bitwise reproducible (dQ accumulated per query tile in a fixed order)."""
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale, causal, window, workspace, stream, deterministic)
+    bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale, causal, window, workspace, stream, deterministic, alibi_slopes)
     return dq, dk, dv
 
 
@@ -253,10 +285,15 @@ def flash_attention(q, k, v, scale=None, causal=False, window=(-1, -1)):
 
 
 def decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale=None, causal=False, window=(-1, -1),
-                      splits=0, workspace=None, stream=None) -> None:
+                      splits=0, workspace=None, stream=None, k_new=None, v_new=None) -> None:
     """fa_decode_paged: q (B,Sq,H,d) bf16 new rows; k_cache, v_cache (num_pages,page_size,H,d) bf16;
-    block_table (B,max_pages) int32; seqlens (B,) int32; into o (B,Sq,H,d) bf16, lse (B,H,Sq) float32."""
+    block_table (B,max_pages) int32; seqlens (B,) int32; into o (B,Sq,H,d) bf16, lse (B,H,Sq) float32.
+    k_new, v_new: optional (B,Sq,H,d) bf16 rows written into the caches first (in place)."""
     B, Sq, H, d = _check_qkv(q, o)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("give both k_new and v_new, or neither")
+    if k_new is not None:
+        _check_qkv(q, k_new, v_new)
     _check_qkv(k_cache, v_cache)
     num_pages, page_size, Hc, dc = k_cache.shape
     if (Hc, dc) != (H, d):
@@ -269,11 +306,20 @@ def decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale=N
     if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Sq) or not lse.is_contiguous() or not lse.is_cuda:
         raise ValueError("lse must be a contiguous (B, H, Sq) float32 CUDA tensor")
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
-    st = load().fa_decode_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+    kn, vn = (None, None) if k_new is None else (k_new.data_ptr(), v_new.data_ptr())
+    st = load().fa_decode_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), kn, vn, block_table.data_ptr(),
                                 seqlens.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Sq, H, d, num_pages, page_size,
                                 int(block_table.shape[1]), _scale(scale, d), int(bool(causal)), int(window[0]),
                                 int(window[1]), int(splits), ws_ptr, ws_bytes, _stream_handle(stream))
     _raise(st, "fa_decode_paged")
+
+
+def decode_splits(B: int, H: int, max_keys: int) -> int:
+    """The split count fa_decode_paged picks for splits=0 on the current device."""
+    n = int(load().fa_decode_splits(B, H, max_keys))
+    if n < 0:
+        _raise(-n, "fa_decode_splits")
+    return n
 
 
 def decode_workspace_bytes(B: int, Sq: int, H: int, d: int, splits: int) -> int:
@@ -281,10 +327,12 @@ def decode_workspace_bytes(B: int, Sq: int, H: int, d: int, splits: int) -> int:
 
 
 def attention_decode_paged(q, k_cache, v_cache, block_table, seqlens, scale=None, causal=False, window=(-1, -1),
-                           splits=0, stream=None):
-    """Paged-KV decode: returns (o, lse), o (B,Sq,H,d) bf16 and lse (B,H,Sq) float32."""
+                           splits=0, stream=None, k_new=None, v_new=None):
+    """Paged-KV decode: returns (o, lse), o (B,Sq,H,d) bf16 and lse (B,H,Sq) float32. With k_new, v_new the
+    new rows are first written into the caches (in place) at positions seqlens[b] - Sq + i."""
     B, Sq, H, d = q.shape
     o = torch.empty_like(q)
     lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
-    decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale, causal, window, splits, None, stream)
+    decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale, causal, window, splits, None, stream,
+                      k_new, v_new)
     return o, lse

@@ -53,6 +53,31 @@ bool log_enabled() {
 }
 
 // Per-device set-up: SM count, sm_100 check, dynamic shared memory opt-in of every kernel.
+template <int D>
+bool bwd_attributes() {
+  const int smem = fa::BwdCfg<D>::kSmemBytes, smem_dq = fa::BwdDqCfg<D>::kSmemBytes;
+  const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  return cudaFuncSetAttribute(fa::fa_bwd_kernel<D, true, false>, attr, smem) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_bwd_kernel<D, false, false>, attr, smem) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_bwd_kernel<D, true, true>, attr, smem) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_bwd_kernel<D, false, true>, attr, smem) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<D, false>, attr, smem_dq) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<D, true>, attr, smem_dq) == cudaSuccess;
+}
+
+template <int D>
+bool decode_attributes() {
+  const int smem = fa::DecCfg<D>::kSmemBytes;
+  return cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+             cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+             cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+             cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
+             cudaSuccess;
+}
+
 int device_setup(int* dev_out, int* sm_count) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
@@ -72,22 +97,12 @@ int device_setup(int* dev_out, int* sm_count) {
                                fa::FwdCfg<128>::kSmemBytes) != cudaSuccess ||
           cudaFuncSetAttribute(fa::fa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fa::FwdCfg<128, true>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_decode_split_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::DecCfg<64>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_decode_split_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::DecCfg<128>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_bwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdCfg<64>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_bwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdCfg<128>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_bwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdCfg<64>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_bwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdCfg<128>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdDqCfg<64>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::BwdDqCfg<128>::kSmemBytes) != cudaSuccess)
+          !decode_attributes<64>() || !decode_attributes<128>() ||
+          cudaFuncSetAttribute(fa::fa_fwd_kernel<64, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::FwdCfg<64>::kSmemBytes) != cudaSuccess ||
+          cudaFuncSetAttribute(fa::fa_fwd_kernel<128, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fa::FwdCfg<128>::kSmemBytes) != cudaSuccess ||
+          !bwd_attributes<64>() || !bwd_attributes<128>())
         return FA_ERR_CUDA;
     }
     g_attr_done[dev] = true;
@@ -221,9 +236,10 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_
 // ---------------------------------------------------------------- launches (arguments already checked)
 
 // descales != nullptr: q, k, v hold E4M3 codes (head dim 128) with (B, H) descale factors.
+// alibi != nullptr: (B, H) ALiBi slopes (bf16 inputs).
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& s, float scale,
                int causal, int win_l, int win_r, int sm_count, cudaStream_t stream,
-               const float* const* descales = nullptr) {
+               const float* const* descales = nullptr, const float* alibi = nullptr) {
   CUtensorMap mq, mk, mv, mo;
   int st;
   auto in_map = descales ? make_map_u8 : make_map;
@@ -234,6 +250,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.q_descale = descales ? descales[0] : nullptr;
   p.k_descale = descales ? descales[1] : nullptr;
   p.v_descale = descales ? descales[2] : nullptr;
+  p.alibi_slopes = alibi;
   p.B = s.B;
   p.N = s.N;
   p.H = s.H;
@@ -256,6 +273,12 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (descales)
     fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128, true>::kThreads, fa::FwdCfg<128, true>::kSmemBytes,
                                    stream>>>(mq, mk, mv, mo, p);
+  else if (alibi && s.d == 64)
+    fa::fa_fwd_kernel<64, false, true><<<grid, fa::FwdCfg<64>::kThreads, fa::FwdCfg<64>::kSmemBytes, stream>>>(
+        mq, mk, mv, mo, p);
+  else if (alibi)
+    fa::fa_fwd_kernel<128, false, true><<<grid, fa::FwdCfg<128>::kThreads, fa::FwdCfg<128>::kSmemBytes, stream>>>(
+        mq, mk, mv, mo, p);
   else if (s.d == 64)
     fa::fa_fwd_kernel<64><<<grid, fa::FwdCfg<64>::kThreads, fa::FwdCfg<64>::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
   else
@@ -279,8 +302,10 @@ int launch_pre(const void* o, const float* lse, const void* dO, const Shape& s, 
   return launch_status();
 }
 
-fa::BwdParams bwd_params(const Shape& s, float scale, int causal, int win_l, int win_r, const Workspace& w) {
+fa::BwdParams bwd_params(const Shape& s, float scale, int causal, int win_l, int win_r, const Workspace& w,
+                         const float* alibi = nullptr) {
   fa::BwdParams p;
+  p.alibi_slopes = alibi;
   p.B = s.B;
   p.N = s.N;
   p.H = s.H;
@@ -299,53 +324,69 @@ fa::BwdParams bwd_params(const Shape& s, float scale, int causal, int win_l, int
   return p;
 }
 
+template <int D, bool kDQ>
+void main_kernel(bool alibi, int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
+                 const CUtensorMap& mv, const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
+                 const CUtensorMap& mdq, const fa::BwdParams& p) {
+  if (alibi)
+    fa::fa_bwd_kernel<D, kDQ, true><<<grid, fa::BwdCfg<D>::kThreads, fa::BwdCfg<D>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  else
+    fa::fa_bwd_kernel<D, kDQ, false><<<grid, fa::BwdCfg<D>::kThreads, fa::BwdCfg<D>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdk, mdv, mdq, p);
+}
+
 // Main backward kernel; with_dq = false computes dK and dV only (the deterministic backward).
 int launch_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, const Shape& s,
                 float scale, int causal, int win_l, int win_r, const Workspace& w, int sm_count,
-                cudaStream_t stream, bool with_dq = true) {
+                cudaStream_t stream, bool with_dq = true, const float* alibi = nullptr) {
   CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
   int st;
   if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
       (st = make_map(&mdo, dO, s)) || (st = make_map(&mdk, dk, s)) || (st = make_map(&mdv, dv, s)) ||
       (st = make_map_f32_acc(&mdq, w.dq_acc, s)))
     return st;
-  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w);
+  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, alibi);
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   if (log_enabled())
     std::fprintf(stderr, "[fa] bwd B=%d N=%d H=%d d=%d causal=%d win=(%d,%d) items=%d grid=%d smem=%d\n", s.B, s.N,
                  s.H, s.d, p.causal, win_l, win_r, p.num_items, grid,
                  s.d == 64 ? fa::BwdCfg<64>::kSmemBytes : fa::BwdCfg<128>::kSmemBytes);
+  const bool a = alibi != nullptr;
   if (s.d == 64 && with_dq)
-    fa::fa_bwd_kernel<64, true><<<grid, fa::BwdCfg<64>::kThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    main_kernel<64, true>(a, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
   else if (s.d == 64)
-    fa::fa_bwd_kernel<64, false><<<grid, fa::BwdCfg<64>::kThreads, fa::BwdCfg<64>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    main_kernel<64, false>(a, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
   else if (with_dq)
-    fa::fa_bwd_kernel<128, true><<<grid, fa::BwdCfg<128>::kThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    main_kernel<128, true>(a, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
   else
-    fa::fa_bwd_kernel<128, false><<<grid, fa::BwdCfg<128>::kThreads, fa::BwdCfg<128>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    main_kernel<128, false>(a, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
   return launch_status();
 }
 
 // dQ of the deterministic backward: one item per (b, h, Q tile), dQ accumulated in TMEM.
 int launch_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, const Shape& s, float scale,
-              int causal, int win_l, int win_r, const Workspace& w, int sm_count, cudaStream_t stream) {
+              int causal, int win_l, int win_r, const Workspace& w, int sm_count, cudaStream_t stream,
+              const float* alibi = nullptr) {
   CUtensorMap mq, mk, mv, mdo, mdq;
   int st;
   if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
       (st = make_map(&mdo, dO, s)) || (st = make_map(&mdq, dq, s)))
     return st;
-  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w);
+  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, alibi);
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
-  if (s.d == 64)
-    fa::fa_bwd_dq_kernel<64><<<grid, fa::BwdDqCfg<64>::kThreads, fa::BwdDqCfg<64>::kSmemBytes, stream>>>(
+  if (s.d == 64 && alibi)
+    fa::fa_bwd_dq_kernel<64, true><<<grid, fa::BwdDqCfg<64>::kThreads, fa::BwdDqCfg<64>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdq, p);
+  else if (s.d == 64)
+    fa::fa_bwd_dq_kernel<64, false><<<grid, fa::BwdDqCfg<64>::kThreads, fa::BwdDqCfg<64>::kSmemBytes, stream>>>(
+        mq, mk, mv, mdo, mdq, p);
+  else if (alibi)
+    fa::fa_bwd_dq_kernel<128, true><<<grid, fa::BwdDqCfg<128>::kThreads, fa::BwdDqCfg<128>::kSmemBytes, stream>>>(
         mq, mk, mv, mdo, mdq, p);
   else
-    fa::fa_bwd_dq_kernel<128><<<grid, fa::BwdDqCfg<128>::kThreads, fa::BwdDqCfg<128>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdq, p);
+    fa::fa_bwd_dq_kernel<128, false><<<grid, fa::BwdDqCfg<128>::kThreads, fa::BwdDqCfg<128>::kSmemBytes,
+                                        stream>>>(mq, mk, mv, mdo, mdq, p);
   return launch_status();
 }
 
@@ -427,6 +468,27 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int fa_fwd_ex(const void* q, const void* k, const void* v, const float* alibi_slopes, void* o, float* lse, int B,
+              int N, int H, int d, float scale, int causal, int win_l, int win_r, fa_stream_t stream) {
+  int st = check_problem(B, N, H, d, scale, causal, &win_l, &win_r);
+  if (st) return st;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(alibi_slopes, 4))
+    return FA_ERR_INVALID_ARG;
+  const Shape s{B, N, H, d};
+  const size_t tb = s.tensor_bytes(), lb = s.rowvec_bytes(), ab = (size_t)B * H * 4;
+  if (overlap(o, tb, q, tb) || overlap(o, tb, k, tb) || overlap(o, tb, v, tb) || overlap(lse, lb, q, tb) ||
+      overlap(lse, lb, k, tb) || overlap(lse, lb, v, tb) || overlap(lse, lb, o, tb))
+    return FA_ERR_INVALID_ARG;
+  if (alibi_slopes && (overlap(o, tb, alibi_slopes, ab) || overlap(lse, lb, alibi_slopes, ab)))
+    return FA_ERR_INVALID_ARG;
+  int dev, sms;
+  if ((st = device_setup(&dev, &sms))) return st;
+  return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream),
+                    nullptr, alibi_slopes);
+}
+
 int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale, const float* k_descale,
                const float* v_descale, void* o, float* lse, int B, int N, int H, int d, float scale, int causal,
                int win_l, int win_r, fa_stream_t stream) {
@@ -455,6 +517,21 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_desca
 
 namespace {
 
+template <int D>
+int launch_decode(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
+                  cudaStream_t cs) {
+  const int smem = fa::DecCfg<D>::kSmemBytes;
+  if (p.Sq == 1)
+    fa::fa_decode_split_kernel<D, 1><<<grid, fa::kDecThreads, smem, cs>>>(mk, mv, p);
+  else if (p.Sq == 2)
+    fa::fa_decode_split_kernel<D, 2><<<grid, fa::kDecThreads, smem, cs>>>(mk, mv, p);
+  else if (p.Sq <= 4)
+    fa::fa_decode_split_kernel<D, 4><<<grid, fa::kDecThreads, smem, cs>>>(mk, mv, p);
+  else
+    fa::fa_decode_split_kernel<D, 8><<<grid, fa::kDecThreads, smem, cs>>>(mk, mv, p);
+  return launch_status();
+}
+
 size_t decode_workspace_bytes(int B, int Sq, int H, int d, int splits) {
   if (splits <= 1) return 0;
   const size_t rows = (size_t)B * H * Sq * splits;
@@ -476,13 +553,21 @@ int decode_auto_splits(int B, int H, int max_keys, int sm_count) {
 
 extern "C" {
 
+int fa_decode_splits(int B, int H, int max_keys) {
+  if (B < 1 || H < 1 || max_keys < 1) return -FA_ERR_INVALID_ARG;
+  int dev, sms, st;
+  if ((st = device_setup(&dev, &sms))) return -st;
+  return decode_auto_splits(B, H, max_keys, sms);
+}
+
 size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits) {
   if (B < 1 || Sq < 1 || H < 1 || (d != 64 && d != 128) || splits < 0) return 0;
   return decode_workspace_bytes(B, Sq, H, d, splits);
 }
 
-int fa_decode_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
-                    const int* seqlens, void* o, float* lse, int B, int Sq, int H, int d, int num_pages,
+int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                    const int* block_table, const int* seqlens, void* o, float* lse, int B, int Sq, int H, int d,
+                    int num_pages,
                     int page_size, int max_pages, float scale, int causal, int win_l, int win_r, int splits,
                     void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
   if (B < 1 || H < 1 || Sq < 1 || num_pages < 1 || max_pages < 1 || page_size < 1 || splits < 0)
@@ -494,24 +579,29 @@ int fa_decode_paged(const void* q, const void* k_cache, const void* v_cache, con
       (double)max_pages * page_size >= 2147483647.0)
     return FA_ERR_INVALID_ARG;
   if (!q || !k_cache || !v_cache || !block_table || !seqlens || !o || !lse) return FA_ERR_INVALID_ARG;
+  if ((k_new == nullptr) != (v_new == nullptr)) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
-      !aligned(block_table, 4) || !aligned(seqlens, 4))
+      !aligned(block_table, 4) || !aligned(seqlens, 4) || !aligned(k_new, 16) || !aligned(v_new, 16))
     return FA_ERR_INVALID_ARG;
   if (causal) win_r = 0;
   const size_t qb = (size_t)B * Sq * H * d * 2, cb = (size_t)num_pages * page_size * H * d * 2;
   const size_t lb = (size_t)B * H * Sq * 4, tb = (size_t)B * max_pages * 4, sb = (size_t)B * 4;
-  const void* ins[5] = {q, k_cache, v_cache, block_table, seqlens};
-  const size_t in_bytes[5] = {qb, cb, cb, tb, sb};
-  for (int i = 0; i < 5; ++i)
+  const void* ins[7] = {q, k_cache, v_cache, block_table, seqlens, k_new, v_new};
+  const size_t in_bytes[7] = {qb, cb, cb, tb, sb, k_new ? qb : 0, v_new ? qb : 0};
+  for (int i = 0; i < 7; ++i)
     if (overlap(o, qb, ins[i], in_bytes[i]) || overlap(lse, lb, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
-  if (overlap(o, qb, lse, lb)) return FA_ERR_INVALID_ARG;
+  if (overlap(o, qb, lse, lb) || overlap(k_cache, cb, v_cache, cb)) return FA_ERR_INVALID_ARG;
+  for (int i = 0; i < 7; ++i)  // the caches are written when new rows are given: nothing may alias them
+    if (k_new && i != 1 && i != 2 &&
+        (overlap(k_cache, cb, ins[i], in_bytes[i]) || overlap(v_cache, cb, ins[i], in_bytes[i])))
+      return FA_ERR_INVALID_ARG;
   int dev, sms, st;
   if ((st = device_setup(&dev, &sms))) return st;
   if (splits == 0) splits = decode_auto_splits(B, H, max_pages * page_size, sms);
   const size_t wbytes = decode_workspace_bytes(B, Sq, H, d, splits);
   if (wbytes > 0 && workspace) {
     if (!aligned(workspace, 256) || workspace_bytes_ < wbytes) return FA_ERR_INVALID_ARG;
-    for (int i = 0; i < 5; ++i)
+    for (int i = 0; i < 7; ++i)
       if (overlap(workspace, wbytes, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
     if (overlap(workspace, wbytes, o, qb) || overlap(workspace, wbytes, lse, lb)) return FA_ERR_INVALID_ARG;
   }
@@ -547,12 +637,21 @@ int fa_decode_paged(const void* q, const void* k_cache, const void* v_cache, con
   p.lse_part = wbytes ? reinterpret_cast<float*>(static_cast<char*>(ws) +
                                                  align256((size_t)B * H * Sq * splits * d * 4))
                       : nullptr;
-  const dim3 grid(splits, H, B);
-  if (d == 64)
-    fa::fa_decode_split_kernel<64><<<grid, fa::kDecThreads, fa::DecCfg<64>::kSmemBytes, cs>>>(mk, mv, p);
-  else
-    fa::fa_decode_split_kernel<128><<<grid, fa::kDecThreads, fa::DecCfg<128>::kSmemBytes, cs>>>(mk, mv, p);
-  st = launch_status();
+  st = FA_OK;
+  if (k_new) {
+    fa::fa_decode_append_kernel<<<dim3(Sq, B), 256, 0, cs>>>(p, d, static_cast<const __nv_bfloat16*>(k_new),
+                                                             static_cast<const __nv_bfloat16*>(v_new),
+                                                             static_cast<__nv_bfloat16*>(k_cache),
+                                                             static_cast<__nv_bfloat16*>(v_cache));
+    st = launch_status();
+  }
+  if (!st) {
+    const dim3 grid(H, splits, B);  // heads fastest: concurrent CTAs share cache rows
+    if (d == 64)
+      st = launch_decode<64>(grid, mk, mv, p, cs);
+    else
+      st = launch_decode<128>(grid, mk, mv, p, cs);
+  }
   if (!st && splits > 1) {
     const dim3 cgrid(Sq, H, B);
     if (d == 64)
@@ -622,7 +721,8 @@ int fa_bwd_dq_convert(void* dq, int B, int N, int H, int d, void* workspace, siz
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                     void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale, int causal, int win_l,
-                    int win_r, void* workspace, size_t workspace_bytes_, fa_stream_t stream, bool deterministic) {
+                    int win_r, void* workspace, size_t workspace_bytes_, fa_stream_t stream, bool deterministic,
+                    const float* alibi = nullptr) {
   int st = check_problem(B, N, H, d, scale, causal, &win_l, &win_r);
   if (st) return st;
   const Shape s{B, N, H, d};
@@ -640,8 +740,14 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
     if (overlap(out, tb, lse, lb)) return FA_ERR_INVALID_ARG;
   }
   if (overlap(dq, tb, dk, tb) || overlap(dq, tb, dv, tb) || overlap(dk, tb, dv, tb)) return FA_ERR_INVALID_ARG;
+  if (alibi) {
+    if (!aligned(alibi, 4)) return FA_ERR_INVALID_ARG;
+    for (void* out : outs)
+      if (overlap(out, tb, alibi, (size_t)B * H * 4)) return FA_ERR_INVALID_ARG;
+  }
   if (workspace) {
     if ((st = check_workspace(workspace, workspace_bytes_, s))) return st;
+    if (alibi && overlap(workspace, workspace_bytes(s), alibi, (size_t)B * H * 4)) return FA_ERR_INVALID_ARG;
     const size_t wb = workspace_bytes(s);
     for (const void* in : ins)
       if (overlap(workspace, wb, in, tb)) return FA_ERR_INVALID_ARG;
@@ -663,10 +769,10 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   const Workspace w = carve(ws, s);
   st = launch_pre(o, lse, dO, s, w, cs);
   if (deterministic) {
-    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs, false);
-    if (!st) st = launch_dq(q, k, v, dO, dq, s, scale, causal, win_l, win_r, w, sms, cs);
+    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs, false, alibi);
+    if (!st) st = launch_dq(q, k, v, dO, dq, s, scale, causal, win_l, win_r, w, sms, cs, alibi);
   } else {
-    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs);
+    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs, true, alibi);
     if (!st) st = launch_convert(dq, s, w, cs);
   }
   if (!workspace && cudaFreeAsync(ws, cs) != cudaSuccess && !st) st = FA_ERR_CUDA;
@@ -680,6 +786,14 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, N, H, d, scale, causal, win_l, win_r, workspace,
                   workspace_bytes_, stream, false);
+}
+
+int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+              const float* alibi_slopes, void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale,
+              int causal, int win_l, int win_r, int deterministic, void* workspace, size_t workspace_bytes_,
+              fa_stream_t stream) {
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, N, H, d, scale, causal, win_l, win_r, workspace,
+                  workspace_bytes_, stream, deterministic != 0, alibi_slopes);
 }
 
 int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,

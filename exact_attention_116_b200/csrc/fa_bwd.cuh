@@ -31,7 +31,6 @@
 
 namespace fa {
 
-constexpr float kLog2e = 1.4426950408889634074f;
 
 struct BwdParams {
   int B, N, H, N_pad;  // N_pad = N rounded up to 128 (row stride of LSE2 and D)
@@ -46,6 +45,7 @@ struct BwdParams {
   const float* lse2;   // (B, H, N_pad) fp32: -LSE * log2(e)
   const float* dvec;   // (B, H, N_pad) fp32: -rowsum(dO * O)
   int* next_item;      // work counters (zeroed by the preprocess kernel): [0] main kernel, [1] dQ kernel
+  const float* alibi_slopes;  // ALiBi only: (B, H) slopes m, bias -m |i - j| on the scaled scores
 };
 
 // Heads per scheduling group: items of a group are handed out before the next group's, so the
@@ -209,9 +209,11 @@ __device__ __forceinline__ bool bwd_tile_unmasked(const BwdParams& p, int j, int
 // P^T for 64 query columns of this thread's key row: exp2(S^T * c - LSE_q * log2(e)), zero
 // where masked (kMasked), packed to bf16 pairs (even column low). nlse2 holds -LSE * log2(e)
 // of the same 64 queries.
-template <bool kMasked>
+template <bool kMasked, bool kAlibi = false>
 __device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[32], const uint32_t (&s1)[32], float c,
-                                          const float* nlse2, int qbase, int qlo, int qhi, uint32_t (&pk)[32]) {
+                                          const float* nlse2, int qbase, int qlo, int qhi, uint32_t (&pk)[32],
+                                          float d0 = 0.0f, float nslope2 = 0.0f) {
+  // ALiBi: d0 = qbase - key; the bias of column f is nslope2 * |d0 + f| (nslope2 = -m log2(e)).
   const float2 c2 = make_float2(c, c);
 #pragma unroll
   for (int e = 0; e < 64; e += 4) {
@@ -221,7 +223,11 @@ __device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[32], const uint32
       const int f = e + h2;
       const float2 sv = make_float2(__uint_as_float(f < 32 ? s0[f] : s1[f - 32]),
                                     __uint_as_float(f < 32 ? s0[f + 1] : s1[f - 31]));
-      const float2 xv = fma2(sv, c2, h2 ? make_float2(nl.z, nl.w) : make_float2(nl.x, nl.y));
+      float2 xv = fma2(sv, c2, h2 ? make_float2(nl.z, nl.w) : make_float2(nl.x, nl.y));
+      if (kAlibi) {
+        xv.x = fmaf(fabsf(d0 + (float)f), nslope2, xv.x);
+        xv.y = fmaf(fabsf(d0 + (float)(f + 1)), nslope2, xv.y);
+      }
       float2 pv;
       if (((f >> 1) % kBwdPolyDen) < kBwdPolyNum) {
         pv = exp2_poly2(xv);
@@ -238,7 +244,7 @@ __device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[32], const uint32
   }
 }
 
-template <int D, bool kDQ>
+template <int D, bool kDQ, bool kAlibi = false>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -507,6 +513,7 @@ __global__ void __launch_bounds__(512, 1)
       int lo, hi;
       bwd_q_range(p, j, lo, hi);
       const int k = j * 128 + row;
+      const float nslope2 = kAlibi ? -p.alibi_slopes[b * p.H + h] * kLog2e : 0.0f;
       const int qlo = p.win_r >= 0 ? k - p.win_r : 0;
       const int qhi = (k >= p.N) ? -1 : (p.win_l >= 0 ? min(p.N - 1, k + p.win_l) : p.N - 1);
       for (int i = lo; i <= hi; ++i, ++n) {
@@ -525,10 +532,11 @@ __global__ void __launch_bounds__(512, 1)
         tmem_wait_ld(s0);
         tmem_wait_ld(s1);
         uint32_t pk[32];
+        const float dist0 = (float)(qbase - k);
         if (masked)
-          bwd_probs<true>(s0, s1, c, nlse2 + 64 * grp, qbase, qlo, qhi, pk);
+          bwd_probs<true, kAlibi>(s0, s1, c, nlse2 + 64 * grp, qbase, qlo, qhi, pk, dist0, nslope2);
         else
-          bwd_probs<false>(s0, s1, c, nlse2 + 64 * grp, qbase, qlo, qhi, pk);
+          bwd_probs<false, kAlibi>(s0, s1, c, nlse2 + 64 * grp, qbase, qlo, qhi, pk, dist0, nslope2);
         {
           uint32_t lo16[16], hi16[16];
 #pragma unroll

@@ -89,7 +89,7 @@ __device__ __forceinline__ FwdParams bwd_dq_as_fwd(const BwdParams& p) {
   return f;
 }
 
-template <int D>
+template <int D, bool kAlibi = false>
 __global__ void __launch_bounds__(256, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -269,6 +269,7 @@ __global__ void __launch_bounds__(256, 1)
       const size_t stat = ((size_t)b * p.H + h) * (size_t)p.N_pad + q;  // padded rows hold 0
       const float nlse2 = p.lse2[stat];                                 // -LSE * log2(e)
       const float nd = p.dvec[stat];                                     // -D
+      const float nslope2 = kAlibi ? -p.alibi_slopes[b * p.H + h] * kLog2e : 0.0f;  // ALiBi: -m log2(e)
       const int kmin = p.win_l >= 0 ? q - p.win_l : 0;
       const int kmax = (q >= p.N) ? -1 : (p.win_r >= 0 ? min(p.N - 1, q + p.win_r) : p.N - 1);
       for (int j = lo; j <= hi; ++j, ++n) {
@@ -283,8 +284,13 @@ __global__ void __launch_bounds__(256, 1)
           tmem_wait_ld(sv);
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float2 xv = fma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
-                                   make_float2(c, c), make_float2(nlse2, nlse2));
+            float2 xv = fma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
+                             make_float2(c, c), make_float2(nlse2, nlse2));
+            if (kAlibi) {  // bias -m |q - key| with key = j * 128 + q4 * 32 + e
+              const float d0 = (float)(q - j * 128 - q4 * 32);
+              xv.x = fmaf(fabsf(d0 - (float)e), nslope2, xv.x);
+              xv.y = fmaf(fabsf(d0 - (float)(e + 1)), nslope2, xv.y);
+            }
             float2 pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
             if (masked) {
               const int key = j * 128 + q4 * 32 + e;

@@ -20,6 +20,13 @@
 //   B: warp w owns rows w and w + 4: mask, tile max, exponentials, running max / sum, rescale
 //      factor alpha_i; P goes to shared memory
 //   C: thread (column pair, key group) accumulates O_i += P_i,t v_t over its keys
+// The kernel is compiled for kSq = 1, 2, 4, 8 rows (the call's Sq rounded up; the extra rows
+// have q = 0 and are not written). CTAs of the same (b, split) for consecutive heads are
+// launched next to each other (head is the fastest grid index), so the 128-byte rows of one
+// cache row (H x d bf16, contiguous) are read by concurrent CTAs.
+//
+// With new K/V rows given (flash_attn_with_kvcache's in-place update of the cache),
+// fa_decode_append_kernel first writes them into the cache at their positions.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -78,7 +85,7 @@ __device__ __forceinline__ bool dec_tile_range(const DecParams& p, int n, int s,
   return n > 0 && t1 > t0;
 }
 
-template <int D>
+template <int D, int kSq>
 __global__ void __launch_bounds__(kDecThreads)
     fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                            const DecParams p) {
@@ -95,7 +102,8 @@ __global__ void __launch_bounds__(kDecThreads)
   float* sRed = reinterpret_cast<float*>(sm + Cfg::kOffRed);
   const Abort ab{abort_flag};
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  static_assert(kSq >= 1 && kSq <= kDecMaxSq, "rows per CTA");
+  const int h = blockIdx.x, s = blockIdx.y, b = blockIdx.z;
   const int Sq = p.Sq;
   int n = p.seqlens[b];
   if (n < 0 || n > p.max_pages * p.page_size) {  // reported by fa_check; the sequence is treated as empty
@@ -111,6 +119,7 @@ __global__ void __launch_bounds__(kDecThreads)
     for (int st = 0; st < kDecStages; ++st) mbar_init(smem_u32(&full[st]), 1);
     fence_barrier_init();
   }
+  if (tid < kDecMaxSq) sAlpha[tid] = 0.0f;  // rows past Sq keep alpha = 0 (their O stays 0)
   // q rows -> shared memory (fp32); rows >= Sq are zero
   for (int e = tid; e < kDecMaxSq * D; e += kDecThreads) {
     const int i = e / D, c = e - i * D;
@@ -146,9 +155,9 @@ __global__ void __launch_bounds__(kDecThreads)
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
   // O accumulators of this thread: rows 0..Sq-1, columns 2 cp and 2 cp + 1, keys of group kg
   const int cp = tid % Cfg::kPairs, kg = tid / Cfg::kPairs;
-  float acc[kDecMaxSq][2];
+  float acc[kSq][2];
 #pragma unroll
-  for (int i = 0; i < kDecMaxSq; ++i) acc[i][0] = acc[i][1] = 0.0f;
+  for (int i = 0; i < kSq; ++i) acc[i][0] = acc[i][1] = 0.0f;
   const float c = p.scale_log2;
 
   for (int t = t0; t < t1; ++t) {
@@ -159,9 +168,9 @@ __global__ void __launch_bounds__(kDecThreads)
     // ---- A: half dot products, key kt = tid % 64, dims [half * D/2, half * D/2 + D/2)
     {
       const int kt = tid % kDecTile, half = tid / kDecTile;
-      float part[kDecMaxSq];
+      float part[kSq];
 #pragma unroll
-      for (int i = 0; i < kDecMaxSq; ++i) part[i] = 0.0f;
+      for (int i = 0; i < kSq; ++i) part[i] = 0.0f;
 #pragma unroll
       for (int ch = 0; ch < D / 16; ++ch) {  // 16-byte chunks of this thread's half row
         const int col0 = half * (D / 2) + ch * 8;
@@ -175,31 +184,28 @@ __global__ void __launch_bounds__(kDecThreads)
           kv[2 * e + 1] = bf16hi_to_f32(w[e]);
         }
 #pragma unroll
-        for (int i = 0; i < kDecMaxSq; ++i) {
-          if (i < Sq) {
-            const float4 qa = *reinterpret_cast<const float4*>(&sQ[i * D + col0]);
-            const float4 qb = *reinterpret_cast<const float4*>(&sQ[i * D + col0 + 4]);
-            part[i] = fmaf(qa.x, kv[0], part[i]);
-            part[i] = fmaf(qa.y, kv[1], part[i]);
-            part[i] = fmaf(qa.z, kv[2], part[i]);
-            part[i] = fmaf(qa.w, kv[3], part[i]);
-            part[i] = fmaf(qb.x, kv[4], part[i]);
-            part[i] = fmaf(qb.y, kv[5], part[i]);
-            part[i] = fmaf(qb.z, kv[6], part[i]);
-            part[i] = fmaf(qb.w, kv[7], part[i]);
-          }
+        for (int i = 0; i < kSq; ++i) {  // rows past Sq have q = 0
+          const float4 qa = *reinterpret_cast<const float4*>(&sQ[i * D + col0]);
+          const float4 qb = *reinterpret_cast<const float4*>(&sQ[i * D + col0 + 4]);
+          part[i] = fmaf(qa.x, kv[0], part[i]);
+          part[i] = fmaf(qa.y, kv[1], part[i]);
+          part[i] = fmaf(qa.z, kv[2], part[i]);
+          part[i] = fmaf(qa.w, kv[3], part[i]);
+          part[i] = fmaf(qb.x, kv[4], part[i]);
+          part[i] = fmaf(qb.y, kv[5], part[i]);
+          part[i] = fmaf(qb.z, kv[6], part[i]);
+          part[i] = fmaf(qb.w, kv[7], part[i]);
         }
       }
 #pragma unroll
-      for (int i = 0; i < kDecMaxSq; ++i)
-        if (i < Sq) sS[(half * kDecMaxSq + i) * kDecTile + kt] = part[i];
+      for (int i = 0; i < kSq; ++i) sS[(half * kDecMaxSq + i) * kDecTile + kt] = part[i];
     }
     __syncthreads();
     // every thread has finished with the previous tile's slot: refill it
     if (tid == 0 && t > t0 && t - 1 + kDecStages < t1) issue(t - 1 + kDecStages);
     // ---- B: softmax bookkeeping, warp w -> rows w, w + 4
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < (kSq + 3) / 4; ++r) {
       const int i = warp + 4 * r;
       if (i < Sq) {
         const int pos = n - Sq + i;
@@ -237,12 +243,10 @@ __global__ void __launch_bounds__(kDecThreads)
     {
       const int col = 2 * cp, bx = col / 64, chunk = (col % 64) / 8, within = (col % 8) * 2;
 #pragma unroll
-      for (int i = 0; i < kDecMaxSq; ++i) {
-        if (i < Sq) {
-          const float a = sAlpha[i];
-          acc[i][0] *= a;
-          acc[i][1] *= a;
-        }
+      for (int i = 0; i < kSq; ++i) {  // rows past Sq stay 0
+        const float a = sAlpha[i];
+        acc[i][0] *= a;
+        acc[i][1] *= a;
       }
 #pragma unroll 4
       for (int kt = kg; kt < kDecTile; kt += Cfg::kKeyGroups) {
@@ -250,12 +254,10 @@ __global__ void __launch_bounds__(kDecThreads)
                                                               within);
         const float v0 = bf16lo_to_f32(w), v1 = bf16hi_to_f32(w);
 #pragma unroll
-        for (int i = 0; i < kDecMaxSq; ++i) {
-          if (i < Sq) {
-            const float pv = sP[i * kDecTile + kt];
-            acc[i][0] = fmaf(pv, v0, acc[i][0]);
-            acc[i][1] = fmaf(pv, v1, acc[i][1]);
-          }
+        for (int i = 0; i < kSq; ++i) {
+          const float pv = sP[i * kDecTile + kt];
+          acc[i][0] = fmaf(pv, v0, acc[i][0]);
+          acc[i][1] = fmaf(pv, v1, acc[i][1]);
         }
       }
     }
@@ -271,16 +273,14 @@ __global__ void __launch_bounds__(kDecThreads)
   __syncthreads();  // the K/V ring is free: it holds the reduction below
   // ---- combine the key groups' partial sums, normalise, write
 #pragma unroll
-  for (int i = 0; i < kDecMaxSq; ++i) {
-    if (i < Sq) {
-      sRed[(kg * kDecMaxSq + i) * D + 2 * cp] = acc[i][0];
-      sRed[(kg * kDecMaxSq + i) * D + 2 * cp + 1] = acc[i][1];
-    }
+  for (int i = 0; i < kSq; ++i) {
+    sRed[(kg * kDecMaxSq + i) * D + 2 * cp] = acc[i][0];
+    sRed[(kg * kDecMaxSq + i) * D + 2 * cp + 1] = acc[i][1];
   }
   // row statistics of warp-owned rows -> shared (reuse the alpha slots as 1/l, S as log2 l + m)
   __syncthreads();
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
+  for (int r = 0; r < (kSq + 3) / 4; ++r) {
     const int i = warp + 4 * r;
     if (i < Sq && lane == 0) {
       sAlpha[i] = l_run[r] > 0.0f ? 1.0f / l_run[r] : 0.0f;
@@ -306,6 +306,31 @@ __global__ void __launch_bounds__(kDecThreads)
       p.lse[((size_t)b * p.H + h) * Sq + tid] = l2 == -INFINITY ? -INFINITY : l2 * kDecLn2;
     else
       p.lse_part[(((size_t)b * p.H + h) * Sq + tid) * p.splits + s] = l2;
+  }
+}
+
+// Write the new rows' K and V (B, Sq, H, d) into the cache at positions seqlen_b - Sq + i:
+// one CTA per (i, b), each copying the row's H*d contiguous values of K and of V.
+__global__ void __launch_bounds__(256)
+    fa_decode_append_kernel(const DecParams p, int d, const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                            __nv_bfloat16* k_cache, __nv_bfloat16* v_cache) {
+  const int i = blockIdx.x, b = blockIdx.y;
+  const int n = p.seqlens[b];
+  if (n < 0 || n > p.max_pages * p.page_size) return;  // reported by the split kernel
+  const int pos = n - p.Sq + i;
+  if (pos < 0) return;  // the sequence is shorter than its new rows: nothing to place
+  const int page = p.block_table[(size_t)b * p.max_pages + pos / p.page_size];
+  if (page < 0 || page >= p.num_pages) {
+    if (threadIdx.x == 0) atomicOr(&g_fa_error, kErrBadInput);
+    return;
+  }
+  const size_t row_elems = (size_t)p.H * d;
+  const size_t src = ((size_t)b * p.Sq + i) * row_elems;
+  const size_t dst = ((size_t)page * p.page_size + pos % p.page_size) * row_elems;
+  const int chunks = (int)(row_elems / 8);  // 16-byte chunks (d is 64 or 128)
+  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+    reinterpret_cast<uint4*>(k_cache + dst)[c] = reinterpret_cast<const uint4*>(k_new + src)[c];
+    reinterpret_cast<uint4*>(v_cache + dst)[c] = reinterpret_cast<const uint4*>(v_new + src)[c];
   }
 }
 

@@ -49,6 +49,7 @@ struct FwdParams {
   const float* q_descale;   // E4M3 inputs only: (B, H) factors, value = descale * code
   const float* k_descale;
   const float* v_descale;
+  const float* alibi_slopes;  // ALiBi only: (B, H) slopes m, bias -m |i - j| on the scaled scores
 };
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
@@ -135,11 +136,18 @@ __device__ __forceinline__ bool fwd_tile_unmasked(const FwdParams& p, int r0, in
 // ------------------------------------------------------------------ softmax role
 
 // Row maximum of a 128-key tile (scaled, log2 units) with masking, and the lazy update of
-// the reference maximum. x is scaled in place when the scale is not positive.
-template <bool kPosScale>
+// the reference maximum. x is scaled in place when the scale is not positive, and always with
+// ALiBi, whose bias nslope2 * |d0 - cc| (nslope2 = -m log2(e), d0 = row - kbase) is added
+// after the scaling.
+template <bool kPosScale, bool kAlibi = false>
 __device__ __forceinline__ void fwd_row_max(float (&x)[128], bool masked, int kbase, int kmin, int kmax, float c,
-                                            float& m_run, float& alpha, bool& updated) {
-  if (!kPosScale) {  // then masking must follow the scaling
+                                            float& m_run, float& alpha, bool& updated, float d0 = 0.0f,
+                                            float nslope2 = 0.0f) {
+  static_assert(!(kAlibi && kPosScale), "the ALiBi bias is added to scaled scores");
+  if (kAlibi) {
+#pragma unroll
+    for (int cc = 0; cc < 128; ++cc) x[cc] = fmaf(fabsf(d0 - (float)cc), nslope2, x[cc] * c);
+  } else if (!kPosScale) {  // then masking must follow the scaling
 #pragma unroll
     for (int cc = 0; cc < 128; cc += 2) {
       const float2 v = mul2(make_float2(x[cc], x[cc + 1]), make_float2(c, c));
@@ -222,7 +230,7 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
-template <int D, bool kF8 = false>
+template <int D, bool kF8 = false, bool kAlibi = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -230,6 +238,7 @@ __global__ void __launch_bounds__(384, 1)
   using Cfg = FwdCfg<D, kF8>;
   using Bars = FwdBars<Cfg>;
   static_assert(!kF8 || D == 128, "E4M3 inputs: head dim 128 (one 128-byte row per TMA box)");
+  static_assert(!(kF8 && kAlibi), "ALiBi is built for bf16 inputs");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
@@ -498,6 +507,8 @@ __global__ void __launch_bounds__(384, 1)
       fwd_kv_range(p, r0, lo, hi);
       if (hi < lo) continue;
       float c = p.scale_log2, o_mul = 1.0f;  // log2-domain score factor; O factor
+      float nslope2 = 0.0f;                  // ALiBi: -m log2(e)
+      if constexpr (kAlibi) nslope2 = -p.alibi_slopes[b * p.H + h] * kLog2e;
       if constexpr (kF8) {
         const int bh = b * p.H + h;
         c *= p.q_descale[bh] * p.k_descale[bh];
@@ -528,7 +539,11 @@ __global__ void __launch_bounds__(384, 1)
         const bool masked = !fwd_tile_unmasked(p, r0, j);
         float alpha;
         bool updated;
-        if (c > 0.0f)
+        const bool pos_scale = !kAlibi && c > 0.0f;  // with ALiBi the scores are scaled before the max
+        if constexpr (kAlibi)
+          fwd_row_max<false, true>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated, (float)(i - j * 128),
+                                   nslope2);
+        else if (pos_scale)
           fwd_row_max<true>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated);
         else
           fwd_row_max<false>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated);
@@ -544,14 +559,14 @@ __global__ void __launch_bounds__(384, 1)
         for (int q4 = 0; q4 < 4; ++q4) {
           if constexpr (kF8) {
             uint32_t pk[8];
-            if (c > 0.0f)
+            if (pos_scale)
               fwd_exp_chunk_e4m3<true>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
             else
               fwd_exp_chunk_e4m3<false>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
             tmem_st8(tP + q4 * 8, pk);
           } else {
             uint32_t pk[16];
-            if (c > 0.0f)
+            if (pos_scale)
               fwd_exp_chunk<true>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
             else
               fwd_exp_chunk<false>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);

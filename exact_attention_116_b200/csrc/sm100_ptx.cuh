@@ -21,6 +21,8 @@ namespace fa {
 // cleared by the host. The library is a single translation unit, so it is defined here.
 __device__ int g_fa_error = 0;
 
+constexpr float kLog2e = 1.4426950408889634074f;
+
 enum DeviceError : int {
   kErrWaitTimeout = 1,  // a bounded mbarrier wait gave up
   kErrSmemAlign = 2,    // dynamic shared memory not at the alignment a kernel's layout needs

@@ -63,6 +63,18 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            fa_stream_t stream);
 
 /*
+ * Forward with an optional ALiBi bias (the call's alibi_slopes, "FlashAttention技术解析：
+ * 加速GPT训练的核心优化" §2.2): alibi_slopes is NULL (same as fa_fwd) or a device (B,H)
+ * float32 array of slopes m; the score of query i and key j becomes
+ * scale * q_i . k_j - m[b*H+h] * |i - j| before the mask and the softmax, and lse is the
+ * log-sum-exp of those biased scores. Other arguments and errors as fa_fwd; the slopes must
+ * be 4-byte aligned and must not overlap o or lse.
+ */
+int fa_fwd_ex(const void* q, const void* k, const void* v, const float* alibi_slopes, void* o, float* lse,
+              int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
+              fa_stream_t stream);
+
+/*
  * FP8 forward ("突破大模型训练瓶颈：Flash-Attention编译优化与内存占用解决方案", 混合精度计算:
  * FP8 inputs with q_descale / k_descale factors). q, k, v are (B,N,H,d) tensors of E4M3
  * codes (OCP 8-bit format: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits), one byte
@@ -80,6 +92,14 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_desca
                fa_stream_t stream);
 
 /*
+ * The split count fa_decode_paged uses when called with splits = 0, for B sequences, H heads
+ * and at most max_keys keys per sequence (max_pages * page_size), on the current device: about
+ * four CTAs per SM over B*H, at most one per 64-key tile and at most 128. Negative status on
+ * error (-FA_ERR_INVALID_ARG, -FA_ERR_UNSUPPORTED without an sm_100 device, -FA_ERR_CUDA).
+ */
+int fa_decode_splits(int B, int H, int max_keys);
+
+/*
  * Bytes of device workspace fa_decode_paged needs with `splits` splits per (b, h): the
  * float32 partial outputs (B,H,Sq,splits,d) and their log-sum-exps (B,H,Sq,splits), each
  * region 256-byte aligned; 0 when splits <= 1 (nothing to merge) or for invalid sizes.
@@ -94,6 +114,11 @@ size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits);
  *                position seqlens[b] - Sq + i (the new tokens are already in the cache).
  *   k_cache,
  *   v_cache      (num_pages,page_size,H,d) bf16 page pools; page_size a multiple of 64.
+ *   k_new,
+ *   v_new        NULL, or (B,Sq,H,d) bf16 rows of the new tokens: written into the caches at
+ *                positions seqlens[b] - Sq + i (as flash_attn_with_kvcache updates its cache in
+ *                place) before the attention reads them. Both or neither; they, q, o, lse, the
+ *                block table and the lengths must not overlap the caches.
  *   block_table  device (B,max_pages) int32: key j of sequence b is row j % page_size of page
  *                block_table[b*max_pages + j/page_size].
  *   seqlens      device (B) int32: keys held by sequence b (0 <= seqlens[b] <= max_pages*page_size).
@@ -104,13 +129,13 @@ size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits);
  * merged by log-sum-exp; 0 chooses a count from B*H and the SM count. With splits > 1 a
  * workspace of fa_decode_workspace_bytes(B,Sq,H,d,splits) bytes (256-byte aligned) is used; if
  * `workspace` is NULL the call allocates it with cudaMallocAsync/cudaFreeAsync on `stream`.
- * One or two launches on `stream`. Sequence lengths or page indices that are out of range are
+ * One to three launches on `stream` (append, split kernel, merge). Sequence lengths or page indices that are out of range are
  * not read: the sequence counts as empty (or the page as zeros) and fa_check() returns
  * FA_ERR_DEVICE. Host-visible errors as fa_fwd; Sq > 8 or a page_size that is not a multiple
  * of 64 give FA_ERR_UNSUPPORTED.
  */
-int fa_decode_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table,
-                    const int* seqlens, void* o, float* lse,
+int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                    const int* block_table, const int* seqlens, void* o, float* lse,
                     int B, int Sq, int H, int d, int num_pages, int page_size, int max_pages,
                     float scale, int causal, int win_l, int win_r, int splits,
                     void* workspace, size_t workspace_bytes, fa_stream_t stream);
@@ -148,6 +173,17 @@ int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void
                          const void* dO, void* dq, void* dk, void* dv,
                          int B, int N, int H, int d, float scale, int causal, int win_l, int win_r,
                          void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * Backward of fa_fwd_ex: alibi_slopes as there (NULL for none; the slopes are constants of
+ * the call and get no gradient), o and lse from fa_fwd_ex with the same slopes;
+ * deterministic != 0 selects the algorithm of fa_bwd_deterministic, 0 that of fa_bwd. Other
+ * arguments, workspace and errors as fa_bwd.
+ */
+int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+              const float* alibi_slopes, void* dq, void* dk, void* dv,
+              int B, int N, int H, int d, float scale, int causal, int win_l, int win_r, int deterministic,
+              void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * The three launches of fa_bwd, exposed so that a caller can time or interleave them.

@@ -97,3 +97,27 @@ def test_decode_out_of_range_length_is_reported_not_read():
     assert e.value.status == 6  # FA_ERR_DEVICE
     assert torch.isinf(lse[1]).all() and (o[1] == 0).all()  # the bad sequence counts as empty
     fa.check()  # the error word was cleared; the context is usable
+
+
+@pytest.mark.parametrize("Sq", [1, 3])
+def test_decode_appends_new_rows_in_place(Sq):
+    """k_new / v_new are written into the caches at positions len - Sq + i, then attended."""
+    cfg = DecodeConfig("append", 3, Sq, 2, 128, 2, 600, 128, True, seed=66 + Sq)
+    q, kc, vc, table, lens = make_decode_inputs(cfg)
+    g = torch.Generator().manual_seed(9)
+    k_new = torch.randn((cfg.B, Sq, cfg.H, cfg.d), generator=g).to(torch.bfloat16)
+    v_new = torch.randn((cfg.B, Sq, cfg.H, cfg.d), generator=g).to(torch.bfloat16)
+    kc_d, vc_d = kc.cuda(), vc.cuda()
+    o, lse = fa.attention_decode_paged(q.cuda(), kc_d, vc_d, table.cuda(), lens.cuda(), cfg.scale, True, (-1, -1), 0,
+                                       k_new=k_new.cuda(), v_new=v_new.cuda())
+    fa.check()
+    o_ref, lse_ref = oracle_dec.decode_forward(q.double().numpy(), kc.double().numpy(), vc.double().numpy(),
+                                               table.numpy(), lens.numpy(), cfg.scale, True,
+                                               k_new=k_new.double().numpy(), v_new=v_new.double().numpy())
+    assert_fwd_close(o.double().cpu().numpy(), lse.double().cpu().numpy(), o_ref, lse_ref, f"append Sq={Sq}")
+    # the caches now hold the new rows at their positions and are unchanged elsewhere
+    k_exp = oracle_dec.append_rows(kc.double().numpy(), k_new.double().numpy(), table.numpy(), lens.numpy(),
+                                   cfg.page_size)
+    v_exp = oracle_dec.append_rows(vc.double().numpy(), v_new.double().numpy(), table.numpy(), lens.numpy(),
+                                   cfg.page_size)
+    assert np.array_equal(kc_d.double().cpu().numpy(), k_exp) and np.array_equal(vc_d.double().cpu().numpy(), v_exp)
