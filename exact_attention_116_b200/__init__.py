@@ -9,9 +9,11 @@ from .binding import (  # noqa: F401
     FaError,
     FlashAttention,
     attention_bwd,
+    attention_bwd_varlen,
     attention_decode_paged,
     attention_fwd,
     attention_fwd_fp8,
+    attention_fwd_varlen,
     bwd_into,
     bwd_stages,
     check,

@@ -19,8 +19,8 @@ LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
 FA_OK = 0
 STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
                 4: "FA_ERR_TIMEOUT", 5: "FA_ERR_NO_MEMORY", 6: "FA_ERR_DEVICE"}
-EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_fwd_fp8", "fa_decode_splits", "fa_decode_workspace_bytes", "fa_decode_paged",
-           "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_ex", "fa_bwd_deterministic", "fa_bwd_preprocess",
+EXPORTS = ("fa_fwd", "fa_fwd_ex", "fa_fwd_varlen", "fa_fwd_fp8", "fa_decode_splits", "fa_decode_workspace_bytes", "fa_decode_paged",
+           "fa_bwd_workspace_bytes", "fa_bwd", "fa_bwd_ex", "fa_bwd_varlen", "fa_bwd_deterministic", "fa_bwd_preprocess",
            "fa_bwd_main", "fa_bwd_dq_convert", "fa_bwd_static_workspace", "fa_check", "fa_status_string")
 
 _lib = None
@@ -44,6 +44,8 @@ def load() -> ctypes.CDLL:
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
     lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
     lib.fa_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, i, vp, sz, vp]
     lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, i, vp, sz, vp]
     lib.fa_decode_splits.argtypes = [i, i, i]
     lib.fa_decode_splits.restype = i
@@ -61,7 +63,7 @@ def load() -> ctypes.CDLL:
     lib.fa_check.argtypes = [vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
-    for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_fp8", "fa_decode_paged", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
+    for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_fp8", "fa_decode_paged", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
                  "fa_check"):
         getattr(lib, name).restype = i
     _lib = lib
@@ -336,3 +338,53 @@ def attention_decode_paged(q, k_cache, v_cache, block_table, seqlens, scale=None
     decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale, causal, window, splits, None, stream,
                       k_new, v_new)
     return o, lse
+
+
+def _check_packed(cu_seqlens, *ts):
+    total, H, d = ts[0].shape
+    for t in ts:
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != (total, H, d):
+            raise ValueError("packed tensors must be contiguous (total, H, d) bfloat16 CUDA tensors")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1 or \
+            not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous (B + 1,) int32 CUDA tensor")
+    return int(cu_seqlens.numel()) - 1, total, H, d
+
+
+def _check_head_slopes(alibi_slopes, H):
+    if alibi_slopes is None:
+        return None
+    if alibi_slopes.dtype != torch.float32 or not alibi_slopes.is_cuda or tuple(alibi_slopes.shape) != (H,) or \
+            not alibi_slopes.is_contiguous():
+        raise ValueError("alibi_slopes must be a contiguous (H,) float32 CUDA tensor for packed batches")
+    return alibi_slopes.data_ptr()
+
+
+def attention_fwd_varlen(q, k, v, cu_seqlens, scale=None, causal=False, window=(-1, -1), stream=None,
+                         alibi_slopes=None):
+    """Packed variable-length forward: q, k, v (total, H, d) bf16, cu_seqlens (B + 1,) int32.
+    Returns (o (total, H, d) bf16, lse (H, total) float32)."""
+    B, total, H, d = _check_packed(cu_seqlens, q, k, v)
+    o = torch.empty_like(q)
+    lse = torch.empty((H, total), dtype=torch.float32, device=q.device)
+    st = load().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens.data_ptr(),
+                              _check_head_slopes(alibi_slopes, H), o.data_ptr(), lse.data_ptr(), B, total, H, d,
+                              _scale(scale, d), int(bool(causal)), int(window[0]), int(window[1]),
+                              _stream_handle(stream))
+    _raise(st, "fa_fwd_varlen")
+    return o, lse
+
+
+def attention_bwd_varlen(q, k, v, o, lse, do, cu_seqlens, scale=None, causal=False, window=(-1, -1), workspace=None,
+                         stream=None, deterministic=False, alibi_slopes=None):
+    """Backward of attention_fwd_varlen: returns (dq, dk, dv), each (total, H, d) bf16."""
+    B, total, H, d = _check_packed(cu_seqlens, q, k, v, o, do)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    st = load().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                              cu_seqlens.data_ptr(), _check_head_slopes(alibi_slopes, H), dq.data_ptr(),
+                              dk.data_ptr(), dv.data_ptr(), B, total, H, d, _scale(scale, d), int(bool(causal)),
+                              int(window[0]), int(window[1]), int(bool(deterministic)), ws_ptr, ws_bytes,
+                              _stream_handle(stream))
+    _raise(st, "fa_bwd_varlen")
+    return dq, dk, dv

@@ -53,16 +53,22 @@ bool log_enabled() {
 }
 
 // Per-device set-up: SM count, sm_100 check, dynamic shared memory opt-in of every kernel.
+// Shared-memory attributes of every (ALiBi, packed) variant of the bf16 kernels of head dim D.
+template <int D, bool kAlibi, bool kVarlen>
+bool variant_attributes() {
+  const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  const int smem = fa::BwdCfg<D>::kSmemBytes, smem_dq = fa::BwdDqCfg<D>::kSmemBytes;
+  return cudaFuncSetAttribute(fa::fa_fwd_kernel<D, false, kAlibi, kVarlen>, attr, fa::FwdCfg<D>::kSmemBytes) ==
+             cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_bwd_kernel<D, true, kAlibi, kVarlen>, attr, smem) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_bwd_kernel<D, false, kAlibi, kVarlen>, attr, smem) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<D, kAlibi, kVarlen>, attr, smem_dq) == cudaSuccess;
+}
+
 template <int D>
 bool bwd_attributes() {
-  const int smem = fa::BwdCfg<D>::kSmemBytes, smem_dq = fa::BwdDqCfg<D>::kSmemBytes;
-  const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
-  return cudaFuncSetAttribute(fa::fa_bwd_kernel<D, true, false>, attr, smem) == cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_bwd_kernel<D, false, false>, attr, smem) == cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_bwd_kernel<D, true, true>, attr, smem) == cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_bwd_kernel<D, false, true>, attr, smem) == cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<D, false>, attr, smem_dq) == cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<D, true>, attr, smem_dq) == cudaSuccess;
+  return variant_attributes<D, false, false>() && variant_attributes<D, true, false>() &&
+         variant_attributes<D, false, true>() && variant_attributes<D, true, true>();
 }
 
 template <int D>
@@ -91,17 +97,9 @@ int device_setup(int* dev_out, int* sm_count) {
     g_is_sm100[dev] = (major == 10 && minor == 0);
     g_sm_count[dev] = sms;
     if (g_is_sm100[dev]) {
-      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::FwdCfg<64>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::FwdCfg<128>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(fa::fa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                fa::FwdCfg<128, true>::kSmemBytes) != cudaSuccess ||
           !decode_attributes<64>() || !decode_attributes<128>() ||
-          cudaFuncSetAttribute(fa::fa_fwd_kernel<64, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::FwdCfg<64>::kSmemBytes) != cudaSuccess ||
-          cudaFuncSetAttribute(fa::fa_fwd_kernel<128, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               fa::FwdCfg<128>::kSmemBytes) != cudaSuccess ||
           !bwd_attributes<64>() || !bwd_attributes<128>())
         return FA_ERR_CUDA;
     }
@@ -236,10 +234,41 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_
 // ---------------------------------------------------------------- launches (arguments already checked)
 
 // descales != nullptr: q, k, v hold E4M3 codes (head dim 128) with (B, H) descale factors.
+template <int D, bool kAlibi, bool kVarlen>
+void fwd_launch(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                const CUtensorMap& mo, const fa::FwdParams& p) {
+  fa::fa_fwd_kernel<D, false, kAlibi, kVarlen><<<grid, fa::FwdCfg<D>::kThreads, fa::FwdCfg<D>::kSmemBytes, stream>>>(
+      mq, mk, mv, mo, p);
+}
+
+template <int D>
+void fwd_variant(bool alibi, bool varlen, int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
+                 const CUtensorMap& mv, const CUtensorMap& mo, const fa::FwdParams& p) {
+  if (alibi && varlen) fwd_launch<D, true, true>(grid, stream, mq, mk, mv, mo, p);
+  else if (alibi) fwd_launch<D, true, false>(grid, stream, mq, mk, mv, mo, p);
+  else if (varlen) fwd_launch<D, false, true>(grid, stream, mq, mk, mv, mo, p);
+  else fwd_launch<D, false, false>(grid, stream, mq, mk, mv, mo, p);
+}
+
+// Offsets of a packed batch: cu[0] = 0, non-decreasing, cu[nseg] = n; a violation is reported
+// through fa_check (the kernels clamp every bound, so bad offsets cannot send work out of range).
+__global__ void __launch_bounds__(256) fa_check_cu_kernel(const int* cu, int nseg, int n) {
+  bool bad = false;
+  if (threadIdx.x == 0) bad = cu[0] != 0 || cu[nseg] != n;
+  for (int i = threadIdx.x; i < nseg; i += blockDim.x) bad |= cu[i + 1] < cu[i];
+  if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(&fa::g_fa_error, fa::kErrBadInput);
+}
+
+int launch_check_cu(const int* cu, int nseg, int n, cudaStream_t stream) {
+  fa_check_cu_kernel<<<1, 256, 0, stream>>>(cu, nseg, n);
+  return launch_status();
+}
+
 // alibi != nullptr: (B, H) ALiBi slopes (bf16 inputs).
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& s, float scale,
                int causal, int win_l, int win_r, int sm_count, cudaStream_t stream,
-               const float* const* descales = nullptr, const float* alibi = nullptr) {
+               const float* const* descales = nullptr, const float* alibi = nullptr, const int* cu = nullptr,
+               int nseg = 0) {
   CUtensorMap mq, mk, mv, mo;
   int st;
   auto in_map = descales ? make_map_u8 : make_map;
@@ -247,6 +276,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
       (st = make_map(&mo, o, s)))
     return st;
   fa::FwdParams p;
+  p.cu_seqlens = cu;
+  p.nseg = nseg;
   p.q_descale = descales ? descales[0] : nullptr;
   p.k_descale = descales ? descales[1] : nullptr;
   p.v_descale = descales ? descales[2] : nullptr;
@@ -273,17 +304,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   if (descales)
     fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128, true>::kThreads, fa::FwdCfg<128, true>::kSmemBytes,
                                    stream>>>(mq, mk, mv, mo, p);
-  else if (alibi && s.d == 64)
-    fa::fa_fwd_kernel<64, false, true><<<grid, fa::FwdCfg<64>::kThreads, fa::FwdCfg<64>::kSmemBytes, stream>>>(
-        mq, mk, mv, mo, p);
-  else if (alibi)
-    fa::fa_fwd_kernel<128, false, true><<<grid, fa::FwdCfg<128>::kThreads, fa::FwdCfg<128>::kSmemBytes, stream>>>(
-        mq, mk, mv, mo, p);
   else if (s.d == 64)
-    fa::fa_fwd_kernel<64><<<grid, fa::FwdCfg<64>::kThreads, fa::FwdCfg<64>::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+    fwd_variant<64>(alibi != nullptr, cu != nullptr, grid, stream, mq, mk, mv, mo, p);
   else
-    fa::fa_fwd_kernel<128><<<grid, fa::FwdCfg<128>::kThreads, fa::FwdCfg<128>::kSmemBytes, stream>>>(mq, mk, mv, mo,
-                                                                                                     p);
+    fwd_variant<128>(alibi != nullptr, cu != nullptr, grid, stream, mq, mk, mv, mo, p);
   return launch_status();
 }
 
@@ -302,10 +326,19 @@ int launch_pre(const void* o, const float* lse, const void* dO, const Shape& s, 
   return launch_status();
 }
 
+// Packed sequences travel with the backward's other options.
+struct BwdOptions {
+  const float* alibi = nullptr;
+  const int* cu = nullptr;
+  int nseg = 0;
+};
+
 fa::BwdParams bwd_params(const Shape& s, float scale, int causal, int win_l, int win_r, const Workspace& w,
-                         const float* alibi = nullptr) {
+                         const BwdOptions& opt) {
   fa::BwdParams p;
-  p.alibi_slopes = alibi;
+  p.alibi_slopes = opt.alibi;
+  p.cu_seqlens = opt.cu;
+  p.nseg = opt.nseg;
   p.B = s.B;
   p.N = s.N;
   p.H = s.H;
@@ -324,69 +357,83 @@ fa::BwdParams bwd_params(const Shape& s, float scale, int causal, int win_l, int
   return p;
 }
 
+template <int D, bool kDQ, bool kAlibi, bool kVarlen>
+void main_launch(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                 const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv, const CUtensorMap& mdq,
+                 const fa::BwdParams& p) {
+  fa::fa_bwd_kernel<D, kDQ, kAlibi, kVarlen><<<grid, fa::BwdCfg<D>::kThreads, fa::BwdCfg<D>::kSmemBytes, stream>>>(
+      mq, mk, mv, mdo, mdk, mdv, mdq, p);
+}
+
 template <int D, bool kDQ>
-void main_kernel(bool alibi, int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
+void main_kernel(bool alibi, bool varlen, int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
                  const CUtensorMap& mv, const CUtensorMap& mdo, const CUtensorMap& mdk, const CUtensorMap& mdv,
                  const CUtensorMap& mdq, const fa::BwdParams& p) {
-  if (alibi)
-    fa::fa_bwd_kernel<D, kDQ, true><<<grid, fa::BwdCfg<D>::kThreads, fa::BwdCfg<D>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdk, mdv, mdq, p);
-  else
-    fa::fa_bwd_kernel<D, kDQ, false><<<grid, fa::BwdCfg<D>::kThreads, fa::BwdCfg<D>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  if (alibi && varlen) main_launch<D, kDQ, true, true>(grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  else if (alibi) main_launch<D, kDQ, true, false>(grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  else if (varlen) main_launch<D, kDQ, false, true>(grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
+  else main_launch<D, kDQ, false, false>(grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
+}
+
+template <int D, bool kAlibi, bool kVarlen>
+void dq_launch(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const CUtensorMap& mdo, const CUtensorMap& mdq, const fa::BwdParams& p) {
+  fa::fa_bwd_dq_kernel<D, kAlibi, kVarlen><<<grid, fa::BwdDqCfg<D>::kThreads, fa::BwdDqCfg<D>::kSmemBytes, stream>>>(
+      mq, mk, mv, mdo, mdq, p);
+}
+
+template <int D>
+void dq_kernel(bool alibi, bool varlen, int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
+               const CUtensorMap& mv, const CUtensorMap& mdo, const CUtensorMap& mdq, const fa::BwdParams& p) {
+  if (alibi && varlen) dq_launch<D, true, true>(grid, stream, mq, mk, mv, mdo, mdq, p);
+  else if (alibi) dq_launch<D, true, false>(grid, stream, mq, mk, mv, mdo, mdq, p);
+  else if (varlen) dq_launch<D, false, true>(grid, stream, mq, mk, mv, mdo, mdq, p);
+  else dq_launch<D, false, false>(grid, stream, mq, mk, mv, mdo, mdq, p);
 }
 
 // Main backward kernel; with_dq = false computes dK and dV only (the deterministic backward).
 int launch_main(const void* q, const void* k, const void* v, const void* dO, void* dk, void* dv, const Shape& s,
                 float scale, int causal, int win_l, int win_r, const Workspace& w, int sm_count,
-                cudaStream_t stream, bool with_dq = true, const float* alibi = nullptr) {
+                cudaStream_t stream, bool with_dq = true, const BwdOptions& opt = BwdOptions()) {
   CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
   int st;
   if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
       (st = make_map(&mdo, dO, s)) || (st = make_map(&mdk, dk, s)) || (st = make_map(&mdv, dv, s)) ||
       (st = make_map_f32_acc(&mdq, w.dq_acc, s)))
     return st;
-  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, alibi);
+  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, opt);
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   if (log_enabled())
     std::fprintf(stderr, "[fa] bwd B=%d N=%d H=%d d=%d causal=%d win=(%d,%d) items=%d grid=%d smem=%d\n", s.B, s.N,
                  s.H, s.d, p.causal, win_l, win_r, p.num_items, grid,
                  s.d == 64 ? fa::BwdCfg<64>::kSmemBytes : fa::BwdCfg<128>::kSmemBytes);
-  const bool a = alibi != nullptr;
+  const bool a = opt.alibi != nullptr, vl = opt.cu != nullptr;
   if (s.d == 64 && with_dq)
-    main_kernel<64, true>(a, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    main_kernel<64, true>(a, vl, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
   else if (s.d == 64)
-    main_kernel<64, false>(a, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    main_kernel<64, false>(a, vl, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
   else if (with_dq)
-    main_kernel<128, true>(a, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    main_kernel<128, true>(a, vl, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
   else
-    main_kernel<128, false>(a, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
+    main_kernel<128, false>(a, vl, grid, stream, mq, mk, mv, mdo, mdk, mdv, mdq, p);
   return launch_status();
 }
 
 // dQ of the deterministic backward: one item per (b, h, Q tile), dQ accumulated in TMEM.
 int launch_dq(const void* q, const void* k, const void* v, const void* dO, void* dq, const Shape& s, float scale,
               int causal, int win_l, int win_r, const Workspace& w, int sm_count, cudaStream_t stream,
-              const float* alibi = nullptr) {
+              const BwdOptions& opt = BwdOptions()) {
   CUtensorMap mq, mk, mv, mdo, mdq;
   int st;
   if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
       (st = make_map(&mdo, dO, s)) || (st = make_map(&mdq, dq, s)))
     return st;
-  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, alibi);
+  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, opt);
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
-  if (s.d == 64 && alibi)
-    fa::fa_bwd_dq_kernel<64, true><<<grid, fa::BwdDqCfg<64>::kThreads, fa::BwdDqCfg<64>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdq, p);
-  else if (s.d == 64)
-    fa::fa_bwd_dq_kernel<64, false><<<grid, fa::BwdDqCfg<64>::kThreads, fa::BwdDqCfg<64>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdq, p);
-  else if (alibi)
-    fa::fa_bwd_dq_kernel<128, true><<<grid, fa::BwdDqCfg<128>::kThreads, fa::BwdDqCfg<128>::kSmemBytes, stream>>>(
-        mq, mk, mv, mdo, mdq, p);
+  if (s.d == 64)
+    dq_kernel<64>(opt.alibi != nullptr, opt.cu != nullptr, grid, stream, mq, mk, mv, mdo, mdq, p);
   else
-    fa::fa_bwd_dq_kernel<128, false><<<grid, fa::BwdDqCfg<128>::kThreads, fa::BwdDqCfg<128>::kSmemBytes,
-                                        stream>>>(mq, mk, mv, mdo, mdq, p);
+    dq_kernel<128>(opt.alibi != nullptr, opt.cu != nullptr, grid, stream, mq, mk, mv, mdo, mdq, p);
   return launch_status();
 }
 
@@ -487,6 +534,30 @@ int fa_fwd_ex(const void* q, const void* k, const void* v, const float* alibi_sl
   if ((st = device_setup(&dev, &sms))) return st;
   return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream),
                     nullptr, alibi_slopes);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, const int* cu_seqlens, const float* alibi_slopes,
+                  void* o, float* lse, int B, int total, int H, int d, float scale, int causal, int win_l,
+                  int win_r, fa_stream_t stream) {
+  if (B < 1 || !cu_seqlens || !aligned(cu_seqlens, 4)) return FA_ERR_INVALID_ARG;
+  int st = check_problem(1, total, H, d, scale, causal, &win_l, &win_r);
+  if (st) return st;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(alibi_slopes, 4))
+    return FA_ERR_INVALID_ARG;
+  const Shape s{1, total, H, d};
+  const size_t tb = s.tensor_bytes(), lb = s.rowvec_bytes(), ab = (size_t)H * 4, cb = (size_t)(B + 1) * 4;
+  const void* ins[5] = {q, k, v, cu_seqlens, alibi_slopes};
+  const size_t in_bytes[5] = {tb, tb, tb, cb, alibi_slopes ? ab : 0};
+  for (int i = 0; i < 5; ++i)
+    if (overlap(o, tb, ins[i], in_bytes[i]) || overlap(lse, lb, ins[i], in_bytes[i])) return FA_ERR_INVALID_ARG;
+  if (overlap(o, tb, lse, lb)) return FA_ERR_INVALID_ARG;
+  int dev, sms;
+  if ((st = device_setup(&dev, &sms))) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = launch_check_cu(cu_seqlens, B, total, cs))) return st;
+  return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, cs, nullptr, alibi_slopes, cu_seqlens, B);
 }
 
 int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale, const float* k_descale,
@@ -722,7 +793,7 @@ int fa_bwd_dq_convert(void* dq, int B, int N, int H, int d, void* workspace, siz
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                     void* dq, void* dk, void* dv, int B, int N, int H, int d, float scale, int causal, int win_l,
                     int win_r, void* workspace, size_t workspace_bytes_, fa_stream_t stream, bool deterministic,
-                    const float* alibi = nullptr) {
+                    const float* alibi = nullptr, const int* cu = nullptr, int nseg = 0) {
   int st = check_problem(B, N, H, d, scale, causal, &win_l, &win_r);
   if (st) return st;
   const Shape s{B, N, H, d};
@@ -768,11 +839,16 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   }
   const Workspace w = carve(ws, s);
   st = launch_pre(o, lse, dO, s, w, cs);
+  BwdOptions opt;
+  opt.alibi = alibi;
+  opt.cu = cu;
+  opt.nseg = nseg;
+  if (!st && cu) st = launch_check_cu(cu, nseg, N, cs);
   if (deterministic) {
-    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs, false, alibi);
-    if (!st) st = launch_dq(q, k, v, dO, dq, s, scale, causal, win_l, win_r, w, sms, cs, alibi);
+    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs, false, opt);
+    if (!st) st = launch_dq(q, k, v, dO, dq, s, scale, causal, win_l, win_r, w, sms, cs, opt);
   } else {
-    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs, true, alibi);
+    if (!st) st = launch_main(q, k, v, dO, dk, dv, s, scale, causal, win_l, win_r, w, sms, cs, true, opt);
     if (!st) st = launch_convert(dq, s, w, cs);
   }
   if (!workspace && cudaFreeAsync(ws, cs) != cudaSuccess && !st) st = FA_ERR_CUDA;
@@ -794,6 +870,19 @@ int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const 
               fa_stream_t stream) {
   return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, B, N, H, d, scale, causal, win_l, win_r, workspace,
                   workspace_bytes_, stream, deterministic != 0, alibi_slopes);
+}
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                  const int* cu_seqlens, const float* alibi_slopes, void* dq, void* dk, void* dv, int B, int total,
+                  int H, int d, float scale, int causal, int win_l, int win_r, int deterministic, void* workspace,
+                  size_t workspace_bytes_, fa_stream_t stream) {
+  if (B < 1 || !cu_seqlens || !aligned(cu_seqlens, 4)) return FA_ERR_INVALID_ARG;
+  const size_t tb = (size_t)total * H * d * 2, cb = (size_t)(B + 1) * 4;
+  void* outs[3] = {dq, dk, dv};
+  for (void* out : outs)
+    if (out && total > 0 && H > 0 && d > 0 && overlap(out, tb, cu_seqlens, cb)) return FA_ERR_INVALID_ARG;
+  return bwd_impl(q, k, v, o, lse, dO, dq, dk, dv, 1, total, H, d, scale, causal, win_l, win_r, workspace,
+                  workspace_bytes_, stream, deterministic != 0, alibi_slopes, cu_seqlens, B);
 }
 
 int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,

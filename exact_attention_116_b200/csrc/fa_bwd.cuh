@@ -46,6 +46,8 @@ struct BwdParams {
   const float* dvec;   // (B, H, N_pad) fp32: -rowsum(dO * O)
   int* next_item;      // work counters (zeroed by the preprocess kernel): [0] main kernel, [1] dQ kernel
   const float* alibi_slopes;  // ALiBi only: (B, H) slopes m, bias -m |i - j| on the scaled scores
+  const int* cu_seqlens;      // packed variable-length batch (B = 1, N = total): nseg + 1 offsets, or null
+  int nseg;
 };
 
 // Heads per scheduling group: items of a group are handed out before the next group's, so the
@@ -189,20 +191,30 @@ __device__ __forceinline__ int bwd_take_item(BwdBars* bars, uint32_t n, bool arr
 }
 
 // Q tiles whose rows see any key of KV tile j.
+template <bool kVarlen>
 __device__ __forceinline__ void bwd_q_range(const BwdParams& p, int j, int& lo, int& hi) {
   const int k0 = j * 128;
   const int k1 = min(k0 + 127, p.N - 1);
-  const int qlo = p.win_r >= 0 ? max(0, k0 - p.win_r) : 0;
-  const int qhi = p.win_l >= 0 ? min(p.N - 1, k1 + p.win_l) : p.N - 1;
+  int first = 0, last = p.N - 1, dummy;
+  if (kVarlen) {  // packed sequences: the first key's sequence start to the last key's end
+    seg_bounds(p.cu_seqlens, p.nseg, p.N, k0, first, dummy);
+    seg_bounds(p.cu_seqlens, p.nseg, p.N, k1, dummy, last);
+  }
+  const int qlo = p.win_r >= 0 ? max(first, k0 - p.win_r) : first;
+  const int qhi = p.win_l >= 0 ? min(last, k1 + p.win_l) : last;
   lo = qlo >> 7;
   hi = qhi >> 7;
 }
 
-__device__ __forceinline__ bool bwd_tile_unmasked(const BwdParams& p, int j, int i) {
+// Packed sequences (kVarlen): [seg_first, seg_last] are the rows of the sequence of key j * 128.
+template <bool kVarlen>
+__device__ __forceinline__ bool bwd_tile_unmasked(const BwdParams& p, int j, int i, int seg_first = 0,
+                                                  int seg_last = 0) {
   const int k0 = j * 128, k1 = k0 + 127, q0 = i * 128, q1 = q0 + 127;
   if (k1 >= p.N || q1 >= p.N) return false;
   if (p.win_l >= 0 && k0 < q1 - p.win_l) return false;
   if (p.win_r >= 0 && k1 > q0 + p.win_r) return false;
+  if (kVarlen && (k1 > seg_last || q0 < seg_first || q1 > seg_last)) return false;  // one sequence only
   return true;
 }
 
@@ -244,7 +256,7 @@ __device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[32], const uint32
   }
 }
 
-template <int D, bool kDQ, bool kAlibi = false>
+template <int D, bool kDQ, bool kAlibi = false, bool kVarlen = false>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -326,7 +338,7 @@ __global__ void __launch_bounds__(512, 1)
         int b, h, j;
         bwd_decode(p, w, b, h, j);
         int lo, hi;
-        bwd_q_range(p, j, lo, hi);
+        bwd_q_range<kVarlen>(p, j, lo, hi);
         mbar_wait(bar(bars->kv_empty), (items & 1) ^ 1, ab);
         mbar_arrive_expect_tx(bar(bars->kv_full), 2 * Cfg::kTileBytes);
 #pragma unroll
@@ -388,7 +400,7 @@ __global__ void __launch_bounds__(512, 1)
         int b, h, j;
         bwd_decode(p, w, b, h, j);
         int lo, hi;
-        bwd_q_range(p, j, lo, hi);
+        bwd_q_range<kVarlen>(p, j, lo, hi);
         mbar_wait(bar(bars->kv_full), items & 1, ab);
         tc_fence_after_sync();
         issue_s(qs, qphase);  // S(lo)
@@ -456,7 +468,7 @@ __global__ void __launch_bounds__(512, 1)
       int b, h, j;
       bwd_decode(p, w, b, h, j);
       int lo, hi;
-      bwd_q_range(p, j, lo, hi);
+      bwd_q_range<kVarlen>(p, j, lo, hi);
       // Without kDQ, dQ comes from its own kernel: these warps only follow the items.
       for (int i = lo; kDQ && i <= hi; ++i, ++n) {
         mbar_wait(bar(bars->dq_full), n & 1, ab);
@@ -511,17 +523,21 @@ __global__ void __launch_bounds__(512, 1)
       int b, h, j;
       bwd_decode(p, w, b, h, j);
       int lo, hi;
-      bwd_q_range(p, j, lo, hi);
+      bwd_q_range<kVarlen>(p, j, lo, hi);
       const int k = j * 128 + row;
       const float nslope2 = kAlibi ? -p.alibi_slopes[b * p.H + h] * kLog2e : 0.0f;
-      const int qlo = p.win_r >= 0 ? k - p.win_r : 0;
-      const int qhi = (k >= p.N) ? -1 : (p.win_l >= 0 ? min(p.N - 1, k + p.win_l) : p.N - 1);
+      int first = 0, last = p.N - 1;
+      if (kVarlen && k < p.N) seg_bounds(p.cu_seqlens, p.nseg, p.N, k, first, last);
+      int seg_first = 0, seg_last = 0;  // sequence of the tile's first key (packed batches)
+      if (kVarlen) seg_bounds(p.cu_seqlens, p.nseg, p.N, j * 128, seg_first, seg_last);
+      const int qlo = p.win_r >= 0 ? max(first, k - p.win_r) : first;
+      const int qhi = (k >= p.N) ? -1 : (p.win_l >= 0 ? min(last, k + p.win_l) : last);
       for (int i = lo; i <= hi; ++i, ++n) {
         // the Q slot's LSE2_i / D_i rows are read here
         mbar_wait(bar(bars->q_full[qs]), qphase, ab);
         const float* nlse2 = reinterpret_cast<const float*>(smem_raw + Cfg::kOffStat + qs * 1024);  // -LSE*log2(e)
         const float* nd = nlse2 + 128;                                                              // -D
-        const bool masked = !bwd_tile_unmasked(p, j, i);
+        const bool masked = !bwd_tile_unmasked<kVarlen>(p, j, i, seg_first, seg_last);
         const int qbase = i * 128 + 64 * grp;
 
         mbar_wait(bar(bars->s_full), n & 1, ab);

@@ -86,10 +86,12 @@ __device__ __forceinline__ FwdParams bwd_dq_as_fwd(const BwdParams& p) {
   f.win_l = p.win_l;
   f.win_r = p.win_r;
   f.causal = p.causal;
+  f.cu_seqlens = p.cu_seqlens;
+  f.nseg = p.nseg;
   return f;
 }
 
-template <int D, bool kAlibi = false>
+template <int D, bool kAlibi = false, bool kVarlen = false>
 __global__ void __launch_bounds__(256, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -157,7 +159,7 @@ __global__ void __launch_bounds__(256, 1)
         int b, h, i;
         bwd_dq_decode(p, w, b, h, i);
         int lo, hi;
-        fwd_kv_range(fp, i * 128, lo, hi);
+        fwd_kv_range<kVarlen>(fp, i * 128, lo, hi);
         mbar_wait(bar(bars->q_empty), (qn & 1) ^ 1, ab);
         mbar_arrive_expect_tx(bar(bars->q_full), 2 * Cfg::kTileBytes);
 #pragma unroll
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(256, 1)
         int b, h, i;
         bwd_dq_decode(p, w, b, h, i);
         int lo, hi;
-        fwd_kv_range(fp, i * 128, lo, hi);
+        fwd_kv_range<kVarlen>(fp, i * 128, lo, hi);
         mbar_wait(bar(bars->q_full), qn & 1, ab);
         tc_fence_after_sync();
         uint32_t k_slot, v_slot;
@@ -264,16 +266,23 @@ __global__ void __launch_bounds__(256, 1)
       int b, h, i;
       bwd_dq_decode(p, w, b, h, i);
       int lo, hi;
-      fwd_kv_range(fp, i * 128, lo, hi);
+      fwd_kv_range<kVarlen>(fp, i * 128, lo, hi);
       const int q = i * 128 + row;
       const size_t stat = ((size_t)b * p.H + h) * (size_t)p.N_pad + q;  // padded rows hold 0
       const float nlse2 = p.lse2[stat];                                 // -LSE * log2(e)
       const float nd = p.dvec[stat];                                     // -D
       const float nslope2 = kAlibi ? -p.alibi_slopes[b * p.H + h] * kLog2e : 0.0f;  // ALiBi: -m log2(e)
-      const int kmin = p.win_l >= 0 ? q - p.win_l : 0;
-      const int kmax = (q >= p.N) ? -1 : (p.win_r >= 0 ? min(p.N - 1, q + p.win_r) : p.N - 1);
+      int kmin, kmax;
+      if constexpr (kVarlen) {
+        fwd_row_keys<true>(fp, q, kmin, kmax);
+      } else {
+        kmin = p.win_l >= 0 ? q - p.win_l : 0;
+        kmax = (q >= p.N) ? -1 : (p.win_r >= 0 ? min(p.N - 1, q + p.win_r) : p.N - 1);
+      }
+      int seg_first = 0, seg_last = 0;  // sequence of the tile's first row (packed batches)
+      if (kVarlen) seg_bounds(p.cu_seqlens, p.nseg, p.N, i * 128, seg_first, seg_last);
       for (int j = lo; j <= hi; ++j, ++n) {
-        const bool masked = !fwd_tile_unmasked(fp, i * 128, j) || (i * 128 + 127 >= p.N);
+        const bool masked = !fwd_tile_unmasked<kVarlen>(fp, i * 128, j, seg_first, seg_last) || (i * 128 + 127 >= p.N);
         mbar_wait(bar(bars->s_full), n & 1, ab);
         tc_fence_after_sync();
         uint32_t pk[64];  // P(q, keys) as bf16 pairs

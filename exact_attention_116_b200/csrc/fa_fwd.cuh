@@ -50,6 +50,8 @@ struct FwdParams {
   const float* k_descale;
   const float* v_descale;
   const float* alibi_slopes;  // ALiBi only: (B, H) slopes m, bias -m |i - j| on the scaled scores
+  const int* cu_seqlens;      // packed variable-length batch (B = 1, N = total): nseg + 1 offsets, or null
+  int nseg;
 };
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
@@ -114,22 +116,43 @@ __device__ __forceinline__ void fwd_decode(const FwdParams& p, int w, int& b, in
 }
 
 // KV tiles visible from Q rows [r0, min(r0+127, N-1)]; empty (hi < lo) if r0 >= N.
+// Packed sequences (kVarlen): the keys of the first row's sequence start to the last row's
+// sequence end.
+template <bool kVarlen>
 __device__ __forceinline__ void fwd_kv_range(const FwdParams& p, int r0, int& lo, int& hi) {
   if (r0 >= p.N) { lo = 0; hi = -1; return; }
   const int r1 = min(r0 + 127, p.N - 1);
-  const int kmin = p.win_l >= 0 ? max(0, r0 - p.win_l) : 0;
-  const int kmax = p.win_r >= 0 ? min(p.N - 1, r1 + p.win_r) : p.N - 1;
+  int first = 0, last = p.N - 1, dummy;
+  if (kVarlen) {
+    seg_bounds(p.cu_seqlens, p.nseg, p.N, r0, first, dummy);
+    seg_bounds(p.cu_seqlens, p.nseg, p.N, r1, dummy, last);
+  }
+  const int kmin = p.win_l >= 0 ? max(first, r0 - p.win_l) : first;
+  const int kmax = p.win_r >= 0 ? min(last, r1 + p.win_r) : last;
   lo = kmin >> 7;
   hi = kmax >> 7;
 }
 
+// Visible keys [kmin, kmax] of query row i (its own sequence only when packed).
+template <bool kVarlen>
+__device__ __forceinline__ void fwd_row_keys(const FwdParams& p, int i, int& kmin, int& kmax) {
+  int first = 0, last = p.N - 1;
+  if (kVarlen && i < p.N) seg_bounds(p.cu_seqlens, p.nseg, p.N, i, first, last);
+  kmin = p.win_l >= 0 ? max(first, i - p.win_l) : first;
+  kmax = (i >= p.N) ? -1 : (p.win_r >= 0 ? min(last, i + p.win_r) : last);
+}
+
 // True when every valid row of the Q tile sees every key of KV tile j (no masking needed).
-__device__ __forceinline__ bool fwd_tile_unmasked(const FwdParams& p, int r0, int j) {
+// Packed sequences (kVarlen): [seg_first, seg_last] are the rows of the sequence of row r0.
+template <bool kVarlen>
+__device__ __forceinline__ bool fwd_tile_unmasked(const FwdParams& p, int r0, int j, int seg_first = 0,
+                                                  int seg_last = 0) {
   const int r1 = min(r0 + 127, p.N - 1);
   const int k0 = j * 128, k1 = k0 + 127;
   if (k1 >= p.N) return false;
   if (p.win_l >= 0 && k0 < r1 - p.win_l) return false;
   if (p.win_r >= 0 && k1 > r0 + p.win_r) return false;
+  if (kVarlen && (r1 > seg_last || k0 < seg_first || k1 > seg_last)) return false;  // one sequence only
   return true;
 }
 
@@ -230,7 +253,7 @@ __device__ __forceinline__ float lg2_approx(float x) {
   return y;
 }
 
-template <int D, bool kF8 = false, bool kAlibi = false>
+template <int D, bool kF8 = false, bool kAlibi = false, bool kVarlen = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -239,6 +262,7 @@ __global__ void __launch_bounds__(384, 1)
   using Bars = FwdBars<Cfg>;
   static_assert(!kF8 || D == 128, "E4M3 inputs: head dim 128 (one 128-byte row per TMA box)");
   static_assert(!(kF8 && kAlibi), "ALiBi is built for bf16 inputs");
+  static_assert(!(kF8 && kVarlen), "packed batches are built for bf16 inputs");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
@@ -298,8 +322,8 @@ __global__ void __launch_bounds__(384, 1)
         int b, h, pair;
         fwd_decode(p, w, b, h, pair);
         int lo_t[2], hi_t[2];
-        fwd_kv_range(p, pair * 256, lo_t[0], hi_t[0]);
-        fwd_kv_range(p, pair * 256 + 128, lo_t[1], hi_t[1]);
+        fwd_kv_range<kVarlen>(p, pair * 256, lo_t[0], hi_t[0]);
+        fwd_kv_range<kVarlen>(p, pair * 256 + 128, lo_t[1], hi_t[1]);
         const bool act1 = hi_t[1] >= lo_t[1];
         const int lo = act1 ? min(lo_t[0], lo_t[1]) : lo_t[0];
         const int hi = act1 ? max(hi_t[0], hi_t[1]) : hi_t[0];
@@ -375,8 +399,8 @@ __global__ void __launch_bounds__(384, 1)
         int b, h, pair;
         fwd_decode(p, w, b, h, pair);
         int lo_t[2], hi_t[2];
-        fwd_kv_range(p, pair * 256, lo_t[0], hi_t[0]);
-        fwd_kv_range(p, pair * 256 + 128, lo_t[1], hi_t[1]);
+        fwd_kv_range<kVarlen>(p, pair * 256, lo_t[0], hi_t[0]);
+        fwd_kv_range<kVarlen>(p, pair * 256 + 128, lo_t[1], hi_t[1]);
         const bool act[2] = {true, hi_t[1] >= lo_t[1]};
         const int lo = act[1] ? min(lo_t[0], lo_t[1]) : lo_t[0];
         const int hi = act[1] ? max(hi_t[0], hi_t[1]) : hi_t[0];
@@ -504,7 +528,7 @@ __global__ void __launch_bounds__(384, 1)
       fwd_decode(p, w, b, h, pair);
       const int r0 = pair * 256 + t * 128;
       int lo, hi;
-      fwd_kv_range(p, r0, lo, hi);
+      fwd_kv_range<kVarlen>(p, r0, lo, hi);
       if (hi < lo) continue;
       float c = p.scale_log2, o_mul = 1.0f;  // log2-domain score factor; O factor
       float nslope2 = 0.0f;                  // ALiBi: -m log2(e)
@@ -515,8 +539,15 @@ __global__ void __launch_bounds__(384, 1)
         o_mul = p.v_descale[bh];
       }
       const int i = r0 + row;
-      const int kmin = p.win_l >= 0 ? i - p.win_l : 0;
-      const int kmax = p.win_r >= 0 ? min(p.N - 1, i + p.win_r) : p.N - 1;
+      int kmin, kmax;
+      if constexpr (kVarlen) {
+        fwd_row_keys<true>(p, i, kmin, kmax);
+      } else {
+        kmin = p.win_l >= 0 ? i - p.win_l : 0;
+        kmax = p.win_r >= 0 ? min(p.N - 1, i + p.win_r) : p.N - 1;
+      }
+      int seg_first = 0, seg_last = 0;  // sequence of the tile's first row (packed batches)
+      if (kVarlen) seg_bounds(p.cu_seqlens, p.nseg, p.N, r0, seg_first, seg_last);
       float m_run = -INFINITY, l_run = 0.0f;
 
       for (int j = lo; j <= hi; ++j) {
@@ -536,7 +567,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int cc = 0; cc < 128; ++cc) x[cc] = __uint_as_float(r[cc >> 5][cc & 31]);
 
-        const bool masked = !fwd_tile_unmasked(p, r0, j);
+        const bool masked = !fwd_tile_unmasked<kVarlen>(p, r0, j, seg_first, seg_last);
         float alpha;
         bool updated;
         const bool pos_scale = !kAlibi && c > 0.0f;  // with ALiBi the scores are scaled before the max

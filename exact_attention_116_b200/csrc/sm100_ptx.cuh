@@ -23,6 +23,26 @@ __device__ int g_fa_error = 0;
 
 constexpr float kLog2e = 1.4426950408889634074f;
 
+// Packed variable-length batches: sequence b holds rows [cu[b], cu[b+1]) of the token axis.
+// seg_of returns the sequence of `row` (the largest b < nseg with cu[b] <= row); seg_bounds
+// gives its first and last row, clamped into [0, n - 1] so that malformed offsets (reported
+// separately) can only shrink the work, never send it out of range.
+__device__ __forceinline__ int seg_of(const int* cu, int nseg, int row) {
+  int lo = 0, hi = nseg - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= row) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void seg_bounds(const int* cu, int nseg, int n, int row, int& first, int& last) {
+  const int s = seg_of(cu, nseg, row);
+  first = min(max(__ldg(cu + s), 0), n - 1);
+  last = min(max(__ldg(cu + s + 1) - 1, 0), n - 1);
+}
+
 enum DeviceError : int {
   kErrWaitTimeout = 1,  // a bounded mbarrier wait gave up
   kErrSmemAlign = 2,    // dynamic shared memory not at the alignment a kernel's layout needs

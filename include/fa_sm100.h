@@ -75,6 +75,21 @@ int fa_fwd_ex(const void* q, const void* k, const void* v, const float* alibi_sl
               fa_stream_t stream);
 
 /*
+ * Variable-length batch ("Flash Attention V2核心网络算子解析" §五: variable sequence lengths):
+ * B sequences packed along the token axis, sequence b in rows [cu_seqlens[b], cu_seqlens[b+1])
+ * of (total,H,d) bf16 tensors q, k, v, o; cu_seqlens is a device (B+1) int32 array with
+ * cu_seqlens[0] = 0, non-decreasing, cu_seqlens[B] = total (empty sequences allowed). Each
+ * sequence is attended on its own: positions, causal mask and window count from its first
+ * token and no token sees another sequence. lse is (H,total) float32. alibi_slopes is NULL or
+ * a device (H) float32 array (one slope per head, shared by the sequences). Offsets that break
+ * the rules are reported by fa_check() as FA_ERR_DEVICE (every bound the kernels use is
+ * clamped into the packed tensor). Other arguments and errors as fa_fwd.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, const int* cu_seqlens, const float* alibi_slopes,
+                  void* o, float* lse, int B, int total, int H, int d, float scale, int causal, int win_l,
+                  int win_r, fa_stream_t stream);
+
+/*
  * FP8 forward ("突破大模型训练瓶颈：Flash-Attention编译优化与内存占用解决方案", 混合精度计算:
  * FP8 inputs with q_descale / k_descale factors). q, k, v are (B,N,H,d) tensors of E4M3
  * codes (OCP 8-bit format: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits), one byte
@@ -184,6 +199,16 @@ int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const 
               const float* alibi_slopes, void* dq, void* dk, void* dv,
               int B, int N, int H, int d, float scale, int causal, int win_l, int win_r, int deterministic,
               void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * Backward of fa_fwd_varlen (same packing, cu_seqlens and alibi_slopes; o and lse from
+ * fa_fwd_varlen); deterministic as in fa_bwd_ex. The workspace is that of a single sequence
+ * of `total` tokens: fa_bwd_workspace_bytes(1, total, H, d).
+ */
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                  const int* cu_seqlens, const float* alibi_slopes, void* dq, void* dk, void* dv,
+                  int B, int total, int H, int d, float scale, int causal, int win_l, int win_r,
+                  int deterministic, void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * The three launches of fa_bwd, exposed so that a caller can time or interleave them.
