@@ -137,25 +137,32 @@ struct BwdCfg {
   static constexpr int kThreads = 512;
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBoxes = D / 64;
-  static constexpr int kOffK = 0;
+  // d = 64: two K/V slots and two dK/dV TMEM buffers, alternating per work item, so that the
+  // next item's K/V load and first MMAs overlap this item's tail and dK/dV epilogue.
+  static constexpr int kKVSlots = (D == 64) ? 2 : 1;
+  static constexpr int kOffK = 0;                     // slot s: K at 2 s tiles, V right after
   static constexpr int kOffV = kTileBytes;
-  static constexpr int kOffQ = 2 * kTileBytes;        // two Q slots
-  static constexpr int kOffDO = 4 * kTileBytes;       // one dO slot
-  static constexpr int kOffDS = 5 * kTileBytes;       // dS^T, 128 x 128 bf16
+  static constexpr int kOffQ = 2 * kKVSlots * kTileBytes;        // two Q slots
+  static constexpr int kDOSlots = kKVSlots;                      // dO slots (two at d = 64)
+  static constexpr int kOffDO = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffDS = kOffDO + kDOSlots * kTileBytes;  // dS^T, 128 x 128 bf16
   static constexpr int kOffDQ = kOffDS + 32768;       // dQ staging: 128 rows x 64 fp32 (two 32-column boxes)
   static constexpr int kOffStat = kOffDQ + 32768;     // per Q slot: LSE2[128], D[128]
   static constexpr int kOffBar = kOffStat + 2 * 1024;
   static constexpr int kSmemBytes = kOffBar + 256;
   static constexpr int kDqRounds = D / 64;            // staging rounds per dQ tile
   static constexpr uint32_t kColDK = 0, kColDV = D, kColDP = 2 * D, kColS = 2 * D + 128;
+  static constexpr uint32_t kColDK1 = 2 * D + 256, kColDV1 = 3 * D + 256;  // second dK/dV buffer (d = 64)
   static constexpr uint32_t kTmemCols = 512;
+  static_assert(kKVSlots == 1 || kColDV1 + D <= kTmemCols, "TMEM budget");
 };
 
 struct BwdBars {
-  uint64_t kv_full, kv_empty;
+  uint64_t kv_full[2], kv_empty[2];      // per K/V slot
   uint64_t q_full[2], q_empty[2];  // Q_i and its LSE2 / D rows
-  uint64_t do_full, do_empty;
-  uint64_t s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_empty, dkv_full, dkv_empty;
+  uint64_t do_full[2], do_empty[2];     // per dO slot
+  uint64_t s_full, dp_full, p_full, ds_full, ds_empty, dq_full, dq_empty;
+  uint64_t dkv_full[2], dkv_empty[2];    // per dK/dV buffer
   uint64_t mma_done;
   uint64_t item_full[2], item_empty[2];  // ring of fetched work items, producer -> other roles
   int item_w[2];
@@ -263,6 +270,7 @@ __global__ void __launch_bounds__(512, 1)
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                   const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
   using Cfg = BwdCfg<D>;
+  static_assert(sizeof(BwdBars) <= 256, "barrier block");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = smem_u32(smem_raw);
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw + Cfg::kOffBar);
@@ -278,16 +286,20 @@ __global__ void __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     bars->abort_flag = 0;
-    mbar_init(bar(bars->kv_full), 1);
-    mbar_init(bar(bars->kv_empty), 2);
     for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(bars->kv_full[s]), 1);
+      mbar_init(bar(bars->kv_empty[s]), 2);
+      mbar_init(bar(bars->dkv_full[s]), 1);
+      mbar_init(bar(bars->dkv_empty[s]), 256);
       mbar_init(bar(bars->q_full[s]), 1);
       mbar_init(bar(bars->q_empty[s]), 1);
       mbar_init(bar(bars->item_full[s]), 1);
       mbar_init(bar(bars->item_empty[s]), kBwdItemConsumers);
     }
-    mbar_init(bar(bars->do_full), 1);
-    mbar_init(bar(bars->do_empty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(bars->do_full[s]), 1);
+      mbar_init(bar(bars->do_empty[s]), 1);
+    }
     mbar_init(bar(bars->s_full), 1);
     mbar_init(bar(bars->dp_full), 1);
     mbar_init(bar(bars->p_full), 256);
@@ -295,8 +307,6 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(bar(bars->ds_empty), 1);
     mbar_init(bar(bars->dq_full), 1);
     mbar_init(bar(bars->dq_empty), 128);
-    mbar_init(bar(bars->dkv_full), 1);
-    mbar_init(bar(bars->dkv_empty), 256);
     mbar_init(bar(bars->mma_done), 1);
     fence_barrier_init();
     prefetch_tmap(&tmQ);
@@ -316,8 +326,11 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
-  const uint32_t sK = smem_base + Cfg::kOffK, sV = smem_base + Cfg::kOffV;
-  const uint32_t sDO = smem_base + Cfg::kOffDO;
+  // K/V slot of the items-th work item of a role (the items of a CTA alternate between slots)
+  auto sKs = [&](uint32_t items) { return smem_base + Cfg::kOffK + (items % Cfg::kKVSlots) * 2 * Cfg::kTileBytes; };
+  auto sVs = [&](uint32_t items) { return smem_base + Cfg::kOffV + (items % Cfg::kKVSlots) * 2 * Cfg::kTileBytes; };
+  // dO slot of the n-th Q tile a role handles (Q tiles of a CTA alternate between the slots)
+  auto sDOs = [&](uint32_t n) { return smem_base + Cfg::kOffDO + (n % Cfg::kDOSlots) * Cfg::kTileBytes; };
   const uint32_t sDS = smem_base + Cfg::kOffDS;
   const uint32_t sDQ = smem_base + Cfg::kOffDQ;
   auto sQ = [&](int s) { return smem_base + Cfg::kOffQ + s * Cfg::kTileBytes; };
@@ -339,12 +352,13 @@ __global__ void __launch_bounds__(512, 1)
         bwd_decode(p, w, b, h, j);
         int lo, hi;
         bwd_q_range<kVarlen>(p, j, lo, hi);
-        mbar_wait(bar(bars->kv_empty), (items & 1) ^ 1, ab);
-        mbar_arrive_expect_tx(bar(bars->kv_full), 2 * Cfg::kTileBytes);
+        const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
+        mbar_wait(bar(bars->kv_empty[kvs]), kvphase ^ 1, ab);
+        mbar_arrive_expect_tx(bar(bars->kv_full[kvs]), 2 * Cfg::kTileBytes);
 #pragma unroll
         for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-          tma_load_4d(sK + bx * 16384, &tmK, bar(bars->kv_full), bx * 64, j * 128, h, b);
-          tma_load_4d(sV + bx * 16384, &tmV, bar(bars->kv_full), bx * 64, j * 128, h, b);
+          tma_load_4d(sKs(items) + bx * 16384, &tmK, bar(bars->kv_full[kvs]), bx * 64, j * 128, h, b);
+          tma_load_4d(sVs(items) + bx * 16384, &tmV, bar(bars->kv_full[kvs]), bx * 64, j * 128, h, b);
         }
         ++items;
         const size_t stat_row = ((size_t)b * p.H + h) * (size_t)p.N_pad;
@@ -360,17 +374,20 @@ __global__ void __launch_bounds__(512, 1)
           last_q_parity[qs] = qphase;
           if (++qs == 2) { qs = 0; qphase ^= 1; }
           // dO_i into the single dO slot (freed when dV_{i-1} is done)
-          mbar_wait(bar(bars->do_empty), (dn & 1) ^ 1, ab);
-          mbar_arrive_expect_tx(bar(bars->do_full), Cfg::kTileBytes);
+          const uint32_t dos = dn % Cfg::kDOSlots, dophase = (dn / Cfg::kDOSlots) & 1;
+          mbar_wait(bar(bars->do_empty[dos]), dophase ^ 1, ab);
+          mbar_arrive_expect_tx(bar(bars->do_full[dos]), Cfg::kTileBytes);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_4d(sDO + bx * 16384, &tmdO, bar(bars->do_full), bx * 64, i * 128, h, b);
+            tma_load_4d(sDOs(dn) + bx * 16384, &tmdO, bar(bars->do_full[dos]), bx * 64, i * 128, h, b);
         }
       }
       for (int s = 0; s < 2; ++s)
         if (last_q_parity[s] >= 0) mbar_drain(bar(bars->q_full[s]), last_q_parity[s]);
-      if (dn > 0) mbar_drain(bar(bars->do_full), (dn - 1) & 1);
-      if (items > 0) mbar_drain(bar(bars->kv_full), (items - 1) & 1);
+      for (uint32_t t = (dn > Cfg::kDOSlots ? dn - Cfg::kDOSlots : 0); t < dn; ++t)
+        mbar_drain(bar(bars->do_full[t % Cfg::kDOSlots]), (t / Cfg::kDOSlots) & 1);
+      for (uint32_t t = (items > Cfg::kKVSlots ? items - Cfg::kKVSlots : 0); t < items; ++t)
+        mbar_drain(bar(bars->kv_full[t % Cfg::kKVSlots]), (t / Cfg::kKVSlots) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -380,9 +397,9 @@ __global__ void __launch_bounds__(512, 1)
       constexpr uint32_t idSP = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T: K-major A and B
       constexpr uint32_t idKV = idesc_bf16_f32(128, D, false, true);     // dV, dK: B (dO, Q) MN-major
       constexpr uint32_t idQ = idesc_bf16_f32(128, D, true, true);       // dQ: A (dS) and B (K) MN-major
-      const uint32_t tDK = tmem + Cfg::kColDK, tDV = tmem + Cfg::kColDV;
       const uint32_t tDP = tmem + Cfg::kColDP, tS = tmem + Cfg::kColS;
       uint32_t items = 0, n = 0, qs = 0, qphase = 0;
+      uint32_t sK = sKs(0), sV = sVs(0);
       auto issue_s = [&](uint32_t slot, uint32_t phase) {
         mbar_wait(bar(bars->q_full[slot]), phase, ab);
         tc_fence_after_sync();
@@ -401,14 +418,20 @@ __global__ void __launch_bounds__(512, 1)
         bwd_decode(p, w, b, h, j);
         int lo, hi;
         bwd_q_range<kVarlen>(p, j, lo, hi);
-        mbar_wait(bar(bars->kv_full), items & 1, ab);
+        const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
+        sK = sKs(items);
+        sV = sVs(items);
+        const uint32_t tDK = tmem + (kvs ? Cfg::kColDK1 : Cfg::kColDK);
+        const uint32_t tDV = tmem + (kvs ? Cfg::kColDV1 : Cfg::kColDV);
+        mbar_wait(bar(bars->kv_full[kvs]), kvphase, ab);
         tc_fence_after_sync();
         issue_s(qs, qphase);  // S(lo)
         for (int i = lo; i <= hi; ++i, ++n) {
           const bool first = (i == lo);
           const uint32_t q = sQ(qs);
           // dP^T = V_j dO_i^T into the columns dQ_{i-1} occupied
-          mbar_wait(bar(bars->do_full), n & 1, ab);
+          const uint32_t sDO = sDOs(n), dos = n % Cfg::kDOSlots;
+          mbar_wait(bar(bars->do_full[dos]), (n / Cfg::kDOSlots) & 1, ab);
           if (kDQ) mbar_wait(bar(bars->dq_empty), (n & 1) ^ 1, ab);
           tc_fence_after_sync();
 #pragma unroll
@@ -419,14 +442,14 @@ __global__ void __launch_bounds__(512, 1)
           mma_commit(bar(bars->dp_full));
           // dV += P^T dO_i (P^T packed in TMEM: queries [0,64) in S columns [0,32), [64,128) in [64,96))
           mbar_wait(bar(bars->p_full), n & 1, ab);
-          if (first) mbar_wait(bar(bars->dkv_empty), (items & 1) ^ 1, ab);
+          if (first) mbar_wait(bar(bars->dkv_empty[kvs]), kvphase ^ 1, ab);
           tc_fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t acol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
             mma_ts(tDV, tS + acol, sdesc_mnmajor(sDO + kk * 2048, 16384), idKV, !first || kk > 0);
           }
-          mma_commit(bar(bars->do_empty));
+          mma_commit(bar(bars->do_empty[dos]));
           // S(i+1): overwrites P^T(i), which dV(i) (issued before) has read
           const uint32_t nqs = qs ^ 1, nqphase = qs ? (qphase ^ 1) : qphase;
           if (i < hi) issue_s(nqs, nqphase);
@@ -449,7 +472,7 @@ __global__ void __launch_bounds__(512, 1)
           qs = nqs;
           qphase = nqphase;
         }
-        mma_commit(bar(bars->dkv_full));
+        mma_commit(bar(bars->dkv_full[kvs]));
         ++items;
       }
       mma_commit(bar(bars->mma_done));
@@ -600,10 +623,12 @@ __global__ void __launch_bounds__(512, 1)
       }
 
       // Epilogue: dK (group 0, times scale) or dV (group 1) -> bf16 -> the K_j / V_j buffer -> TMA store.
-      mbar_wait(bar(bars->dkv_full), items & 1, ab);
+      const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
+      mbar_wait(bar(bars->dkv_full[kvs]), kvphase, ab);
       tc_fence_after_sync();
-      const uint32_t src = tmem + lane_field + (grp ? Cfg::kColDV : Cfg::kColDK);
-      const uint32_t stage_buf = grp ? sV : sK;
+      const uint32_t src =
+          tmem + lane_field + (grp ? (kvs ? Cfg::kColDV1 : Cfg::kColDV) : (kvs ? Cfg::kColDK1 : Cfg::kColDK));
+      const uint32_t stage_buf = grp ? sVs(items) : sKs(items);  // this item's K/V slot: its MMAs are done
       const float mult = grp ? 1.0f : p.scale;
 #pragma unroll 1
       for (int cc = 0; cc < D; cc += 32) {
@@ -621,7 +646,7 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
       tc_fence_before_sync();
-      mbar_arrive(bar(bars->dkv_empty));
+      mbar_arrive(bar(bars->dkv_empty[kvs]));
       fence_proxy_async_smem();
       named_bar_sync(1 + grp, 128);
       if (row == 0) {
@@ -630,7 +655,7 @@ __global__ void __launch_bounds__(512, 1)
           tma_store_4d(grp ? &tmdV : &tmdK, stage_buf + bx * 16384, bx * 64, j * 128, h, b);
         bulk_commit_group();
         bulk_wait_group_read0();
-        mbar_arrive(bar(bars->kv_empty));
+        mbar_arrive(bar(bars->kv_empty[kvs]));
       }
       ++items;
     }
