@@ -49,8 +49,6 @@ UNIT = "TFLOPS"
 L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "ncu_traffic.json")
-KERNEL_SOURCES = [os.path.join(ROOT, "exact_attention_116_b200", "csrc", f)
-                  for f in ("fa_api.cu", "fa_fwd.cuh", "fa_bwd.cuh", "fa_bwd_dq.cuh", "sm100_ptx.cuh")]
 
 
 def peaks():
@@ -62,24 +60,24 @@ def peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
-        with open(p, "rb") as f:
+    for name in sources:
+        with open(os.path.join(ROOT, "exact_attention_116_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it still matches the source."""
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the sources that
+    define the kernel still hash to the value recorded with the measurement."""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
     with open(PROFILE_TRAFFIC) as f:
-        d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
+        k = json.load(f).get("kernels", {}).get(kernel)
+    if k is None or k.get("source_hash") != kernel_source_hash(k.get("sources", [])):
         return None
-    k = d.get("kernels", {}).get(kernel)
-    return None if k is None else k.get("dram_bytes_per_launch")
+    return k.get("dram_bytes_per_launch")
 
 
 # ----------------------------------------------------------------------------- clocks

@@ -201,8 +201,9 @@ __global__ void __launch_bounds__(kDecThreads)
       for (int i = 0; i < kSq; ++i) sS[(half * kDecMaxSq + i) * kDecTile + kt] = part[i];
     }
     __syncthreads();
-    // every thread has finished with the previous tile's slot: refill it
-    if (tid == 0 && t > t0 && t - 1 + kDecStages < t1) issue(t - 1 + kDecStages);
+    // every thread has finished with the previous tile's slot: refill it (not after a wait gave
+    // up: that slot's barrier may still be waiting for bytes, and must not be armed twice)
+    if (tid == 0 && t > t0 && t - 1 + kDecStages < t1 && !ab.raised()) issue(t - 1 + kDecStages);
     // ---- B: softmax bookkeeping, warp w -> rows w, w + 4
 #pragma unroll
     for (int r = 0; r < (kSq + 3) / 4; ++r) {
