@@ -73,15 +73,11 @@ bool bwd_attributes() {
 
 template <int D>
 bool decode_attributes() {
-  const int smem = fa::DecCfg<D>::kSmemBytes;
-  return cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
-             cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
-             cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
-             cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ==
-             cudaSuccess;
+  const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  return cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 1>, attr, fa::DecCfg<D, 1>::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 2>, attr, fa::DecCfg<D, 2>::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 4>, attr, fa::DecCfg<D, 4>::kSmemBytes) == cudaSuccess &&
+         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 8>, attr, fa::DecCfg<D, 8>::kSmemBytes) == cudaSuccess;
 }
 
 int device_setup(int* dev_out, int* sm_count) {
@@ -591,15 +587,14 @@ namespace {
 template <int D>
 int launch_decode(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
                   cudaStream_t cs) {
-  const int smem = fa::DecCfg<D>::kSmemBytes;
   if (p.Sq == 1)
-    fa::fa_decode_split_kernel<D, 1><<<grid, fa::kDecThreads, smem, cs>>>(mk, mv, p);
+    fa::fa_decode_split_kernel<D, 1><<<grid, fa::kDecThreads, fa::DecCfg<D, 1>::kSmemBytes, cs>>>(mk, mv, p);
   else if (p.Sq == 2)
-    fa::fa_decode_split_kernel<D, 2><<<grid, fa::kDecThreads, smem, cs>>>(mk, mv, p);
+    fa::fa_decode_split_kernel<D, 2><<<grid, fa::kDecThreads, fa::DecCfg<D, 2>::kSmemBytes, cs>>>(mk, mv, p);
   else if (p.Sq <= 4)
-    fa::fa_decode_split_kernel<D, 4><<<grid, fa::kDecThreads, smem, cs>>>(mk, mv, p);
+    fa::fa_decode_split_kernel<D, 4><<<grid, fa::kDecThreads, fa::DecCfg<D, 4>::kSmemBytes, cs>>>(mk, mv, p);
   else
-    fa::fa_decode_split_kernel<D, 8><<<grid, fa::kDecThreads, smem, cs>>>(mk, mv, p);
+    fa::fa_decode_split_kernel<D, 8><<<grid, fa::kDecThreads, fa::DecCfg<D, 8>::kSmemBytes, cs>>>(mk, mv, p);
   return launch_status();
 }
 
@@ -609,11 +604,12 @@ size_t decode_workspace_bytes(int B, int Sq, int H, int d, int splits) {
   return align256(rows * d * 4) + align256(rows * 4);
 }
 
-// Splits per (b, h) when the caller passes 0: about four CTAs per SM in total (two fit at a
-// time), never more than the 64-key tiles of the longest possible sequence, at most 128.
+// Splits per (b, h) when the caller passes 0: about seven CTAs per SM in total (two or three
+// fit at a time; measured best on a B8 H16 batch of 4-8K-key sequences), never more than the
+// 64-key tiles of the longest possible sequence, at most 128.
 int decode_auto_splits(int B, int H, int max_keys, int sm_count) {
   const long long bh = (long long)B * H;
-  long long s = (4LL * sm_count + bh - 1) / bh;
+  long long s = (7LL * sm_count + bh / 2) / bh;
   const long long tiles = (max_keys + fa::kDecTile - 1) / fa::kDecTile;
   if (s > tiles) s = tiles;
   if (s > 128) s = 128;

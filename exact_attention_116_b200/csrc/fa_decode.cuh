@@ -35,7 +35,7 @@ namespace fa {
 
 constexpr int kDecMaxSq = 8;       // new query rows per call
 constexpr int kDecTile = 64;       // keys per tile
-constexpr int kDecStages = 3;      // K/V ring depth
+constexpr int kStagesMax = 3;   // K/V ring depth for 8 new rows
 constexpr int kDecThreads = 128;
 constexpr float kDecLn2 = 0.69314718055994530942f;
 
@@ -53,22 +53,26 @@ struct DecParams {
   float* lse_part;         // (B, H, Sq, splits), log2 domain (splits > 1)
 };
 
-template <int D>
+// Shared memory of a CTA compiled for kSq rows: up to 4 rows a 2-stage ring (about 67 KB at
+// d = 128, so that three CTAs share an SM and hide each other's per-tile latency), 8 rows a
+// 3-stage ring (two CTAs per SM).
+template <int D, int kSq>
 struct DecCfg {
+  static constexpr int kStages = (kSq <= 4) ? 2 : kStagesMax;
   static constexpr int kBoxes = D / 64;                       // 64-column (128-byte) boxes per row
   static constexpr int kTileBytes = kDecTile * D * 2;         // one K or V tile
   static constexpr int kStageBytes = 2 * kTileBytes;          // K and V
   static constexpr int kOffKV = 0;
-  static constexpr int kOffQ = kDecStages * kStageBytes;       // q rows, fp32 (kDecMaxSq x D)
-  static constexpr int kOffS = kOffQ + kDecMaxSq * D * 4;      // half-dot products (2 x kDecMaxSq x 64)
-  static constexpr int kOffP = kOffS + 2 * kDecMaxSq * kDecTile * 4;  // P (kDecMaxSq x 64)
-  static constexpr int kOffAlpha = kOffP + kDecMaxSq * kDecTile * 4;  // rescale factor per row
-  static constexpr int kPairs = D / 2;                                // column pairs
-  static constexpr int kKeyGroups = kDecThreads / kPairs;             // 2 (D=128) or 4 (D=64)
-  static constexpr int kOffRed = kOffKV;  // final reduction (key groups x Sq x D), over the drained ring
-  static_assert(kKeyGroups * kDecMaxSq * D * 4 <= kDecStages * kStageBytes, "reduction buffer");
-  static constexpr int kOffBar = kOffAlpha + kDecMaxSq * 4 + 64;
-  static constexpr int kSmemBytes = kOffBar + 128 + 1024;             // barriers + alignment slack
+  static constexpr int kOffQ = kStages * kStageBytes;          // q rows, fp32 (kSq x D)
+  static constexpr int kOffS = kOffQ + kSq * D * 4;            // half-dot products (2 x kSq x 64)
+  static constexpr int kOffP = kOffS + 2 * kSq * kDecTile * 4;  // P (kSq x 64)
+  static constexpr int kOffAlpha = kOffP + kSq * kDecTile * 4;  // rescale factor per row
+  static constexpr int kPairs = D / 2;                          // column pairs
+  static constexpr int kKeyGroups = kDecThreads / kPairs;       // 2 (D=128) or 4 (D=64)
+  static constexpr int kOffRed = kOffKV;  // final reduction (key groups x kSq x D), over the drained ring
+  static_assert(kKeyGroups * kSq * D * 4 <= kStages * kStageBytes, "reduction buffer");
+  static constexpr int kOffBar = (kOffAlpha + kSq * 4 + 63) & ~63;
+  static constexpr int kSmemBytes = kOffBar + 128 + 1024;       // barriers + alignment slack
 };
 
 // Keys [t0 * 64, t1 * 64) of sequence b that split s covers, clipped to what rows
@@ -89,7 +93,8 @@ template <int D, int kSq>
 __global__ void __launch_bounds__(kDecThreads)
     fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                            const DecParams p) {
-  using Cfg = DecCfg<D>;
+  using Cfg = DecCfg<D, kSq>;
+  constexpr int kStages = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sm = smem_raw + (smem_base - smem_u32(smem_raw));
@@ -116,12 +121,12 @@ __global__ void __launch_bounds__(kDecThreads)
 
   if (tid == 0) {
     *abort_flag = 0;
-    for (int st = 0; st < kDecStages; ++st) mbar_init(smem_u32(&full[st]), 1);
+    for (int st = 0; st < kStages; ++st) mbar_init(smem_u32(&full[st]), 1);
     fence_barrier_init();
   }
-  if (tid < kDecMaxSq) sAlpha[tid] = 0.0f;  // rows past Sq keep alpha = 0 (their O stays 0)
+  if (tid < kSq) sAlpha[tid] = 0.0f;  // rows past Sq keep alpha = 0 (their O stays 0)
   // q rows -> shared memory (fp32); rows >= Sq are zero
-  for (int e = tid; e < kDecMaxSq * D; e += kDecThreads) {
+  for (int e = tid; e < kSq * D; e += kDecThreads) {
     const int i = e / D, c = e - i * D;
     sQ[e] = i < Sq ? __bfloat162float(p.q[(((size_t)b * Sq + i) * p.H + h) * D + c]) : 0.0f;
   }
@@ -129,7 +134,7 @@ __global__ void __launch_bounds__(kDecThreads)
 
   // TMA: tile t of this sequence -> stage slot; keys [64 t, 64 t + 64) lie in one page.
   auto issue = [&](int t) {
-    const int st = (t - t0) % kDecStages;
+    const int st = (t - t0) % kStages;
     const int key = t * kDecTile;
     int page = p.block_table[(size_t)b * p.max_pages + key / p.page_size];
     if (page < 0 || page >= p.num_pages) {  // the TMA would read zeros there; report it
@@ -148,7 +153,7 @@ __global__ void __launch_bounds__(kDecThreads)
   if (tid == 0) {
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
-    for (int t = t0; t < t1 && t < t0 + kDecStages; ++t) issue(t);
+    for (int t = t0; t < t1 && t < t0 + kStages; ++t) issue(t);
   }
 
   // running state: warp w owns rows w and w + 4 (warp-uniform values)
@@ -161,8 +166,8 @@ __global__ void __launch_bounds__(kDecThreads)
   const float c = p.scale_log2;
 
   for (int t = t0; t < t1; ++t) {
-    const int st = (t - t0) % kDecStages;
-    mbar_wait(smem_u32(&full[st]), ((t - t0) / kDecStages) & 1, ab);
+    const int st = (t - t0) % kStages;
+    mbar_wait(smem_u32(&full[st]), ((t - t0) / kStages) & 1, ab);
     const uint8_t* kgen = sm + Cfg::kOffKV + st * Cfg::kStageBytes;
     const uint8_t* vgen = kgen + Cfg::kTileBytes;
     // ---- A: half dot products, key kt = tid % 64, dims [half * D/2, half * D/2 + D/2)
@@ -198,12 +203,12 @@ __global__ void __launch_bounds__(kDecThreads)
         }
       }
 #pragma unroll
-      for (int i = 0; i < kSq; ++i) sS[(half * kDecMaxSq + i) * kDecTile + kt] = part[i];
+      for (int i = 0; i < kSq; ++i) sS[(half * kSq + i) * kDecTile + kt] = part[i];
     }
     __syncthreads();
     // every thread has finished with the previous tile's slot: refill it (not after a wait gave
     // up: that slot's barrier may still be waiting for bytes, and must not be armed twice)
-    if (tid == 0 && t > t0 && t - 1 + kDecStages < t1 && !ab.raised()) issue(t - 1 + kDecStages);
+    if (tid == 0 && t > t0 && t - 1 + kStages < t1 && !ab.raised()) issue(t - 1 + kStages);
     // ---- B: softmax bookkeeping, warp w -> rows w, w + 4
 #pragma unroll
     for (int r = 0; r < (kSq + 3) / 4; ++r) {
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(kDecThreads)
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int kt = lane + 32 * u, key = t * kDecTile + kt;
-          const float sc = (sS[i * kDecTile + kt] + sS[(kDecMaxSq + i) * kDecTile + kt]) * c;
+          const float sc = (sS[i * kDecTile + kt] + sS[(kSq + i) * kDecTile + kt]) * c;
           x[u] = (key >= kmin && key <= kmax) ? sc : -INFINITY;
         }
         float tmax = fmaxf(x[0], x[1]);
@@ -266,17 +271,17 @@ __global__ void __launch_bounds__(kDecThreads)
 
   // drain: loads issued past a wait that gave up must land before the ring is reused
   if (tid == 0 && ab.raised()) {
-    for (int t = max(t0, t1 - kDecStages); t < t1; ++t) {
-      const int st = (t - t0) % kDecStages;
-      mbar_drain(smem_u32(&full[st]), ((t - t0) / kDecStages) & 1);
+    for (int t = max(t0, t1 - kStages); t < t1; ++t) {
+      const int st = (t - t0) % kStages;
+      mbar_drain(smem_u32(&full[st]), ((t - t0) / kStages) & 1);
     }
   }
   __syncthreads();  // the K/V ring is free: it holds the reduction below
   // ---- combine the key groups' partial sums, normalise, write
 #pragma unroll
   for (int i = 0; i < kSq; ++i) {
-    sRed[(kg * kDecMaxSq + i) * D + 2 * cp] = acc[i][0];
-    sRed[(kg * kDecMaxSq + i) * D + 2 * cp + 1] = acc[i][1];
+    sRed[(kg * kSq + i) * D + 2 * cp] = acc[i][0];
+    sRed[(kg * kSq + i) * D + 2 * cp + 1] = acc[i][1];
   }
   // row statistics of warp-owned rows -> shared (reuse the alpha slots as 1/l, S as log2 l + m)
   __syncthreads();
@@ -293,7 +298,7 @@ __global__ void __launch_bounds__(kDecThreads)
     const int i = e / D, col = e - i * D;
     float v = 0.0f;
 #pragma unroll
-    for (int g = 0; g < Cfg::kKeyGroups; ++g) v += sRed[(g * kDecMaxSq + i) * D + col];
+    for (int g = 0; g < Cfg::kKeyGroups; ++g) v += sRed[(g * kSq + i) * D + col];
     v *= sAlpha[i];
     if (p.splits == 1) {
       p.o[(((size_t)b * Sq + i) * p.H + h) * D + col] = __float2bfloat16_rn(v);

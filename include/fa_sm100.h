@@ -109,7 +109,7 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_desca
 /*
  * The split count fa_decode_paged uses when called with splits = 0, for B sequences, H heads
  * and at most max_keys keys per sequence (max_pages * page_size), on the current device: about
- * four CTAs per SM over B*H, at most one per 64-key tile and at most 128. Negative status on
+ * seven CTAs per SM over B*H, at most one per 64-key tile and at most 128. Negative status on
  * error (-FA_ERR_INVALID_ARG, -FA_ERR_UNSUPPORTED without an sm_100 device, -FA_ERR_CUDA).
  */
 int fa_decode_splits(int B, int H, int max_keys);
