@@ -5,7 +5,8 @@ followed by the backward's three launches (preprocess, main, dQ conversion). The
 workload is the training configuration B=2, H=16, N=8192, d=128, causal, bf16.
 ``--config train_fwd_fp8`` instead times the E4M3 forward (fa_fwd_fp8) on the same shape:
 one step = one launch. ``--config decode_paged`` times the paged-KV decode (fa_decode_paged):
-one step = one call (split kernel + merge) over every sequence, reported in GB/s of cache read.
+one step = one call (append, split kernel and merge in one kernel) over every sequence, reported
+in GB/s of cache read.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
 
@@ -289,8 +290,11 @@ def run_gpu_decode(args):
     stream = torch.cuda.current_stream()
     # workspace of the split count in use (the library's choice unless --splits is given)
     ws = torch.empty(max(1, binding.decode_workspace_bytes(B, Sq, H, d, splits)), dtype=torch.uint8, device=dev)
-    # L2 flush between steps: the cache is 2x268 MiB > L2 already, q/O are tiny
+    # L2 flush between steps (the cache is 2x268 MiB > L2 already, q/O are tiny): a buffer larger
+    # than L2 is written, then another one read, so that the step starts with a clean L2 and does
+    # not pay for writing the flush's dirty lines back
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
     def step():
         binding.decode_paged_into(q, kc, vc, table, lens, o, lse, cfg.scale, cfg.causal, (cfg.win_l, cfg.win_r),
@@ -307,6 +311,7 @@ def run_gpu_decode(args):
     ms = 0.0
     for _ in range(args.steps):
         flush.zero_()
+        flush_r.sum()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         step()
@@ -362,16 +367,18 @@ def run_gpu_decode(args):
                    "B": B, "Sq": Sq, "H": H, "d": d,
                    "page_size": cfg.page_size, "lengths": [int(x) for x in host[4]], "causal": cfg.causal,
                    "splits": splits, "seed": cfg.seed,
-                   "l2": "L2 flushed (512 MiB write) before every timed step; KV cache > L2",
+                   "l2": "L2 flushed before every timed step (512 MiB written, then 512 MiB read: no dirty lines "
+                         "left to write back inside the step); KV cache > L2",
                    "bytes": "K and V rows of every visible key + q, O, LSE"},
-        "roofline": {"kernel": "fa_decode_split_kernel<128> + combine", "bound": "hbm", "achieved": round(gbs, 1),
+        "roofline": {"kernel": "fa_decode_split_kernel<128> (append and merge fused; timed with the counter-"
+                               "zeroing launch before it)", "bound": "hbm", "achieved": round(gbs, 1),
                      "peak": peak["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peak["hbm_gbs"], 4),
-                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)", "traffic": None,
-                     "algorithmic_bytes": nbytes},
+                     "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                     "traffic": recorded_traffic("fa_decode_split_kernel"), "algorithmic_bytes": nbytes},
         "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4},
-        "gpu_launches": (3 if splits > 1 else 2) * args.steps,  # append, split kernel, merge
+        "gpu_launches": (2 if splits > 1 else 1) * args.steps,  # counter zeroing, split kernel
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -15,7 +15,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "fa_api.cu")
-HEADERS = [os.path.join(PKG, "csrc", f) for f in ("fa_fwd.cuh", "fa_bwd.cuh", "fa_bwd_dq.cuh", "sm100_ptx.cuh")] + [
+HEADERS = [os.path.join(PKG, "csrc", f) for f in ("fa_fwd.cuh", "fa_bwd.cuh", "fa_bwd_dq.cuh", "fa_decode.cuh", "sm100_ptx.cuh")] + [
     os.path.join(ROOT, "include", "fa_sm100.h")
 ]
 LIB = os.path.join(PKG, "libfa_sm100.so")

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -584,24 +585,42 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_desca
 
 namespace {
 
-template <int D>
-int launch_decode(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
-                  cudaStream_t cs) {
-  if (p.Sq == 1)
-    fa::fa_decode_split_kernel<D, 1><<<grid, fa::kDecThreads, fa::DecCfg<D, 1>::kSmemBytes, cs>>>(mk, mv, p);
-  else if (p.Sq == 2)
-    fa::fa_decode_split_kernel<D, 2><<<grid, fa::kDecThreads, fa::DecCfg<D, 2>::kSmemBytes, cs>>>(mk, mv, p);
-  else if (p.Sq <= 4)
-    fa::fa_decode_split_kernel<D, 4><<<grid, fa::kDecThreads, fa::DecCfg<D, 4>::kSmemBytes, cs>>>(mk, mv, p);
-  else
-    fa::fa_decode_split_kernel<D, 8><<<grid, fa::kDecThreads, fa::DecCfg<D, 8>::kSmemBytes, cs>>>(mk, mv, p);
+// The split kernel compiled for Sq rounded up to 1, 2, 4 or 8, launched as the programmatic
+// dependent of the kernel before it on the stream (the prep kernel, when there are splits).
+template <int D, int kSq>
+int launch_decode_sq(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
+                     cudaStream_t cs) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(fa::kDecThreads);
+  cfg.dynamicSmemBytes = fa::DecCfg<D, kSq>::kSmemBytes;
+  cfg.stream = cs;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa::fa_decode_split_kernel<D, kSq>, mk, mv, p) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
   return launch_status();
 }
 
+template <int D>
+int launch_decode(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
+                  cudaStream_t cs) {
+  if (p.Sq == 1) return launch_decode_sq<D, 1>(grid, mk, mv, p, cs);
+  if (p.Sq == 2) return launch_decode_sq<D, 2>(grid, mk, mv, p, cs);
+  if (p.Sq <= 4) return launch_decode_sq<D, 4>(grid, mk, mv, p, cs);
+  return launch_decode_sq<D, 8>(grid, mk, mv, p, cs);
+}
+
+// Workspace of a split call: partial O (fp32), partial LSE, one arrival counter per (b, h).
 size_t decode_workspace_bytes(int B, int Sq, int H, int d, int splits) {
   if (splits <= 1) return 0;
   const size_t rows = (size_t)B * H * Sq * splits;
-  return align256(rows * d * 4) + align256(rows * 4);
+  return align256(rows * d * 4) + align256(rows * 4) + align256((size_t)B * H * 4);
 }
 
 // Splits per (b, h) when the caller passes 0: about seven CTAs per SM in total (two or three
@@ -645,6 +664,7 @@ int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_n
   if ((double)num_pages * page_size * H * d * 2 >= 1099511627776.0 ||
       (double)max_pages * page_size >= 2147483647.0)
     return FA_ERR_INVALID_ARG;
+  if (B > 65535 || splits > 65535 || (long long)B * H >= 2147483647LL) return FA_ERR_INVALID_ARG;  // grid limits
   if (!q || !k_cache || !v_cache || !block_table || !seqlens || !o || !lse) return FA_ERR_INVALID_ARG;
   if ((k_new == nullptr) != (v_new == nullptr)) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
@@ -701,15 +721,19 @@ int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_n
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.o_part = static_cast<float*>(ws);
-  p.lse_part = wbytes ? reinterpret_cast<float*>(static_cast<char*>(ws) +
-                                                 align256((size_t)B * H * Sq * splits * d * 4))
-                      : nullptr;
+  const size_t part_bytes = align256((size_t)B * H * Sq * splits * d * 4);
+  const size_t lse_part_bytes = align256((size_t)B * H * Sq * splits * 4);
+  p.lse_part = wbytes ? reinterpret_cast<float*>(static_cast<char*>(ws) + part_bytes) : nullptr;
+  p.arrivals = wbytes ? reinterpret_cast<int*>(static_cast<char*>(ws) + part_bytes + lse_part_bytes) : nullptr;
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(v_cache);
   st = FA_OK;
-  if (k_new) {
-    fa::fa_decode_append_kernel<<<dim3(Sq, B), 256, 0, cs>>>(p, d, static_cast<const __nv_bfloat16*>(k_new),
-                                                             static_cast<const __nv_bfloat16*>(v_new),
-                                                             static_cast<__nv_bfloat16*>(k_cache),
-                                                             static_cast<__nv_bfloat16*>(v_cache));
+  if (splits > 1) {
+    const int count = B * H;
+    const int blocks = (int)std::min<long long>((count + 255) / 256, sms);
+    fa::fa_decode_prep_kernel<<<blocks, 256, 0, cs>>>(p.arrivals, count);
     st = launch_status();
   }
   if (!st) {
@@ -718,14 +742,6 @@ int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_n
       st = launch_decode<64>(grid, mk, mv, p, cs);
     else
       st = launch_decode<128>(grid, mk, mv, p, cs);
-  }
-  if (!st && splits > 1) {
-    const dim3 cgrid(Sq, H, B);
-    if (d == 64)
-      fa::fa_decode_combine_kernel<64><<<cgrid, 64, 0, cs>>>(p);
-    else
-      fa::fa_decode_combine_kernel<128><<<cgrid, 128, 0, cs>>>(p);
-    st = launch_status();
   }
   if (wbytes > 0 && !workspace && cudaFreeAsync(ws, cs) != cudaSuccess && !st) st = FA_ERR_CUDA;
   return st;

@@ -12,8 +12,11 @@
 // cut into `splits` contiguous ranges, one CTA each; a CTA streams its 64-key K/V tiles by TMA
 // into a 3-stage ring (a 64-key tile never straddles a page: page_size is a multiple of 64),
 // keeps a running maximum and sum per row (log2 domain) and writes a partial (O / l, log2 l + m).
-// fa_decode_combine_kernel merges the partials by their log-sum-exp; with one split the CTA
-// writes the final O and LSE itself.
+// The last CTA of a (b, h) to finish (an arrival counter per (b, h)) merges the partials by
+// their log-sum-exp and writes O and LSE; with one split the CTA writes them itself. The
+// counters are zeroed by fa_decode_prep_kernel, launched just before on the same stream; the
+// split kernel is launched as its programmatic dependent, so it streams the cache while the
+// prep kernel runs and waits for it only before its first arrival.
 //
 // CTA (128 threads), per tile of 64 keys:
 //   A: thread (key t = tid % 64, half = tid / 64) forms half of q_i . k_t for every row i
@@ -25,8 +28,10 @@
 // launched next to each other (head is the fastest grid index), so the 128-byte rows of one
 // cache row (H x d bf16, contiguous) are read by concurrent CTAs.
 //
-// With new K/V rows given (flash_attn_with_kvcache's in-place update of the cache),
-// fa_decode_append_kernel first writes them into the cache at their positions.
+// With new K/V rows given (flash_attn_with_kvcache's in-place update of the cache), the CTA
+// whose key range holds a new row writes that row's d columns of its head into the cache
+// before it loads any tile: every new row is visible to the newest query row, so exactly one
+// split of each head covers it, and no other CTA reads those bytes.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -38,6 +43,21 @@ constexpr int kDecTile = 64;       // keys per tile
 constexpr int kStagesMax = 3;   // K/V ring depth for 8 new rows
 constexpr int kDecThreads = 128;
 constexpr float kDecLn2 = 0.69314718055994530942f;
+
+// Generic-proxy writes to global memory by this thread are ordered before later async-proxy
+// (TMA) accesses that a barrier orders after this fence.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Programmatic dependent launch: let the next kernel on the stream (launched with the
+// programmatic-serialization attribute) start, and, in that kernel, wait until the grids it
+// depends on have finished and their writes are visible. The wait returns at once in a
+// kernel launched without the attribute.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 struct DecParams {
   int B, Sq, H, page_size, max_pages, num_pages;
@@ -51,6 +71,11 @@ struct DecParams {
   float* lse;              // (B, H, Sq), natural log
   float* o_part;           // (B, H, Sq, splits, d) fp32 (splits > 1)
   float* lse_part;         // (B, H, Sq, splits), log2 domain (splits > 1)
+  int* arrivals;           // (B, H) split CTAs finished (splits > 1), zeroed by the prep kernel
+  const __nv_bfloat16* k_new;  // (B, Sq, H, d) rows to write into the cache, or null
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* k_cache;  // (num_pages, page_size, H, d)
+  __nv_bfloat16* v_cache;
 };
 
 // Shared memory of a CTA compiled for kSq rows: up to 4 rows a 2-stage ring (about 67 KB at
@@ -118,6 +143,31 @@ __global__ void __launch_bounds__(kDecThreads)
 
   int t0 = 0, t1 = 0;
   if (!dec_tile_range(p, n, s, t0, t1)) t1 = t0;
+
+  // new rows in this CTA's key range: head h's columns go into the cache before any tile load
+  if (p.k_new != nullptr && t1 > t0) {
+    const int key_lo = t0 * kDecTile, key_hi = t1 * kDecTile;
+    constexpr int kChunks = D / 8;  // 16-byte chunks of one head's row
+    bool wrote = false;
+    for (int i = 0; i < Sq; ++i) {
+      const int pos = n - Sq + i;
+      if (pos < key_lo || pos >= key_hi) continue;  // another split's (or, pos < 0, nobody's)
+      const int page = p.block_table[(size_t)b * p.max_pages + pos / p.page_size];
+      if (page < 0 || page >= p.num_pages) {  // reported below when the tile is loaded
+        continue;
+      }
+      const size_t src = (((size_t)b * Sq + i) * p.H + h) * D;
+      const size_t dst = (((size_t)page * p.page_size + pos % p.page_size) * p.H + h) * D;
+      if (tid < kChunks) {
+        reinterpret_cast<uint4*>(p.k_cache + dst)[tid] = reinterpret_cast<const uint4*>(p.k_new + src)[tid];
+      } else if (tid < 2 * kChunks) {
+        reinterpret_cast<uint4*>(p.v_cache + dst)[tid - kChunks] =
+            reinterpret_cast<const uint4*>(p.v_new + src)[tid - kChunks];
+      }
+      wrote = true;
+    }
+    if (wrote) fence_proxy_async_global();  // ordered before the TMA loads by the barrier below
+  }
 
   if (tid == 0) {
     *abort_flag = 0;
@@ -313,52 +363,46 @@ __global__ void __launch_bounds__(kDecThreads)
     else
       p.lse_part[(((size_t)b * p.H + h) * Sq + tid) * p.splits + s] = l2;
   }
-}
+  if (p.splits == 1) return;
 
-// Write the new rows' K and V (B, Sq, H, d) into the cache at positions seqlen_b - Sq + i:
-// one CTA per (i, b), each copying the row's H*d contiguous values of K and of V.
-__global__ void __launch_bounds__(256)
-    fa_decode_append_kernel(const DecParams p, int d, const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
-                            __nv_bfloat16* k_cache, __nv_bfloat16* v_cache) {
-  const int i = blockIdx.x, b = blockIdx.y;
-  const int n = p.seqlens[b];
-  if (n < 0 || n > p.max_pages * p.page_size) return;  // reported by the split kernel
-  const int pos = n - p.Sq + i;
-  if (pos < 0) return;  // the sequence is shorter than its new rows: nothing to place
-  const int page = p.block_table[(size_t)b * p.max_pages + pos / p.page_size];
-  if (page < 0 || page >= p.num_pages) {
-    if (threadIdx.x == 0) atomicOr(&g_fa_error, kErrBadInput);
-    return;
+  // ---- arrival: the last split of (b, h) merges all partials
+  __threadfence();  // this thread's partials are visible device-wide before the arrival
+  __syncthreads();
+  int* last = abort_flag + 1;
+  if (tid == 0) {
+    griddep_wait();  // the prep kernel has zeroed the counters
+    const int before = atomicAdd(&p.arrivals[(size_t)b * p.H + h], 1);
+    *last = before == p.splits - 1;
   }
-  const size_t row_elems = (size_t)p.H * d;
-  const size_t src = ((size_t)b * p.Sq + i) * row_elems;
-  const size_t dst = ((size_t)page * p.page_size + pos % p.page_size) * row_elems;
-  const int chunks = (int)(row_elems / 8);  // 16-byte chunks (d is 64 or 128)
-  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
-    reinterpret_cast<uint4*>(k_cache + dst)[c] = reinterpret_cast<const uint4*>(k_new + src)[c];
-    reinterpret_cast<uint4*>(v_cache + dst)[c] = reinterpret_cast<const uint4*>(v_new + src)[c];
-  }
-}
-
-// Merge the splits of one (b, h, i): O = sum_s 2^(L_s - L) O_s, L = log2 sum_s 2^L_s.
-template <int D>
-__global__ void __launch_bounds__(D) fa_decode_combine_kernel(const DecParams p) {
-  const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z, col = threadIdx.x;
-  const size_t row = ((size_t)b * p.H + h) * p.Sq + i;
-  const float* lp = p.lse_part + row * p.splits;
-  float mx = -INFINITY;
-  for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, lp[s]);
-  float wsum = 0.0f, v = 0.0f;
-  if (mx != -INFINITY) {
-    for (int s = 0; s < p.splits; ++s) {
-      const float w = ex2_approx(lp[s] - mx);
-      wsum += w;
-      v = fmaf(w, p.o_part[(row * p.splits + s) * D + col], v);
+  __syncthreads();
+  if (!*last) return;
+  __threadfence();
+  // O = sum_s 2^(L_s - L) O_s, L = log2 sum_s 2^L_s, in split order (the same sum whichever
+  // CTA arrives last)
+  for (int e = tid; e < Sq * D; e += kDecThreads) {
+    const int i = e / D, col = e - i * D;
+    const size_t row = ((size_t)b * p.H + h) * Sq + i;
+    const float* lp = p.lse_part + row * p.splits;
+    float mx = -INFINITY;
+    for (int u = 0; u < p.splits; ++u) mx = fmaxf(mx, __ldcg(lp + u));
+    float wsum = 0.0f, v = 0.0f;
+    if (mx != -INFINITY) {
+      for (int u = 0; u < p.splits; ++u) {
+        const float w = ex2_approx(__ldcg(lp + u) - mx);
+        wsum += w;
+        v = fmaf(w, __ldcg(p.o_part + (row * p.splits + u) * D + col), v);
+      }
     }
+    p.o[(((size_t)b * Sq + i) * p.H + h) * D + col] = __float2bfloat16_rn(wsum > 0.0f ? v / wsum : 0.0f);
+    if (col == 0) p.lse[row] = mx == -INFINITY ? -INFINITY : (mx + __log2f(wsum)) * kDecLn2;
   }
-  const float out = wsum > 0.0f ? v / wsum : 0.0f;
-  p.o[(((size_t)b * p.Sq + i) * p.H + h) * D + col] = __float2bfloat16_rn(out);
-  if (col == 0) p.lse[row] = mx == -INFINITY ? -INFINITY : (mx + __log2f(wsum)) * kDecLn2;
+}
+
+// Zero the (b, h) arrival counters of a split call. It lets the split kernel launch at once
+// (that kernel waits for this one only before its first arrival).
+__global__ void __launch_bounds__(256) fa_decode_prep_kernel(int* arrivals, int count) {
+  griddep_launch_dependents();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += gridDim.x * blockDim.x) arrivals[i] = 0;
 }
 
 }  // namespace fa

@@ -116,8 +116,9 @@ int fa_decode_splits(int B, int H, int max_keys);
 
 /*
  * Bytes of device workspace fa_decode_paged needs with `splits` splits per (b, h): the
- * float32 partial outputs (B,H,Sq,splits,d) and their log-sum-exps (B,H,Sq,splits), each
- * region 256-byte aligned; 0 when splits <= 1 (nothing to merge) or for invalid sizes.
+ * float32 partial outputs (B,H,Sq,splits,d), their log-sum-exps (B,H,Sq,splits) and one int32
+ * arrival counter per (b,h), each region 256-byte aligned; 0 when splits <= 1 (nothing to
+ * merge) or for invalid sizes.
  */
 size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits);
 
@@ -133,7 +134,9 @@ size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits);
  *   v_new        NULL, or (B,Sq,H,d) bf16 rows of the new tokens: written into the caches at
  *                positions seqlens[b] - Sq + i (as flash_attn_with_kvcache updates its cache in
  *                place) before the attention reads them. Both or neither; they, q, o, lse, the
- *                block table and the lengths must not overlap the caches.
+ *                block table and the lengths must not overlap the caches, and a cache row that
+ *                receives a new row must not be read by another sequence of the same call (no
+ *                page holding a new row is shared, and none appears twice in a block table).
  *   block_table  device (B,max_pages) int32: key j of sequence b is row j % page_size of page
  *                block_table[b*max_pages + j/page_size].
  *   seqlens      device (B) int32: keys held by sequence b (0 <= seqlens[b] <= max_pages*page_size).
@@ -144,10 +147,13 @@ size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits);
  * merged by log-sum-exp; 0 chooses a count from B*H and the SM count. With splits > 1 a
  * workspace of fa_decode_workspace_bytes(B,Sq,H,d,splits) bytes (256-byte aligned) is used; if
  * `workspace` is NULL the call allocates it with cudaMallocAsync/cudaFreeAsync on `stream`.
- * One to three launches on `stream` (append, split kernel, merge). Sequence lengths or page indices that are out of range are
- * not read: the sequence counts as empty (or the page as zeros) and fa_check() returns
- * FA_ERR_DEVICE. Host-visible errors as fa_fwd; Sq > 8 or a page_size that is not a multiple
- * of 64 give FA_ERR_UNSUPPORTED.
+ * One launch on `stream` with one split; with more, a small kernel that zeroes the arrival
+ * counters and the split kernel, launched as its programmatic dependent: each split CTA
+ * writes the new rows that fall in its key range, streams its range, and the last of a
+ * (b, h) to finish merges the partials. Sequence lengths or page indices that are out of
+ * range are not read: the sequence counts as empty (or the page as zeros) and fa_check()
+ * returns FA_ERR_DEVICE. Host-visible errors as fa_fwd (B or splits above 65535 are
+ * invalid); Sq > 8 or a page_size that is not a multiple of 64 give FA_ERR_UNSUPPORTED.
  */
 int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
                     const int* block_table, const int* seqlens, void* o, float* lse,

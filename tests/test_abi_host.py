@@ -130,6 +130,41 @@ def test_bwd_stage_calls_reject_invalid_arguments(lib):
     assert lib.fa_bwd_dq_convert(P, 1, 128, 2, 48, P + 6 * T, wsb, None) == UNSUPPORTED
 
 
+def test_decode_workspace_bytes(lib):
+    def expect(B, Sq, H, d, splits):
+        a = lambda x: (x + 255) // 256 * 256  # noqa: E731
+        rows = B * H * Sq * splits
+        return a(rows * d * 4) + a(rows * 4) + a(B * H * 4)  # partial O, partial LSE, arrival counters
+
+    for shape in [(3, 2, 4, 128, 6), (8, 1, 16, 128, 8), (1, 8, 1, 64, 2), (5, 3, 7, 64, 40)]:
+        assert lib.fa_decode_workspace_bytes(*shape) == expect(*shape)
+    assert lib.fa_decode_workspace_bytes(8, 1, 16, 128, 1) == 0  # one split: nothing to merge
+    assert lib.fa_decode_workspace_bytes(8, 1, 16, 96, 4) == 0
+    assert lib.fa_decode_workspace_bytes(0, 1, 16, 128, 4) == 0
+
+
+def _decode(lib, q=P, kc=P + T, vc=P + 2 * T, kn=None, vn=None, table=P + 3 * T, lens=P + 4 * T, o=P + 5 * T,
+            lse=P + 6 * T, B=2, Sq=1, H=2, d=128, num_pages=4, page_size=64, max_pages=2, scale=0.1, splits=0,
+            ws=None, ws_bytes=0):
+    return lib.fa_decode_paged(q, kc, vc, kn, vn, table, lens, o, lse, B, Sq, H, d, num_pages, page_size, max_pages,
+                               ctypes.c_float(scale), 1, -1, -1, splits, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(q=0), INVALID), (dict(table=0), INVALID), (dict(B=0), INVALID), (dict(Sq=0), INVALID),
+    (dict(Sq=9), UNSUPPORTED), (dict(d=96), UNSUPPORTED), (dict(page_size=96), UNSUPPORTED),
+    (dict(splits=-1), INVALID), (dict(splits=70000), INVALID), (dict(B=70000), INVALID),
+    (dict(kn=P + 7 * T), INVALID),                    # k_new without v_new
+    (dict(o=P + 8), INVALID), (dict(lse=P + 6 * T + 2), INVALID),
+    (dict(o=P), INVALID),                             # output aliases q
+    (dict(vc=P + T + 1024), INVALID),                 # the caches overlap
+    (dict(kn=P + 7 * T, vn=P + 8 * T, table=P + T + 64), INVALID),  # a written cache overlaps the table
+    (dict(scale=float("nan")), INVALID),
+])
+def test_decode_rejects_invalid_arguments(lib, kw, expected):
+    assert _decode(lib, **kw) == expected
+
+
 def test_binding_has_no_cpu_path():
     q = torch.zeros(1, 16, 1, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):

@@ -121,3 +121,71 @@ def test_decode_appends_new_rows_in_place(Sq):
     v_exp = oracle_dec.append_rows(vc.double().numpy(), v_new.double().numpy(), table.numpy(), lens.numpy(),
                                    cfg.page_size)
     assert np.array_equal(kc_d.double().cpu().numpy(), k_exp) and np.array_equal(vc_d.double().cpu().numpy(), v_exp)
+
+
+def _expect_rows(o, lse, o_ref, lse_ref, seqlens, what):
+    dead = ~np.isfinite(lse_ref)
+    assert np.array_equal(dead, ~np.isfinite(lse)), f"{what}: rows without keys differ"
+    if dead.any():
+        assert (o[dead.transpose(0, 2, 1)] == 0).all()
+    B, H = lse_ref.shape[:2]
+    for b in range(B):
+        for h in range(H):
+            rows = np.nonzero(~dead[b, h])[0]
+            if len(rows):
+                assert_fwd_close(o[b, rows, h], lse[b, h, rows], o_ref[b, rows, h], lse_ref[b, h, rows],
+                                 f"{what} b={b} h={h} len={int(seqlens[b])}")
+
+
+@pytest.mark.parametrize("splits", [1, 5, 40])
+@pytest.mark.parametrize("Sq,d,causal,win", [(8, 128, True, (-1, -1)), (2, 64, False, (3, 0)), (5, 128, True, (6, -1))])
+def test_decode_append_across_splits(splits, Sq, d, causal, win):
+    """Each new row is written by the split CTA whose key range holds it: rows that straddle a
+    tile (and, with many splits, a split) boundary, sequences shorter than Sq, an empty one,
+    window masks."""
+    cfg = DecodeConfig("append_splits", 5, Sq, 3, d, 1, 700, 64, causal, seed=80 + Sq + splits)
+    q, kc, vc, table, _ = make_decode_inputs(cfg)
+    lens = torch.tensor([0, Sq - 1, 644, 64, 1], dtype=torch.int32)
+    g = torch.Generator().manual_seed(90 + Sq)
+    k_new = torch.randn((cfg.B, Sq, cfg.H, d), generator=g).to(torch.bfloat16)
+    v_new = torch.randn((cfg.B, Sq, cfg.H, d), generator=g).to(torch.bfloat16)
+    kc_d, vc_d = kc.cuda(), vc.cuda()
+    o, lse = fa.attention_decode_paged(q.cuda(), kc_d, vc_d, table.cuda(), lens.cuda(), cfg.scale, causal, win, splits,
+                                       k_new=k_new.cuda(), v_new=v_new.cuda())
+    fa.check()
+    o_ref, lse_ref = oracle_dec.decode_forward(q.double().numpy(), kc.double().numpy(), vc.double().numpy(),
+                                               table.numpy(), lens.numpy(), cfg.scale, causal, *win,
+                                               k_new=k_new.double().numpy(), v_new=v_new.double().numpy())
+    _expect_rows(o.double().cpu().numpy(), lse.double().cpu().numpy(), o_ref, lse_ref, lens,
+                 f"append Sq={Sq} d={d} splits={splits}")
+    for cache_d, cache, new in ((kc_d, kc, k_new), (vc_d, vc, v_new)):
+        exp = oracle_dec.append_rows(cache.double().numpy(), new.double().numpy(), table.numpy(), lens.numpy(),
+                                     cfg.page_size)
+        assert np.array_equal(cache_d.double().cpu().numpy(), exp)
+
+
+def test_decode_workspace_contents_do_not_matter():
+    """The per-(b, h) arrival counters live in the caller's workspace and are zeroed by every
+    call: a workspace filled with splits - 1 everywhere (a counter that would make the first
+    arrival merge at once) and reused across calls gives the oracle's rows, bitwise the same
+    every time (the merge sums the splits in a fixed order)."""
+    cfg = DecodeConfig("workspace", 3, 2, 4, 128, 500, 1500, 128, True, seed=67)
+    q, kc, vc, table, lens = (t.cuda() for t in make_decode_inputs(cfg))
+    splits = 6
+    nbytes = fa.decode_workspace_bytes(cfg.B, cfg.Sq, cfg.H, cfg.d, splits)
+    assert nbytes > 0 and nbytes % 4 == 0
+    ws = torch.full((nbytes // 4,), splits - 1, dtype=torch.int32, device="cuda").view(torch.uint8)
+    o = torch.empty_like(q)
+    lse = torch.empty((cfg.B, cfg.H, cfg.Sq), dtype=torch.float32, device="cuda")
+    outs = []
+    for _ in range(3):
+        fa.decode_paged_into(q, kc, vc, table, lens, o, lse, cfg.scale, True, (-1, -1), splits, ws)
+        fa.check()
+        outs.append((o.clone(), lse.clone()))
+    for o2, l2 in outs[1:]:
+        assert torch.equal(o2, outs[0][0]) and torch.equal(l2, outs[0][1])
+    o_ref, lse_ref = oracle_dec.decode_forward(q.cpu().double().numpy(), kc.cpu().double().numpy(),
+                                               vc.cpu().double().numpy(), table.cpu().numpy(), lens.cpu().numpy(),
+                                               cfg.scale, True)
+    _expect_rows(outs[0][0].double().cpu().numpy(), outs[0][1].double().cpu().numpy(), o_ref, lse_ref,
+                 lens.cpu(), "garbage workspace")
