@@ -286,7 +286,7 @@ def run_gpu_decode(args):
     B, Sq, H, d = q.shape
     o = torch.empty_like(q)
     lse = torch.empty((B, H, Sq), dtype=torch.float32, device=dev)
-    splits = int(args.splits) or binding.decode_splits(B, H, cfg.max_pages * cfg.page_size)
+    splits = int(args.splits) or binding.decode_splits(B, Sq, H, d, cfg.max_pages * cfg.page_size)
     stream = torch.cuda.current_stream()
     # workspace of the split count in use (the library's choice unless --splits is given)
     ws = torch.empty(max(1, binding.decode_workspace_bytes(B, Sq, H, d, splits)), dtype=torch.uint8, device=dev)

@@ -47,7 +47,7 @@ def load() -> ctypes.CDLL:
     lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
     lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, i, vp, sz, vp]
     lib.fa_bwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, i, vp, sz, vp]
-    lib.fa_decode_splits.argtypes = [i, i, i]
+    lib.fa_decode_splits.argtypes = [i, i, i, i, i]
     lib.fa_decode_splits.restype = i
     lib.fa_decode_workspace_bytes.argtypes = [i, i, i, i, i]
     lib.fa_decode_workspace_bytes.restype = sz
@@ -316,9 +316,9 @@ def decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale=N
     _raise(st, "fa_decode_paged")
 
 
-def decode_splits(B: int, H: int, max_keys: int) -> int:
-    """The split count fa_decode_paged picks for splits=0 on the current device."""
-    n = int(load().fa_decode_splits(B, H, max_keys))
+def decode_splits(B: int, Sq: int, H: int, d: int, max_keys: int) -> int:
+    """The pieces per head fa_decode_paged picks for splits=0 on the current device."""
+    n = int(load().fa_decode_splits(B, Sq, H, d, max_keys))
     if n < 0:
         _raise(-n, "fa_decode_splits")
     return n

@@ -616,34 +616,58 @@ int launch_decode(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const
   return launch_decode_sq<D, 8>(grid, mk, mv, p, cs);
 }
 
-// Workspace of a split call: partial O (fp32), partial LSE, one arrival counter per (b, h).
-size_t decode_workspace_bytes(int B, int Sq, int H, int d, int splits) {
-  if (splits <= 1) return 0;
-  const size_t rows = (size_t)B * H * Sq * splits;
+// Workspace of a call with P > 1 pieces per head: partial O (fp32) and partial LSE for the
+// B + P - 1 (sequence, piece) slots, one arrival counter per (b, h).
+size_t decode_workspace_bytes(int B, int Sq, int H, int d, int pieces) {
+  if (pieces <= 1) return 0;
+  const size_t rows = ((size_t)B + pieces - 1) * H * Sq;
   return align256(rows * d * 4) + align256(rows * 4) + align256((size_t)B * H * 4);
 }
 
-// Splits per (b, h) when the caller passes 0: about seven CTAs per SM in total (two or three
-// fit at a time; measured best on a B8 H16 batch of 4-8K-key sequences), never more than the
-// 64-key tiles of the longest possible sequence, at most 128.
-int decode_auto_splits(int B, int H, int max_keys, int sm_count) {
-  const long long bh = (long long)B * H;
-  long long s = (7LL * sm_count + bh / 2) / bh;
-  const long long tiles = (max_keys + fa::kDecTile - 1) / fa::kDecTile;
-  if (s > tiles) s = tiles;
-  if (s > 128) s = 128;
-  return s < 1 ? 1 : (int)s;
+// CTAs of the split kernel for (d, Sq) that fit on one SM at a time (0 on error).
+template <int D>
+int decode_ctas_per_sm(int Sq) {
+  int n = 0;
+  cudaError_t e;
+  if (Sq == 1)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 1>, fa::kDecThreads,
+                                                      fa::DecCfg<D, 1>::kSmemBytes);
+  else if (Sq == 2)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 2>, fa::kDecThreads,
+                                                      fa::DecCfg<D, 2>::kSmemBytes);
+  else if (Sq <= 4)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 4>, fa::kDecThreads,
+                                                      fa::DecCfg<D, 4>::kSmemBytes);
+  else
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 8>, fa::kDecThreads,
+                                                      fa::DecCfg<D, 8>::kSmemBytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// Pieces per head when the caller passes 0: as many as fill every CTA slot of the GPU once
+// (H x P <= resident CTAs), at least 1, no more than the batch can have tiles, at most 65535.
+int decode_auto_pieces(int B, int Sq, int H, int d, int max_keys, int sm_count) {
+  const int per_sm = d == 64 ? decode_ctas_per_sm<64>(Sq) : decode_ctas_per_sm<128>(Sq);
+  long long pieces = (long long)std::max(per_sm, 1) * sm_count / H;
+  const long long tiles = (long long)B * ((max_keys + fa::kDecTile - 1) / fa::kDecTile);
+  pieces = std::min(pieces, std::min(tiles, 65535LL));
+  return pieces < 1 ? 1 : (int)pieces;
 }
 
 }  // namespace
 
 extern "C" {
 
-int fa_decode_splits(int B, int H, int max_keys) {
-  if (B < 1 || H < 1 || max_keys < 1) return -FA_ERR_INVALID_ARG;
+int fa_decode_splits(int B, int Sq, int H, int d, int max_keys) {
+  if (B < 1 || Sq < 1 || H < 1 || max_keys < 1 || d < 1) return -FA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || Sq > fa::kDecMaxSq) return -FA_ERR_UNSUPPORTED;
   int dev, sms, st;
   if ((st = device_setup(&dev, &sms))) return -st;
-  return decode_auto_splits(B, H, max_keys, sms);
+  return decode_auto_pieces(B, Sq, H, d, max_keys, sms);
 }
 
 size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits) {
@@ -664,7 +688,7 @@ int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_n
   if ((double)num_pages * page_size * H * d * 2 >= 1099511627776.0 ||
       (double)max_pages * page_size >= 2147483647.0)
     return FA_ERR_INVALID_ARG;
-  if (B > 65535 || splits > 65535 || (long long)B * H >= 2147483647LL) return FA_ERR_INVALID_ARG;  // grid limits
+  if (splits > 65535 || (long long)B * H >= 2147483647LL) return FA_ERR_INVALID_ARG;  // grid and counter limits
   if (!q || !k_cache || !v_cache || !block_table || !seqlens || !o || !lse) return FA_ERR_INVALID_ARG;
   if ((k_new == nullptr) != (v_new == nullptr)) return FA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
@@ -684,7 +708,7 @@ int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_n
       return FA_ERR_INVALID_ARG;
   int dev, sms, st;
   if ((st = device_setup(&dev, &sms))) return st;
-  if (splits == 0) splits = decode_auto_splits(B, H, max_pages * page_size, sms);
+  if (splits == 0) splits = decode_auto_pieces(B, Sq, H, d, max_pages * page_size, sms);
   const size_t wbytes = decode_workspace_bytes(B, Sq, H, d, splits);
   if (wbytes > 0 && workspace) {
     if (!aligned(workspace, 256) || workspace_bytes_ < wbytes) return FA_ERR_INVALID_ARG;
@@ -714,15 +738,16 @@ int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_n
   p.scale_log2 = scale * fa::kLog2e;
   p.win_l = win_l;
   p.win_r = win_r;
-  p.splits = splits;
+  p.pieces = splits;
   p.block_table = block_table;
   p.seqlens = seqlens;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.o_part = static_cast<float*>(ws);
-  const size_t part_bytes = align256((size_t)B * H * Sq * splits * d * 4);
-  const size_t lse_part_bytes = align256((size_t)B * H * Sq * splits * 4);
+  const size_t part_rows = ((size_t)B + splits - 1) * H * Sq;  // (sequence, piece) slots
+  const size_t part_bytes = align256(part_rows * d * 4);
+  const size_t lse_part_bytes = align256(part_rows * 4);
   p.lse_part = wbytes ? reinterpret_cast<float*>(static_cast<char*>(ws) + part_bytes) : nullptr;
   p.arrivals = wbytes ? reinterpret_cast<int*>(static_cast<char*>(ws) + part_bytes + lse_part_bytes) : nullptr;
   p.k_new = static_cast<const __nv_bfloat16*>(k_new);
@@ -737,7 +762,7 @@ int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_n
     st = launch_status();
   }
   if (!st) {
-    const dim3 grid(H, splits, B);  // heads fastest: concurrent CTAs share cache rows
+    const dim3 grid(H, splits);  // heads fastest: concurrent CTAs share cache rows
     if (d == 64)
       st = launch_decode<64>(grid, mk, mv, p, cs);
     else

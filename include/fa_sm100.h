@@ -107,18 +107,21 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_desca
                fa_stream_t stream);
 
 /*
- * The split count fa_decode_paged uses when called with splits = 0, for B sequences, H heads
- * and at most max_keys keys per sequence (max_pages * page_size), on the current device: about
- * seven CTAs per SM over B*H, at most one per 64-key tile and at most 128. Negative status on
- * error (-FA_ERR_INVALID_ARG, -FA_ERR_UNSUPPORTED without an sm_100 device, -FA_ERR_CUDA).
+ * The number of pieces per head fa_decode_paged uses when called with splits = 0, for B
+ * sequences of Sq new rows, H heads of dim d and at most max_keys keys per sequence
+ * (max_pages * page_size), on the current device: as many as let the H x pieces CTAs run at
+ * once (CTAs per SM x SM count / H), at least 1, at most the B * ceil(max_keys / 64) tiles
+ * the batch can have and 65535. Negative status on error (-FA_ERR_INVALID_ARG,
+ * -FA_ERR_UNSUPPORTED for d other than 64 / 128, Sq > 8 or without an sm_100 device,
+ * -FA_ERR_CUDA).
  */
-int fa_decode_splits(int B, int H, int max_keys);
+int fa_decode_splits(int B, int Sq, int H, int d, int max_keys);
 
 /*
- * Bytes of device workspace fa_decode_paged needs with `splits` splits per (b, h): the
- * float32 partial outputs (B,H,Sq,splits,d), their log-sum-exps (B,H,Sq,splits) and one int32
- * arrival counter per (b,h), each region 256-byte aligned; 0 when splits <= 1 (nothing to
- * merge) or for invalid sizes.
+ * Bytes of device workspace fa_decode_paged needs with `splits` pieces per head: the float32
+ * partial outputs (B+splits-1,H,Sq,d) and their log-sum-exps (B+splits-1,H,Sq) of the
+ * (sequence, piece) slots, and one int32 arrival counter per (b,h), each region 256-byte
+ * aligned; 0 when splits <= 1 (nothing to merge) or for invalid sizes.
  */
 size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits);
 
@@ -143,16 +146,18 @@ size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits);
  *   o, lse       (B,Sq,H,d) bf16 and (B,H,Sq) float32 natural-log LSE; a row that sees no key
  *                gets O = 0 and LSE = -inf.
  * Masks as fa_fwd, taken at each row's position (causal keeps keys j <= position). d is 64 or
- * 128. `splits` cuts every (b, h)'s keys into that many ranges processed in parallel and then
- * merged by log-sum-exp; 0 chooses a count from B*H and the SM count. With splits > 1 a
- * workspace of fa_decode_workspace_bytes(B,Sq,H,d,splits) bytes (256-byte aligned) is used; if
- * `workspace` is NULL the call allocates it with cudaMallocAsync/cudaFreeAsync on `stream`.
- * One launch on `stream` with one split; with more, a small kernel that zeroes the arrival
- * counters and the split kernel, launched as its programmatic dependent: each split CTA
- * writes the new rows that fall in its key range, streams its range, and the last of a
- * (b, h) to finish merges the partials. Sequence lengths or page indices that are out of
- * range are not read: the sequence counts as empty (or the page as zeros) and fa_check()
- * returns FA_ERR_DEVICE. Host-visible errors as fa_fwd (B or splits above 65535 are
+ * 128. `splits` is the number of CTAs per head: each head's visible 64-key tiles, listed
+ * sequence after sequence, are cut into that many equal contiguous pieces processed in
+ * parallel; a sequence spread over several pieces is merged by log-sum-exp. 0 chooses
+ * fa_decode_splits(B,Sq,H,d,max_pages*page_size). With splits > 1 a workspace of
+ * fa_decode_workspace_bytes(B,Sq,H,d,splits) bytes (256-byte aligned, any contents) is used;
+ * if `workspace` is NULL the call allocates it with cudaMallocAsync/cudaFreeAsync on `stream`.
+ * One launch on `stream` with one piece per head; with more, a small kernel that zeroes the
+ * arrival counters and the split kernel, launched as its programmatic dependent: each CTA
+ * writes the new rows that fall in its piece, streams its piece, and the last piece of a
+ * sequence to finish merges that sequence's partials. Sequence lengths or page indices that
+ * are out of range are not read: the sequence counts as empty (or the page as zeros) and
+ * fa_check() returns FA_ERR_DEVICE. Host-visible errors as fa_fwd (splits above 65535 is
  * invalid); Sq > 8 or a page_size that is not a multiple of 64 give FA_ERR_UNSUPPORTED.
  */
 int fa_decode_paged(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,

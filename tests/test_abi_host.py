@@ -131,9 +131,9 @@ def test_bwd_stage_calls_reject_invalid_arguments(lib):
 
 
 def test_decode_workspace_bytes(lib):
-    def expect(B, Sq, H, d, splits):
+    def expect(B, Sq, H, d, pieces):
         a = lambda x: (x + 255) // 256 * 256  # noqa: E731
-        rows = B * H * Sq * splits
+        rows = (B + pieces - 1) * H * Sq  # (sequence, piece) slots
         return a(rows * d * 4) + a(rows * 4) + a(B * H * 4)  # partial O, partial LSE, arrival counters
 
     for shape in [(3, 2, 4, 128, 6), (8, 1, 16, 128, 8), (1, 8, 1, 64, 2), (5, 3, 7, 64, 40)]:
@@ -153,7 +153,7 @@ def _decode(lib, q=P, kc=P + T, vc=P + 2 * T, kn=None, vn=None, table=P + 3 * T,
 @pytest.mark.parametrize("kw,expected", [
     (dict(q=0), INVALID), (dict(table=0), INVALID), (dict(B=0), INVALID), (dict(Sq=0), INVALID),
     (dict(Sq=9), UNSUPPORTED), (dict(d=96), UNSUPPORTED), (dict(page_size=96), UNSUPPORTED),
-    (dict(splits=-1), INVALID), (dict(splits=70000), INVALID), (dict(B=70000), INVALID),
+    (dict(splits=-1), INVALID), (dict(splits=70000), INVALID),
     (dict(kn=P + 7 * T), INVALID),                    # k_new without v_new
     (dict(o=P + 8), INVALID), (dict(lse=P + 6 * T + 2), INVALID),
     (dict(o=P), INVALID),                             # output aliases q
@@ -163,6 +163,14 @@ def _decode(lib, q=P, kc=P + T, vc=P + 2 * T, kn=None, vn=None, table=P + 3 * T,
 ])
 def test_decode_rejects_invalid_arguments(lib, kw, expected):
     assert _decode(lib, **kw) == expected
+
+
+def test_decode_splits_rejects_invalid_arguments(lib):
+    assert lib.fa_decode_splits(0, 1, 16, 128, 4096) == -INVALID
+    assert lib.fa_decode_splits(8, 0, 16, 128, 4096) == -INVALID
+    assert lib.fa_decode_splits(8, 1, 16, 128, 0) == -INVALID
+    assert lib.fa_decode_splits(8, 9, 16, 128, 4096) == -UNSUPPORTED
+    assert lib.fa_decode_splits(8, 1, 16, 96, 4096) == -UNSUPPORTED
 
 
 def test_binding_has_no_cpu_path():

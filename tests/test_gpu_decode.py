@@ -4,8 +4,9 @@ The kernel computes scores, the online softmax and P·V in fp32 on the CUDA core
 exact bf16 inputs (P is not rounded), so the forward's tolerances apply: per row
 max |ΔO| / max(1, |O_ref|) <= 1e-2 and max |ΔLSE| <= 1e-3. Cases cover ragged lengths (empty,
 shorter than Sq, one key, page and tile boundaries), causal / window / full masks, Sq = 1..8,
-page sizes 64..512, split counts 1, automatic and more splits than tiles, and the full decode
-workload compared row by row.
+page sizes 64..512, piece counts 1, automatic and more pieces than tiles, pieces that span
+several sequences and sequences spread over several pieces, and the full decode workload
+compared row by row.
 """
 
 from __future__ import annotations
@@ -71,6 +72,25 @@ def test_decode_masks(causal, win, d):
 def test_decode_rows_and_page_sizes(Sq, page):
     cfg = DecodeConfig("pages", 4, Sq, 4, 128, 1, 1500, page, True, seed=63 + Sq)
     check(cfg, splits=0, what=f"Sq={Sq} page={page}")
+
+
+@pytest.mark.parametrize("splits", [1, 2, 7, 0])
+def test_decode_pieces_cross_sequences(splits):
+    """Pieces of the concatenated tile list that span several short (and empty) sequences, and
+    sequences spread over several pieces."""
+    lens = [0, 1, 2, 63, 64, 65, 0, 130, 3, 700, 1, 0, 257, 5, 64, 1]
+    cfg = DecodeConfig("cross", len(lens), 2, 3, 128, 1, 704, 64, True, seed=69)
+    check(cfg, lens=lens, splits=splits, what=f"pieces={splits}")
+
+
+@pytest.mark.parametrize("splits", [3, 0])
+def test_decode_many_sequences(splits):
+    """More sequences than threads in a CTA (the tile prefix sums run over several sequences per
+    thread), d = 64, a window."""
+    g = np.random.default_rng(70)
+    lens = [int(x) for x in g.integers(0, 200, size=300)]
+    cfg = DecodeConfig("many", 300, 1, 2, 64, 1, 200, 64, False, seed=70)
+    check(cfg, lens=lens, splits=splits, causal=False, win=(90, 0), what=f"B=300 pieces={splits}")
 
 
 def test_decode_split_counts_agree():
