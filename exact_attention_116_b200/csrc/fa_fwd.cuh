@@ -17,12 +17,19 @@
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
 // P_t (bf16, two per column) is the A operand of O_t += P_t V_j, read straight from TMEM.
 //
-// D = 128 (TMEM full): P_t overwrites the first 64 columns of S_t. MMA issue order per KV
-// tile j: S0(j), PV1(j-1), S1(j), PV0(j). tcgen05.mma operations issued by one thread
-// execute in order, so S_t(j) never overwrites P_t(j-1) before PV_t(j-1) has read it, and
-// the commit that signals "S_t(j) ready" also covers PV_t(j-1): when a softmax thread sees
-// S_t(j), O_t is quiescent and may be rescaled in place. The O tile is staged for its TMA
-// store in the Q_t buffer.
+// D = 128, bf16 (kShareS): the two tiles share one S buffer (columns [0,128)), P_t has its
+// own columns (P0 [128,192), P1 [192,256)), O0 [256,384), O1 [384,512). The S buffer holds
+// S0(j), S1(j), S0(j+1), ... in turn, each issued as soon as the softmax threads have read the
+// previous one into registers ("S empty"), so a tile's next scores do not wait for its P·V.
+// MMA issue order per KV tile j: S0(j+1), PV0(j), S1(j+1), PV1(j). A softmax thread writes
+// P_t(j+1) and rescales O_t only after the commit of PV_t(j) ("PV done"). The O tile is staged
+// for its TMA store in the Q_t buffer (free once the item's last PV_t is done).
+//
+// D = 128, E4M3: P_t overwrites the first 32 columns of S_t. MMA issue order per KV tile j:
+// S0(j), PV1(j-1), S1(j), PV0(j). tcgen05.mma operations issued by one thread execute in
+// order, so S_t(j) never overwrites P_t(j-1) before PV_t(j-1) has read it, and the commit that
+// signals "S_t(j) ready" also covers PV_t(j-1): when a softmax thread sees S_t(j), O_t is
+// quiescent and may be rescaled in place.
 //
 // D = 64 (kSepP): P_t has its own columns P0 [384,448), P1 [448,512), so S_t(j+1) is issued
 // as soon as the softmax threads have read S_t(j) into registers ("S empty"), one tile ahead
@@ -80,8 +87,9 @@ struct FwdCfg {
   static constexpr int kBoxElems = 128 / kElem;       // elements per box row
   static constexpr int kOBoxes = D / 64;              // 64-column boxes per O tile
   static constexpr int kSlots = (kTileBytes == 32768) ? 4 : 8;
-  static constexpr bool kSepP = (D == 64 && !kF8);    // P apart from S in TMEM
-  static constexpr bool kSepO = kSepP || kF8;         // O staging apart from Q; Q freed by the last S
+  static constexpr bool kShareS = (D == 128 && !kF8);  // one S buffer for both tiles
+  static constexpr bool kSepP = (D == 64 && !kF8) || kShareS;  // P apart from S in TMEM
+  static constexpr bool kSepO = (D == 64) || kF8;     // O staging apart from Q; Q freed by the last S
   static constexpr int kKSteps = D * kElem / 32;      // MMA steps over d (32 bytes of K each)
   static constexpr int kPvSteps = kF8 ? 4 : 8;        // MMA steps over the 128 keys of P
   static constexpr int kOffQ = 0;                     // Q0, Q1 (also O staging unless kSepO)
@@ -89,8 +97,9 @@ struct FwdCfg {
   static constexpr int kOffKV = kSepO ? kOffO + 2 * kOTileBytes : 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
-  static constexpr uint32_t kColP0 = kSepP ? 384 : kColS0, kColP1 = kSepP ? 448 : kColS1;
+  static constexpr uint32_t kColS0 = 0, kColS1 = kShareS ? 0 : 128, kColO0 = 256, kColO1 = 256 + D;
+  static constexpr uint32_t kColP0 = kShareS ? 128 : kSepP ? 384 : kColS0;
+  static constexpr uint32_t kColP1 = kShareS ? 192 : kSepP ? 448 : kColS1;
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -100,7 +109,7 @@ struct FwdBars {
   uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[Cfg::kSlots], kv_empty[Cfg::kSlots];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
-  uint64_t s_empty[2], pv_done[2];  // kSepP only
+  uint64_t s_empty[2], pv_done[2];  // kSepP only (kShareS: s_empty[0] for the shared S)
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -410,7 +419,54 @@ __global__ void __launch_bounds__(384, 1)
           if (act[t]) mbar_wait(bar(bars->q_full[t]), qn[t] & 1, ab);
         tc_fence_after_sync();
 
-        if constexpr (Cfg::kSepP) {
+        if constexpr (Cfg::kShareS) {
+          // K(j) is tile n0 + 2(j - lo) of the K/V stream and V(j) the next one; stream tile n
+          // sits in slot n % kSlots, filled for the (n / kSlots)-th time.
+          const uint32_t n0 = kvn;
+          auto kv_wait = [&](uint32_t n) {
+            const uint32_t s = n % Cfg::kSlots;
+            mbar_wait(bar(bars->kv_full[s]), (n / Cfg::kSlots) & 1, ab);
+            tc_fence_after_sync();
+            return s;
+          };
+          auto s_shared = [&](int t, uint32_t ks) {  // S_t into the shared buffer once the last S is read
+            mbar_wait(bar(bars->s_empty[0]), (sq[0] & 1) ^ 1, ab);
+            ++sq[0];
+            tc_fence_after_sync();
+            issue_s(t, sKV + ks * Cfg::kTileBytes);
+            if (drop_s_signal) drop_s_signal = false;
+            else mma_commit(bar(bars->s_full[t]));
+          };
+          auto pv = [&](int t, uint32_t vs) {
+            mbar_wait(bar(bars->p_full[t]), pn[t] & 1, ab);
+            ++pn[t];
+            tc_fence_after_sync();
+            issue_pv(t, sKV + vs * Cfg::kTileBytes, !first_pv[t]);
+            first_pv[t] = false;
+            mma_commit(bar(bars->pv_done[t]));
+          };
+          {
+            const uint32_t ks = kv_wait(n0);  // S0(lo), S1(lo)
+            for (int t = 0; t < 2; ++t)
+              if (active(t, lo)) s_shared(t, ks);
+            mma_commit(bar(bars->kv_empty[ks]));
+          }
+          for (int j = lo; j <= hi; ++j) {
+            const bool more = j < hi;
+            const uint32_t vs = kv_wait(n0 + 2 * (j - lo) + 1);
+            const uint32_t ks = more ? kv_wait(n0 + 2 * (j + 1 - lo)) : 0;
+            if (more && active(0, j + 1)) s_shared(0, ks);
+            if (active(0, j)) pv(0, vs);
+            if (more && active(1, j + 1)) s_shared(1, ks);
+            if (more) mma_commit(bar(bars->kv_empty[ks]));
+            if (active(1, j)) pv(1, vs);
+            mma_commit(bar(bars->kv_empty[vs]));
+          }
+          kvn = n0 + 2 * (hi - lo + 1);
+          for (int t = 0; t < 2; ++t)
+            if (act[t]) ++qn[t];
+          continue;
+        } else if constexpr (Cfg::kSepP) {
           // K(j) is tile n0 + 2(j - lo) of the K/V stream and V(j) the next one; stream tile n
           // sits in slot n % kSlots, filled for the (n / kSlots)-th time.
           const uint32_t n0 = kvn;
@@ -559,9 +615,9 @@ __global__ void __launch_bounds__(384, 1)
         for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, r[q4]);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) tmem_wait_ld(r[q4]);
-        if constexpr (Cfg::kSepP) {  // S_t may now be overwritten by the next tile's scores
+        if constexpr (Cfg::kSepP) {  // S_t may now be overwritten by the next scores
           tc_fence_before_sync();
-          mbar_arrive(bar(bars->s_empty[t]));
+          mbar_arrive(bar(bars->s_empty[Cfg::kShareS ? 0 : t]));
         }
         float x[128];
 #pragma unroll
@@ -584,7 +640,7 @@ __global__ void __launch_bounds__(384, 1)
           ++pvn;
           tc_fence_after_sync();
         }
-        // P in 32-column chunks straight into TMEM (D = 128: over S columns already read into registers)
+        // P in 32-column chunks straight into TMEM (E4M3: over S columns already read into registers)
         float2 sum0 = make_float2(0.0f, 0.0f), sum1 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
