@@ -14,29 +14,26 @@
 //   warps 2-3   : no role
 //   warps 4-7   : softmax + epilogue for Q tile 0 (one thread per query row / TMEM lane)
 //   warps 8-11  : softmax + epilogue for Q tile 1
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
-// P_t (bf16, two per column) is the A operand of O_t += P_t V_j, read straight from TMEM.
+// TMEM (512 columns): O0 [256,256+D), O1 [256+D, 256+2D); S and P as below. P_t (bf16, two
+// per column; E4M3, four) is the A operand of O_t += P_t V_j, read straight from TMEM.
 //
-// D = 128, bf16 (kShareS): the two tiles share one S buffer (columns [0,128)), P_t has its
-// own columns (P0 [128,192), P1 [192,256)), O0 [256,384), O1 [384,512). The S buffer holds
-// S0(j), S1(j), S0(j+1), ... in turn, each issued as soon as the softmax threads have read the
-// previous one into registers ("S empty"), so a tile's next scores do not wait for its P·V.
-// MMA issue order per KV tile j: S0(j+1), PV0(j), S1(j+1), PV1(j). A softmax thread writes
-// P_t(j+1) and rescales O_t only after the commit of PV_t(j) ("PV done"). The O tile is staged
-// for its TMA store in the Q_t buffer (free once the item's last PV_t is done).
+// D = 128 (kShareS): the two tiles share one S buffer (columns [0,128)), P_t has its own
+// columns (P0 from 128, P1 from 192: 64 columns of bf16 pairs or 32 of E4M3 quads), O0
+// [256,384), O1 [384,512). The S buffer holds S0(j), S1(j), S0(j+1), ... in turn, each issued
+// as soon as the softmax threads have read the previous one into registers ("S empty"), so a
+// tile's next scores do not wait for its P·V. MMA issue order per KV tile j: S0(j+1), PV0(j),
+// S1(j+1), PV1(j). A softmax thread writes P_t(j+1) and rescales O_t only after the commit of
+// PV_t(j) ("PV done"). bf16: the O tile is staged for its TMA store in the Q_t buffer (free
+// once the item's last PV_t is done); E4M3: O has staging buffers of its own and Q_t is
+// released by the commit of the item's last S_t.
 //
-// D = 128, E4M3: P_t overwrites the first 32 columns of S_t. MMA issue order per KV tile j:
-// S0(j), PV1(j-1), S1(j), PV0(j). tcgen05.mma operations issued by one thread execute in
-// order, so S_t(j) never overwrites P_t(j-1) before PV_t(j-1) has read it, and the commit that
-// signals "S_t(j) ready" also covers PV_t(j-1): when a softmax thread sees S_t(j), O_t is
-// quiescent and may be rescaled in place.
-//
-// D = 64 (kSepP): P_t has its own columns P0 [384,448), P1 [448,512), so S_t(j+1) is issued
-// as soon as the softmax threads have read S_t(j) into registers ("S empty"), one tile ahead
-// of PV_t(j): the next scores are ready when a softmax thread finishes a tile. A softmax
-// thread writes P_t(j+1) and rescales O_t only after the commit of PV_t(j) ("PV done"). O is
-// staged in buffers of its own, so Q_t is released by the commit of the item's last S_t and
-// the next item's Q and K/V loads overlap this item's last tiles and epilogue.
+// D = 64: each tile has its own S (S0 [0,128), S1 [128,256)) and P (P0 [384,448), P1
+// [448,512)) columns, so S_t(j+1) is issued as soon as the softmax threads have read S_t(j)
+// into registers ("S empty"), one tile ahead of PV_t(j): the next scores are ready when a
+// softmax thread finishes a tile. A softmax thread writes P_t(j+1) and rescales O_t only after
+// the commit of PV_t(j) ("PV done"). O is staged in buffers of its own, so Q_t is released by
+// the commit of the item's last S_t and the next item's Q and K/V loads overlap this item's
+// last tiles and epilogue.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -87,8 +84,8 @@ struct FwdCfg {
   static constexpr int kBoxElems = 128 / kElem;       // elements per box row
   static constexpr int kOBoxes = D / 64;              // 64-column boxes per O tile
   static constexpr int kSlots = (kTileBytes == 32768) ? 4 : 8;
-  static constexpr bool kShareS = (D == 128 && !kF8);  // one S buffer for both tiles
-  static constexpr bool kSepP = (D == 64 && !kF8) || kShareS;  // P apart from S in TMEM
+  static constexpr bool kShareS = (D == 128);          // one S buffer for both tiles
+  static_assert(D == 128 || !kF8, "E4M3 tiles are 128 bytes wide: d = 128");
   static constexpr bool kSepO = (D == 64) || kF8;     // O staging apart from Q; Q freed by the last S
   static constexpr int kKSteps = D * kElem / 32;      // MMA steps over d (32 bytes of K each)
   static constexpr int kPvSteps = kF8 ? 4 : 8;        // MMA steps over the 128 keys of P
@@ -98,8 +95,7 @@ struct FwdCfg {
   static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
   static constexpr uint32_t kColS0 = 0, kColS1 = kShareS ? 0 : 128, kColO0 = 256, kColO1 = 256 + D;
-  static constexpr uint32_t kColP0 = kShareS ? 128 : kSepP ? 384 : kColS0;
-  static constexpr uint32_t kColP1 = kShareS ? 192 : kSepP ? 448 : kColS1;
+  static constexpr uint32_t kColP0 = kShareS ? 128 : 384, kColP1 = kShareS ? 192 : 448;  // P apart from S
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -108,8 +104,8 @@ template <class Cfg>
 struct FwdBars {
   uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[Cfg::kSlots], kv_empty[Cfg::kSlots];
-  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
-  uint64_t s_empty[2], pv_done[2];  // kSepP only (kShareS: s_empty[0] for the shared S)
+  uint64_t s_full[2], p_full[2];
+  uint64_t s_empty[2], pv_done[2];  // kShareS: s_empty[0] for the shared S
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -288,8 +284,6 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(bars->q_empty[t]), 1);
       mbar_init(bar(bars->s_full[t]), 1);
       mbar_init(bar(bars->p_full[t]), 128);
-      mbar_init(bar(bars->o_full[t]), 1);
-      mbar_init(bar(bars->o_empty[t]), 128);
       mbar_init(bar(bars->s_empty[t]), 128);
       mbar_init(bar(bars->pv_done[t]), 1);
     }
@@ -375,9 +369,8 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t tS[2] = {tmem + Cfg::kColS0, tmem + Cfg::kColS1};
       const uint32_t tO[2] = {tmem + Cfg::kColO0, tmem + Cfg::kColO1};
       const uint32_t tP[2] = {tmem + Cfg::kColP0, tmem + Cfg::kColP1};
-      uint32_t slot = 0, phase = 0;
       uint32_t qn[2] = {0, 0}, pn[2] = {0, 0};
-      uint32_t kvn = 0, sq[2] = {0, 0};  // kSepP: K/V stream position, S_t issued
+      uint32_t kvn = 0, sq[2] = {0, 0};  // K/V stream position, S issued (per tile, or shared)
       bool drop_s_signal = p.debug_drop_s_signal != 0;
 
       auto issue_s = [&](int t, uint32_t k_smem) {
@@ -429,13 +422,14 @@ __global__ void __launch_bounds__(384, 1)
             tc_fence_after_sync();
             return s;
           };
-          auto s_shared = [&](int t, uint32_t ks) {  // S_t into the shared buffer once the last S is read
+          auto s_shared = [&](int t, int j, uint32_t ks) {  // S_t(j) into the shared buffer once the last S is read
             mbar_wait(bar(bars->s_empty[0]), (sq[0] & 1) ^ 1, ab);
             ++sq[0];
             tc_fence_after_sync();
             issue_s(t, sKV + ks * Cfg::kTileBytes);
             if (drop_s_signal) drop_s_signal = false;
             else mma_commit(bar(bars->s_full[t]));
+            if (Cfg::kSepO && j == hi_t[t]) mma_commit(bar(bars->q_empty[t]));  // last read of Q_t (O staged apart)
           };
           auto pv = [&](int t, uint32_t vs) {
             mbar_wait(bar(bars->p_full[t]), pn[t] & 1, ab);
@@ -448,16 +442,16 @@ __global__ void __launch_bounds__(384, 1)
           {
             const uint32_t ks = kv_wait(n0);  // S0(lo), S1(lo)
             for (int t = 0; t < 2; ++t)
-              if (active(t, lo)) s_shared(t, ks);
+              if (active(t, lo)) s_shared(t, lo, ks);
             mma_commit(bar(bars->kv_empty[ks]));
           }
           for (int j = lo; j <= hi; ++j) {
             const bool more = j < hi;
             const uint32_t vs = kv_wait(n0 + 2 * (j - lo) + 1);
             const uint32_t ks = more ? kv_wait(n0 + 2 * (j + 1 - lo)) : 0;
-            if (more && active(0, j + 1)) s_shared(0, ks);
+            if (more && active(0, j + 1)) s_shared(0, j + 1, ks);
             if (active(0, j)) pv(0, vs);
-            if (more && active(1, j + 1)) s_shared(1, ks);
+            if (more && active(1, j + 1)) s_shared(1, j + 1, ks);
             if (more) mma_commit(bar(bars->kv_empty[ks]));
             if (active(1, j)) pv(1, vs);
             mma_commit(bar(bars->kv_empty[vs]));
@@ -465,8 +459,7 @@ __global__ void __launch_bounds__(384, 1)
           kvn = n0 + 2 * (hi - lo + 1);
           for (int t = 0; t < 2; ++t)
             if (act[t]) ++qn[t];
-          continue;
-        } else if constexpr (Cfg::kSepP) {
+        } else {
           // K(j) is tile n0 + 2(j - lo) of the K/V stream and V(j) the next one; stream tile n
           // sits in slot n % kSlots, filled for the (n / kSlots)-th time.
           const uint32_t n0 = kvn;
@@ -508,61 +501,8 @@ __global__ void __launch_bounds__(384, 1)
           kvn = n0 + 2 * (hi - lo + 1);
           for (int t = 0; t < 2; ++t)
             if (act[t]) ++qn[t];
-          continue;
         }
 
-        uint32_t v_prev_slot = 0;
-        auto wait_p_and_o = [&](int t) {
-          mbar_wait(bar(bars->p_full[t]), pn[t] & 1, ab);
-          ++pn[t];
-          if (first_pv[t]) mbar_wait(bar(bars->o_empty[t]), (qn[t] & 1) ^ 1, ab);
-          tc_fence_after_sync();
-        };
-        for (int j = lo; j <= hi + 1; ++j) {
-          uint32_t k_slot = 0;
-          if (j <= hi) {
-            k_slot = slot;
-            mbar_wait(bar(bars->kv_full[slot]), phase, ab);
-            if (++slot == Cfg::kSlots) { slot = 0; phase ^= 1; }
-            tc_fence_after_sync();
-            if (active(0, j)) {
-              issue_s(0, sKV + k_slot * Cfg::kTileBytes);
-              if (drop_s_signal) drop_s_signal = false;
-              else mma_commit(bar(bars->s_full[0]));
-              if (Cfg::kSepO && j == hi_t[0]) mma_commit(bar(bars->q_empty[0]));  // last read of Q_0
-            }
-          }
-          if (j - 1 >= lo) {
-            if (active(1, j - 1)) {
-              wait_p_and_o(1);
-              issue_pv(1, sKV + v_prev_slot * Cfg::kTileBytes, !first_pv[1]);
-              first_pv[1] = false;
-              if (j - 1 == hi_t[1]) mma_commit(bar(bars->o_full[1]));
-            }
-            mma_commit(bar(bars->kv_empty[v_prev_slot]));
-          }
-          if (j <= hi) {
-            if (active(1, j)) {
-              issue_s(1, sKV + k_slot * Cfg::kTileBytes);
-              mma_commit(bar(bars->s_full[1]));
-              if (Cfg::kSepO && j == hi_t[1]) mma_commit(bar(bars->q_empty[1]));  // last read of Q_1
-            }
-            mma_commit(bar(bars->kv_empty[k_slot]));
-            const uint32_t v_slot = slot;
-            mbar_wait(bar(bars->kv_full[slot]), phase, ab);
-            if (++slot == Cfg::kSlots) { slot = 0; phase ^= 1; }
-            tc_fence_after_sync();
-            if (active(0, j)) {
-              wait_p_and_o(0);
-              issue_pv(0, sKV + v_slot * Cfg::kTileBytes, !first_pv[0]);
-              first_pv[0] = false;
-              if (j == hi_t[0]) mma_commit(bar(bars->o_full[0]));
-            }
-            v_prev_slot = v_slot;
-          }
-        }
-        for (int t = 0; t < 2; ++t)
-          if (act[t]) ++qn[t];
       }
       mma_commit(bar(bars->mma_done));
       mbar_drain(bar(bars->mma_done), 0);
@@ -575,7 +515,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = tmem + lane_field + (t ? Cfg::kColS1 : Cfg::kColS0);
     const uint32_t tO = tmem + lane_field + (t ? Cfg::kColO1 : Cfg::kColO0);
     const uint32_t tP = tmem + lane_field + (t ? Cfg::kColP1 : Cfg::kColP0);
-    uint32_t sn = 0, on = 0, pvn = 0;
+    uint32_t sn = 0, pvn = 0;
 
     for (int round = 0;; ++round) {
       const int w = sched_item(round, blockIdx.x, gridDim.x);
@@ -615,10 +555,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, r[q4]);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) tmem_wait_ld(r[q4]);
-        if constexpr (Cfg::kSepP) {  // S_t may now be overwritten by the next scores
-          tc_fence_before_sync();
-          mbar_arrive(bar(bars->s_empty[Cfg::kShareS ? 0 : t]));
-        }
+        tc_fence_before_sync();  // the S buffer may now take the next scores
+        mbar_arrive(bar(bars->s_empty[Cfg::kShareS ? 0 : t]));
         float x[128];
 #pragma unroll
         for (int cc = 0; cc < 128; ++cc) x[cc] = __uint_as_float(r[cc >> 5][cc & 31]);
@@ -635,7 +573,7 @@ __global__ void __launch_bounds__(384, 1)
         else
           fwd_row_max<false>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated);
         const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
-        if (Cfg::kSepP && j > lo) {  // PV_t(j-1) has read P_t and O_t is quiescent
+        if (j > lo) {  // PV_t(j-1) has read P_t and O_t is quiescent
           mbar_wait(bar(bars->pv_done[t]), pvn & 1, ab);
           ++pvn;
           tc_fence_after_sync();
@@ -682,13 +620,8 @@ __global__ void __launch_bounds__(384, 1)
       }
 
       // Epilogue: O_t / l -> bf16 -> staging (the Q_t buffer, free once the last PV_t is done) -> TMA store.
-      if constexpr (Cfg::kSepP) {
-        mbar_wait(bar(bars->pv_done[t]), pvn & 1, ab);  // the item's last PV_t
-        ++pvn;
-      } else {
-        mbar_wait(bar(bars->o_full[t]), on & 1, ab);
-        ++on;
-      }
+      mbar_wait(bar(bars->pv_done[t]), pvn & 1, ab);  // the item's last PV_t
+      ++pvn;
       tc_fence_after_sync();
       if constexpr (Cfg::kSepO) {
         if (row == 0) bulk_wait_group_read0();  // the previous store has read the staging tile
@@ -710,10 +643,6 @@ __global__ void __launch_bounds__(384, 1)
             w4[e] = pack_bf16x2(__uint_as_float(o[ch * 8 + 2 * e]) * inv_l, __uint_as_float(o[ch * 8 + 2 * e + 1]) * inv_l);
           st_shared_v4(box + sw128_offset(row, ((cc & 63) >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
         }
-      }
-      if constexpr (!Cfg::kSepP) {
-        tc_fence_before_sync();
-        mbar_arrive(bar(bars->o_empty[t]));
       }
       fence_proxy_async_smem();
       named_bar_sync(1 + t, 128);
