@@ -476,7 +476,8 @@ def run_gpu_fp8(args):
                      "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
                      "frac_of_bf16_peak": round(achieved / peak["bf16_tflops"], 4),
                      "peak_source": f"{peak_src} bf16_tflops x {FP8_PER_BF16} (nominal dense FP8/BF16 ratio)",
-                     "traffic": None, "algorithmic_bytes": in_bytes + B * N * H * d * 2 + B * H * N * 4},
+                     "traffic": recorded_traffic("fa_fwd_kernel<128, E4M3>"),
+                     "algorithmic_bytes": in_bytes + B * N * H * d * 2 + B * H * N * 4},
         "e2e": {"value": round(mg.aggregate_rate(f_fwd, world, e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": B * N * H * d * 2 + B * H * N * 4},
