@@ -310,8 +310,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 
 int launch_pre(const void* o, const float* lse, const void* dO, const Shape& s, const Workspace& w,
                cudaStream_t stream) {
-  const long long warps = (long long)s.B * s.n_pad() * s.H;
-  const long long blocks = (warps + 7) / 8;
+  const long long rows_per_cta = s.d == 64 ? fa::PreCfg<64>::kRows : fa::PreCfg<128>::kRows;
+  const long long blocks = (long long)s.B * s.H * (s.n_pad() / rows_per_cta);
   if (s.d == 64)
     fa::fa_bwd_pre_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, w.lse2, w.dvec, w.dq_acc,

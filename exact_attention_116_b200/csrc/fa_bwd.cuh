@@ -67,9 +67,17 @@ constexpr int kBwdPolyNum = FA_BWD_POLY_NUM, kBwdPolyDen = FA_BWD_POLY_DEN;
 
 // ------------------------------------------------------------------ preprocess
 
-// One warp per (b, n, h) row with n < N_pad: -D = -sum_c dO*O in fp32 and -LSE*log2(e)
-// (0 for padding rows; stored negated so that the main kernel adds them), and the row of the
-// dQ accumulator set to zero. Also resets the main kernel's work counter.
+// Per (b, h) row n < N_pad: -D = -sum_c dO*O in fp32 and -LSE*log2(e) (0 for padding rows;
+// stored negated so that the main kernel adds them), and the row of the dQ accumulator set to
+// zero. A CTA takes kPreRows consecutive rows of one (b, h), D/8 threads per row with 16-byte
+// loads of O and dO, so the row vectors are read and written contiguously. Also resets the
+// main kernel's work counters.
+template <int D>
+struct PreCfg {
+  static constexpr int kThreadsPerRow = D / 8;                // 8 bf16 (16 bytes) per thread
+  static constexpr int kRows = 256 / kThreadsPerRow;           // rows per CTA: 16 (D=128), 32 (D=64)
+};
+
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
@@ -77,40 +85,33 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
                                                          float* __restrict__ dvec, float* __restrict__ dq_acc,
                                                          int* __restrict__ next_item, int B, int N, int H,
                                                          int N_pad) {
-  const long long warp_g = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  using Cfg = PreCfg<D>;
   if (blockIdx.x == 0 && threadIdx.x < 2) next_item[threadIdx.x] = 0;
-  const long long total = (long long)B * N_pad * H;
-  if (warp_g >= total) return;
-  const int h = (int)(warp_g % H);
-  const long long bn = warp_g / H;
-  const int n = (int)(bn % N_pad);
-  const int b = (int)(bn / N_pad);
-  const size_t stat = ((size_t)b * H + h) * (size_t)N_pad + n;
-  if (n >= N) {
-    if (lane == 0) { lse2[stat] = 0.0f; dvec[stat] = 0.0f; }
-    return;
-  }
-  const size_t row = (((size_t)b * N + n) * H + h) * (size_t)D;
-  constexpr int kPer = D / 32;  // bf16 elements per lane: 2 (D=64) or 4 (D=128)
+  const int blocks_per_head = N_pad / Cfg::kRows;
+  const long long bh = blockIdx.x / blocks_per_head;  // b * H + h
+  const int n = (int)(blockIdx.x % blocks_per_head) * Cfg::kRows + (int)threadIdx.x / Cfg::kThreadsPerRow;
+  const int part = (int)threadIdx.x % Cfg::kThreadsPerRow;
+  if (bh >= (long long)B * H) return;
+  const int b = (int)(bh / H), h = (int)(bh % H);
+  const size_t stat = (size_t)bh * (size_t)N_pad + n;
   float acc = 0.0f;
-  if (kPer == 4) {
-    const uint2 ov = *reinterpret_cast<const uint2*>(o + row + lane * 4);
-    const uint2 gv = *reinterpret_cast<const uint2*>(dout + row + lane * 4);
-    acc = bf16lo_to_f32(ov.x) * bf16lo_to_f32(gv.x) + bf16hi_to_f32(ov.x) * bf16hi_to_f32(gv.x) +
-          bf16lo_to_f32(ov.y) * bf16lo_to_f32(gv.y) + bf16hi_to_f32(ov.y) * bf16hi_to_f32(gv.y);
-    *reinterpret_cast<float4*>(dq_acc + row + lane * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-  } else {
-    const uint32_t ov = *reinterpret_cast<const uint32_t*>(o + row + lane * 2);
-    const uint32_t gv = *reinterpret_cast<const uint32_t*>(dout + row + lane * 2);
-    acc = bf16lo_to_f32(ov) * bf16lo_to_f32(gv) + bf16hi_to_f32(ov) * bf16hi_to_f32(gv);
-    *reinterpret_cast<float2*>(dq_acc + row + lane * 2) = make_float2(0.f, 0.f);
+  if (n < N) {
+    const size_t row = (((size_t)b * N + n) * H + h) * (size_t)D + part * 8;
+    const uint4 ov = *reinterpret_cast<const uint4*>(o + row);
+    const uint4 gv = *reinterpret_cast<const uint4*>(dout + row);
+    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      acc += bf16lo_to_f32(ow[e]) * bf16lo_to_f32(gw[e]) + bf16hi_to_f32(ow[e]) * bf16hi_to_f32(gw[e]);
+    float4* z = reinterpret_cast<float4*>(dq_acc + row);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    dvec[stat] = -acc;
-    lse2[stat] = -lse[((size_t)b * H + h) * (size_t)N + n] * kLog2e;
+  for (int off = Cfg::kThreadsPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (part == 0) {
+    dvec[stat] = n < N ? -acc : 0.0f;
+    lse2[stat] = n < N ? -lse[(size_t)bh * (size_t)N + n] * kLog2e : 0.0f;
   }
 }
 
