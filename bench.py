@@ -759,7 +759,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default="train_fwd_bwd",
                     choices=sorted(CONFIGS) + sorted(FP8_CONFIGS) + sorted(DECODE_CONFIGS))
-    ap.add_argument("--splits", type=int, default=0, help="decode: KV splits per (b, h); 0 = library's choice")
+    ap.add_argument("--splits", type=int, default=0, help="decode: CTAs (pieces) per head; 0 = library's choice")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
