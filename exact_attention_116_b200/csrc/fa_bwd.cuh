@@ -22,9 +22,11 @@
 //   warps 12-15  P/dS for query columns [64, 128); dV epilogue
 // TMEM: dK [0,D), dV [D,2D), dP^T / dQ [2D, 2D+128), S^T / P^T [2D+128, 2D+256).
 // Per Q tile i the MMA warp issues dP^T = V dO_i^T, dV += P^T dO_i (P^T from TMEM), then
-// S^T for tile i+1 (= K Q_{i+1}^T), then dQ_i = dS K_j and dK += dS^T Q_i (dS^T in shared
-// memory, read MN-major for dQ and K-major for dK). Issuing S(i+1) early lets the P of tile
-// i+1 be computed while dQ and dK of tile i run; dQ goes first so its columns free up early.
+// S^T for tile i+1 (= K Q_{i+1}^T), dQ_i = dS K_j and dK += dS^T Q_i (dS^T in shared memory,
+// read MN-major for dQ and K-major for dK). At d = 64, S(i+1) goes before dQ(i): the P of tile
+// i+1 is computed while dQ and dK of tile i run. At d = 128, dQ(i) goes before S(i+1): its
+// columns, which dP(i+1) reuses, free up one matrix product earlier (measured faster at each
+// head dim respectively). dQ always precedes dK.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -272,6 +274,7 @@ __global__ void __launch_bounds__(512, 1)
                   const __grid_constant__ CUtensorMap tmdQacc, const BwdParams p) {
   using Cfg = BwdCfg<D>;
   static_assert(sizeof(BwdBars) <= 256, "barrier block");
+  constexpr bool kDqFirst = D == 128;  // MMA order per Q tile: see the issuer
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = smem_u32(smem_raw);
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw + Cfg::kOffBar);
@@ -392,8 +395,9 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    // Per Q tile i: dP(i), dV(i), then S(i+1) ahead of dQ(i), dK(i), so that the P of tile i+1
-    // is computed while the tensor core works on dQ and dK of tile i.
+    // Per Q tile i: dP(i), dV(i), then S(i+1), dQ(i), dK(i) at d = 64 (the P of tile i+1 is
+    // computed while the tensor core works on dQ and dK of tile i) or dQ(i), S(i+1), dK(i) at
+    // d = 128 (dQ(i) and its drain from TMEM, which the next dP waits for, start earlier).
     if (elect_one()) {
       constexpr uint32_t idSP = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T: K-major A and B
       constexpr uint32_t idKV = idesc_bf16_f32(128, D, false, true);     // dV, dK: B (dO, Q) MN-major
@@ -451,9 +455,11 @@ __global__ void __launch_bounds__(512, 1)
             mma_ts(tDV, tS + acol, sdesc_mnmajor(sDO + kk * 2048, 16384), idKV, !first || kk > 0);
           }
           mma_commit(bar(bars->do_empty[dos]));
-          // S(i+1): overwrites P^T(i), which dV(i) (issued before) has read
+          // S(i+1): overwrites P^T(i), which dV(i) (issued before) has read. d = 64 issues it
+          // here, ahead of dQ(i), so that the P of tile i+1 is computed meanwhile; d = 128
+          // issues dQ(i) first, which shortens the chain dS(i) -> dQ(i) -> dQ drained -> dP(i+1).
           const uint32_t nqs = qs ^ 1, nqphase = qs ? (qphase ^ 1) : qphase;
-          if (i < hi) issue_s(nqs, nqphase);
+          if (!kDqFirst && i < hi) issue_s(nqs, nqphase);
           // dQ_i = dS K_j, then dK += dS^T Q_i
           mbar_wait(bar(bars->ds_full), n & 1, ab);
           tc_fence_after_sync();
@@ -463,6 +469,7 @@ __global__ void __launch_bounds__(512, 1)
               mma_ss(tDP, sdesc_mnmajor(sDS + kk * 2048, 16384), sdesc_mnmajor(sK + kk * 2048, 16384), idQ, kk > 0);
             mma_commit(bar(bars->dq_full));
           }
+          if (kDqFirst && i < hi) issue_s(nqs, nqphase);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
