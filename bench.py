@@ -81,6 +81,77 @@ def recorded_traffic(kernel: str):
     return k.get("dram_bytes_per_launch")
 
 
+# ----------------------------------------------------------------------------- end to end
+
+def pipelined_e2e(info, dev, sets, copy_in, compute, copy_out, steps: int, warm: int = 4) -> float:
+    """Time `steps` end-to-end steps through the public API, pipelined over three streams and
+    len(sets) device buffer sets: every step copies its inputs host -> device (copy_in(set)),
+    runs the path (compute(set, stream)) and copies its outputs device -> host (copy_out(set)).
+    Step k's outputs travel down while step k+1's inputs travel up and step k+1 computes (PCIe
+    is full duplex), so throughput is bounded by the slowest of the three, not their sum. A set
+    is refilled only after its previous compute has read it, and recomputed only after its
+    previous outputs are on the host. Returns the device time per step (ms, max over ranks) from
+    the first copy-in to the last copy-out."""
+    s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    n = len(sets)
+    ev = {name: [torch.cuda.Event() for _ in range(n)] for name in ("in", "comp", "out")}
+    started = [False] * n
+
+    def one(k):
+        b = k % n
+        with torch.cuda.stream(s_in):
+            if started[b]:
+                s_in.wait_event(ev["comp"][b])  # the set's previous compute has read its inputs
+            copy_in(sets[b])
+            ev["in"][b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev["in"][b])
+            if started[b]:
+                s_comp.wait_event(ev["out"][b])  # the set's previous outputs are on the host
+            compute(sets[b], s_comp)
+            ev["comp"][b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev["comp"][b])
+            copy_out(sets[b])
+            ev["out"][b].record(s_out)
+        started[b] = True
+
+    for k in range(warm):
+        one(k)
+    torch.cuda.synchronize()
+    mg.barrier(info)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    s_comp.wait_event(e0)
+    s_out.wait_event(e0)
+    for k in range(steps):
+        one(k)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_comp)
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    mg.barrier(info)
+    return mg.max_over_ranks(info, e0.elapsed_time(e1), dev) / steps
+
+
+def packed_buffers(dev, specs, pin=False):
+    """One byte buffer holding tensors of the given (shape, dtype) specs at 256-byte aligned
+    offsets, and views of it: a single copy moves them all."""
+    offs, total = [], 0
+    for shape, dt in specs:
+        total = (total + 255) // 256 * 256
+        offs.append(total)
+        total += int(np.prod(shape)) * torch.empty((), dtype=dt).element_size()
+    buf = torch.empty(total, dtype=torch.uint8, device=dev)
+    if pin:
+        buf = buf.pin_memory()
+    views = []
+    for (shape, dt), off in zip(specs, offs):
+        nb = int(np.prod(shape)) * torch.empty((), dtype=dt).element_size()
+        views.append(buf[off:off + nb].view(dt).view(shape))
+    return buf, views
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -328,34 +399,31 @@ def run_gpu_decode(args):
     gbs = nbytes / (ms_step * 1e-3) / 1e9
 
     # a step's host inputs: the new rows' q, K, V, the block table and the lengths (the cache is
-    # device-resident state, as in a serving loop)
+    # device-resident state, as in a serving loop), packed in one pinned buffer so that a step is
+    # one copy up and one copy down (O and LSE packed likewise)
     step_inputs = (host[0], kn_h, vn_h, host[3], host[4])
-    pin = [x.pin_memory() for x in step_inputs]
-    o_h = torch.empty_like(host[0]).pin_memory()
-    lse_h = torch.empty((B, H, Sq), dtype=torch.float32).pin_memory()
-
-    def e2e_step():
-        for src, dst in zip(pin, (q, k_new, v_new, table, lens)):
-            dst.copy_(src, non_blocking=True)
-        step()
-        o_h.copy_(o, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
-
-    e2e_steps = max(3, min(args.steps, 10))
+    in_specs = [(tuple(x.shape), x.dtype) for x in step_inputs]
+    out_specs = [(tuple(o.shape), o.dtype), (tuple(lse.shape), lse.dtype)]
+    in_h, in_h_views = packed_buffers("cpu", in_specs, pin=True)
+    for dst, src in zip(in_h_views, step_inputs):
+        dst.copy_(src)
+    out_h, _ = packed_buffers("cpu", out_specs, pin=True)
+    e2e_sets = []
     for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    mg.barrier(info)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    mg.barrier(info)
+        in_d, in_v = packed_buffers(dev, in_specs)
+        out_d, out_v = packed_buffers(dev, out_specs)
+        e2e_sets.append((in_d, in_v, out_d, out_v))
+
+    def dec_compute(st, s):
+        (qd, knd, vnd, td, ld), (od, lsed) = st[1], st[3]
+        binding.decode_paged_into(qd, kc, vc, td, ld, od, lsed, cfg.scale, cfg.causal, (cfg.win_l, cfg.win_r),
+                                  splits, ws, stream=s, k_new=knd, v_new=vnd)
+
+    e2e_steps = max(4, min(args.steps, 50))
+    e2e_ms = pipelined_e2e(info, dev, e2e_sets, lambda st: st[0].copy_(in_h, non_blocking=True), dec_compute,
+                           lambda st: out_h.copy_(st[2], non_blocking=True), e2e_steps)
     binding.check()
-    e2e_ms = mg.max_over_ranks(info, e0.elapsed_time(e1), dev) / e2e_steps
-    h2d = sum(x.numel() * x.element_size() for x in step_inputs)
+    h2d = in_h.numel()
 
     peak, peak_src = peaks()
     res = {
@@ -377,7 +445,10 @@ def run_gpu_decode(args):
                      "traffic": recorded_traffic("fa_decode_split_kernel"), "algorithmic_bytes": nbytes},
         "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4},
+                "d2h_bytes_per_step": out_h.numel(),
+                "pipelining": "one packed copy up (q, new K/V rows, block table, lengths) and one down (O, LSE) per "
+                              "step, on their own streams, overlapping the previous and next steps' compute (two "
+                              "device buffer sets)"},
         "gpu_launches": (2 if splits > 1 else 1) * args.steps,  # counter zeroing, split kernel
         "clocks": clocks,
     }
@@ -435,28 +506,23 @@ def run_gpu_fp8(args):
     pin = [x.pin_memory() for x in (*codes_h, *desc_h)]
     o_h = torch.empty((B, N, H, d), dtype=torch.bfloat16).pin_memory()
     lse_h = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    e2e_sets = [((*codes, *desc), (o, lse))]
+    e2e_sets.append((tuple(torch.empty_like(x) for x in (*codes, *desc)), (torch.empty_like(o), torch.empty_like(lse))))
 
-    def e2e_step():
-        for src, dst in zip(pin, (*codes, *desc)):
+    def fp8_copy_in(st):
+        for src, dst in zip(pin, st[0]):
             dst.copy_(src, non_blocking=True)
-        binding.fwd_fp8_into(*codes, *desc, o, lse, scale, causal, win)
-        o_h.copy_(o, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
 
-    e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    mg.barrier(info)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    mg.barrier(info)
+    def fp8_compute(st, s):
+        binding.fwd_fp8_into(*st[0], *st[1], scale, causal, win, stream=s)
+
+    def fp8_copy_out(st):
+        o_h.copy_(st[1][0], non_blocking=True)
+        lse_h.copy_(st[1][1], non_blocking=True)
+
+    e2e_steps = max(4, min(args.steps, 20))
+    e2e_ms = pipelined_e2e(info, dev, e2e_sets, fp8_copy_in, fp8_compute, fp8_copy_out, e2e_steps)
     binding.check()
-    e2e_ms = mg.max_over_ranks(info, e0.elapsed_time(e1), dev) / e2e_steps
 
     peak, peak_src = peaks()
     fp8_peak = peak["bf16_tflops"] * FP8_PER_BF16
@@ -480,7 +546,9 @@ def run_gpu_fp8(args):
                      "algorithmic_bytes": in_bytes + B * N * H * d * 2 + B * H * N * 4},
         "e2e": {"value": round(mg.aggregate_rate(f_fwd, world, e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": in_bytes,
-                "d2h_bytes_per_step": B * N * H * d * 2 + B * H * N * 4},
+                "d2h_bytes_per_step": B * N * H * d * 2 + B * H * N * 4,
+                "pipelining": "copy-in, fa_fwd_fp8 and copy-out of consecutive steps on three streams with two "
+                              "device buffer sets (every step copies its own inputs and outputs)"},
         "gpu_launches": args.steps,
         "clocks": clocks,
     }
@@ -559,63 +627,32 @@ def run_gpu(args):
     bwd_ms = pre_ms + main_ms + conv_ms
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region.
-    # Every step copies its inputs host -> device, runs fa_fwd + fa_bwd and copies its outputs back.
-    # Steps are pipelined over three streams and two device buffer sets: step k's outputs travel
-    # device -> host while step k+1's inputs travel host -> device and step k+1 computes (PCIe is
-    # full duplex), so throughput is bounded by the slowest of the three, not their sum.
+    # Every step copies its inputs host -> device, runs fa_fwd + fa_bwd and copies its outputs back,
+    # pipelined over three streams and two device buffer sets (pipelined_e2e).
     pin = [x.pin_memory() for x in (q_h, k_h, v_h, do_h)]
     out_h = [torch.empty_like(q_h).pin_memory() for _ in range(4)]
     lse_h = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
     sets = [((q, k, v, do), (o, dq, dk, dv), lse, ws)]
     sets.append((tuple(torch.empty_like(x) for x in (q, k, v, do)), tuple(torch.empty_like(x) for x in (o, dq, dk, dv)),
                  torch.empty_like(lse), torch.empty_like(ws)))
-    s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("in", "comp", "out")}
-    started = [False, False]
 
-    def e2e_step(kstep):
-        b_ = kstep % 2
-        (qi, ki, vi, doi), (oo, dqo, dko, dvo), lseo, wso = sets[b_]
-        with torch.cuda.stream(s_in):
-            if started[b_]:
-                s_in.wait_event(ev["comp"][b_])  # the set's previous compute has read its inputs
-            for src, dst in zip(pin, (qi, ki, vi, doi)):
-                dst.copy_(src, non_blocking=True)
-            ev["in"][b_].record(s_in)
-        with torch.cuda.stream(s_comp):
-            s_comp.wait_event(ev["in"][b_])
-            if started[b_]:
-                s_comp.wait_event(ev["out"][b_])  # the set's previous outputs are on the host
-            binding.fwd_into(qi, ki, vi, oo, lseo, scale, causal, win, stream=s_comp)
-            binding.bwd_into(qi, ki, vi, oo, lseo, doi, dqo, dko, dvo, scale, causal, win, workspace=wso,
-                             stream=s_comp)
-            ev["comp"][b_].record(s_comp)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev["comp"][b_])
-            for src, dst in zip((oo, dqo, dko, dvo), out_h):
-                dst.copy_(src, non_blocking=True)
-            lse_h.copy_(lseo, non_blocking=True)
-            ev["out"][b_].record(s_out)
-        started[b_] = True
+    def train_copy_in(st):
+        for src, dst in zip(pin, st[0]):
+            dst.copy_(src, non_blocking=True)
+
+    def train_compute(st, s):
+        (qi, ki, vi, doi), (oo, dqo, dko, dvo), lseo, wso = st
+        binding.fwd_into(qi, ki, vi, oo, lseo, scale, causal, win, stream=s)
+        binding.bwd_into(qi, ki, vi, oo, lseo, doi, dqo, dko, dvo, scale, causal, win, workspace=wso, stream=s)
+
+    def train_copy_out(st):
+        for src, dst in zip(st[1], out_h):
+            dst.copy_(src, non_blocking=True)
+        lse_h.copy_(st[2], non_blocking=True)
 
     e2e_steps = max(4, min(args.steps, 20))
-    for kstep in range(4):
-        e2e_step(kstep)
-    torch.cuda.synchronize()
-    mg.barrier(info)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    s_comp.wait_event(e0)
-    s_out.wait_event(e0)
-    for kstep in range(e2e_steps):
-        e2e_step(kstep)
-    s_out.wait_stream(s_in)
-    s_out.wait_stream(s_comp)
-    e1.record(s_out)
-    torch.cuda.synchronize()
-    mg.barrier(info)
+    e2e_ms = pipelined_e2e(info, dev, sets, train_copy_in, train_compute, train_copy_out, e2e_steps)
     binding.check()
-    e2e_ms = mg.max_over_ranks(info, e0.elapsed_time(e1), dev) / e2e_steps
 
     peak, peak_src = peaks()
     main_tflops = f_bwd / (main_ms * 1e-3) / 1e12
