@@ -18,6 +18,7 @@ from .binding import (  # noqa: F401
     bwd_stages,
     check,
     decode_paged_into,
+    decode_splits,
     decode_workspace_bytes,
     flash_attention,
     fwd_fp8_into,

@@ -209,3 +209,16 @@ def test_decode_workspace_contents_do_not_matter():
                                                cfg.scale, True)
     _expect_rows(outs[0][0].double().cpu().numpy(), outs[0][1].double().cpu().numpy(), o_ref, lse_ref,
                  lens.cpu(), "garbage workspace")
+
+
+def test_decode_auto_pieces_fill_the_gpu_once():
+    """fa_decode_splits: the automatic piece count lets all H x P CTAs run at once (no second
+    wave) and uses at least one CTA per SM; it never exceeds the batch's possible tiles."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    for B, Sq, H, d, keys in [(8, 1, 16, 128, 8192), (8, 8, 16, 128, 8192), (4, 2, 8, 64, 4096), (1, 1, 2, 128, 65536)]:
+        pieces = fa.decode_splits(B, Sq, H, d, keys)
+        assert 1 <= pieces <= 65535
+        assert pieces <= B * -(-keys // 64)
+        assert H * pieces >= sms, (B, Sq, H, d, pieces)  # at least one CTA per SM
+        assert H * pieces <= 8 * sms, (B, Sq, H, d, pieces)  # bounded by CTAs that fit per SM
+    assert fa.decode_splits(1, 1, 2, 128, 64) == 1  # one tile: one piece
