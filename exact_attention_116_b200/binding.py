@@ -290,7 +290,10 @@ def decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale=N
                       splits=0, workspace=None, stream=None, k_new=None, v_new=None) -> None:
     """fa_decode_paged: q (B,Sq,H,d) bf16 new rows; k_cache, v_cache (num_pages,page_size,H,d) bf16;
     block_table (B,max_pages) int32; seqlens (B,) int32; into o (B,Sq,H,d) bf16, lse (B,H,Sq) float32.
-    k_new, v_new: optional (B,Sq,H,d) bf16 rows written into the caches first (in place)."""
+    k_new, v_new: optional (B,Sq,H,d) bf16 rows written into the caches first (in place).
+    splits: CTAs per head (each head's visible tiles, listed sequence after sequence, cut into that
+    many equal pieces); 0 = decode_splits(). workspace: decode_workspace_bytes(B,Sq,H,d,splits)
+    bytes (any contents), or None to allocate on the stream."""
     B, Sq, H, d = _check_qkv(q, o)
     if (k_new is None) != (v_new is None):
         raise ValueError("give both k_new and v_new, or neither")
