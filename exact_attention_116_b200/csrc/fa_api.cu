@@ -59,8 +59,8 @@ template <int D, bool kAlibi, bool kVarlen>
 bool variant_attributes() {
   const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
   const int smem = fa::BwdCfg<D>::kSmemBytes, smem_dq = fa::BwdDqCfg<D>::kSmemBytes;
-  return cudaFuncSetAttribute(fa::fa_fwd_kernel<D, false, kAlibi, kVarlen>, attr, fa::FwdCfg<D>::kSmemBytes) ==
-             cudaSuccess &&
+  const int smem_fwd = fa::FwdCfg<D>::kSmemBytes + (kVarlen ? fa::kFwdSortBytes : 0);
+  return cudaFuncSetAttribute(fa::fa_fwd_kernel<D, false, kAlibi, kVarlen>, attr, smem_fwd) == cudaSuccess &&
          cudaFuncSetAttribute(fa::fa_bwd_kernel<D, true, kAlibi, kVarlen>, attr, smem) == cudaSuccess &&
          cudaFuncSetAttribute(fa::fa_bwd_kernel<D, false, kAlibi, kVarlen>, attr, smem) == cudaSuccess &&
          cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<D, kAlibi, kVarlen>, attr, smem_dq) == cudaSuccess;
@@ -234,8 +234,8 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_
 template <int D, bool kAlibi, bool kVarlen>
 void fwd_launch(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                 const CUtensorMap& mo, const fa::FwdParams& p) {
-  fa::fa_fwd_kernel<D, false, kAlibi, kVarlen><<<grid, fa::FwdCfg<D>::kThreads, fa::FwdCfg<D>::kSmemBytes, stream>>>(
-      mq, mk, mv, mo, p);
+  constexpr int smem = fa::FwdCfg<D>::kSmemBytes + (kVarlen ? fa::kFwdSortBytes : 0);
+  fa::fa_fwd_kernel<D, false, kAlibi, kVarlen><<<grid, fa::FwdCfg<D>::kThreads, smem, stream>>>(mq, mk, mv, mo, p);
 }
 
 template <int D>

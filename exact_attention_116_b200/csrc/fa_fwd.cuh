@@ -60,6 +60,13 @@ struct FwdParams {
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
 
+// Packed batches: the cost of a pair of Q tiles (its visible KV tiles) does not fall with its
+// index, so every CTA sorts the pairs by decreasing cost (ties: higher index first) before
+// dealing them out; the same deterministic order in every CTA keeps each item dealt once.
+// Up to kFwdSortMaxPairs pairs (524288 tokens); above that the index order is kept.
+constexpr int kFwdSortMaxPairs = 2048;
+constexpr int kFwdSortBytes = 4 * kFwdSortMaxPairs;  // uint16 cost and order per pair
+
 // Share of the exponentials computed by exp2_poly on the FMA pipes instead of MUFU: pair p of
 // a row's 64 pairs uses the polynomial when p % kPolyDen < kPolyNum.
 #ifndef FA_FWD_POLY_NUM
@@ -94,6 +101,7 @@ struct FwdCfg {
   static constexpr int kOffKV = kSepO ? kOffO + 2 * kOTileBytes : 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
+  static constexpr int kOffSort = kOffBar + 512;            // packed batches: pair costs and order
   static constexpr uint32_t kColS0 = 0, kColS1 = kShareS ? 0 : 128, kColO0 = 256, kColO1 = 256 + D;
   static constexpr uint32_t kColP0 = kShareS ? 128 : 384, kColP1 = kShareS ? 192 : 448;  // P apart from S
   static constexpr uint32_t kTmemCols = 512;
@@ -111,11 +119,13 @@ struct FwdBars {
   int abort_flag;
 };
 
-// Item w -> (b, h, pair). Under causal masking pairs are visited longest first.
-__device__ __forceinline__ void fwd_decode(const FwdParams& p, int w, int& b, int& h, int& pair) {
+// Item w -> (b, h, pair). Under causal masking pairs are visited longest first; for a packed
+// batch `order` (when given) lists the pairs by decreasing cost.
+__device__ __forceinline__ void fwd_decode(const FwdParams& p, int w, int& b, int& h, int& pair,
+                                           const uint16_t* order = nullptr) {
   const int bh_count = p.B * p.H;
   const int r = w / bh_count, bh = w - r * bh_count;
-  pair = p.causal ? (p.num_pairs - 1 - r) : r;
+  pair = order ? (int)order[r] : p.causal ? (p.num_pairs - 1 - r) : r;
   b = bh / p.H;
   h = bh - b * p.H;
 }
@@ -303,6 +313,31 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
     tc_fence_before_sync();
   }
+  // packed batch: pair order by decreasing cost, computed by the whole CTA
+  const uint16_t* order = nullptr;
+  if constexpr (kVarlen) {
+    if (p.num_pairs <= kFwdSortMaxPairs) {
+      uint16_t* sCost = reinterpret_cast<uint16_t*>(smem_gen + Cfg::kOffSort);
+      uint16_t* sOrder = sCost + kFwdSortMaxPairs;
+      for (int q = threadIdx.x; q < p.num_pairs; q += blockDim.x) {
+        int lo0, hi0, lo1, hi1;
+        fwd_kv_range<true>(p, q * 256, lo0, hi0);
+        fwd_kv_range<true>(p, q * 256 + 128, lo1, hi1);
+        sCost[q] = (uint16_t)(max(0, hi0 - lo0 + 1) + max(0, hi1 - lo1 + 1));
+      }
+      __syncthreads();
+      for (int q = threadIdx.x; q < p.num_pairs; q += blockDim.x) {
+        const int c = sCost[q];
+        int rank = 0;
+        for (int u = 0; u < p.num_pairs; ++u) {
+          const int cu = sCost[u];
+          rank += (cu > c) | ((cu == c) & (u > q));
+        }
+        sOrder[rank] = (uint16_t)q;
+      }
+      order = sOrder;
+    }
+  }
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
@@ -323,7 +358,7 @@ __global__ void __launch_bounds__(384, 1)
         const int w = sched_item(round, blockIdx.x, gridDim.x);
         if (w >= p.num_items || ab.raised()) break;
         int b, h, pair;
-        fwd_decode(p, w, b, h, pair);
+        fwd_decode(p, w, b, h, pair, order);
         int lo_t[2], hi_t[2];
         fwd_kv_range<kVarlen>(p, pair * 256, lo_t[0], hi_t[0]);
         fwd_kv_range<kVarlen>(p, pair * 256 + 128, lo_t[1], hi_t[1]);
@@ -399,7 +434,7 @@ __global__ void __launch_bounds__(384, 1)
         const int w = sched_item(round, blockIdx.x, gridDim.x);
         if (w >= p.num_items || ab.raised()) break;
         int b, h, pair;
-        fwd_decode(p, w, b, h, pair);
+        fwd_decode(p, w, b, h, pair, order);
         int lo_t[2], hi_t[2];
         fwd_kv_range<kVarlen>(p, pair * 256, lo_t[0], hi_t[0]);
         fwd_kv_range<kVarlen>(p, pair * 256 + 128, lo_t[1], hi_t[1]);
@@ -521,7 +556,7 @@ __global__ void __launch_bounds__(384, 1)
       const int w = sched_item(round, blockIdx.x, gridDim.x);
       if (w >= p.num_items || ab.raised()) break;
       int b, h, pair;
-      fwd_decode(p, w, b, h, pair);
+      fwd_decode(p, w, b, h, pair, order);
       const int r0 = pair * 256 + t * 128;
       int lo, hi;
       fwd_kv_range<kVarlen>(p, r0, lo, hi);
