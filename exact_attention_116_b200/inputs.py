@@ -121,6 +121,9 @@ DECODE_CONFIGS: dict[str, DecodeConfig] = {
     "decode_paged": DecodeConfig("decode_paged", 8, 1, 16, 128, 4096, 8192, 256, True, seed=107,
                                  note="B8 H16 d128, 1 new row per sequence, context 4096-8192 keys (uniform), "
                                       "256-key pages in random order"),
+    "decode_paged_sq4": DecodeConfig("decode_paged_sq4", 8, 4, 16, 128, 4096, 8192, 256, True, seed=108,
+                                     note="B8 H16 d128, 4 new rows per sequence (a speculative step), context "
+                                          "4096-8192 keys (uniform), 256-key pages in random order"),
 }
 
 

@@ -101,9 +101,10 @@ def test_decode_split_counts_agree():
         assert np.abs(o - outs[0][0]).max() < 1e-2 and np.abs(lse - outs[0][1]).max() < 1e-4
 
 
-def test_decode_workload_all_rows():
-    cfg = DECODE_CONFIGS["decode_paged"]
-    check(cfg, splits=0, what="decode_paged")
+@pytest.mark.parametrize("name", ["decode_paged", "decode_paged_sq4"])
+def test_decode_workload_all_rows(name):
+    cfg = DECODE_CONFIGS[name]
+    check(cfg, splits=0, what=name)
 
 
 def test_decode_out_of_range_length_is_reported_not_read():
