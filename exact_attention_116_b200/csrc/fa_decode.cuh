@@ -352,9 +352,9 @@ __global__ void __launch_bounds__(kDecThreads)
     // running state: warp w owns rows w and w + 4 (warp-uniform values)
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
     // O accumulators of this thread: rows 0..kSq-1, columns 2 cp and 2 cp + 1, keys of group kg
-    float acc[kSq][2];
+    float2 acc[kSq];
 #pragma unroll
-    for (int i = 0; i < kSq; ++i) acc[i][0] = acc[i][1] = 0.0f;
+    for (int i = 0; i < kSq; ++i) acc[i] = make_float2(0.0f, 0.0f);
 
     for (int t = w.t0; t < w.t1; ++t, ++k) {
       const int st = (int)(k % kStages);
@@ -364,9 +364,9 @@ __global__ void __launch_bounds__(kDecThreads)
       // ---- A: half dot products, key kt = tid % 64, dims [half * D/2, half * D/2 + D/2)
       {
         const int kt = tid % kDecTile, half = tid / kDecTile;
-        float part[kSq];
+        float2 part[kSq];  // even / odd columns, packed f32x2 arithmetic
 #pragma unroll
-        for (int i = 0; i < kSq; ++i) part[i] = 0.0f;
+        for (int i = 0; i < kSq; ++i) part[i] = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int ch = 0; ch < D / 16; ++ch) {  // 16-byte chunks of this thread's half row
           const int col0 = half * (D / 2) + ch * 8;
@@ -374,28 +374,21 @@ __global__ void __launch_bounds__(kDecThreads)
           const uint4 raw =
               *reinterpret_cast<const uint4*>(kgen + bx * (kDecTile * 128) + sw128_offset(kt, chunk));
           const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-          float kv[8];
+          float2 kv[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            kv[2 * e] = bf16lo_to_f32(wv[e]);
-            kv[2 * e + 1] = bf16hi_to_f32(wv[e]);
-          }
+          for (int e = 0; e < 4; ++e) kv[e] = make_float2(bf16lo_to_f32(wv[e]), bf16hi_to_f32(wv[e]));
 #pragma unroll
           for (int i = 0; i < kSq; ++i) {  // rows past Sq have q = 0
             const float4 qa = *reinterpret_cast<const float4*>(&sQ[i * D + col0]);
             const float4 qb = *reinterpret_cast<const float4*>(&sQ[i * D + col0 + 4]);
-            part[i] = fmaf(qa.x, kv[0], part[i]);
-            part[i] = fmaf(qa.y, kv[1], part[i]);
-            part[i] = fmaf(qa.z, kv[2], part[i]);
-            part[i] = fmaf(qa.w, kv[3], part[i]);
-            part[i] = fmaf(qb.x, kv[4], part[i]);
-            part[i] = fmaf(qb.y, kv[5], part[i]);
-            part[i] = fmaf(qb.z, kv[6], part[i]);
-            part[i] = fmaf(qb.w, kv[7], part[i]);
+            part[i] = fma2(make_float2(qa.x, qa.y), kv[0], part[i]);
+            part[i] = fma2(make_float2(qa.z, qa.w), kv[1], part[i]);
+            part[i] = fma2(make_float2(qb.x, qb.y), kv[2], part[i]);
+            part[i] = fma2(make_float2(qb.z, qb.w), kv[3], part[i]);
           }
         }
 #pragma unroll
-        for (int i = 0; i < kSq; ++i) sS[(half * kSq + i) * kDecTile + kt] = part[i];
+        for (int i = 0; i < kSq; ++i) sS[(half * kSq + i) * kDecTile + kt] = part[i].x + part[i].y;
       }
       __syncthreads();
       // every thread has finished with the previous tile's slot: refill it (not after a wait
@@ -444,19 +437,17 @@ __global__ void __launch_bounds__(kDecThreads)
 #pragma unroll
         for (int i = 0; i < kSq; ++i) {  // rows past Sq stay 0
           const float a = sAlpha[i];
-          acc[i][0] *= a;
-          acc[i][1] *= a;
+          acc[i] = mul2(acc[i], make_float2(a, a));
         }
 #pragma unroll 4
         for (int kt = kg; kt < kDecTile; kt += Cfg::kKeyGroups) {
           const uint32_t wv = *reinterpret_cast<const uint32_t*>(vgen + bx * (kDecTile * 128) +
                                                                  sw128_offset(kt, chunk) + within);
-          const float v0 = bf16lo_to_f32(wv), v1 = bf16hi_to_f32(wv);
+          const float2 v = make_float2(bf16lo_to_f32(wv), bf16hi_to_f32(wv));
 #pragma unroll
           for (int i = 0; i < kSq; ++i) {
             const float pv = sP[i * kDecTile + kt];
-            acc[i][0] = fmaf(pv, v0, acc[i][0]);
-            acc[i][1] = fmaf(pv, v1, acc[i][1]);
+            acc[i] = fma2(make_float2(pv, pv), v, acc[i]);
           }
         }
       }
@@ -466,8 +457,8 @@ __global__ void __launch_bounds__(kDecThreads)
     __syncthreads();  // every thread is past phase C (sAlpha, sS are reused below)
 #pragma unroll
     for (int i = 0; i < kSq; ++i) {
-      sRed[(kg * kSq + i) * D + 2 * cp] = acc[i][0];
-      sRed[(kg * kSq + i) * D + 2 * cp + 1] = acc[i][1];
+      sRed[(kg * kSq + i) * D + 2 * cp] = acc[i].x;
+      sRed[(kg * kSq + i) * D + 2 * cp + 1] = acc[i].y;
     }
 #pragma unroll
     for (int r = 0; r < (kSq + 3) / 4; ++r) {  // row statistics: alpha slots -> 1 / l, S -> log2 l + m
