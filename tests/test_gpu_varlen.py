@@ -103,3 +103,18 @@ def test_varlen_bad_offsets_are_reported_not_followed():
     assert e.value.status == 6  # FA_ERR_DEVICE
     assert torch.isfinite(o[:150].float()).all()
     fa.check()  # cleared; the context is usable
+
+
+def test_varlen_forward_is_bitwise_reproducible_and_ordered_by_cost():
+    """Many sequences of mixed lengths, so that the cost-sorted pair order differs from the index
+    order: two calls give the same bits, and rows match the oracle."""
+    lens = [900, 3, 0, 1500, 77, 640, 256, 1, 1100, 300, 2049, 128]
+    (q, k, v, do), cu = packed_inputs(lens, 2, 128, seed=91)
+    dev = [x.cuda() for x in (q, k, v)]
+    cu_d = cu.cuda()
+    o1, l1 = fa.attention_fwd_varlen(*dev, cu_d, None, True)
+    o2, l2 = fa.attention_fwd_varlen(*dev, cu_d, None, True)
+    fa.check()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2), "packed forward is not bitwise reproducible"
+    o_ref, lse_ref = oracle_vl.varlen_forward(to_np(q), to_np(k), to_np(v), cu.numpy(), 128 ** -0.5, True, -1, -1)
+    assert_fwd_close(to_np(o1), to_np(l1).T, o_ref, lse_ref.T, "mixed packed forward")
