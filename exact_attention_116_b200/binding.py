@@ -102,6 +102,32 @@ def _check_qkv(*ts: torch.Tensor, dtype=torch.bfloat16) -> tuple[int, int, int, 
     return tuple(int(x) for x in shape)  # type: ignore[return-value]
 
 
+def _check_lse(lse: torch.Tensor, shape: tuple[int, ...]) -> None:
+    """LSE / row statistics: a contiguous float32 CUDA tensor of the given shape. Checked before any
+    launch: the C layer sees only a pointer, so a wrong dtype or layout would be read out of bounds."""
+    if lse.dtype != torch.float32:
+        raise ValueError(f"lse must be float32 (got {lse.dtype})")
+    if tuple(lse.shape) != tuple(shape):
+        raise ValueError(f"lse must have shape {tuple(shape)} (got {tuple(lse.shape)})")
+    if not lse.is_contiguous():
+        raise ValueError("lse must be contiguous")
+    if not lse.is_cuda:
+        raise ValueError("lse must be on a CUDA device (there is no CPU path)")
+
+
+def _check_workspace(workspace) -> tuple[int | None, int]:
+    """Optional backward workspace: a contiguous uint8 CUDA tensor; returns (pointer, bytes)."""
+    if workspace is None:
+        return None, 0
+    if workspace.dtype != torch.uint8:
+        raise ValueError(f"workspace must be a uint8 tensor (got {workspace.dtype})")
+    if not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    if not workspace.is_cuda:
+        raise ValueError("workspace must be on a CUDA device")
+    return workspace.data_ptr(), workspace.numel()
+
+
 def _scale(scale: float | None, d: int) -> float:
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
@@ -118,8 +144,7 @@ def _check_slopes(alibi_slopes, B: int, H: int):
 def fwd_into(q, k, v, o, lse, scale=None, causal=False, window=(-1, -1), stream=None, alibi_slopes=None) -> None:
     """fa_fwd (fa_fwd_ex with ALiBi slopes) into caller-provided o (B,N,H,d) bf16 and lse (B,H,N) fp32."""
     B, N, H, d = _check_qkv(q, k, v, o)
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous() or not lse.is_cuda:
-        raise ValueError("lse must be a contiguous (B, H, N) float32 CUDA tensor")
+    _check_lse(lse, (B, H, N))
     slopes = _check_slopes(alibi_slopes, B, H)
     if slopes is None:
         st = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), B, N, H, d,
@@ -157,8 +182,7 @@ def fwd_fp8_into(q8, k8, v8, q_descale, k_descale, v_descale, o, lse, scale=None
     _check_qkv(o)
     if tuple(o.shape) != (B, N, H, d):
         raise ValueError("o must have the shape of q")
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N) or not lse.is_contiguous() or not lse.is_cuda:
-        raise ValueError("lse must be a contiguous (B, H, N) float32 CUDA tensor")
+    _check_lse(lse, (B, H, N))
     for t in (q_descale, k_descale, v_descale):
         if t.dtype != torch.float32 or tuple(t.shape) != (B, H) or not t.is_contiguous() or not t.is_cuda:
             raise ValueError("descales must be contiguous (B, H) float32 CUDA tensors")
@@ -187,9 +211,10 @@ def bwd_into(q, k, v, o, lse, do, dq, dk, dv, scale=None, causal=False, window=(
     """fa_bwd (or fa_bwd_deterministic; fa_bwd_ex with ALiBi slopes) into caller-provided dq, dk, dv.
     ``workspace``: uint8 CUDA tensor or None."""
     B, N, H, d = _check_qkv(q, k, v, o, do, dq, dk, dv)
-    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
-    lib = load()
+    _check_lse(lse, (B, H, N))
+    ws_ptr, ws_bytes = _check_workspace(workspace)
     slopes = _check_slopes(alibi_slopes, B, H)
+    lib = load()
     if slopes is not None:
         st = lib.fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
                            slopes, dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, d, _scale(scale, d),
@@ -218,8 +243,11 @@ def bwd_stages(q, k, v, o, lse, do, dq, dk, dv, workspace, scale=None, causal=Fa
     """The three launches of the backward issued one by one; ``between(i)`` runs before stage i
     (i = 0, 1, 2) and once more after the last (i = 3) — e.g. to record CUDA events."""
     B, N, H, d = _check_qkv(q, k, v, o, do, dq, dk, dv)
+    _check_lse(lse, (B, H, N))
+    if workspace is None:
+        raise ValueError("bwd_stages needs a workspace of workspace_bytes(B, N, H, d) bytes")
+    ws, wb = _check_workspace(workspace)
     lib, s = load(), _stream_handle(stream)
-    ws, wb = workspace.data_ptr(), workspace.numel()
     sc = _scale(scale, d)
     if between:
         between(0)
@@ -247,6 +275,7 @@ def bwd_into_static_workspace(q, k, v, o, lse, do, dq, dk, dv, scale=None, causa
     issue them one after another. Make the first call on each device outside stream capture.
     """
     B, N, H, d = _check_qkv(q, k, v, o, do, dq, dk, dv)
+    _check_lse(lse, (B, H, N))
     lib = load()
     fn = lib.fa_bwd_static_workspace
     if fn.argtypes is None:
@@ -308,9 +337,8 @@ def decode_paged_into(q, k_cache, v_cache, block_table, seqlens, o, lse, scale=N
             raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
     if block_table.dim() != 2 or block_table.shape[0] != B or tuple(seqlens.shape) != (B,):
         raise ValueError("block_table must be (B, max_pages) and seqlens (B,)")
-    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, Sq) or not lse.is_contiguous() or not lse.is_cuda:
-        raise ValueError("lse must be a contiguous (B, H, Sq) float32 CUDA tensor")
-    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    _check_lse(lse, (B, H, Sq))
+    ws_ptr, ws_bytes = _check_workspace(workspace)
     kn, vn = (None, None) if k_new is None else (k_new.data_ptr(), v_new.data_ptr())
     st = load().fa_decode_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), kn, vn, block_table.data_ptr(),
                                 seqlens.data_ptr(), o.data_ptr(), lse.data_ptr(), B, Sq, H, d, num_pages, page_size,
@@ -382,8 +410,9 @@ def attention_bwd_varlen(q, k, v, o, lse, do, cu_seqlens, scale=None, causal=Fal
                          stream=None, deterministic=False, alibi_slopes=None):
     """Backward of attention_fwd_varlen: returns (dq, dk, dv), each (total, H, d) bf16."""
     B, total, H, d = _check_packed(cu_seqlens, q, k, v, o, do)
+    _check_lse(lse, (H, total))
+    ws_ptr, ws_bytes = _check_workspace(workspace)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
     st = load().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
                               cu_seqlens.data_ptr(), _check_head_slopes(alibi_slopes, H), dq.data_ptr(),
                               dk.data_ptr(), dv.data_ptr(), B, total, H, d, _scale(scale, d), int(bool(causal)),

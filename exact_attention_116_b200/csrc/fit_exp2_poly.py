@@ -41,8 +41,8 @@ def f32_coeffs(degree: int = 3):
 
 def exp2_poly_f32(x, coeffs):
     """float32 emulation of the kernel's sequence of operations (for the error check)."""
-    x = np.asarray(x, dtype=np.float32)
-    x = np.maximum(x, np.float32(-125.0))  # keeps 2^j * p(f) a normal float
+    x_in = np.asarray(x, dtype=np.float32)
+    x = np.maximum(x_in, np.float32(-125.0))  # keeps 2^j * p(f) a normal float
     magic = np.float32(12582912.0)  # 1.5 * 2^23: adding it rounds to an integer in the low bits
     t = (x + magic).astype(np.float32)
     j_f = (t - magic).astype(np.float32)
@@ -52,7 +52,8 @@ def exp2_poly_f32(x, coeffs):
     p = (p * f + c1).astype(np.float32)
     p = (p * f + c0).astype(np.float32)
     bits = p.view(np.int32) + (t.view(np.int32) << 23)
-    return bits.astype(np.int32).view(np.float32)
+    r = bits.astype(np.int32).view(np.float32)
+    return np.where(x_in >= np.float32(-125.0), r, np.float32(0.0))  # below -125 (and -inf): exactly 0
 
 
 if __name__ == "__main__":

@@ -363,21 +363,23 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // Cody-Waite split x = j + f with j = round(x) and |f| <= 1/2 (adding 1.5 * 2^23 rounds x to
 // an integer held in the low mantissa bits), a degree-3 minimax polynomial for 2^f on
 // [-1/2, 1/2] (coefficients fitted by csrc/fit_exp2_poly.py, max relative error 7.5e-5), and
-// j added to the exponent field of the polynomial's value. x is clamped at -125 so the
-// result stays a normal float: for x < -125 (including -inf) it returns about 2^-125.
+// j added to the exponent field of the polynomial's value. The reduction runs on x clamped at
+// -125 (so that 2^j p(f) stays a normal float), and for x < -125, -inf included, the result is
+// exactly 0: a masked score (-inf) must carry no weight, as 2^-inf = 0 does on MUFU.
 constexpr float kExp2C0 = 9.999280572e-01f;
 constexpr float kExp2C1 = 6.932608485e-01f;
 constexpr float kExp2C2 = 2.426111549e-01f;
 constexpr float kExp2C3 = 5.517221987e-02f;
 
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.0f);
+__device__ __forceinline__ float exp2_poly(float x_in) {
+  const float x = fmaxf(x_in, -125.0f);
   const float t = x + 12582912.0f;
   const float f = x - (t - 12582912.0f);
   float p = fmaf(kExp2C3, f, kExp2C2);
   p = fmaf(p, f, kExp2C1);
   p = fmaf(p, f, kExp2C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x_in >= -125.0f ? r : 0.0f;
 }
 
 // Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of a float2) and the
@@ -407,17 +409,17 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 
 // exp2_poly on a pair, with the same operations as the scalar version done as packed pairs.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -125.0f);
-  x.y = fmaxf(x.y, -125.0f);
+__device__ __forceinline__ float2 exp2_poly2(float2 x_in) {
+  const float2 x = make_float2(fmaxf(x_in.x, -125.0f), fmaxf(x_in.y, -125.0f));
   const float2 t = add2(x, make_float2(12582912.0f, 12582912.0f));
   const float2 jf = add2(t, make_float2(-12582912.0f, -12582912.0f));
   const float2 f = fma2(jf, make_float2(-1.0f, -1.0f), x);
   float2 p = fma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
   p = fma2(p, f, make_float2(kExp2C1, kExp2C1));
   p = fma2(p, f, make_float2(kExp2C0, kExp2C0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+  const float rx = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
+  const float ry = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
+  return make_float2(x_in.x >= -125.0f ? rx : 0.0f, x_in.y >= -125.0f ? ry : 0.0f);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

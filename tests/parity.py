@@ -1,9 +1,11 @@
 """Shared helpers of the GPU parity tests: run the CUDA path and compare with the oracle.
 
 Tolerances (bf16 inputs and outputs, fp32 accumulation):
-* forward: max_i |O_gpu - O_ref|_inf / max(1, |O_ref,i|_inf) <= 1e-2, and max |LSE_gpu - LSE_ref| <= 1e-3.
-  The relative form matters only for |O| >= 1: bf16's half-ulp in [4, 8) is 2^-6 ~ 0.0156,
-  so rounding the output alone can exceed a raw 1e-2 there; the raw maximum is reported too.
+* forward: every element obeys |O_gpu - O_ref| <= 1e-2 + ulp_bf16(O_gpu) / 2, and
+  max |LSE_gpu - LSE_ref| <= 1e-3. The kernel rounds its fp32 result o32 to bf16 once at the end,
+  so |O_gpu - O_ref| <= |O_gpu - o32| + |o32 - O_ref| <= ulp/2 + |o32 - O_ref|: the check is
+  exactly the 1e-2 bound on the kernel's own error plus that last rounding, which alone can
+  exceed 1e-2 (bf16's half-ulp in [4, 8) is 2^-6 ~ 0.0156). The raw maximum is reported too.
 * backward: relative L2 error ||g - g_ref|| / ||g_ref|| <= 1e-2 per gradient (per sampled head
   at the large sizes). Where the exact dQ or dK vanishes (a query that sees only itself has
   dS = 0 exactly, so dQ = dK = 0), the GPU returns rounding noise of (dP - D) and the
@@ -31,19 +33,25 @@ def window_args(causal: bool, win: tuple[int, int]):
     return bool(causal), int(win[0]), int(win[1])
 
 
+def half_ulp_bf16(x: np.ndarray) -> np.ndarray:
+    """Half the spacing of bf16 values at |x| (8 significant bits): 2^(e - 8) for |x| in [2^e, 2^(e+1))."""
+    _, e = np.frexp(np.abs(np.asarray(x, dtype=np.float64)))  # |x| = m 2^e with m in [0.5, 1)
+    return np.ldexp(1.0, e - 9)
+
+
 def fwd_errors(o_gpu: np.ndarray, lse_gpu: np.ndarray, o_ref: np.ndarray, lse_ref: np.ndarray):
-    """(scaled max O error, raw max O error, max LSE error) over the rows present in the refs."""
-    diff = np.abs(o_gpu - o_ref).max(axis=-1)
-    scale = np.maximum(1.0, np.abs(o_ref).max(axis=-1))
-    return float((diff / scale).max()), float(diff.max()), float(np.abs(lse_gpu - lse_ref).max())
+    """(O error beyond the output's last rounding, raw max O error, max LSE error) over the refs' rows."""
+    diff = np.abs(o_gpu - o_ref)
+    excess = diff - half_ulp_bf16(o_gpu)
+    return float(excess.max()), float(diff.max()), float(np.abs(lse_gpu - lse_ref).max())
 
 
 def assert_fwd_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
-    e_rel, e_raw, e_lse = fwd_errors(o_gpu, lse_gpu, o_ref, lse_ref)
+    e_o, e_raw, e_lse = fwd_errors(o_gpu, lse_gpu, o_ref, lse_ref)
     assert np.isfinite(o_gpu).all() and np.isfinite(lse_gpu).all(), what
-    assert e_rel <= FWD_O_TOL, f"{what}: O error {e_rel:.3e} (raw {e_raw:.3e})"
+    assert e_o <= FWD_O_TOL, f"{what}: O error {e_o:.3e} beyond the bf16 output rounding (raw {e_raw:.3e})"
     assert e_lse <= FWD_LSE_TOL, f"{what}: LSE error {e_lse:.3e}"
-    return e_rel, e_raw, e_lse
+    return e_o, e_raw, e_lse
 
 
 def rel_l2(g: np.ndarray, ref: np.ndarray) -> float:

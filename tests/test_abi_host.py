@@ -184,3 +184,58 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="not built"):
         binding.load()
+
+
+def _no_launch(*_a, **_k):
+    raise AssertionError("validation passed: the call would have reached the library")
+
+
+def _qkv_any_device(*ts, dtype=torch.bfloat16):
+    """_check_qkv without its CUDA requirement, so that the later checks run on CPU tensors."""
+    shape = ts[0].shape
+    for t in ts:
+        assert t.dtype == dtype and t.shape == shape
+    return tuple(int(x) for x in shape)
+
+
+@pytest.mark.parametrize("case", ["dtype", "shape", "transposed", "cpu"])
+def test_backward_wrappers_validate_lse_before_any_launch(monkeypatch, case):
+    """A bf16, mis-shaped, non-contiguous or host LSE is refused by every backward wrapper
+    before the library is touched (the C layer only checks its pointer's alignment)."""
+    monkeypatch.setattr(binding, "_check_qkv", _qkv_any_device)
+    monkeypatch.setattr(binding, "load", _no_launch)
+    B, N, H, d = 1, 16, 2, 64
+    t = torch.zeros(B, N, H, d, dtype=torch.bfloat16)
+    lse = {"dtype": torch.zeros(B, H, N, dtype=torch.bfloat16),
+           "shape": torch.zeros(B, N, H, dtype=torch.float32),
+           "transposed": torch.zeros(B, N, H, dtype=torch.float32).transpose(1, 2),
+           "cpu": torch.zeros(B, H, N, dtype=torch.float32)}[case]
+    msg = {"dtype": "float32", "shape": "shape", "transposed": "contiguous", "cpu": "CUDA"}[case]
+    ws = torch.zeros(64, dtype=torch.uint8)
+    calls = [
+        lambda: binding.bwd_into(t, t, t, t, lse, t, t, t, t),
+        lambda: binding.bwd_stages(t, t, t, t, lse, t, t, t, t, ws),
+        lambda: binding.bwd_into_static_workspace(t, t, t, t, lse, t, t, t, t),
+        lambda: binding.fwd_into(t, t, t, t, lse),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError, match=msg):
+            call()
+
+
+@pytest.mark.parametrize("case", ["dtype", "strided", "cpu"])
+def test_backward_wrappers_validate_workspace_before_any_launch(monkeypatch, case):
+    monkeypatch.setattr(binding, "_check_qkv", _qkv_any_device)
+    monkeypatch.setattr(binding, "_check_lse", lambda *_a: None)
+    monkeypatch.setattr(binding, "load", _no_launch)
+    t = torch.zeros(1, 16, 2, 64, dtype=torch.bfloat16)
+    ws = {"dtype": torch.zeros(64, dtype=torch.float32),
+          "strided": torch.zeros(128, dtype=torch.uint8)[::2],
+          "cpu": torch.zeros(64, dtype=torch.uint8)}[case]
+    msg = {"dtype": "uint8", "strided": "contiguous", "cpu": "CUDA"}[case]
+    for call in (lambda: binding.bwd_into(t, t, t, t, None, t, t, t, t, workspace=ws),
+                 lambda: binding.bwd_stages(t, t, t, t, None, t, t, t, t, ws)):
+        with pytest.raises(ValueError, match=msg):
+            call()
+    with pytest.raises(ValueError, match="workspace"):
+        binding.bwd_stages(t, t, t, t, None, t, t, t, t, None)

@@ -3,8 +3,8 @@
 The coefficients in the header must be the ones csrc/fit_exp2_poly.py fits (a minimax fit of
 2^f on [-1/2, 1/2]); a float32 emulation of the kernel's exact sequence of operations must
 stay within 1e-4 relative error of 2^x on [-125, 8] (the kernels feed its result, rounded to
-bf16 with relative error up to 2^-9, to the tensor cores); -inf must give a tiny positive
-normal number.
+bf16 with relative error up to 2^-9, to the tensor cores); below -125, and at -inf (a masked
+score), it must return exactly 0, as 2^-inf = 0 does: a masked key carries no weight.
 """
 
 from __future__ import annotations
@@ -46,5 +46,17 @@ def test_emulated_error_bound():
                          np.float32([-0.5, 0.5, -1.5, 1.5, 0.0, -124.5, 7.999])])
     rel = np.abs(mod.exp2_poly_f32(xs, c).astype(np.float64) / np.exp2(xs.astype(np.float64)) - 1.0)
     assert rel.max() < 1e-4
-    tiny = mod.exp2_poly_f32(np.float32([-np.inf, -1000.0, -126.0]), c)
-    assert (tiny > 0).all() and (tiny < 1e-37).all() and (tiny >= np.finfo(np.float32).tiny).all()
+    zero = mod.exp2_poly_f32(np.float32([-np.inf, -1000.0, -126.0, -125.001]), c)
+    assert (zero == 0).all(), zero
+    edge = mod.exp2_poly_f32(np.float32([-125.0]), c)
+    assert edge[0] > 0 and abs(float(edge[0]) / 2.0 ** -125 - 1.0) < 1e-4
+
+
+def test_header_zeroes_below_the_clamp():
+    """Both header forms (scalar and pair) select 0 below the clamp from the unclamped input."""
+    with open(os.path.join(CSRC, "sm100_ptx.cuh")) as f:
+        text = f.read()
+    body1 = text[text.index("float exp2_poly(float x_in)"):text.index("// Packed fp32 pair")]
+    assert "x_in >= -125.0f ? r : 0.0f" in body1
+    body2 = text[text.index("float2 exp2_poly2(float2 x_in)"):text.index("pack_bf16x2")]
+    assert "x_in.x >= -125.0f ? rx : 0.0f" in body2 and "x_in.y >= -125.0f ? ry : 0.0f" in body2

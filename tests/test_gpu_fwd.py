@@ -1,8 +1,8 @@
 """GPU parity of the forward pass (CUDA path through the C ABI) against the fp64 oracle.
 
-Small and ragged shapes are compared element by element over whole tensors; the large
-workloads run in the same launch configuration the bench uses and are compared on sampled
-heads (whole heads) or sampled rows (each row computed on its own by the oracle).
+Small and ragged shapes and the GPT-style workload are compared element by element over whole
+tensors; the large workloads run in the same launch configuration the bench uses and are
+compared over every row of sampled heads.
 """
 
 from __future__ import annotations
@@ -84,36 +84,37 @@ def test_fwd_tiny_config_full():
     assert_fwd_close(to_np(o), to_np(lse), o_ref, lse_ref, "tiny_fwd")
 
 
-def test_fwd_gpt_config_sampled_heads_and_determinism():
+def test_fwd_gpt_config_full_and_determinism():
+    """The GPT-style workload (B4 H16 N2048 d64 causal) against the oracle over all 64 heads, element
+    by element, and bitwise equal across two calls."""
     cfg = CONFIGS["gpt_fwd"]
     q, k, v, _ = make_inputs(cfg)
     o, lse = gpu_fwd(q, k, v, cfg.scale, cfg.causal, (cfg.win_l, cfg.win_r))
     o2, lse2 = gpu_fwd(q, k, v, cfg.scale, cfg.causal, (cfg.win_l, cfg.win_r))
     assert torch.equal(o, o2) and torch.equal(lse, lse2), "forward is not bitwise reproducible"
-    heads = [(0, 0), (cfg.B - 1, cfg.H - 1), (1, 7), (2, 11)]
     o_ref, lse_ref = oracle.attention_forward(to_np(q), to_np(k), to_np(v), cfg.scale, cfg.causal, cfg.win_l,
-                                              cfg.win_r, heads=heads)
-    on, ln_ = to_np(o), to_np(lse)
-    for b, h in heads:
-        assert_fwd_close(on[b, :, h], ln_[b, h], o_ref[b, :, h], lse_ref[b, h], f"gpt_fwd head {(b, h)}")
-    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+                                              cfg.win_r)
+    assert_fwd_close(to_np(o), to_np(lse), o_ref, lse_ref, "gpt_fwd (all heads)")
 
 
 @pytest.mark.parametrize("name", ["train_fwd_bwd", "long_fwd_bwd", "window_fwd_bwd"])
-def test_fwd_full_size_sampled_rows(name):
+def test_fwd_full_size_whole_heads(name):
+    """The large workloads in the bench's launch configuration: every row of three heads, the first,
+    the last and one drawn at random (heads are independent, so each comparison is exact for its head),
+    and finite outputs everywhere."""
     cfg = CONFIGS[name]
     q, k, v, _ = make_inputs(cfg)
     o, lse = gpu_fwd(q, k, v, cfg.scale, cfg.causal, (cfg.win_l, cfg.win_r))
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
-    rng = np.random.default_rng(hash(name) % 2**32)
-    rows = sorted(set([0, 1, 127, 128, 255, 256, cfg.N // 2, cfg.N - 129, cfg.N - 128, cfg.N - 1]
-                      + rng.integers(0, cfg.N, 40).tolist()))
+    rng = np.random.default_rng(sum(map(ord, name)))
     heads = [(0, 0), (cfg.B - 1, cfg.H - 1), (int(rng.integers(cfg.B)), int(rng.integers(cfg.H)))]
     on, ln_ = to_np(o), to_np(lse)
+    qn, kn, vn = (x.float().numpy() for x in (q, k, v))
     for b, h in heads:
-        o_ref, lse_ref = oracle.forward_rows(q.float().numpy(), k.float().numpy(), v.float().numpy(), b, h, rows,
-                                             cfg.scale, cfg.causal, cfg.win_l, cfg.win_r)
-        assert_fwd_close(on[b, rows, h], ln_[b, h, rows], o_ref, lse_ref, f"{name} head {(b, h)}")
+        o_ref, lse_ref = oracle.head_forward(qn[b, :, h].astype(np.float64), kn[b, :, h].astype(np.float64),
+                                             vn[b, :, h].astype(np.float64), cfg.scale, cfg.causal, cfg.win_l,
+                                             cfg.win_r, block_rows=1024)
+        assert_fwd_close(on[b, :, h], ln_[b, h], o_ref, lse_ref, f"{name} head {(b, h)}")
 
 
 def test_fwd_autograd_wrapper_matches():
