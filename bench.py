@@ -1,12 +1,14 @@
 """Benchmark: exact attention forward + backward on B200 through the C ABI.
 
 One step = one pass of the whole hot path over one batch of synthetic input: fa_fwd (O, LSE)
-followed by the backward's three launches (preprocess, main, dQ conversion). The default
-workload is the training configuration B=2, H=16, N=8192, d=128, causal, bf16.
-``--config train_fwd_fp8`` instead times the E4M3 forward (fa_fwd_fp8) on the same shape:
-one step = one launch. ``--config decode_paged`` times the paged-KV decode (fa_decode_paged):
-one step = one call (append, split kernel and merge in one kernel) over every sequence, reported
-in GB/s of cache read.
+followed by the backward's launches (preprocess, main, dQ conversion). The default workload is
+the long-context configuration B=1, H=16, N=32768, d=128, causal, bf16 (the largest of the
+workloads, which fits one GPU). The same run also reports device-timed forward / backward
+figures of the other workloads (GPT-style forward, training shape, sliding window, tiny) under
+"configs". ``--config train_fwd_fp8`` instead times the E4M3 forward (fa_fwd_fp8) on the training
+shape: one step = one launch. ``--config decode_paged`` times the paged-KV decode
+(fa_decode_paged): one step = one call (append, split kernel and merge in one kernel) over every
+sequence, reported in GB/s of cache read.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
 
@@ -40,7 +42,7 @@ from exact_attention_116_b200 import binding  # noqa: E402
 from exact_attention_116_b200 import distributed as mg  # noqa: E402
 from exact_attention_116_b200.inputs import (CONFIGS, DECODE_CONFIGS, FP8_CONFIGS, make_decode_inputs,  # noqa: E402
                                              make_fp8_inputs, make_inputs)
-from exact_attention_116_b200.workload import flops, hbm_bytes, visible_pairs  # noqa: E402
+from exact_attention_116_b200.workload import flops, flops_tile_granular, hbm_bytes, visible_pairs  # noqa: E402
 
 METRIC = "attention fwd/bwd TFLOPS (bf16, causal) and % of B200 dense BF16 peak"
 METRIC_FP8 = "attention fwd TFLOPS (E4M3 inputs, causal) and % of B200 dense FP8 peak"
@@ -69,16 +71,42 @@ def kernel_source_hash(sources) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the sources that
-    define the kernel still hash to the value recorded with the measurement."""
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary (entry
+    "kernel@workload"), if the sources that define the kernel still hash to the value recorded
+    with the measurement."""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
     with open(PROFILE_TRAFFIC) as f:
-        k = json.load(f).get("kernels", {}).get(kernel)
+        k = json.load(f).get("kernels", {}).get(f"{kernel}@{workload}")
     if k is None or k.get("source_hash") != kernel_source_hash(k.get("sources", [])):
         return None
     return k.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- L2 flush, config record
+
+def l2_flusher(dev):
+    """A callable that writes one buffer larger than L2 and then reads another, so that the next
+    timed launch starts with a clean L2 (nothing of its inputs cached, no dirty lines of the flush
+    left to write back). It runs on the current stream, outside the timed interval."""
+    w = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    r = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        w.zero_()
+        r.sum()
+    return flush
+
+
+L2_NOTE = ("L2 flushed before every timed step outside the timed interval (252 MiB written, then 252 MiB read); "
+           "each step timed with CUDA events on the launching stream")
+
+
+def attn_config(cfg) -> dict:
+    """The workload record of a bf16 config: the same keys in the GPU arm and the reference arm."""
+    return {"workload": f"{cfg.name}: {cfg.note}", "B": cfg.B, "N": cfg.N, "H": cfg.H, "d": cfg.d,
+            "causal": cfg.causal, "window": [cfg.win_l, cfg.win_r], "seed": cfg.seed}
 
 
 # ----------------------------------------------------------------------------- end to end
@@ -442,7 +470,7 @@ def run_gpu_decode(args):
                                "zeroing launch before it)", "bound": "hbm", "achieved": round(gbs, 1),
                      "peak": peak["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peak["hbm_gbs"], 4),
                      "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
-                     "traffic": recorded_traffic("fa_decode_split_kernel"), "algorithmic_bytes": nbytes},
+                     "traffic": recorded_traffic("fa_decode_split_kernel", cfg.name), "algorithmic_bytes": nbytes},
         "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": out_h.numel(),
@@ -542,7 +570,7 @@ def run_gpu_fp8(args):
                      "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
                      "frac_of_bf16_peak": round(achieved / peak["bf16_tflops"], 4),
                      "peak_source": f"{peak_src} bf16_tflops x {FP8_PER_BF16} (nominal dense FP8/BF16 ratio)",
-                     "traffic": recorded_traffic("fa_fwd_kernel<128, E4M3>"),
+                     "traffic": recorded_traffic("fa_fwd_kernel<128, E4M3>", cfg.name),
                      "algorithmic_bytes": in_bytes + B * N * H * d * 2 + B * H * N * 4},
         "e2e": {"value": round(mg.aggregate_rate(f_fwd, world, e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": in_bytes,
@@ -562,6 +590,87 @@ def run_gpu_fp8(args):
         print(json.dumps(res), flush=True)
 
 
+def time_attention(cfg, dev, iters: int, warm: int, flush) -> dict:
+    """Device time of one workload's forward and backward stages (the bench's launch configuration):
+    every iteration flushes L2, then times fa_fwd and each backward launch with CUDA events on the
+    launching stream. Returns mean milliseconds per launch."""
+    q_h, k_h, v_h, do_h = make_inputs(cfg)
+    q, k, v, do = (x.to(dev) for x in (q_h, k_h, v_h, do_h))
+    B, N, H, d = cfg.shape
+    o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ws = torch.empty(binding.workspace_bytes(B, N, H, d), dtype=torch.uint8, device=dev) if cfg.backward else None
+    stream = torch.cuda.current_stream()
+    win = (cfg.win_l, cfg.win_r)
+    marks = {}
+
+    def one(record: bool):
+        flush()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        evs[0].record(stream)
+        binding.fwd_into(q, k, v, o, lse, cfg.scale, cfg.causal, win)
+        evs[1].record(stream)
+        if cfg.backward:
+            binding.bwd_stages(q, k, v, o, lse, do, dq, dk, dv, ws, cfg.scale, cfg.causal, win,
+                               between=lambda i: i > 0 and evs[1 + i].record(stream))
+        if record:
+            marks.setdefault("ev", []).append(evs)
+
+    for _ in range(warm):
+        one(False)
+    for _ in range(iters):
+        one(True)
+    torch.cuda.synchronize()
+    binding.check()
+    ev = marks["ev"]
+    out = {"fwd_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in ev)}
+    if cfg.backward:
+        out["pre_ms"] = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+        out["main_ms"] = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+        out["conv_ms"] = statistics.mean(e[3].elapsed_time(e[4]) for e in ev)
+    del q, k, v, do, o, dq, dk, dv, lse, ws
+    return out
+
+
+def config_figures(cfg, t: dict, peak: dict) -> dict:
+    """TFLOP/s (exact pair count and tile-granular count), fractions of the measured bf16 peak and,
+    for the window workload, achieved algorithmic bytes per second against the HBM copy bandwidth."""
+    B, N, H, d = cfg.shape
+    win = (cfg.win_l, cfg.win_r)
+    f_fwd, f_bwd = flops(B, N, H, d, cfg.causal, *win)
+    g_fwd, g_bwd = flops_tile_granular(B, N, H, d, cfg.causal, *win)
+    by_fwd, by_bwd = hbm_bytes(B, N, H, d)
+    pk = peak["bf16_tflops"]
+    r = {"workload": f"{cfg.name}: {cfg.note}", "fwd_ms": round(t["fwd_ms"], 4),
+         "fwd_tflops": round(f_fwd / (t["fwd_ms"] * 1e-3) / 1e12, 2),
+         "fwd_tflops_tile_granular": round(g_fwd / (t["fwd_ms"] * 1e-3) / 1e12, 2),
+         "fwd_frac_of_peak": round(f_fwd / (t["fwd_ms"] * 1e-3) / 1e12 / pk, 4),
+         "fwd_gflop": round(f_fwd / 1e9, 3), "fwd_gflop_tile_granular": round(g_fwd / 1e9, 3)}
+    if cfg.backward:
+        bwd_ms = t["pre_ms"] + t["main_ms"] + t["conv_ms"]
+        r.update({"bwd_ms": round(bwd_ms, 4),
+                  "bwd_stage_ms": {"preprocess": round(t["pre_ms"], 4), "main": round(t["main_ms"], 4),
+                                   "dq_convert": round(t["conv_ms"], 4)},
+                  "bwd_tflops": round(f_bwd / (bwd_ms * 1e-3) / 1e12, 2),
+                  "bwd_tflops_tile_granular": round(g_bwd / (bwd_ms * 1e-3) / 1e12, 2),
+                  "bwd_main_tflops": round(f_bwd / (t["main_ms"] * 1e-3) / 1e12, 2),
+                  "bwd_frac_of_peak": round(f_bwd / (bwd_ms * 1e-3) / 1e12 / pk, 4),
+                  "bwd_gflop": round(f_bwd / 1e9, 3), "bwd_gflop_tile_granular": round(g_bwd / 1e9, 3)})
+    if cfg.win_l >= 0 or cfg.win_r >= 0:  # a narrow window is bound by its algorithmic bytes
+        hb = peak["hbm_gbs"]
+        r["fwd_gbs"] = round(by_fwd / (t["fwd_ms"] * 1e-3) / 1e9, 1)
+        r["fwd_frac_of_hbm"] = round(r["fwd_gbs"] / hb, 4)
+        if cfg.backward:
+            r["bwd_gbs"] = round(by_bwd / (r["bwd_ms"] * 1e-3) / 1e9, 1)
+            r["bwd_frac_of_hbm"] = round(r["bwd_gbs"] / hb, 4)
+        r["algorithmic_bytes"] = {"fwd": by_fwd, "bwd": by_bwd, "convention": "fwd 4T+L, bwd 8T+L"}
+    return r
+
+
+EXTRA_CONFIGS = {"tiny_fwd": (50, 5), "gpt_fwd": (50, 5), "train_fwd_bwd": (20, 3), "window_fwd_bwd": (40, 5),
+                 "long_fwd_bwd": (6, 2)}
+
+
 def run_gpu(args):
     info = mg.rank_info()
     world, rank, local = info.world, info.rank, info.local_rank
@@ -579,51 +688,46 @@ def run_gpu(args):
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     ws = torch.empty(binding.workspace_bytes(B, N, H, d), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    flush = l2_flusher(dev)
 
-    ev = {}
-
-    def mark(name):
-        def rec(i):
-            e = torch.cuda.Event(enable_timing=True)
-            e.record(stream)
-            ev.setdefault(f"{name}{i}", []).append(e)
-        return rec
-
-    def step(record: bool):
-        if record:
-            mark("f")(0)
+    def step(evs=None):
+        """One step; with evs (5 events): fwd start, preprocess, main, convert, end marks."""
+        if evs:
+            evs[0].record(stream)
         binding.fwd_into(q, k, v, o, lse, scale, causal, win)
+        if evs:
+            evs[1].record(stream)
         binding.bwd_stages(q, k, v, o, lse, do, dq, dk, dv, ws, scale, causal, win,
-                           between=mark("b") if record else None)
+                           between=(lambda i: i > 0 and evs[1 + i].record(stream)) if evs else None)
 
     for _ in range(args.warmup):
-        step(False)
+        flush()
+        step()
     binding.check()
     torch.cuda.synchronize()
 
+    steps_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     sampler = ClockSampler(dev.index) if local == 0 else None
     mg.barrier(info)
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(args.steps):
-        step(True)
-    end.record(stream)
+    for evs in steps_ev:
+        flush()  # outside the step's timed interval
+        step(evs)
     torch.cuda.synchronize()
     mg.barrier(info)
     t_wall1 = time.time()
     binding.check()
     clocks = sampler.stop(t_wall0, t_wall1) if sampler else None
 
-    ms_total = start.elapsed_time(end)
-    ms_total = mg.max_over_ranks(info, ms_total, dev)
+    ms_total = mg.max_over_ranks(info, sum(e[0].elapsed_time(e[4]) for e in steps_ev), dev)
     ms_step = ms_total / args.steps
     f_fwd, f_bwd = flops(B, N, H, d, causal, *win)
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["f0"], ev["b0"]))
-    pre_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["b0"], ev["b1"]))
-    main_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["b1"], ev["b2"]))
-    conv_ms = statistics.mean(a.elapsed_time(b) for a, b in zip(ev["b2"], ev["b3"]))
+    g_fwd, g_bwd = flops_tile_granular(B, N, H, d, causal, *win)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in steps_ev)
+    pre_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in steps_ev)
+    main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in steps_ev)
+    conv_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in steps_ev)
     bwd_ms = pre_ms + main_ms + conv_ms
 
     # ---- end to end through the public API with host buffers (pinned), copies inside the timed region.
@@ -653,6 +757,7 @@ def run_gpu(args):
     e2e_steps = max(4, min(args.steps, 20))
     e2e_ms = pipelined_e2e(info, dev, sets, train_copy_in, train_compute, train_copy_out, e2e_steps)
     binding.check()
+    del sets, pin, out_h, lse_h
 
     peak, peak_src = peaks()
     main_tflops = f_bwd / (main_ms * 1e-3) / 1e12
@@ -661,7 +766,7 @@ def run_gpu(args):
     dominant = "fa_bwd_kernel" if main_ms >= fwd_ms else "fa_fwd_kernel"
     dom_ms, dom_flops = (main_ms, f_bwd) if dominant == "fa_bwd_kernel" else (fwd_ms, f_fwd)
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    traffic = recorded_traffic(dominant)
+    traffic = recorded_traffic(dominant, cfg.name)
     t_bytes = B * N * H * d * 2
     res = {
         "metric": METRIC, "value": round(mg.aggregate_rate(f_fwd + f_bwd, world, ms_step * 1e-3) / 1e12, 3),
@@ -669,15 +774,18 @@ def run_gpu(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16)",
-        "config": {"workload": f"{cfg.name}: {cfg.note}", "B": B, "N": N, "H": H, "d": d, "causal": causal,
-                   "window": list(win), "seed": cfg.seed,
-                   "l2": f"inputs larger than L2 (q,k,v,dO = {4 * t_bytes / 2**20:.0f} MiB > 126 MiB); no flush",
-                   "flops": "fwd 4*d*pairs + bwd 10*d*pairs over exactly counted visible pairs",
-                   "per_rank": "each rank runs the whole workload on its own inputs"},
+        "config": attn_config(cfg),
+        "notes": {"l2": L2_NOTE,
+                  "flops": "fwd 4*d*pairs + bwd 10*d*pairs over exactly counted visible pairs; the tile-granular "
+                           "count (every touched 128x128 block in full) is reported beside it",
+                  "per_rank": "each rank runs the whole workload on its own inputs"},
         "fwd_tflops": round(fwd_tflops, 2), "bwd_tflops": round(bwd_tflops, 2),
         "bwd_main_tflops": round(main_tflops, 2),
         "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
         "bwd_stage_ms": {"preprocess": round(pre_ms, 4), "main": round(main_ms, 4), "dq_convert": round(conv_ms, 4)},
+        "gflop": {"fwd": round(f_fwd / 1e9, 3), "bwd": round(f_bwd / 1e9, 3),
+                  "fwd_tile_granular": round(g_fwd / 1e9, 3), "bwd_tile_granular": round(g_bwd / 1e9, 3)},
+        "value_tile_granular": round(mg.aggregate_rate(g_fwd + g_bwd, world, ms_step * 1e-3) / 1e12, 3),
         "frac_of_peak": {"fwd": round(fwd_tflops / peak["bf16_tflops"], 4),
                          "bwd": round(bwd_tflops / peak["bf16_tflops"], 4),
                          "denominator": f"bf16_tflops {peak['bf16_tflops']} ({peak_src})",
@@ -697,6 +805,17 @@ def run_gpu(args):
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
+    if not args.no_extras:
+        # the other workloads, device-timed in the same run (after the timed region above)
+        extras = {}
+        for name, (iters, warm) in EXTRA_CONFIGS.items():
+            if name == cfg.name:
+                continue
+            t = time_attention(CONFIGS[name], dev, iters, warm, flush)
+            extras[name] = config_figures(CONFIGS[name], t, peak)
+        extras[cfg.name] = config_figures(cfg, {"fwd_ms": fwd_ms, "pre_ms": pre_ms, "main_ms": main_ms,
+                                                "conv_ms": conv_ms}, peak)
+        res["configs"] = extras
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, dt, rows, threads = oracle_sample(cfg, args.cpu_seconds, q_h, k_h, v_h, do_h)
         res["cpu_baseline"] = {"value": round(tf, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
@@ -735,8 +854,7 @@ def run_reference(args):
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / max(1, args.steps) * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic (seeded N(0,1) bf16 widened to fp64)",
-           "config": {"workload": f"{cfg.name}: {cfg.note}", "B": cfg.B, "N": cfg.N, "H": cfg.H, "d": cfg.d,
-                      "causal": cfg.causal, "window": [cfg.win_l, cfg.win_r], "seed": cfg.seed},
+           "config": attn_config(cfg),
            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -794,12 +912,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="train_fwd_bwd",
+    ap.add_argument("--config", default="long_fwd_bwd",
                     choices=sorted(CONFIGS) + sorted(FP8_CONFIGS) + sorted(DECODE_CONFIGS))
     ap.add_argument("--splits", type=int, default=0, help="decode: CTAs (pieces) per head; 0 = library's choice")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the other workloads' device-timed figures")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -230,21 +231,59 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_
 
 // ---------------------------------------------------------------- launches (arguments already checked)
 
-// descales != nullptr: q, k, v hold E4M3 codes (head dim 128) with (B, H) descale factors.
-template <int D, bool kAlibi, bool kVarlen>
-void fwd_launch(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                const CUtensorMap& mo, const fa::FwdParams& p) {
-  constexpr int smem = fa::FwdCfg<D>::kSmemBytes + (kVarlen ? fa::kFwdSortBytes : 0);
-  fa::fa_fwd_kernel<D, false, kAlibi, kVarlen><<<grid, fa::FwdCfg<D>::kThreads, smem, stream>>>(mq, mk, mv, mo, p);
+// The forward's work counter: slots of fa::g_fwd_next_item are handed out in turn per device,
+// so calls in flight at the same time (on different streams) count in different slots as long
+// as fewer than kFwdCounterSlots of them overlap. Each launch zeroes its slot first.
+std::atomic<unsigned> g_fwd_slot_seq[kMaxDevices];
+
+// The counter-reset kernel, then the forward kernel as its programmatic dependent (it sets up
+// while the reset runs and waits for it before taking its first item).
+template <int D, bool kF8, bool kAlibi, bool kVarlen>
+int fwd_launch(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+               const CUtensorMap& mo, const fa::FwdParams& p) {
+  fa::fa_fwd_counter_reset_kernel<<<1, 32, 0, stream>>>(p.counter_slot);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(fa::FwdCfg<D, kF8>::kThreads);
+  cfg.dynamicSmemBytes = fa::FwdCfg<D, kF8>::kSmemBytes + (kVarlen ? fa::kFwdSortBytes : 0);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa::fa_fwd_kernel<D, kF8, kAlibi, kVarlen>, mq, mk, mv, mo, p) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  return FA_OK;
 }
 
 template <int D>
-void fwd_variant(bool alibi, bool varlen, int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
-                 const CUtensorMap& mv, const CUtensorMap& mo, const fa::FwdParams& p) {
-  if (alibi && varlen) fwd_launch<D, true, true>(grid, stream, mq, mk, mv, mo, p);
-  else if (alibi) fwd_launch<D, true, false>(grid, stream, mq, mk, mv, mo, p);
-  else if (varlen) fwd_launch<D, false, true>(grid, stream, mq, mk, mv, mo, p);
-  else fwd_launch<D, false, false>(grid, stream, mq, mk, mv, mo, p);
+int fwd_variant(bool alibi, bool varlen, int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
+                const CUtensorMap& mv, const CUtensorMap& mo, const fa::FwdParams& p) {
+  if (alibi && varlen) return fwd_launch<D, false, true, true>(grid, stream, mq, mk, mv, mo, p);
+  if (alibi) return fwd_launch<D, false, true, false>(grid, stream, mq, mk, mv, mo, p);
+  if (varlen) return fwd_launch<D, false, false, true>(grid, stream, mq, mk, mv, mo, p);
+  return fwd_launch<D, false, false, false>(grid, stream, mq, mk, mv, mo, p);
+}
+
+// Pair ranks of the forward's final phase (all heads, shortest last): enough for two items per
+// CTA, so that the end of the run is made of short items; all of them when that is more.
+int fwd_tail_ranks(const Shape& s, int num_pairs, int sm_count) {
+  const int bh = s.B * s.H;
+  const int k = (2 * sm_count + bh - 1) / bh;
+  return k < num_pairs ? k : num_pairs;
+}
+
+// Heads per scheduling group of the forward: as many as keep the K/V of one group within
+// 24 MiB (two groups in flight stay well inside L2), at least 1.
+int fwd_head_group(const Shape& s, int elem_bytes) {
+  const double kv_per_head = 2.0 * s.N * s.d * elem_bytes;
+  const double g = (24.0 * 1024 * 1024) / kv_per_head;
+  const int bh = s.B * s.H;
+  return g < 1.0 ? 1 : (g >= bh ? bh : (int)g);
 }
 
 // Offsets of a packed batch: cu[0] = 0, non-decreasing, cu[nseg] = n; a violation is reported
@@ -264,7 +303,7 @@ int launch_check_cu(const int* cu, int nseg, int n, cudaStream_t stream) {
 // alibi != nullptr: (B, H) ALiBi slopes (bf16 inputs).
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const Shape& s, float scale,
                int causal, int win_l, int win_r, int sm_count, cudaStream_t stream,
-               const float* const* descales = nullptr, const float* alibi = nullptr, const int* cu = nullptr,
+               int dev, const float* const* descales = nullptr, const float* alibi = nullptr, const int* cu = nullptr,
                int nseg = 0) {
   CUtensorMap mq, mk, mv, mo;
   int st;
@@ -289,6 +328,14 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.num_pairs = (s.N + 255) / 256;
   p.num_items = s.B * s.H * p.num_pairs;
   p.lse = lse;
+  if (cu) {  // packed batch: the cost-sorted pairs in one group (their order already ends short)
+    p.head_group = s.B * s.H;
+    p.tail_ranks = 0;
+  } else {
+    p.head_group = fwd_head_group(s, descales ? 1 : 2);
+    p.tail_ranks = fwd_tail_ranks(s, p.num_pairs, sm_count);
+  }
+  p.counter_slot = (int)(g_fwd_slot_seq[dev].fetch_add(1, std::memory_order_relaxed) % fa::kFwdCounterSlots);
   // Test-only fault knob: the forward withholds one internal signal so that a bounded wait in
   // the kernel runs out (it must report FA_ERR_TIMEOUT through fa_check, not hang).
   const char* drop = std::getenv("FA_DEBUG_DROP_S_SIGNAL");
@@ -299,13 +346,12 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                  s.H, s.d, p.causal, win_l, win_r, p.num_items, grid,
                  s.d == 64 ? fa::FwdCfg<64>::kSmemBytes : fa::FwdCfg<128>::kSmemBytes);
   if (descales)
-    fa::fa_fwd_kernel<128, true><<<grid, fa::FwdCfg<128, true>::kThreads, fa::FwdCfg<128, true>::kSmemBytes,
-                                   stream>>>(mq, mk, mv, mo, p);
+    st = fwd_launch<128, true, false, false>(grid, stream, mq, mk, mv, mo, p);
   else if (s.d == 64)
-    fwd_variant<64>(alibi != nullptr, cu != nullptr, grid, stream, mq, mk, mv, mo, p);
+    st = fwd_variant<64>(alibi != nullptr, cu != nullptr, grid, stream, mq, mk, mv, mo, p);
   else
-    fwd_variant<128>(alibi != nullptr, cu != nullptr, grid, stream, mq, mk, mv, mo, p);
-  return launch_status();
+    st = fwd_variant<128>(alibi != nullptr, cu != nullptr, grid, stream, mq, mk, mv, mo, p);
+  return st ? st : launch_status();
 }
 
 int launch_pre(const void* o, const float* lse, const void* dO, const Shape& s, const Workspace& w,
@@ -509,7 +555,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     return FA_ERR_INVALID_ARG;
   int dev, sms;
   if ((st = device_setup(&dev, &sms))) return st;
-  return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream));
+  return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream),
+                    dev);
 }
 
 int fa_fwd_ex(const void* q, const void* k, const void* v, const float* alibi_slopes, void* o, float* lse, int B,
@@ -530,7 +577,7 @@ int fa_fwd_ex(const void* q, const void* k, const void* v, const float* alibi_sl
   int dev, sms;
   if ((st = device_setup(&dev, &sms))) return st;
   return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream),
-                    nullptr, alibi_slopes);
+                    dev, nullptr, alibi_slopes);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, const int* cu_seqlens, const float* alibi_slopes,
@@ -554,7 +601,8 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, const int* cu_seq
   if ((st = device_setup(&dev, &sms))) return st;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   if ((st = launch_check_cu(cu_seqlens, B, total, cs))) return st;
-  return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, cs, nullptr, alibi_slopes, cu_seqlens, B);
+  return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, cs, dev, nullptr, alibi_slopes, cu_seqlens,
+                    B);
 }
 
 int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_descale, const float* k_descale,
@@ -578,7 +626,7 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_desca
   if ((st = device_setup(&dev, &sms))) return st;
   const float* descales[3] = {q_descale, k_descale, v_descale};
   return launch_fwd(q, k, v, o, lse, s, scale, causal, win_l, win_r, sms, reinterpret_cast<cudaStream_t>(stream),
-                    descales);
+                    dev, descales);
 }
 
 }  // extern "C"

@@ -55,14 +55,7 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Programmatic dependent launch: let the next kernel on the stream (launched with the
-// programmatic-serialization attribute) start, and, in that kernel, wait until the grids it
-// depends on have finished and their writes are visible. The wait returns at once in a
-// kernel launched without the attribute.
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 
 struct DecParams {
   int B, Sq, H, page_size, max_pages, num_pages;

@@ -9,7 +9,13 @@
 //
 // Work decomposition (persistent, one CTA per SM):
 //   work item = (b, h, pair of 128-row Q tiles); the two Q tiles share every K/V tile load.
-//   warp 0      : TMA producer (Q tiles; a ring of K/V tile slots)
+//   Items are dealt dynamically: the producer takes the next item from an atomic counter (one
+//   slot of a library-owned ring per call, zeroed by the kernel launched just before) and hands
+//   it to the other roles through a two-entry ring in shared memory. Items are ordered in groups
+//   of heads small enough that the K/V of the heads in flight stay in L2, longest first
+//   inside a group under causal masking, and the shortest pair ranks of every head come last
+//   (fwd_decode).
+//   warp 0      : work fetch and TMA producer (Q tiles; a ring of K/V tile slots)
 //   warp 1      : tcgen05 MMA issuer (one elected thread) and TMEM owner
 //   warps 2-3   : no role
 //   warps 4-7   : softmax + epilogue for Q tile 0 (one thread per query row / TMEM lane)
@@ -56,7 +62,20 @@ struct FwdParams {
   const float* alibi_slopes;  // ALiBi only: (B, H) slopes m, bias -m |i - j| on the scaled scores
   const int* cu_seqlens;      // packed variable-length batch (B = 1, N = total): nseg + 1 offsets, or null
   int nseg;
+  int head_group;             // heads per scheduling group (>= 1)
+  int tail_ranks;             // shortest pair ranks dealt last over all heads at once (<= num_pairs)
+  int counter_slot;           // this call's work counter: g_fwd_next_item[counter_slot]
 };
+
+// Work counters of the forward, one per call in flight: the host hands out the slots in turn
+// and zeroes a call's slot with fa_fwd_counter_reset_kernel just before the forward kernel.
+constexpr int kFwdCounterSlots = 1024;
+__device__ int g_fwd_next_item[kFwdCounterSlots];
+
+__global__ void fa_fwd_counter_reset_kernel(int slot) {
+  griddep_launch_dependents();  // the forward (its programmatic dependent) may start setting up
+  if (threadIdx.x == 0) g_fwd_next_item[slot] = 0;
+}
 
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P may grow to 2^8 before O is rescaled
 
@@ -115,16 +134,54 @@ struct FwdBars {
   uint64_t s_full[2], p_full[2];
   uint64_t s_empty[2], pv_done[2];  // kShareS: s_empty[0] for the shared S
   uint64_t mma_done;
+  uint64_t item_full[2], item_empty[2];  // ring of fetched work items, producer -> other roles
+  int item_w[2];
   uint32_t tmem_base;
   int abort_flag;
 };
 
-// Item w -> (b, h, pair). Under causal masking pairs are visited longest first; for a packed
-// batch `order` (when given) lists the pairs by decreasing cost.
+// Consumers of a fetched item: the MMA thread and the 8 softmax warps (one arrival each).
+constexpr uint32_t kFwdItemConsumers = 9;
+
+// Next work item of a consumer role (n counts the items this role has taken); values >=
+// num_items mean "no more work".
+template <class Bars>
+__device__ __forceinline__ int fwd_take_item(Bars* bars, uint32_t n, bool arrive, Abort ab) {
+  const uint32_t slot = n & 1;
+  mbar_wait(smem_u32(&bars->item_full[slot]), (n >> 1) & 1, ab);
+  const int w = *reinterpret_cast<volatile int*>(&bars->item_w[slot]);
+  __syncwarp(__activemask());
+  if (arrive) mbar_arrive(smem_u32(&bars->item_empty[slot]));
+  return ab.raised() ? 0x7fffffff : w;
+}
+
+// Item w -> (b, h, pair). Pair rank r is pair num_pairs - 1 - r under causal masking (longest
+// first), order[r] for a packed batch (pairs by decreasing cost), else r. Two phases:
+//   1. ranks [0, num_pairs - tail_ranks): groups of head_group heads in order, inside a group
+//      the rank slowest and the heads fastest, so that the K/V read by the items in flight
+//      belong to few heads and stay in L2;
+//   2. the tail_ranks shortest ranks over all heads, rank-major: the last items dealt are the
+//      shortest, whatever group ran last, so the CTAs finish together (the items of this phase
+//      read only the first few K/V tiles of each head).
 __device__ __forceinline__ void fwd_decode(const FwdParams& p, int w, int& b, int& h, int& pair,
                                            const uint16_t* order = nullptr) {
   const int bh_count = p.B * p.H;
-  const int r = w / bh_count, bh = w - r * bh_count;
+  const int ranks1 = p.num_pairs - p.tail_ranks;
+  const int n1 = bh_count * ranks1;
+  int r, bh;
+  if (w < n1) {
+    const int per_group = p.head_group * ranks1;
+    const int g = w / per_group;
+    const int pos = w - g * per_group;
+    const int gs = min(p.head_group, bh_count - g * p.head_group);  // heads in this group
+    r = pos / gs;
+    bh = g * p.head_group + (pos - r * gs);
+  } else {
+    const int w2 = w - n1;
+    const int r2 = w2 / bh_count;
+    r = ranks1 + r2;
+    bh = w2 - r2 * bh_count;
+  }
   pair = order ? (int)order[r] : p.causal ? (p.num_pairs - 1 - r) : r;
   b = bh / p.H;
   h = bh - b * p.H;
@@ -217,10 +274,14 @@ __device__ __forceinline__ void fwd_row_max(float (&x)[128], bool masked, int kb
 }
 
 // Exponentials of 32 columns (16 pairs starting at pair k0) against the reference maximum,
-// packed to bf16 pairs (even column low) and summed.
+// packed to bf16 pairs (even column low) and summed twice: `sum` adds the fp32 values (the
+// row sum of the log-sum-exp), `rsum` the bf16 values the tensor core multiplies with V (the
+// divisor of O, so that O is a weighted mean of V rows under exactly the weights applied: a
+// row dominated by one key then returns that key's value row, not the row times the
+// relative rounding error of its weight).
 template <bool kPosScale>
 __device__ __forceinline__ void fwd_exp_chunk(const float (&x)[128], int k0, float c, float m_use, uint32_t (&pk)[16],
-                                              float2& sum) {
+                                              float2& sum, float2& rsum) {
   const float2 neg_m = make_float2(-m_use, -m_use);
   const float2 c2 = make_float2(c, c);
 #pragma unroll
@@ -235,6 +296,7 @@ __device__ __forceinline__ void fwd_exp_chunk(const float (&x)[128], int k0, flo
     }
     sum = add2(sum, pv);
     pk[k] = pack_bf16x2(pv.x, pv.y);
+    rsum = add_bf16x2_f32x2(pk[k], rsum);
   }
 }
 
@@ -275,6 +337,7 @@ __global__ void __launch_bounds__(384, 1)
                   const FwdParams p) {
   using Cfg = FwdCfg<D, kF8>;
   using Bars = FwdBars<Cfg>;
+  static_assert(sizeof(Bars) <= 512, "barrier block");
   static_assert(!kF8 || D == 128, "E4M3 inputs: head dim 128 (one 128-byte row per TMA box)");
   static_assert(!(kF8 && kAlibi), "ALiBi is built for bf16 inputs");
   static_assert(!(kF8 && kVarlen), "packed batches are built for bf16 inputs");
@@ -302,6 +365,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(bars->kv_empty[s]), 1);
     }
     mbar_init(bar(bars->mma_done), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(bars->item_full[t]), 1);
+      mbar_init(bar(bars->item_empty[t]), kFwdItemConsumers);
+    }
     fence_barrier_init();
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
@@ -354,9 +421,15 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t qn[2] = {0, 0};
       int last_slot_parity[Cfg::kSlots];
       for (int s = 0; s < Cfg::kSlots; ++s) last_slot_parity[s] = -1;
-      for (int round = 0;; ++round) {
-        const int w = sched_item(round, blockIdx.x, gridDim.x);
-        if (w >= p.num_items || ab.raised()) break;
+      griddep_wait();  // this call's counter slot has been zeroed
+      int* counter = &g_fwd_next_item[p.counter_slot];
+      for (uint32_t n = 0;; ++n) {
+        const uint32_t islot = n & 1;
+        mbar_wait(bar(bars->item_empty[islot]), ((n >> 1) & 1) ^ 1, ab);
+        const int w = ab.raised() ? p.num_items : atomicAdd(counter, 1);
+        bars->item_w[islot] = w;
+        mbar_arrive(bar(bars->item_full[islot]));
+        if (w >= p.num_items) break;
         int b, h, pair;
         fwd_decode(p, w, b, h, pair, order);
         int lo_t[2], hi_t[2];
@@ -430,9 +503,9 @@ __global__ void __launch_bounds__(384, 1)
         }
       };
 
-      for (int round = 0;; ++round) {
-        const int w = sched_item(round, blockIdx.x, gridDim.x);
-        if (w >= p.num_items || ab.raised()) break;
+      for (uint32_t it = 0;; ++it) {
+        const int w = fwd_take_item(bars, it, true, ab);
+        if (w >= p.num_items) break;
         int b, h, pair;
         fwd_decode(p, w, b, h, pair, order);
         int lo_t[2], hi_t[2];
@@ -552,9 +625,9 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tP = tmem + lane_field + (t ? Cfg::kColP1 : Cfg::kColP0);
     uint32_t sn = 0, pvn = 0;
 
-    for (int round = 0;; ++round) {
-      const int w = sched_item(round, blockIdx.x, gridDim.x);
-      if (w >= p.num_items || ab.raised()) break;
+    for (uint32_t it = 0;; ++it) {
+      const int w = fwd_take_item(bars, it, lane_id() == 0, ab);
+      if (w >= p.num_items) break;
       int b, h, pair;
       fwd_decode(p, w, b, h, pair, order);
       const int r0 = pair * 256 + t * 128;
@@ -580,6 +653,7 @@ __global__ void __launch_bounds__(384, 1)
       int seg_first = 0, seg_last = 0;  // sequence of the tile's first row (packed batches)
       if (kVarlen) seg_bounds(p.cu_seqlens, p.nseg, p.N, r0, seg_first, seg_last);
       float m_run = -INFINITY, l_run = 0.0f;
+      float lr_run = 0.0f;  // sum of the bf16-rounded weights (bf16 P): the divisor of O
 
       for (int j = lo; j <= hi; ++j) {
         mbar_wait(bar(bars->s_full[t]), sn & 1, ab);
@@ -615,6 +689,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         // P in 32-column chunks straight into TMEM (E4M3: over S columns already read into registers)
         float2 sum0 = make_float2(0.0f, 0.0f), sum1 = make_float2(0.0f, 0.0f);
+        float2 rs0 = make_float2(0.0f, 0.0f), rs1 = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           if constexpr (kF8) {
@@ -627,14 +702,18 @@ __global__ void __launch_bounds__(384, 1)
           } else {
             uint32_t pk[16];
             if (pos_scale)
-              fwd_exp_chunk<true>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
+              fwd_exp_chunk<true>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0, (q4 & 1) ? rs1 : rs0);
             else
-              fwd_exp_chunk<false>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0);
+              fwd_exp_chunk<false>(x, q4 * 16, c, m_use, pk, (q4 & 1) ? sum1 : sum0, (q4 & 1) ? rs1 : rs0);
             tmem_st16(tP + q4 * 16, pk);
           }
         }
         const float2 s01 = add2(sum0, sum1);
         l_run = l_run * alpha + (s01.x + s01.y);
+        if constexpr (!kF8) {
+          const float2 r01 = add2(rs0, rs1);
+          lr_run = lr_run * alpha + (r01.x + r01.y);
+        }
 
         // Rescale O_t in TMEM when this warp's reference maximum moved (not on the first tile:
         // the first PV of an item overwrites O_t).
@@ -662,7 +741,10 @@ __global__ void __launch_bounds__(384, 1)
         if (row == 0) bulk_wait_group_read0();  // the previous store has read the staging tile
         named_bar_sync(1 + t, 128);
       }
-      const float inv_l = l_run > 0.0f ? o_mul / l_run : 0.0f;
+      // bf16 P: O is divided by the sum of the weights it was accumulated with; E4M3 P keeps the
+      // fp32 sum (its tolerance is derived for that divisor)
+      const float l_o = kF8 ? l_run : lr_run;
+      const float inv_l = l_o > 0.0f ? o_mul / l_o : 0.0f;
       const uint32_t stage = sO[t];
 #pragma unroll 1
       for (int cc = 0; cc < D; cc += 32) {

@@ -436,6 +436,18 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float x0, float x1, float x2, fl
   return (uint32_t)lo | ((uint32_t)hi << 16);
 }
 
+// acc.x += low bf16 of v, acc.y += high bf16 of v: sm_100's mixed-precision add (the bf16
+// operand is widened exactly), so a packed pair is summed without unpacking it first.
+__device__ __forceinline__ float2 add_bf16x2_f32x2(uint32_t v, float2 acc) {
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\t"
+      "add.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "r"(v));
+  return acc;
+}
+
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
@@ -455,12 +467,13 @@ __device__ __forceinline__ void red_add_v4_f32(float* gptr, float a, float b, fl
                : "memory");
 }
 
-// ------------------------------------------------------------------ persistent scheduling
-
-// Work item of a persistent CTA in a given round: snake order over rounds of gridDim.x
-// items, so that a CTA given a long item in one round gets a short one in the next.
-__device__ __forceinline__ int sched_item(int round, int cta, int grid) {
-  return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+// Programmatic dependent launch: let the next kernel on the stream (launched with the
+// programmatic-serialization attribute) start, and, in that kernel, wait until the grids it
+// depends on have finished and their writes are visible. The wait returns at once in a
+// kernel launched without the attribute.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 }  // namespace fa

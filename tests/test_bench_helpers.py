@@ -41,7 +41,33 @@ def test_decode_cache_bytes_counts_visible_rows_and_small_tensors():
 
 
 def test_traffic_lookup():
-    assert bench.recorded_traffic("no_such_kernel") is None
+    assert bench.recorded_traffic("no_such_kernel", "train_fwd_bwd") is None
     h1 = bench.kernel_source_hash(["fa_fwd.cuh", "sm100_ptx.cuh"])
     assert h1 == bench.kernel_source_hash(["fa_fwd.cuh", "sm100_ptx.cuh"]) and len(h1) == 16
     assert h1 != bench.kernel_source_hash(["fa_bwd.cuh", "sm100_ptx.cuh"])
+
+
+def test_tile_granular_count_matches_brute_force_and_the_configs():
+    from exact_attention_116_b200.workload import flops, flops_tile_granular, visible_pairs, visible_tile_pairs
+    import numpy as np
+    for N, causal, wl, wr in [(300, False, -1, -1), (300, True, -1, -1), (700, False, 128, 128), (513, False, 0, 0),
+                              (1030, True, 100, -1), (640, False, -1, 200), (1, False, -1, -1)]:
+        i = np.arange(N)[:, None]
+        j = np.arange(N)[None, :]
+        vis = np.ones((N, N), bool)
+        if wl >= 0:
+            vis &= j >= i - wl
+        r = 0 if causal else wr
+        if r >= 0:
+            vis &= j <= i + r
+        nt = (N + 127) // 128
+        blocks = sum(bool(vis[a * 128:(a + 1) * 128, b * 128:(b + 1) * 128].any()) for a in range(nt) for b in range(nt))
+        assert visible_tile_pairs(N, causal, wl, wr) == blocks
+        assert visible_pairs(N, causal, wl, wr) == int(vis.sum())
+    # the workloads' forward GFLOP, exact and tile-granular
+    assert round(flops(2, 8192, 16, 128, True, -1, -1)[0] / 1e9, 1) == 549.8
+    assert round(flops_tile_granular(2, 8192, 16, 128, True, -1, -1)[0] / 1e9, 1) == 558.3
+    # 256 key tiles, causal: 256 * 257 / 2 = 32896 blocks per head, each 4 * 128 * 128 * 128 FLOPs
+    assert flops_tile_granular(1, 32768, 16, 128, True, -1, -1)[0] == 32896 * 16 * 4 * 128 * 128 * 128
+    assert round(flops_tile_granular(4, 2048, 16, 64, True, -1, -1)[0] / 1e9, 2) == 36.51
+    assert round(flops_tile_granular(2, 16384, 16, 64, False, 128, 128)[0] / 1e9, 2) == 51.27
