@@ -35,11 +35,17 @@ class FaError(RuntimeError):
 def load() -> ctypes.CDLL:
     """Load the in-tree CUDA library (built by ``exact_attention_116_b200.build``)."""
     global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing (run __graft_entry__.build())")
-    lib = ctypes.CDLL(LIB_PATH)
+    if _lib is None:
+        _lib = open_library(LIB_PATH)
+    return _lib
+
+
+def open_library(path: str) -> ctypes.CDLL:
+    """Open a build of the C ABI (the library or its bounds-checking variant, libfa_sm100_debug.so)
+    and declare its argument types. Every wrapper here calls the one ``load()`` returns."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} is missing (run __graft_entry__.build())")
+    lib = ctypes.CDLL(path)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
     lib.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
@@ -63,10 +69,11 @@ def load() -> ctypes.CDLL:
     lib.fa_check.argtypes = [vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
-    for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_fp8", "fa_decode_paged", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
-                 "fa_check"):
+    lib.fa_bwd_static_workspace.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    for name in ("fa_fwd", "fa_fwd_ex", "fa_bwd_ex", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_fp8", "fa_decode_paged",
+                 "fa_bwd", "fa_bwd_deterministic", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_dq_convert",
+                 "fa_bwd_static_workspace", "fa_check"):
         getattr(lib, name).restype = i
-    _lib = lib
     return lib
 
 
@@ -276,13 +283,7 @@ def bwd_into_static_workspace(q, k, v, o, lse, do, dq, dk, dv, scale=None, causa
     """
     B, N, H, d = _check_qkv(q, k, v, o, do, dq, dk, dv)
     _check_lse(lse, (B, H, N))
-    lib = load()
-    fn = lib.fa_bwd_static_workspace
-    if fn.argtypes is None:
-        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-        fn.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
-        fn.restype = i
-    st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+    st = load().fa_bwd_static_workspace(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, H, d, _scale(scale, d), int(bool(causal)),
             int(window[0]), int(window[1]), _stream_handle(stream))
     _raise(st, "fa_bwd_static_workspace")

@@ -19,6 +19,10 @@ HEADERS = [os.path.join(PKG, "csrc", f) for f in ("fa_fwd.cuh", "fa_bwd.cuh", "f
     os.path.join(ROOT, "include", "fa_sm100.h")
 ]
 LIB = os.path.join(PKG, "libfa_sm100.so")
+# The same library with device-side bounds checks (-DFA_DEBUG=1): every computed TMA coordinate,
+# bulk-copy range, shared-memory destination and global index is checked before use; a failed
+# check is reported through fa_check as FA_ERR_DEVICE instead of touching memory out of range.
+LIB_DEBUG = os.path.join(PKG, "libfa_sm100_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -44,14 +48,16 @@ def needs_build(out: str = LIB) -> bool:
     return any(os.path.getmtime(f) > t for f in [SRC, *HEADERS])
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if force or needs_build():
-        tmp = LIB + ".tmp"
-        subprocess.check_call(command(tmp, verbose_ptxas))
-        os.replace(tmp, LIB)
-    return LIB
+def build(force: bool = False, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    """Compile the library (or, with debug=True, its bounds-checking variant) if a source changed."""
+    out = LIB_DEBUG if debug else LIB
+    if force or needs_build(out):
+        tmp = out + ".tmp"
+        subprocess.check_call(command(tmp, verbose_ptxas, ["-DFA_DEBUG=1"] if debug else None))
+        os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv)
-    print(LIB)
+    dbg = "--debug" in sys.argv
+    print(build(force="--force" in sys.argv, verbose_ptxas="-v" in sys.argv, debug=dbg))

@@ -96,9 +96,12 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
   if (bh >= (long long)B * H) return;
   const int b = (int)(bh / H), h = (int)(bh % H);
   const size_t stat = (size_t)bh * (size_t)N_pad + n;
+  const Abort none{nullptr};
+  // (FA_DEBUG: a failed check skips the accesses; every thread still takes part in the shuffle)
+  const bool stat_ok = dbg_range(none, (long long)stat, 1, (long long)B * H * N_pad);
   float acc = 0.0f;
-  if (n < N) {
-    const size_t row = (((size_t)b * N + n) * H + h) * (size_t)D + part * 8;
+  const size_t row = (((size_t)b * N + n) * H + h) * (size_t)D + part * 8;
+  if (n < N && dbg_range(none, (long long)row, 8, (long long)B * N * H * D)) {
     const uint4 ov = *reinterpret_cast<const uint4*>(o + row);
     const uint4 gv = *reinterpret_cast<const uint4*>(dout + row);
     const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w}, gw[4] = {gv.x, gv.y, gv.z, gv.w};
@@ -111,7 +114,7 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
   }
 #pragma unroll
   for (int off = Cfg::kThreadsPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (part == 0) {
+  if (part == 0 && stat_ok) {
     dvec[stat] = n < N ? -acc : 0.0f;
     lse2[stat] = n < N ? -lse[(size_t)bh * (size_t)N + n] * kLog2e : 0.0f;
   }
@@ -287,6 +290,15 @@ __global__ void __launch_bounds__(512, 1)
 
   const int warp = threadIdx.x >> 5;
   const Abort ab{&bars->abort_flag};
+  const uint32_t smem_end = smem_base + Cfg::kSmemBytes;  // for the FA_DEBUG bounds checks
+  // FA_DEBUG: the d/64 boxes of the 128-row bf16 tile at `row` of (b, h)
+  auto tile_ok = [&](uint32_t dst, int row, int b, int h) {
+    bool ok = true;
+#pragma unroll
+    for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+      ok = ok && dbg_tma(ab, bx * 64, row, h, b, D, p.N, p.H, p.B, 2, dst + bx * 16384, 16384, smem_base, smem_end);
+    return ok;
+  };
 
   if (threadIdx.x == 0) {
     bars->abort_flag = 0;
@@ -358,6 +370,7 @@ __global__ void __launch_bounds__(512, 1)
         bwd_q_range<kVarlen>(p, j, lo, hi);
         const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
         mbar_wait(bar(bars->kv_empty[kvs]), kvphase ^ 1, ab);
+        if (!tile_ok(sKs(items), j * 128, b, h) || !tile_ok(sVs(items), j * 128, b, h)) break;
         mbar_arrive_expect_tx(bar(bars->kv_full[kvs]), 2 * Cfg::kTileBytes);
 #pragma unroll
         for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
@@ -370,6 +383,10 @@ __global__ void __launch_bounds__(512, 1)
           // Q_i and its statistics into the next Q slot
           mbar_wait(bar(bars->q_empty[qs]), qphase ^ 1, ab);
           const uint32_t fb = bar(bars->q_full[qs]);
+          const long long stat_size = (long long)p.B * p.H * p.N_pad;
+          if (!tile_ok(sQ(qs), i * 128, b, h) || !dbg_range(ab, (long long)stat_row + i * 128, 128, stat_size) ||
+              !dbg_range(ab, sStat(qs) - smem_base, 1024, smem_end - smem_base))
+            break;
           mbar_arrive_expect_tx(fb, Cfg::kTileBytes + 1024);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx) tma_load_4d(sQ(qs) + bx * 16384, &tmQ, fb, bx * 64, i * 128, h, b);
@@ -380,6 +397,7 @@ __global__ void __launch_bounds__(512, 1)
           // dO_i into the single dO slot (freed when dV_{i-1} is done)
           const uint32_t dos = dn % Cfg::kDOSlots, dophase = (dn / Cfg::kDOSlots) & 1;
           mbar_wait(bar(bars->do_empty[dos]), dophase ^ 1, ab);
+          if (!tile_ok(sDOs(dn), i * 128, b, h)) break;  // (the next fetch then ends the loop)
           mbar_arrive_expect_tx(bar(bars->do_full[dos]), Cfg::kTileBytes);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
@@ -530,7 +548,9 @@ __global__ void __launch_bounds__(512, 1)
           }
           fence_proxy_async_smem();
           named_bar_sync(3, 128);
-          if (row == 0) {
+          if (row == 0 &&
+              dbg_tma(ab, r * 64, i * 128, h, b, D, p.N, p.H, p.B, 4, sDQ, 16384, smem_base, smem_end) &&
+              dbg_tma(ab, r * 64 + 32, i * 128, h, b, D, p.N, p.H, p.B, 4, sDQ + 16384, 16384, smem_base, smem_end)) {
             tma_reduce_add_4d(&tmdQacc, sDQ, r * 64, i * 128, h, b);
             tma_reduce_add_4d(&tmdQacc, sDQ + 16384, r * 64 + 32, i * 128, h, b);
             bulk_commit_group();
@@ -660,7 +680,9 @@ __global__ void __launch_bounds__(512, 1)
       if (row == 0) {
 #pragma unroll
         for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-          tma_store_4d(grp ? &tmdV : &tmdK, stage_buf + bx * 16384, bx * 64, j * 128, h, b);
+          if (dbg_tma(ab, bx * 64, j * 128, h, b, D, p.N, p.H, p.B, 2, stage_buf + bx * 16384, 16384, smem_base,
+                      smem_end))
+            tma_store_4d(grp ? &tmdV : &tmdK, stage_buf + bx * 16384, bx * 64, j * 128, h, b);
         bulk_commit_group();
         bulk_wait_group_read0();
         mbar_arrive(bar(bars->kv_empty[kvs]));

@@ -142,6 +142,14 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
   const uint32_t sQ = smem_base + Cfg::kOffQ, sDO = smem_base + Cfg::kOffDO, sKV = smem_base + Cfg::kOffKV;
+  const uint32_t smem_end = smem_u32(smem_raw) + Cfg::kSmemBytes;  // for the FA_DEBUG bounds checks
+  auto tile_ok = [&](uint32_t dst, int row, int b, int h) {  // FA_DEBUG: the tile's d/64 boxes
+    bool ok = true;
+#pragma unroll
+    for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+      ok = ok && dbg_tma(ab, bx * 64, row, h, b, D, p.N, p.H, p.B, 2, dst + bx * 16384, 16384, smem_base, smem_end);
+    return ok;
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- work fetch + TMA producer
@@ -161,6 +169,7 @@ __global__ void __launch_bounds__(256, 1)
         int lo, hi;
         fwd_kv_range<kVarlen>(fp, i * 128, lo, hi);
         mbar_wait(bar(bars->q_empty), (qn & 1) ^ 1, ab);
+        if (!tile_ok(sQ, i * 128, b, h) || !tile_ok(sDO, i * 128, b, h)) break;
         mbar_arrive_expect_tx(bar(bars->q_full), 2 * Cfg::kTileBytes);
 #pragma unroll
         for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
@@ -168,11 +177,12 @@ __global__ void __launch_bounds__(256, 1)
           tma_load_4d(sDO + bx * 16384, &tmdO, bar(bars->q_full), bx * 64, i * 128, h, b);
         }
         ++qn;
-        for (int j = lo; j <= hi; ++j) {
+        for (int j = lo; j <= hi && !(FA_DEBUG && ab.raised()); ++j) {
           for (int kv = 0; kv < 2; ++kv) {
             mbar_wait(bar(bars->kv_empty[slot]), phase ^ 1, ab);
-            mbar_arrive_expect_tx(bar(bars->kv_full[slot]), Cfg::kTileBytes);
             const uint32_t dst = sKV + slot * Cfg::kTileBytes;
+            if (!tile_ok(dst, j * 128, b, h)) break;
+            mbar_arrive_expect_tx(bar(bars->kv_full[slot]), Cfg::kTileBytes);
 #pragma unroll
             for (int bx = 0; bx < Cfg::kBoxes; ++bx)
               tma_load_4d(dst + bx * 16384, kv ? &tmV : &tmK, bar(bars->kv_full[slot]), bx * 64, j * 128, h, b);
@@ -358,7 +368,9 @@ __global__ void __launch_bounds__(256, 1)
       named_bar_sync(1, 128);
       if (row == 0) {
 #pragma unroll
-        for (int bx = 0; bx < Cfg::kBoxes; ++bx) tma_store_4d(&tmdQ, sQ + bx * 16384, bx * 64, i * 128, h, b);
+        for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+          if (dbg_tma(ab, bx * 64, i * 128, h, b, D, p.N, p.H, p.B, 2, sQ + bx * 16384, 16384, smem_base, smem_end))
+            tma_store_4d(&tmdQ, sQ + bx * 16384, bx * 64, i * 128, h, b);
         bulk_commit_group();
         bulk_wait_group_read0();
         mbar_arrive(bar(bars->q_empty));

@@ -175,19 +175,29 @@ struct DecWalk {
 
 // TMA loads of the piece's next tile (stream index `issued`, at the walk's position) into its
 // ring slot; advances the walk and the count.
+// FA_DEBUG: a tile whose table index, coordinates or ring slot fail the bounds check is neither
+// armed nor loaded (the CTA's abort flag is then raised, so its waits return).
 template <class Cfg>
 __device__ __forceinline__ void dec_issue_tile(const DecParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                                uint32_t smem_base, uint64_t* full, int h, long long u0, long long u1,
-                                               DecWalk& ld, long long& issued) {
+                                               DecWalk& ld, long long& issued, Abort ab, uint32_t smem_end) {
   const int st = (int)(issued % Cfg::kStages);
   const int key = ld.t * kDecTile;
-  int page = p.block_table[(size_t)ld.b * p.max_pages + key / p.page_size];
+  const long long ti = (long long)ld.b * p.max_pages + key / p.page_size;
+  if (!dbg_range(ab, ti, 1, (long long)p.B * p.max_pages)) return;
+  int page = p.block_table[ti];
   if (page < 0 || page >= p.num_pages) {  // the TMA would read zeros there; report it
     atomicOr(&g_fa_error, kErrBadInput);
     page = 0;
   }
   const int row = key % p.page_size;
   const uint32_t dst = smem_base + Cfg::kOffKV + st * Cfg::kStageBytes;
+  bool ok = true;
+#pragma unroll
+  for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+    ok = ok && dbg_tma(ab, bx * 64, h, row, page, Cfg::kBoxes * 64, p.H, p.page_size, p.num_pages, 2,
+                       dst + bx * (kDecTile * 128), 2 * Cfg::kTileBytes - bx * (kDecTile * 128), smem_base, smem_end);
+  if (!ok) return;
   mbar_arrive_expect_tx(smem_u32(&full[st]), Cfg::kStageBytes);
 #pragma unroll
   for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
@@ -217,6 +227,11 @@ __global__ void __launch_bounds__(kDecThreads)
   long long* sSum = reinterpret_cast<long long*>(sm + Cfg::kOffMisc);  // [0, 4) warp sums, [4] first start
   int* sInt = reinterpret_cast<int*>(sm + Cfg::kOffMisc + 48);          // [0] first sequence, [1] last flag
   const Abort ab{abort_flag};
+  const uint32_t smem_end = smem_u32(smem_raw) + Cfg::kSmemBytes;  // for the FA_DEBUG bounds checks
+  // FA_DEBUG: index ranges of the outputs, the partial slots and the cache rows
+  const long long o_size = (long long)p.B * p.Sq * p.H * D, lse_size = (long long)p.B * p.H * p.Sq;
+  const long long part_rows = ((long long)p.B + p.pieces - 1) * p.H * p.Sq;
+  const long long cache_size = (long long)p.num_pages * p.page_size * p.H * D;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   static_assert(kSq >= 1 && kSq <= kDecMaxSq, "rows per CTA");
   static_assert(kDecThreads == 128, "the scan below assumes four warps");
@@ -282,9 +297,11 @@ __global__ void __launch_bounds__(kDecThreads)
     if (dec_vis_tiles(p, dec_len(p, b, false), vt0) != 0) continue;
     for (int e = tid; e < Sq * D; e += kDecThreads) {
       const int i = e / D, col = e - i * D;
-      p.o[(((size_t)b * Sq + i) * p.H + h) * D + col] = __float2bfloat16_rn(0.0f);
+      const long long oi = (((long long)b * Sq + i) * p.H + h) * D + col;
+      if (dbg_range(ab, oi, 1, o_size)) p.o[oi] = __float2bfloat16_rn(0.0f);
     }
-    if (tid < Sq) p.lse[((size_t)b * p.H + h) * Sq + tid] = -INFINITY;
+    const long long li = ((long long)b * p.H + h) * Sq + tid;
+    if (tid < Sq && dbg_range(ab, li, 1, lse_size)) p.lse[li] = -INFINITY;
   }
 
   // ---- new rows in this piece's tiles: head h's columns go into the cache before any tile load
@@ -301,6 +318,7 @@ __global__ void __launch_bounds__(kDecThreads)
         if (page < 0 || page >= p.num_pages) continue;  // reported when the tile is loaded
         const size_t src = (((size_t)w.b * Sq + i) * p.H + h) * D;
         const size_t dst = (((size_t)page * p.page_size + pos % p.page_size) * p.H + h) * D;
+        if (!dbg_range(ab, (long long)src, D, o_size) || !dbg_range(ab, (long long)dst, D, cache_size)) continue;
         if (tid < kChunks) {
           reinterpret_cast<uint4*>(p.k_cache + dst)[tid] = reinterpret_cast<const uint4*>(p.k_new + src)[tid];
         } else if (tid < 2 * kChunks) {
@@ -324,7 +342,7 @@ __global__ void __launch_bounds__(kDecThreads)
     prefetch_tmap(&tmV);
     ld.begin(p, b_first, start_first, u0, u1);
     while (issued < kStages && issued < n_tiles)
-      dec_issue_tile<Cfg>(p, &tmK, &tmV, smem_base, full, h, u0, u1, ld, issued);
+      dec_issue_tile<Cfg>(p, &tmK, &tmV, smem_base, full, h, u0, u1, ld, issued, ab, smem_end);
   }
 
   const float c = p.scale_log2;
@@ -337,7 +355,8 @@ __global__ void __launch_bounds__(kDecThreads)
     // q rows of (b, h) -> shared memory (fp32); rows >= Sq are zero
     for (int e = tid; e < kSq * D; e += kDecThreads) {
       const int i = e / D, col = e - i * D;
-      sQ[e] = i < Sq ? __bfloat162float(p.q[(((size_t)b * Sq + i) * p.H + h) * D + col]) : 0.0f;
+      const long long qi = (((long long)b * Sq + i) * p.H + h) * D + col;
+      sQ[e] = (i < Sq && dbg_range(ab, qi, 1, o_size)) ? __bfloat162float(p.q[qi]) : 0.0f;
     }
     if (tid < kSq) sAlpha[tid] = 0.0f;  // rows past Sq keep alpha = 0 (their O stays 0)
     __syncthreads();
@@ -387,7 +406,7 @@ __global__ void __launch_bounds__(kDecThreads)
       // every thread has finished with the previous tile's slot: refill it (not after a wait
       // gave up: that slot's barrier may still be waiting for bytes, and must not be armed twice)
       if (tid == 0 && k > 0 && issued < n_tiles && !ab.raised())
-        dec_issue_tile<Cfg>(p, &tmK, &tmV, smem_base, full, h, u0, u1, ld, issued);
+        dec_issue_tile<Cfg>(p, &tmK, &tmV, smem_base, full, h, u0, u1, ld, issued, ab, smem_end);
       // ---- B: softmax bookkeeping, warp w -> rows w, w + 4
 #pragma unroll
       for (int r = 0; r < (kSq + 3) / 4; ++r) {
@@ -470,17 +489,22 @@ __global__ void __launch_bounds__(kDecThreads)
 #pragma unroll
       for (int g = 0; g < Cfg::kKeyGroups; ++g) v += sRed[(g * kSq + i) * D + col];
       v *= sAlpha[i];
-      if (pf == pl)
-        p.o[(((size_t)b * Sq + i) * p.H + h) * D + col] = __float2bfloat16_rn(v);
-      else
-        p.o_part[((slot * p.H + h) * Sq + i) * D + col] = v;
+      const long long oi = (((long long)b * Sq + i) * p.H + h) * D + col;
+      const long long pi = (((long long)slot * p.H + h) * Sq + i) * D + col;
+      if (pf == pl) {
+        if (dbg_range(ab, oi, 1, o_size)) p.o[oi] = __float2bfloat16_rn(v);
+      } else if (dbg_range(ab, pi, 1, part_rows * D)) {
+        p.o_part[pi] = v;
+      }
     }
     if (tid < Sq) {
       const float l2 = sS[tid];
-      if (pf == pl)
-        p.lse[((size_t)b * p.H + h) * Sq + tid] = l2 == -INFINITY ? -INFINITY : l2 * kDecLn2;
-      else
-        p.lse_part[(slot * p.H + h) * Sq + tid] = l2;
+      const long long li = ((long long)b * p.H + h) * Sq + tid, pi = ((long long)slot * p.H + h) * Sq + tid;
+      if (pf == pl) {
+        if (dbg_range(ab, li, 1, lse_size)) p.lse[li] = l2 == -INFINITY ? -INFINITY : l2 * kDecLn2;
+      } else if (dbg_range(ab, pi, 1, part_rows)) {
+        p.lse_part[pi] = l2;
+      }
     }
     if (pf != pl) {
       // arrival: the last piece of (b, h) merges all partials
@@ -488,7 +512,8 @@ __global__ void __launch_bounds__(kDecThreads)
       __syncthreads();
       if (tid == 0) {
         griddep_wait();  // the prep kernel has zeroed the counters
-        const int before = atomicAdd(&p.arrivals[(size_t)b * p.H + h], 1);
+        const long long ai = (long long)b * p.H + h;
+        const int before = dbg_range(ab, ai, 1, (long long)p.B * p.H) ? atomicAdd(&p.arrivals[ai], 1) : -1;
         sInt[1] = before == pl - pf;
       }
       __syncthreads();
@@ -499,6 +524,9 @@ __global__ void __launch_bounds__(kDecThreads)
         for (int e = tid; e < Sq * D; e += kDecThreads) {
           const int i = e / D, col = e - i * D;
           float mx = -INFINITY;
+          if (!dbg_range(ab, (((long long)b + pf) * p.H + h) * Sq + i, 1, part_rows) ||
+              !dbg_range(ab, (((long long)b + pl) * p.H + h) * Sq + i, 1, part_rows))
+            continue;
           for (int r = pf; r <= pl; ++r)
             mx = fmaxf(mx, __ldcg(p.lse_part + (((size_t)b + r) * p.H + h) * Sq + i));
           float wsum = 0.0f, v = 0.0f;
@@ -510,9 +538,10 @@ __global__ void __launch_bounds__(kDecThreads)
               v = fmaf(wr, __ldcg(p.o_part + row * D + col), v);
             }
           }
-          p.o[(((size_t)b * Sq + i) * p.H + h) * D + col] = __float2bfloat16_rn(wsum > 0.0f ? v / wsum : 0.0f);
-          if (col == 0)
-            p.lse[((size_t)b * p.H + h) * Sq + i] = mx == -INFINITY ? -INFINITY : (mx + __log2f(wsum)) * kDecLn2;
+          const long long oi = (((long long)b * Sq + i) * p.H + h) * D + col, li = ((long long)b * p.H + h) * Sq + i;
+          if (dbg_range(ab, oi, 1, o_size)) p.o[oi] = __float2bfloat16_rn(wsum > 0.0f ? v / wsum : 0.0f);
+          if (col == 0 && dbg_range(ab, li, 1, lse_size))
+            p.lse[li] = mx == -INFINITY ? -INFINITY : (mx + __log2f(wsum)) * kDecLn2;
         }
       }
     }

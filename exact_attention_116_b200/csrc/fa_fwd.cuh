@@ -344,6 +344,8 @@ __global__ void __launch_bounds__(384, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* smem_gen = smem_raw + (smem_base - smem_u32(smem_raw));
+  // end of this launch's dynamic shared memory (for the FA_DEBUG bounds checks)
+  const uint32_t smem_end = smem_u32(smem_raw) + Cfg::kSmemBytes + (kVarlen ? kFwdSortBytes : 0);
   Bars* bars = reinterpret_cast<Bars*>(smem_gen + Cfg::kOffBar);
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
 
@@ -423,10 +425,11 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < Cfg::kSlots; ++s) last_slot_parity[s] = -1;
       griddep_wait();  // this call's counter slot has been zeroed
       int* counter = &g_fwd_next_item[p.counter_slot];
+      if (!dbg_range(ab, p.counter_slot, 1, kFwdCounterSlots)) counter = nullptr;
       for (uint32_t n = 0;; ++n) {
         const uint32_t islot = n & 1;
         mbar_wait(bar(bars->item_empty[islot]), ((n >> 1) & 1) ^ 1, ab);
-        const int w = ab.raised() ? p.num_items : atomicAdd(counter, 1);
+        const int w = (ab.raised() || !counter) ? p.num_items : atomicAdd(counter, 1);
         bars->item_w[islot] = w;
         mbar_arrive(bar(bars->item_full[islot]));
         if (w >= p.num_items) break;
@@ -438,9 +441,19 @@ __global__ void __launch_bounds__(384, 1)
         const bool act1 = hi_t[1] >= lo_t[1];
         const int lo = act1 ? min(lo_t[0], lo_t[1]) : lo_t[0];
         const int hi = act1 ? max(hi_t[0], hi_t[1]) : hi_t[0];
+        // FA_DEBUG: a tile whose boxes fail the bounds check is neither armed nor loaded
+        auto tile_ok = [&](uint32_t dst, int row) {
+          bool ok = true;
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+            ok = ok && dbg_tma(ab, bx * Cfg::kBoxElems, row, h, b, D, p.N, p.H, p.B, Cfg::kElem, dst + bx * 16384,
+                               16384, smem_base, smem_end);
+          return ok;
+        };
         for (int t = 0; t < 2; ++t) {
           if (hi_t[t] < lo_t[t]) continue;
           mbar_wait(bar(bars->q_empty[t]), (qn[t] & 1) ^ 1, ab);
+          if (!tile_ok(sQ[t], pair * 256 + t * 128)) break;
           mbar_arrive_expect_tx(bar(bars->q_full[t]), Cfg::kTileBytes);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
@@ -448,11 +461,12 @@ __global__ void __launch_bounds__(384, 1)
                         b);
           ++qn[t];
         }
-        for (int j = lo; j <= hi; ++j) {
+        for (int j = lo; j <= hi && !(FA_DEBUG && ab.raised()); ++j) {
           for (int kv = 0; kv < 2; ++kv) {
             mbar_wait(bar(bars->kv_empty[slot]), phase ^ 1, ab);
-            mbar_arrive_expect_tx(bar(bars->kv_full[slot]), Cfg::kTileBytes);
             const uint32_t dst = sKV + slot * Cfg::kTileBytes;
+            if (!tile_ok(dst, j * 128)) break;
+            mbar_arrive_expect_tx(bar(bars->kv_full[slot]), Cfg::kTileBytes);
 #pragma unroll
             for (int bx = 0; bx < Cfg::kBoxes; ++bx)
               tma_load_4d(dst + bx * 16384, kv ? &tmV : &tmK, bar(bars->kv_full[slot]), bx * Cfg::kBoxElems, j * 128,
@@ -461,6 +475,7 @@ __global__ void __launch_bounds__(384, 1)
             if (++slot == Cfg::kSlots) { slot = 0; phase ^= 1; }
           }
         }
+        if (FA_DEBUG && ab.raised()) break;
       }
       // Drain: every load issued must have landed before the CTA can exit.
       for (int s = 0; s < Cfg::kSlots; ++s)
@@ -636,6 +651,7 @@ __global__ void __launch_bounds__(384, 1)
       if (hi < lo) continue;
       float c = p.scale_log2, o_mul = 1.0f;  // log2-domain score factor; O factor
       float nslope2 = 0.0f;                  // ALiBi: -m log2(e)
+      if (!dbg_range(ab, (long long)b * p.H + h, 1, (long long)p.B * p.H)) break;
       if constexpr (kAlibi) nslope2 = -p.alibi_slopes[b * p.H + h] * kLog2e;
       if constexpr (kF8) {
         const int bh = b * p.H + h;
@@ -765,7 +781,9 @@ __global__ void __launch_bounds__(384, 1)
       named_bar_sync(1 + t, 128);
       if (row == 0) {
 #pragma unroll
-        for (int bx = 0; bx < Cfg::kOBoxes; ++bx) tma_store_4d(&tmO, stage + bx * 16384, bx * 64, r0, h, b);
+        for (int bx = 0; bx < Cfg::kOBoxes; ++bx)
+          if (dbg_tma(ab, bx * 64, r0, h, b, D, p.N, p.H, p.B, 2, stage + bx * 16384, 16384, smem_base, smem_end))
+            tma_store_4d(&tmO, stage + bx * 16384, bx * 64, r0, h, b);
         bulk_commit_group();
         if constexpr (!Cfg::kSepO) {  // the Q_t buffer is free again once the store has read it
           bulk_wait_group_read0();
@@ -774,7 +792,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (i < p.N) {
         const float lse = l_run > 0.0f ? (m_run + lg2_approx(l_run)) * kLn2 : -INFINITY;
-        p.lse[((size_t)b * p.H + h) * (size_t)p.N + i] = lse;
+        const long long li = ((long long)b * p.H + h) * (long long)p.N + i;
+        if (dbg_range(ab, li, 1, (long long)p.B * p.H * p.N)) p.lse[li] = lse;
       }
     }
     if (row == 0) bulk_wait_group0();

@@ -108,6 +108,40 @@ struct Abort {
   __device__ __forceinline__ bool raised() const { return *flag != 0; }
 };
 
+// ------------------------------------------------------------------ bounds checks (FA_DEBUG builds)
+//
+// Built with -DFA_DEBUG=1, the kernels check every computed TMA coordinate, bulk-copy range,
+// shared-memory destination and global index before using it. A failed check records
+// kErrBadInput in the device error word, raises the CTA's abort flag (so that its waits return
+// at once and its roles run out their loops) and skips the access; it never traps. In other
+// builds the checks are constant true and compile away. They stand in for a memory checker.
+#ifndef FA_DEBUG
+#define FA_DEBUG 0
+#endif
+
+__device__ __forceinline__ bool dbg_fail(Abort ab) {
+  if (ab.flag) *ab.flag = 1;
+  atomicOr(&g_fa_error, kErrBadInput);
+  return false;
+}
+
+// The box of a tiled TMA copy starts inside the tensor (c0 on a 16-byte boundary of elements of
+// `elem` bytes, 0 <= c_k < e_k) and its `bytes` in shared memory lie in [lo, hi).
+__device__ __forceinline__ bool dbg_tma(Abort ab, int c0, int c1, int c2, int c3, int e0, int e1, int e2, int e3,
+                                        int elem, uint32_t dst, uint32_t bytes, uint32_t lo, uint32_t hi) {
+  if (!FA_DEBUG) return true;
+  const bool ok = c0 >= 0 && c0 < e0 && (c0 * elem) % 16 == 0 && c1 >= 0 && c1 < e1 && c2 >= 0 && c2 < e2 &&
+                  c3 >= 0 && c3 < e3 && dst >= lo && dst + bytes <= hi && (dst & 15u) == 0;
+  return ok || dbg_fail(ab);
+}
+
+// A plain index or element range [first, first + count) inside [0, size).
+__device__ __forceinline__ bool dbg_range(Abort ab, long long first, long long count, long long size) {
+  if (!FA_DEBUG) return true;
+  const bool ok = first >= 0 && count >= 0 && first + count <= size;
+  return ok || dbg_fail(ab);
+}
+
 // Wait until the phase with the given parity has completed. Returns false on timeout
 // or when another role of the CTA has already given up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Abort ab) {

@@ -46,6 +46,14 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(declared_functions()) == set(binding.EXPORTS)
 
 
+def test_debug_library_exports_every_declared_symbol():
+    """The bounds-checking build (-DFA_DEBUG=1) offers the same C ABI."""
+    dbg = binding.open_library(build.build(debug=True))
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+    assert dbg.fa_status_string(0).decode() == "FA_OK"
+
+
 def test_status_strings(lib):
     for code, name in binding.STATUS_NAMES.items():
         assert lib.fa_status_string(code).decode().startswith(name)
