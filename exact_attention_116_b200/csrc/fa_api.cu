@@ -377,7 +377,7 @@ struct BwdOptions {
 };
 
 fa::BwdParams bwd_params(const Shape& s, float scale, int causal, int win_l, int win_r, const Workspace& w,
-                         const BwdOptions& opt) {
+                         const BwdOptions& opt, int sm_count_hint) {
   fa::BwdParams p;
   p.alibi_slopes = opt.alibi;
   p.cu_seqlens = opt.cu;
@@ -393,6 +393,16 @@ fa::BwdParams bwd_params(const Shape& s, float scale, int causal, int win_l, int
   p.causal = causal ? 1 : 0;
   p.num_kv_tiles = (s.N + 127) / 128;
   p.num_items = s.B * s.H * p.num_kv_tiles;
+  // Head groups of the main kernel: the Q, dO (bf16) and dQ accumulator (fp32) rows of a group,
+  // 8 N d bytes per head, within 32 MiB; the last KV tiles (the shortest under causal masking,
+  // enough for four items per CTA) dealt over all heads at the end.
+  const double per_head = 8.0 * s.N * s.d;
+  const double g = (32.0 * 1024 * 1024) / per_head;
+  const int bh = s.B * s.H;
+  p.head_group = g < 1.0 ? 1 : (g >= bh ? bh : (int)g);
+  const int sms = sm_count_hint > 0 ? sm_count_hint : 148;
+  const int k = (4 * sms + bh - 1) / bh;
+  p.tail_tiles = k < p.num_kv_tiles ? k : p.num_kv_tiles;
   p.dq_acc = w.dq_acc;
   p.lse2 = w.lse2;
   p.dvec = w.dvec;
@@ -444,7 +454,7 @@ int launch_main(const void* q, const void* k, const void* v, const void* dO, voi
       (st = make_map(&mdo, dO, s)) || (st = make_map(&mdk, dk, s)) || (st = make_map(&mdv, dv, s)) ||
       (st = make_map_f32_acc(&mdq, w.dq_acc, s)))
     return st;
-  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, opt);
+  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, opt, sm_count);
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   if (log_enabled())
     std::fprintf(stderr, "[fa] bwd B=%d N=%d H=%d d=%d causal=%d win=(%d,%d) items=%d grid=%d smem=%d\n", s.B, s.N,
@@ -471,7 +481,7 @@ int launch_dq(const void* q, const void* k, const void* v, const void* dO, void*
   if ((st = make_map(&mq, q, s)) || (st = make_map(&mk, k, s)) || (st = make_map(&mv, v, s)) ||
       (st = make_map(&mdo, dO, s)) || (st = make_map(&mdq, dq, s)))
     return st;
-  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, opt);
+  const fa::BwdParams p = bwd_params(s, scale, causal, win_l, win_r, w, opt, sm_count);
   const int grid = p.num_items < sm_count ? p.num_items : sm_count;
   if (s.d == 64)
     dq_kernel<64>(opt.alibi != nullptr, opt.cu != nullptr, grid, stream, mq, mk, mv, mdo, mdq, p);

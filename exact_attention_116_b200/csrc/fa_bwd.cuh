@@ -14,7 +14,7 @@
 //   fa_dq_convert_kernel  dQ = bf16(accumulator)
 //
 // fa_bwd_kernel roles (512 threads):
-//   warp 0       work fetch (atomic counter, head-grouped order) and TMA producer: K_j, V_j
+//   warp 0       work fetch (atomic counter, head-grouped order: bwd_decode) and TMA producer: K_j, V_j
 //                per item; Q_i with LSE2_i, D_i in two slots; dO_i in one slot
 //   warp 1       MMA issuer, TMEM owner
 //   warps 4-7    dQ: TMEM -> registers -> shared staging -> TMA reduce-add into the accumulator
@@ -50,11 +50,9 @@ struct BwdParams {
   const float* alibi_slopes;  // ALiBi only: (B, H) slopes m, bias -m |i - j| on the scaled scores
   const int* cu_seqlens;      // packed variable-length batch (B = 1, N = total): nseg + 1 offsets, or null
   int nseg;
+  int head_group;             // heads per scheduling group of the main kernel (>= 1)
+  int tail_tiles;             // the last (shortest under causal masking) KV tiles, dealt over all heads
 };
-
-// Heads per scheduling group: items of a group are handed out before the next group's, so the
-// Q, dO and dQ-accumulator rows of the few heads in flight stay in L2.
-constexpr int kBwdHeadGroup = 4;
 
 // Share of the exponentials computed by exp2_poly on the FMA pipes (pair p of a thread's 32
 // pairs uses the polynomial when p % kPolyDen < kPolyNum).
@@ -179,15 +177,31 @@ struct BwdBars {
 // Consumers of a fetched item: the MMA thread, 4 dQ warps and 8 P/dS warps (one arrival each).
 constexpr uint32_t kBwdItemConsumers = 13;
 
-// Item w -> (b, h, j): groups of kBwdHeadGroup heads in order; inside a group, KV tiles in
-// ascending order (under causal masking the low tiles visit the most Q tiles) across its heads.
+// Item w -> (b, h, j), in two phases:
+//   1. KV tiles [0, num_kv_tiles - tail_tiles): groups of head_group heads in order, inside a
+//      group the KV tile ascending (under causal masking the low tiles visit the most Q tiles)
+//      and the heads fastest, so that the Q, dO and dQ-accumulator rows of the heads in flight
+//      stay in L2;
+//   2. the last tail_tiles KV tiles of every head, tile-major: the items dealt last are the
+//      shortest, whatever group ran last, so the CTAs finish together.
 __device__ __forceinline__ void bwd_decode(const BwdParams& p, int w, int& b, int& h, int& j) {
-  const int per_group = kBwdHeadGroup * p.num_kv_tiles;
-  const int g = w / per_group;
-  const int pos = w - g * per_group;
-  const int gs = min(kBwdHeadGroup, p.B * p.H - g * kBwdHeadGroup);
-  j = pos / gs;
-  const int bh = g * kBwdHeadGroup + (pos - j * gs);
+  const int bh_count = p.B * p.H;
+  const int tiles1 = p.num_kv_tiles - p.tail_tiles;
+  const int n1 = bh_count * tiles1;
+  int bh;
+  if (w < n1) {
+    const int per_group = p.head_group * tiles1;
+    const int g = w / per_group;
+    const int pos = w - g * per_group;
+    const int gs = min(p.head_group, bh_count - g * p.head_group);
+    j = pos / gs;
+    bh = g * p.head_group + (pos - j * gs);
+  } else {
+    const int w2 = w - n1;
+    const int j2 = w2 / bh_count;
+    j = tiles1 + j2;
+    bh = w2 - j2 * bh_count;
+  }
   b = bh / p.H;
   h = bh - b * p.H;
 }

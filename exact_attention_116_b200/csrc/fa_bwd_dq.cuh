@@ -53,6 +53,9 @@ struct BwdDqBars {
 // Consumers of a fetched item: the MMA thread and the 4 compute warps.
 constexpr uint32_t kBwdDqItemConsumers = 5;
 
+// Heads per scheduling group of the dQ kernel: the K/V rows of the few heads in flight stay in L2.
+constexpr int kBwdHeadGroup = 4;
+
 // Item w -> (b, h, i): groups of kBwdHeadGroup heads; inside a group, Q tiles longest first
 // under causal masking (descending i), across the group's heads.
 __device__ __forceinline__ void bwd_dq_decode(const BwdParams& p, int w, int& b, int& h, int& i) {

@@ -416,6 +416,11 @@ __global__ void __launch_bounds__(384, 1)
                           Cfg::kSepO ? smem_base + Cfg::kOffO + Cfg::kOTileBytes : sQ[1]};
   const uint32_t sKV = smem_base + Cfg::kOffKV;
 
+  // Registers: the launch gives every thread 168; the producer / MMA warpgroup (warps 0-3) needs
+  // few and hands some back, and the two softmax warpgroups, which hold a row's 128 scores,
+  // take them: 128 x (96 + 200 + 200) = 63488 <= 384 x 168 = 64512 registers of the launch.
+  if (warp < 4) {  // ---- producer / MMA warpgroup (warps 0-3)
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane_id() == 0) {
@@ -630,7 +635,10 @@ __global__ void __launch_bounds__(384, 1)
       mma_commit(bar(bars->mma_done));
       mbar_drain(bar(bars->mma_done), 0);
     }
-  } else if (warp >= 4) {
+  }
+  } else {  // ---- softmax warpgroups (warps 4-11)
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+  {
     // ---------------------------------------------------------------- softmax + epilogue
     const int t = (warp - 4) >> 2;           // Q tile of the pair handled by this warpgroup
     const int row = threadIdx.x - 128 * (1 + t);  // 0..127: TMEM lane and row within the tile
@@ -797,6 +805,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     if (row == 0) bulk_wait_group0();
+  }
   }
 
   __syncthreads();
