@@ -73,13 +73,21 @@ bool bwd_attributes() {
          variant_attributes<D, false, true>() && variant_attributes<D, true, true>();
 }
 
+// Dynamic shared memory size, and the largest shared-memory carveout (several CTAs of the
+// CUDA-core decode kernel share an SM; the tensor-core kernel takes nearly all of one).
+template <class Kernel>
+bool decode_kernel_attributes(Kernel kernel, int smem_bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) == cudaSuccess &&
+         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared) == cudaSuccess;
+}
+
 template <int D>
 bool decode_attributes() {
-  const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
-  return cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 1>, attr, fa::DecCfg<D, 1>::kSmemBytes) == cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 2>, attr, fa::DecCfg<D, 2>::kSmemBytes) == cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 4>, attr, fa::DecCfg<D, 4>::kSmemBytes) == cudaSuccess &&
-         cudaFuncSetAttribute(fa::fa_decode_split_kernel<D, 8>, attr, fa::DecCfg<D, 8>::kSmemBytes) == cudaSuccess;
+  return decode_kernel_attributes(fa::fa_decode_split_kernel<D, 1>, fa::DecCfg<D, 1>::kSmemBytes) &&
+         decode_kernel_attributes(fa::fa_decode_split_kernel<D, 2>, fa::DecCfg<D, 2>::kSmemBytes) &&
+         decode_kernel_attributes(fa::fa_decode_split_kernel<D, 4>, fa::DecCfg<D, 4>::kSmemBytes) &&
+         decode_kernel_attributes(fa::fa_decode_mma_kernel<D>, fa::DecTcCfg<D>::kSmemBytes);
 }
 
 int device_setup(int* dev_out, int* sm_count) {
@@ -643,35 +651,46 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_desca
 
 namespace {
 
-// The split kernel compiled for Sq rounded up to 1, 2, 4 or 8, launched as the programmatic
-// dependent of the kernel before it on the stream (the prep kernel, when there are splits).
-template <int D, int kSq>
-int launch_decode_sq(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
-                     cudaStream_t cs) {
+// Decode kernel launched as the programmatic dependent of the kernel before it on the stream
+// (the prep kernel, when there are splits).
+template <class Kernel>
+int launch_decode_kernel(Kernel kernel, int threads, int smem_bytes, dim3 grid, const CUtensorMap& mk,
+                         const CUtensorMap& mv, const fa::DecParams& p, cudaStream_t cs) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(fa::kDecThreads);
-  cfg.dynamicSmemBytes = fa::DecCfg<D, kSq>::kSmemBytes;
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = cs;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, fa::fa_decode_split_kernel<D, kSq>, mk, mv, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kernel, mk, mv, p) != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_CUDA;
   }
   return launch_status();
 }
 
+// Up to 3 new rows: the CUDA-core kernel compiled for Sq rounded up to 1, 2 or 4; from 4 rows
+// on: the tensor-core kernel.
+constexpr int kDecMmaMinSq = 4;
+
 template <int D>
 int launch_decode(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
                   cudaStream_t cs) {
-  if (p.Sq == 1) return launch_decode_sq<D, 1>(grid, mk, mv, p, cs);
-  if (p.Sq == 2) return launch_decode_sq<D, 2>(grid, mk, mv, p, cs);
-  if (p.Sq <= 4) return launch_decode_sq<D, 4>(grid, mk, mv, p, cs);
-  return launch_decode_sq<D, 8>(grid, mk, mv, p, cs);
+  constexpr int kT = fa::kDecThreads, kTm = fa::kDecMmaThreads;
+  if (p.Sq == 1)
+    return launch_decode_kernel(fa::fa_decode_split_kernel<D, 1>, kT, fa::DecCfg<D, 1>::kSmemBytes, grid, mk, mv, p,
+                                cs);
+  if (p.Sq == 2)
+    return launch_decode_kernel(fa::fa_decode_split_kernel<D, 2>, kT, fa::DecCfg<D, 2>::kSmemBytes, grid, mk, mv, p,
+                                cs);
+  if (p.Sq < kDecMmaMinSq)
+    return launch_decode_kernel(fa::fa_decode_split_kernel<D, 4>, kT, fa::DecCfg<D, 4>::kSmemBytes, grid, mk, mv, p,
+                                cs);
+  return launch_decode_kernel(fa::fa_decode_mma_kernel<D>, kTm, fa::DecTcCfg<D>::kSmemBytes, grid, mk, mv, p, cs);
 }
 
 // Workspace of a call with P > 1 pieces per head: partial O (fp32) and partial LSE for the
@@ -682,7 +701,7 @@ size_t decode_workspace_bytes(int B, int Sq, int H, int d, int pieces) {
   return align256(rows * d * 4) + align256(rows * 4) + align256((size_t)B * H * 4);
 }
 
-// CTAs of the split kernel for (d, Sq) that fit on one SM at a time (0 on error).
+// CTAs of the decode kernel for (d, Sq) that fit on one SM at a time (0 on error).
 template <int D>
 int decode_ctas_per_sm(int Sq) {
   int n = 0;
@@ -693,12 +712,12 @@ int decode_ctas_per_sm(int Sq) {
   else if (Sq == 2)
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 2>, fa::kDecThreads,
                                                       fa::DecCfg<D, 2>::kSmemBytes);
-  else if (Sq <= 4)
+  else if (Sq < kDecMmaMinSq)
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 4>, fa::kDecThreads,
                                                       fa::DecCfg<D, 4>::kSmemBytes);
   else
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 8>, fa::kDecThreads,
-                                                      fa::DecCfg<D, 8>::kSmemBytes);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_mma_kernel<D>, fa::kDecMmaThreads,
+                                                      fa::DecTcCfg<D>::kSmemBytes);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return 0;

@@ -47,6 +47,7 @@ namespace fa {
 constexpr int kDecMaxSq = 8;  // new query rows per call
 constexpr int kDecTile = 64;  // keys per tile
 constexpr int kDecThreads = 128;
+constexpr int kDecMmaThreads = 192;  // tensor-core kernel: four softmax warps, a producer and an MMA warp
 constexpr float kDecLn2 = 0.69314718055994530942f;
 
 // Generic-proxy writes to global memory by this thread are ordered before later async-proxy
@@ -208,43 +209,26 @@ __device__ __forceinline__ void dec_issue_tile(const DecParams& p, const CUtenso
   if (++ld.t == ld.t1) ld.next_seg(p, u0, u1);
 }
 
-template <int D, int kSq>
-__global__ void __launch_bounds__(kDecThreads)
-    fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                           const DecParams p) {
-  using Cfg = DecCfg<D, kSq>;
-  constexpr int kStages = Cfg::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  uint8_t* sm = smem_raw + (smem_base - smem_u32(smem_raw));
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Cfg::kOffBar);
-  int* abort_flag = reinterpret_cast<int*>(sm + Cfg::kOffBar + 64);
-  float* sQ = reinterpret_cast<float*>(sm + Cfg::kOffQ);
-  float* sS = reinterpret_cast<float*>(sm + Cfg::kOffS);
-  float* sP = reinterpret_cast<float*>(sm + Cfg::kOffP);
-  float* sAlpha = reinterpret_cast<float*>(sm + Cfg::kOffAlpha);
-  float* sRed = reinterpret_cast<float*>(sm + Cfg::kOffRed);
-  long long* sSum = reinterpret_cast<long long*>(sm + Cfg::kOffMisc);  // [0, 4) warp sums, [4] first start
-  int* sInt = reinterpret_cast<int*>(sm + Cfg::kOffMisc + 48);          // [0] first sequence, [1] last flag
-  const Abort ab{abort_flag};
-  const uint32_t smem_end = smem_u32(smem_raw) + Cfg::kSmemBytes;  // for the FA_DEBUG bounds checks
-  // FA_DEBUG: index ranges of the outputs, the partial slots and the cache rows
-  const long long o_size = (long long)p.B * p.Sq * p.H * D, lse_size = (long long)p.B * p.H * p.Sq;
-  const long long part_rows = ((long long)p.B + p.pieces - 1) * p.H * p.Sq;
-  const long long cache_size = (long long)p.num_pages * p.page_size * p.H * D;
+// A CTA's piece of a head's tile list: the list's length T, the pieces in use Pe, this piece's
+// units [u0, u1) and its first segment (sequence b_first, whose tiles start at unit start_first).
+struct DecPiece {
+  long long T, u0, u1, start_first;
+  int Pe, b_first;
+};
+
+// Set-up shared by the decode kernels (all threads of the CTA; threads 0 .. kDecThreads - 1 do the
+// work, any others only meet the barriers): the piece from the lengths (a
+// block-wide prefix sum of tile counts, each thread summing a contiguous run of sequences); O = 0,
+// LSE = -inf for the sequences without a visible tile (written by piece b % P); with new K/V rows
+// given, this piece's new rows of head h written into the cache before any tile load. sSum holds
+// 5 and sInt 1 values of scratch in shared memory.
+template <int D>
+__device__ __forceinline__ DecPiece dec_prologue(const DecParams& p, int h, int piece, Abort ab, long long* sSum,
+                                                 int* sInt) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  static_assert(kSq >= 1 && kSq <= kDecMaxSq, "rows per CTA");
-  static_assert(kDecThreads == 128, "the scan below assumes four warps");
-  const int h = blockIdx.x, piece = blockIdx.y, P = p.pieces;
-  const int Sq = p.Sq;
-
-  if (tid == 0) {
-    *abort_flag = 0;
-    sInt[0] = p.B;
-    for (int st = 0; st < kStages; ++st) mbar_init(smem_u32(&full[st]), 1);
-    fence_barrier_init();
-  }
-
+  const int Sq = p.Sq, P = p.pieces;
+  const long long o_size = (long long)p.B * p.Sq * p.H * D, lse_size = (long long)p.B * p.H * p.Sq;
+  const long long cache_size = (long long)p.num_pages * p.page_size * p.H * D;
   // ---- tile counts of all sequences, prefix sums (each thread a contiguous run of sequences)
   const int run = (p.B + kDecThreads - 1) / kDecThreads;
   const int rb0 = min(p.B, tid * run), rb1 = min(p.B, rb0 + run);
@@ -260,7 +244,7 @@ __global__ void __launch_bounds__(kDecThreads)
     const long long v = __shfl_up_sync(0xffffffffu, incl, off);
     if (lane >= off) incl += v;
   }
-  if (lane == 31) sSum[warp] = incl;
+  if (lane == 31 && warp < 4) sSum[warp] = incl;  // (threads past the first 128 hold no sequences)
   __syncthreads();
   long long T = 0, excl = incl - mine;
 #pragma unroll
@@ -292,7 +276,7 @@ __global__ void __launch_bounds__(kDecThreads)
   const long long start_first = b_first < p.B ? sSum[4] : 0;
 
   // ---- sequences without a visible tile (empty): O = 0, LSE = -inf, written by piece b % P
-  for (int b = piece; b < p.B; b += P) {
+  for (int b = piece; b < p.B && tid < kDecThreads; b += P) {
     int vt0;
     if (dec_vis_tiles(p, dec_len(p, b, false), vt0) != 0) continue;
     for (int e = tid; e < Sq * D; e += kDecThreads) {
@@ -331,6 +315,107 @@ __global__ void __launch_bounds__(kDecThreads)
     if (wrote) fence_proxy_async_global();  // ordered before the TMA loads by the barrier below
   }
   __syncthreads();
+
+  DecPiece pc;
+  pc.T = T;
+  pc.Pe = Pe;
+  pc.u0 = u0;
+  pc.u1 = u1;
+  pc.b_first = b_first;
+  pc.start_first = start_first;
+  return pc;
+}
+
+// Segment end of a sequence spread over pieces pf..pl (threads 0 .. kDecThreads - 1, which meet on
+// named barrier 1, after this piece's partial is written): count this piece on the (b, h) arrival
+// counter; the piece that arrives last merges the partials by their log-sum-exp, in piece order.
+// sInt holds one flag.
+template <int D>
+__device__ __forceinline__ void dec_arrive_merge(const DecParams& p, int b, int h, int pf, int pl, Abort ab,
+                                                 int* sInt) {
+  const int tid = threadIdx.x, Sq = p.Sq;
+  const long long o_size = (long long)p.B * p.Sq * p.H * D, lse_size = (long long)p.B * p.H * p.Sq;
+  const long long part_rows = ((long long)p.B + p.pieces - 1) * p.H * p.Sq;
+  {
+    // arrival: the last piece of (b, h) merges all partials
+    __threadfence();  // this thread's partials are visible device-wide before the arrival
+    named_bar_sync(1, kDecThreads);
+    if (tid == 0) {
+      griddep_wait();  // the prep kernel has zeroed the counters
+      const long long ai = (long long)b * p.H + h;
+      const int before = dbg_range(ab, ai, 1, (long long)p.B * p.H) ? atomicAdd(&p.arrivals[ai], 1) : -1;
+      sInt[1] = before == pl - pf;
+    }
+    named_bar_sync(1, kDecThreads);
+    if (sInt[1]) {
+      __threadfence();
+      // O = sum_r 2^(L_r - L) O_r, L = log2 sum_r 2^L_r, in piece order (the same sum whichever
+      // piece arrives last)
+      for (int e = tid; e < Sq * D; e += kDecThreads) {
+        const int i = e / D, col = e - i * D;
+        float mx = -INFINITY;
+        if (!dbg_range(ab, (((long long)b + pf) * p.H + h) * Sq + i, 1, part_rows) ||
+            !dbg_range(ab, (((long long)b + pl) * p.H + h) * Sq + i, 1, part_rows))
+          continue;
+        for (int r = pf; r <= pl; ++r)
+          mx = fmaxf(mx, __ldcg(p.lse_part + (((size_t)b + r) * p.H + h) * Sq + i));
+        float wsum = 0.0f, v = 0.0f;
+        if (mx != -INFINITY) {
+          for (int r = pf; r <= pl; ++r) {
+            const size_t row = (((size_t)b + r) * p.H + h) * Sq + i;
+            const float wr = ex2_approx(__ldcg(p.lse_part + row) - mx);
+            wsum += wr;
+            v = fmaf(wr, __ldcg(p.o_part + row * D + col), v);
+          }
+        }
+        const long long oi = (((long long)b * Sq + i) * p.H + h) * D + col, li = ((long long)b * p.H + h) * Sq + i;
+        if (dbg_range(ab, oi, 1, o_size)) p.o[oi] = __float2bfloat16_rn(wsum > 0.0f ? v / wsum : 0.0f);
+        if (col == 0 && dbg_range(ab, li, 1, lse_size))
+          p.lse[li] = mx == -INFINITY ? -INFINITY : (mx + __log2f(wsum)) * kDecLn2;
+      }
+    }
+    }
+}
+
+template <int D, int kSq>
+__global__ void __launch_bounds__(kDecThreads)
+    fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                           const DecParams p) {
+  using Cfg = DecCfg<D, kSq>;
+  constexpr int kStages = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sm = smem_raw + (smem_base - smem_u32(smem_raw));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Cfg::kOffBar);
+  int* abort_flag = reinterpret_cast<int*>(sm + Cfg::kOffBar + 64);
+  float* sQ = reinterpret_cast<float*>(sm + Cfg::kOffQ);
+  float* sS = reinterpret_cast<float*>(sm + Cfg::kOffS);
+  float* sP = reinterpret_cast<float*>(sm + Cfg::kOffP);
+  float* sAlpha = reinterpret_cast<float*>(sm + Cfg::kOffAlpha);
+  float* sRed = reinterpret_cast<float*>(sm + Cfg::kOffRed);
+  long long* sSum = reinterpret_cast<long long*>(sm + Cfg::kOffMisc);  // [0, 4) warp sums, [4] first start
+  int* sInt = reinterpret_cast<int*>(sm + Cfg::kOffMisc + 48);          // [0] first sequence, [1] last flag
+  const Abort ab{abort_flag};
+  const uint32_t smem_end = smem_u32(smem_raw) + Cfg::kSmemBytes;  // for the FA_DEBUG bounds checks
+  // FA_DEBUG: index ranges of the outputs and the partial slots
+  const long long o_size = (long long)p.B * p.Sq * p.H * D, lse_size = (long long)p.B * p.H * p.Sq;
+  const long long part_rows = ((long long)p.B + p.pieces - 1) * p.H * p.Sq;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  static_assert(kSq >= 1 && kSq <= kDecMaxSq, "rows per CTA");
+  static_assert(kDecThreads == 128, "the scan below assumes four warps");
+  const int h = blockIdx.x, piece = blockIdx.y;
+  const int Sq = p.Sq;
+
+  if (tid == 0) {
+    *abort_flag = 0;
+    sInt[0] = p.B;
+    for (int st = 0; st < kStages; ++st) mbar_init(smem_u32(&full[st]), 1);
+    fence_barrier_init();
+  }
+
+  const DecPiece pc = dec_prologue<D>(p, h, piece, ab, sSum, sInt);
+  const long long T = pc.T, u0 = pc.u0, u1 = pc.u1, start_first = pc.start_first;
+  const int Pe = pc.Pe, b_first = pc.b_first;
 
   // ---- the piece's tiles, streamed through the ring in list order (stream index k)
   const long long n_tiles = u1 - u0;
@@ -451,8 +536,10 @@ __global__ void __launch_bounds__(kDecThreads)
           const float a = sAlpha[i];
           acc[i] = mul2(acc[i], make_float2(a, a));
         }
+        // keys past the sequence's end are skipped, not weighted by 0: the cache may hold a NaN there
+        const int kv_end = min(kDecTile, n - t * kDecTile);
 #pragma unroll 4
-        for (int kt = kg; kt < kDecTile; kt += Cfg::kKeyGroups) {
+        for (int kt = kg; kt < kv_end; kt += Cfg::kKeyGroups) {
           const uint32_t wv = *reinterpret_cast<const uint32_t*>(vgen + bx * (kDecTile * 128) +
                                                                  sw128_offset(kt, chunk) + within);
           const float2 v = make_float2(bf16lo_to_f32(wv), bf16hi_to_f32(wv));
@@ -506,45 +593,7 @@ __global__ void __launch_bounds__(kDecThreads)
         p.lse_part[pi] = l2;
       }
     }
-    if (pf != pl) {
-      // arrival: the last piece of (b, h) merges all partials
-      __threadfence();  // this thread's partials are visible device-wide before the arrival
-      __syncthreads();
-      if (tid == 0) {
-        griddep_wait();  // the prep kernel has zeroed the counters
-        const long long ai = (long long)b * p.H + h;
-        const int before = dbg_range(ab, ai, 1, (long long)p.B * p.H) ? atomicAdd(&p.arrivals[ai], 1) : -1;
-        sInt[1] = before == pl - pf;
-      }
-      __syncthreads();
-      if (sInt[1]) {
-        __threadfence();
-        // O = sum_r 2^(L_r - L) O_r, L = log2 sum_r 2^L_r, in piece order (the same sum whichever
-        // piece arrives last)
-        for (int e = tid; e < Sq * D; e += kDecThreads) {
-          const int i = e / D, col = e - i * D;
-          float mx = -INFINITY;
-          if (!dbg_range(ab, (((long long)b + pf) * p.H + h) * Sq + i, 1, part_rows) ||
-              !dbg_range(ab, (((long long)b + pl) * p.H + h) * Sq + i, 1, part_rows))
-            continue;
-          for (int r = pf; r <= pl; ++r)
-            mx = fmaxf(mx, __ldcg(p.lse_part + (((size_t)b + r) * p.H + h) * Sq + i));
-          float wsum = 0.0f, v = 0.0f;
-          if (mx != -INFINITY) {
-            for (int r = pf; r <= pl; ++r) {
-              const size_t row = (((size_t)b + r) * p.H + h) * Sq + i;
-              const float wr = ex2_approx(__ldcg(p.lse_part + row) - mx);
-              wsum += wr;
-              v = fmaf(wr, __ldcg(p.o_part + row * D + col), v);
-            }
-          }
-          const long long oi = (((long long)b * Sq + i) * p.H + h) * D + col, li = ((long long)b * p.H + h) * Sq + i;
-          if (dbg_range(ab, oi, 1, o_size)) p.o[oi] = __float2bfloat16_rn(wsum > 0.0f ? v / wsum : 0.0f);
-          if (col == 0 && dbg_range(ab, li, 1, lse_size))
-            p.lse[li] = mx == -INFINITY ? -INFINITY : (mx + __log2f(wsum)) * kDecLn2;
-        }
-      }
-    }
+    if (pf != pl) dec_arrive_merge<D>(p, b, h, pf, pl, ab, sInt);
     __syncthreads();  // the next segment rewrites sQ, sAlpha and the last flag
   }
 
@@ -552,6 +601,446 @@ __global__ void __launch_bounds__(kDecThreads)
   if (tid == 0 && ab.raised()) {
     for (long long j = max(0LL, issued - kStages); j < issued; ++j)
       mbar_drain(smem_u32(&full[j % kStages]), (uint32_t)((j / kStages) & 1));
+  }
+}
+
+// ------------------------------------------------------------------ tensor-core variant (4 to 8 rows)
+//
+// With four or more new rows per sequence the CUDA-core dot products of the kernel above bound
+// it, not the cache read. This variant computes both products on the tensor core, transposed so
+// that the keys, not the few new rows, fill the 128 rows of a tcgen05 tile. Per tile of 128 keys
+// (two 64-key units of one sequence, each from its own page):
+//   S^T = K Q^T    M = 128 keys, N = 16 (the Sq <= 8 new rows, zero-padded), K = d
+//   O^T += V^T P^T M = d, N = 16, K = 128 keys          (d = 128)
+//                  M = 128, N = 32, K = 64 keys         (d = 64: the two 64-key halves stacked in
+//                  M, each half's weights in its own 16 columns of N; the two diagonal blocks are
+//                  added up once per segment, the off-diagonal ones are never read)
+// Thread i of the four softmax warps owns key i of the tile (TMEM lane i of S^T): its scores for
+// every new row come in one TMEM load; the row maxima over the tile are exchanged between the
+// warps through shared memory; P^T goes to shared memory as bf16, the B operand of the second
+// product; O^T stays in TMEM (lane = column of O) across the tiles of a segment. Warp 4 loads the
+// tiles (a ring of 3 stages at d = 128, 6 at d = 64: one CTA per SM), warp 5 issues the products,
+// S(k + 1) ahead of P V(k). O is rescaled only when a row's maximum has grown by more than 2^8.
+// P is rounded to bf16 for the product, so O is divided by the sum of the rounded weights and
+// the log-sum-exp taken from the fp32 sum, as in the training forward. Work split, appends and
+// merge are those of the kernel above (pieces are counted in 64-key units).
+constexpr float kDecRescale = 8.0f;  // log2 units
+constexpr int kDecTcRows = 8;        // new rows a thread handles (Sq <= 8), padded to N = 16
+
+template <int D>
+struct DecTcCfg {
+  static constexpr int kTileKeys = 128;
+  static constexpr int kBoxes = D / 64;                      // 64-column (128-byte) boxes per row
+  static constexpr int kBoxBytes = kTileKeys * 128;          // one box of a 128-key tile (16 KB)
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;      // one K or V tile
+  static constexpr int kStageBytes = 2 * kTileBytes;         // K, then V
+  static constexpr int kStages = D == 64 ? 6 : 3;
+  static constexpr int kOffKV = 0;
+  static constexpr int kOffQ = kStages * kStageBytes;        // Q^T operand: 16 rows x d, K-major boxes of 2 KB
+  static constexpr int kQBytes = 16 * D * 2;
+  static constexpr int kNO = D == 64 ? 32 : 16;              // N of the second product
+  static constexpr int kPBytes = 4096;                       // P^T operand: kNO rows x (2 x 64 or 64) keys
+  static constexpr int kOffP = kOffQ + kQBytes;              // two P^T buffers, by tile parity
+  static constexpr int kOffRed = kOffP + 2 * kPBytes;        // [2][4][8] row maxima of the warps, then [4][16] sums
+  static constexpr int kOffEpi = kOffRed + 512;              // d = 64: [64][8] second-half columns of O
+  static constexpr int kOffMisc = kOffEpi + (D == 64 ? 64 * 8 * 4 : 0);  // scan sums, first segment, flags
+  static constexpr int kOffBar = kOffMisc + 128;             // full, empty [kStages]; s_bar[2], o_bar, p_full, q_full, done
+  static constexpr int kBarBytes = 256;                      // TMEM slot and abort flag in the last 64 bytes
+  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
+  static constexpr uint32_t kColS = 0;                       // S^T buffers at columns 0 and 16
+  static constexpr uint32_t kColO = 32;                      // O^T (kNO columns)
+  static constexpr uint32_t kTmemCols = 64;
+  static_assert((2 * kStages + 6) * 8 <= kBarBytes - 64, "barrier area");
+  static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands sit on 1024-byte boundaries");
+};
+
+// A walk over the 128-key tiles of one piece: the units [t0, t1) of each segment, paired from t0
+// (the last tile of a segment with an odd unit count has one unit).
+struct DecTcWalk {
+  DecWalk w;
+  int ta;  // first unit of the current tile
+  __device__ __forceinline__ void begin(const DecParams& p, int b0, long long s0, long long u0, long long u1) {
+    w.begin(p, b0, s0, u0, u1);
+    ta = w.t0;
+  }
+  __device__ __forceinline__ bool valid(const DecParams& p) const { return w.valid(p); }
+  __device__ __forceinline__ int units() const { return min(2, w.t1 - ta); }
+  // next tile; true when it starts a new segment (false at the end too: then valid() is false)
+  __device__ __forceinline__ bool next(const DecParams& p, long long u0, long long u1) {
+    ta += 2;
+    if (ta < w.t1) return false;
+    const bool more = w.next_seg(p, u0, u1);
+    ta = w.t0;
+    return more;
+  }
+};
+
+// The producer's loads of one tile into its ring slot: one TMA box per 64-column box and unit,
+// for K and for V; a missing second unit is left as it is (its keys are masked, its V rows
+// zeroed by the softmax warps).
+template <int D>
+__device__ __forceinline__ bool dec_tc_issue(const DecParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                             uint32_t dst, uint64_t* full_bar, int h, const DecTcWalk& tw, Abort ab,
+                                             uint32_t smem_lo, uint32_t smem_end) {
+  using Cfg = DecTcCfg<D>;
+  const int nu = tw.units();
+  int page[2] = {0, 0}, row[2] = {0, 0};
+  for (int u = 0; u < nu; ++u) {
+    const int key = (tw.ta + u) * kDecTile;
+    const long long ti = (long long)tw.w.b * p.max_pages + key / p.page_size;
+    if (!dbg_range(ab, ti, 1, (long long)p.B * p.max_pages)) return false;
+    int pg = p.block_table[ti];
+    if (pg < 0 || pg >= p.num_pages) {  // the TMA would read zeros there; report it
+      atomicOr(&g_fa_error, kErrBadInput);
+      pg = 0;
+    }
+    page[u] = pg;
+    row[u] = key % p.page_size;
+    for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+      if (!dbg_tma(ab, bx * 64, h, row[u], pg, Cfg::kBoxes * 64, p.H, p.page_size, p.num_pages, 2,
+                   dst + bx * Cfg::kBoxBytes + u * 8192, Cfg::kStageBytes - bx * Cfg::kBoxBytes - u * 8192, smem_lo,
+                   smem_end))
+        return false;
+  }
+  mbar_arrive_expect_tx(smem_u32(full_bar), (uint32_t)(nu * 2 * Cfg::kBoxes * 8192));
+  for (int u = 0; u < nu; ++u)
+#pragma unroll
+    for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+      const uint32_t off = bx * Cfg::kBoxBytes + u * 8192;
+      tma_load_4d(dst + off, tmK, smem_u32(full_bar), bx * 64, h, row[u], page[u]);
+      tma_load_4d(dst + Cfg::kTileBytes + off, tmV, smem_u32(full_bar), bx * 64, h, row[u], page[u]);
+    }
+  return true;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecMmaThreads, 1)
+    fa_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                         const DecParams p) {
+  using Cfg = DecTcCfg<D>;
+  constexpr int kStages = Cfg::kStages;
+  static_assert(kDecThreads == 128 && kDecMmaThreads == kDecThreads + 64, "four softmax warps, producer, MMA");
+  static_assert(kDecMaxSq <= kDecTcRows, "rows per thread");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t* sm = smem_raw + (smem_base - smem_u32(smem_raw));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Cfg::kOffBar);
+  uint64_t* empty = full + kStages;       // slot free again (P V of its tile completed)
+  uint64_t* s_bar = full + 2 * kStages;   // [2] S(k) done, by k & 1
+  uint64_t* o_bar = s_bar + 2;            // P V(k) done
+  uint64_t* p_full = s_bar + 3;           // P^T(k) written, O rescaled (one arrival per softmax warp)
+  uint64_t* q_full = s_bar + 4;           // Q^T of a segment written (one arrival per softmax warp)
+  uint64_t* done_bar = s_bar + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::kOffBar + Cfg::kBarBytes - 64);
+  int* abort_flag = reinterpret_cast<int*>(sm + Cfg::kOffBar + Cfg::kBarBytes - 60);
+  float* sRed = reinterpret_cast<float*>(sm + Cfg::kOffRed);
+  float* sEpi = reinterpret_cast<float*>(sm + Cfg::kOffEpi);
+  long long* sSum = reinterpret_cast<long long*>(sm + Cfg::kOffMisc);  // [0, 4) warp sums, [4] first start
+  int* sInt = reinterpret_cast<int*>(sm + Cfg::kOffMisc + 48);          // [0] first sequence, [1] last flag
+  const Abort ab{abort_flag};
+  const uint32_t smem_end = smem_u32(smem_raw) + Cfg::kSmemBytes;  // for the FA_DEBUG bounds checks
+  const long long o_size = (long long)p.B * p.Sq * p.H * D, lse_size = (long long)p.B * p.H * p.Sq;
+  const long long part_rows = ((long long)p.B + p.pieces - 1) * p.H * p.Sq;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x, piece = blockIdx.y;
+  const int Sq = p.Sq;
+  const uint32_t sQ = smem_base + Cfg::kOffQ;
+
+  if (tid == 0) {
+    *abort_flag = 0;
+    sInt[0] = p.B;
+    for (int i = 0; i < 2 * kStages; ++i) mbar_init(smem_u32(&full[i]), 1);
+    mbar_init(smem_u32(&s_bar[0]), 1);
+    mbar_init(smem_u32(&s_bar[1]), 1);
+    mbar_init(smem_u32(o_bar), 1);
+    mbar_init(smem_u32(p_full), 4);
+    mbar_init(smem_u32(q_full), 4);
+    mbar_init(smem_u32(done_bar), 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before_sync();
+  }
+  // P^T rows of no new row stay zero: both buffers cleared once
+  for (int e = tid; e < 2 * Cfg::kPBytes / 16; e += kDecMmaThreads)
+    st_shared_v4(smem_base + Cfg::kOffP + e * 16, 0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  const DecPiece pc = dec_prologue<D>(p, h, piece, ab, sSum, sInt);  // (its barriers publish the TMEM base)
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const long long T = pc.T, u0 = pc.u0, u1 = pc.u1, start_first = pc.start_first;
+  const int Pe = pc.Pe, b_first = pc.b_first;
+  auto kv_smem = [&](long long j) { return smem_base + Cfg::kOffKV + (uint32_t)(j % kStages) * Cfg::kStageBytes; };
+
+  if (warp == 4) {
+    // ---- producer: the piece's tiles in order (index j), each into its ring slot once the
+    // P V of the tile before it in that slot has completed
+    if (lane == 0 && u0 < u1) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      DecTcWalk tw;
+      tw.begin(p, b_first, start_first, u0, u1);
+      long long j = 0;
+      for (bool more = tw.valid(p); more && !ab.raised(); ++j) {
+        if (j >= kStages) mbar_wait(smem_u32(&empty[j % kStages]), (uint32_t)(((j / kStages) - 1) & 1), ab);
+        if (ab.raised() ||
+            !dec_tc_issue<D>(p, &tmK, &tmV, kv_smem(j), &full[j % kStages], h, tw, ab, smem_base, smem_end))
+          break;
+        tw.next(p, u0, u1);
+        more = tw.valid(p);
+      }
+      if (ab.raised())  // loads issued past a wait that gave up land before the CTA exits
+        for (long long i = max(0LL, j - kStages); i < j; ++i)
+          mbar_drain(smem_u32(&full[i % kStages]), (uint32_t)((i / kStages) & 1));
+    }
+  } else if (warp == 5) {
+    // ---- MMA issuer: S(k + 1) before P V(k), so that the softmax of tile k + 1 can start as
+    // soon as P(k) is handed over
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 16, false, false);      // S^T: A (K) and B (Q) K-major
+      constexpr uint32_t idO = idesc_bf16_f32(128, Cfg::kNO, true, false);  // O^T: A (V^T) MN-major, B (P^T) K-major
+      auto issue_s = [&](long long j) {
+        mbar_wait(smem_u32(&full[j % kStages]), (uint32_t)((j / kStages) & 1), ab);
+        tc_fence_after_sync();
+        const uint32_t kt = kv_smem(j);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)  // 16 columns of d per step, 4 steps per box
+          mma_ss(tmem + Cfg::kColS + (uint32_t)(j & 1) * 16,
+                 sdesc_kmajor(kt + (kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32),
+                 sdesc_kmajor(sQ + (kk >> 2) * 2048 + (kk & 3) * 32), idS, kk > 0);
+        mma_commit(smem_u32(&s_bar[j & 1]));
+      };
+      long long k = 0;
+      uint32_t seg = 0;
+      DecTcWalk tw;
+      tw.begin(p, b_first, start_first, u0, u1);
+      bool more = tw.valid(p), seg_start = true;
+      while (more) {
+        if (seg_start) {
+          mbar_wait(smem_u32(q_full), seg & 1, ab);  // this segment's Q^T
+          ++seg;
+          issue_s(k);
+        }
+        const bool first = seg_start;
+        seg_start = tw.next(p, u0, u1);
+        more = tw.valid(p);
+        if (more && !seg_start) issue_s(k + 1);  // the next tile is in the same segment
+        mbar_wait(smem_u32(p_full), (uint32_t)(k & 1), ab);
+        tc_fence_after_sync();
+        const uint32_t vt = kv_smem(k) + Cfg::kTileBytes;
+        const uint32_t pb = smem_base + Cfg::kOffP + (uint32_t)(k & 1) * Cfg::kPBytes;
+        if constexpr (D == 128) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // 16 keys per step: 16 rows of V, 32 bytes of each P^T row
+            mma_ss(tmem + Cfg::kColO, sdesc_mnmajor(vt + kk * 2048, Cfg::kBoxBytes),
+                   sdesc_kmajor(pb + (kk >> 2) * 2048 + (kk & 3) * 32), idO, !first || kk > 0);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // keys 16 kk.. of each half; the halves 8 KB apart in M
+            mma_ss(tmem + Cfg::kColO, sdesc_mnmajor(vt + kk * 2048, 8192), sdesc_kmajor(pb + kk * 32), idO,
+                   !first || kk > 0);
+        }
+        mma_commit(smem_u32(o_bar));
+        mma_commit(smem_u32(&empty[k % kStages]));
+        ++k;
+      }
+      mma_commit(smem_u32(done_bar));  // every product has completed before the TMEM is freed
+      mbar_drain(smem_u32(done_bar), 0);
+    }
+  } else {
+    // ---- softmax warps 0-3: thread i owns key i of each tile (TMEM lane i of S^T)
+    const uint32_t my_lanes = (uint32_t)(warp * 32) << 16;
+    // O^T lanes: column d of O for d = 128; for d = 64, lanes 64..127 hold the second half's
+    // sums of column d - 64 in O^T columns 16..23
+    const uint32_t tO = tmem + Cfg::kColO + my_lanes + (D == 64 && warp >= 2 ? 16u : 0u);
+    const float c = p.scale_log2;
+    long long k = 0;
+    DecTcWalk tw;
+    tw.begin(p, b_first, start_first, u0, u1);
+    bool more = tw.valid(p);
+    while (more) {
+      const int b = tw.w.b, n = tw.w.n, t_last = tw.w.t1;  // the segment ends at unit t_last
+      const long long seg_start_unit = tw.w.start, seg_cnt = tw.w.cnt;
+      // Q^T: row i holds new row i of (b, h) (zeros for rows past Sq); the previous segment's
+      // products have all completed
+      for (int e = tid; e < 16 * (D / 8); e += kDecThreads) {
+        const int i = e / (D / 8), ch = e - i * (D / 8);
+        const long long qi = (((long long)b * Sq + i) * p.H + h) * D + ch * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (i < Sq && dbg_range(ab, qi, 8, o_size)) v = *reinterpret_cast<const uint4*>(p.q + qi);
+        st_shared_v4(sQ + (ch >> 3) * 2048 + sw128_offset(i, ch & 7), v.x, v.y, v.z, v.w);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(q_full));
+      // per new row: the visible keys [kmin, khi] of this segment
+      int kmin[kDecTcRows], khi[kDecTcRows];
+#pragma unroll
+      for (int i = 0; i < kDecTcRows; ++i) {
+        const int pos = n - Sq + i;
+        kmin[i] = p.win_l >= 0 ? pos - p.win_l : 0;
+        khi[i] = min(min(n - 1, t_last * kDecTile - 1), p.win_r >= 0 ? pos + p.win_r : n - 1);
+        if (i >= Sq) khi[i] = -1;
+      }
+      float m_used[kDecTcRows], l_part[kDecTcRows], lr_part[kDecTcRows];
+#pragma unroll
+      for (int i = 0; i < kDecTcRows; ++i) {
+        m_used[i] = -INFINITY;
+        l_part[i] = 0.0f;
+        lr_part[i] = 0.0f;
+      }
+      bool seg_end = false;
+      for (bool first = true; !seg_end; first = false, ++k) {
+        const int key0 = tw.ta * kDecTile, nu = tw.units();
+        // ---- scores of key key0 + tid for every new row
+        mbar_wait(smem_u32(&s_bar[k & 1]), (uint32_t)((k >> 1) & 1), ab);
+        tc_fence_after_sync();
+        uint32_t sr[8];
+        tmem_ld8(tmem + Cfg::kColS + (uint32_t)(k & 1) * 16 + my_lanes, sr);
+        tmem_wait_ld(sr);
+        const int key = key0 + tid;
+        float x[kDecTcRows];
+#pragma unroll
+        for (int i = 0; i < kDecTcRows; ++i) {
+          x[i] = (key >= kmin[i] && key <= khi[i]) ? __uint_as_float(sr[i]) * c : -INFINITY;
+          const float wm = warp_max_f32(x[i]);
+          if (lane == 0) sRed[((k & 1) * 4 + warp) * 8 + i] = wm;
+        }
+        named_bar_sync(2, kDecThreads);
+        float alpha[kDecTcRows];
+        bool moved = false;
+#pragma unroll
+        for (int i = 0; i < kDecTcRows; ++i) {
+          const float* rm = sRed + (k & 1) * 32 + i;
+          const float m_tile = fmaxf(fmaxf(rm[0], rm[8]), fmaxf(rm[16], rm[24]));
+          alpha[i] = 1.0f;
+          if (m_tile > m_used[i] + kDecRescale || (m_used[i] == -INFINITY && m_tile != -INFINITY)) {
+            alpha[i] = m_used[i] == -INFINITY ? 0.0f : ex2_approx(m_used[i] - m_tile);
+            m_used[i] = m_tile;
+            moved = true;
+          }
+        }
+        // the P^T buffer of this parity and O^T are free: P V of the previous tile has completed
+        // (the segment's first tile: the last segment end waited for all of them)
+        if (!first) mbar_wait(smem_u32(o_bar), (uint32_t)((k - 1) & 1), ab);
+        const uint32_t pb = smem_base + Cfg::kOffP + (uint32_t)(k & 1) * Cfg::kPBytes;
+        // P^T element (row i, key): d = 128: box key / 64, row i; d = 64: row 16 (key / 64) + i
+        const int kk64 = tid & 63, half = tid >> 6;
+#pragma unroll
+        for (int i = 0; i < kDecTcRows; ++i) {
+          const float m_sub = m_used[i] == -INFINITY ? 0.0f : m_used[i];
+          const float pv = ex2_approx(x[i] - m_sub);  // 2^-inf = 0
+          const __nv_bfloat16 pr = __float2bfloat16_rn(pv);
+          l_part[i] = l_part[i] * alpha[i] + pv;
+          lr_part[i] = lr_part[i] * alpha[i] + __bfloat162float(pr);
+          const int prow = D == 64 ? half * 16 + i : i;
+          const uint32_t addr = pb + (D == 64 ? 0u : (uint32_t)half * 2048u) + (uint32_t)prow * 128u +
+                                ((((uint32_t)kk64 >> 3) ^ ((uint32_t)prow & 7u)) << 4) + ((uint32_t)kk64 & 7u) * 2u;
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(__bfloat16_as_ushort(pr)) : "memory");
+        }
+        // O^T *= alpha (column i of O^T is new row i) for the rows whose maximum moved
+        if (!first && moved) {
+          tc_fence_after_sync();
+          uint32_t o[8];
+          tmem_ld8(tO, o);
+          tmem_wait_ld(o);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha[i]);
+          tmem_st8(tO, o);
+        }
+        // V rows past the last valid key of the tile (the sequence's end, the piece's last unit,
+        // a missing second unit) may hold anything, a NaN among it: zero them before the product
+        const int v_end = min(n, t_last * kDecTile) - key0;
+        if (v_end < nu * kDecTile || nu < 2) {
+          mbar_wait(smem_u32(&full[k % kStages]), (uint32_t)((k / kStages) & 1), ab);
+          const uint32_t vt = kv_smem(k) + Cfg::kTileBytes;
+          const int from = max(0, v_end);
+          for (int e = tid; e < (Cfg::kTileKeys - from) * Cfg::kBoxes * 8; e += kDecThreads) {
+            const int row = from + e / (Cfg::kBoxes * 8), rest = e % (Cfg::kBoxes * 8);
+            st_shared_v4(vt + (rest >> 3) * Cfg::kBoxBytes + row * 128 + (rest & 7) * 16, 0u, 0u, 0u, 0u);
+          }
+        }
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(p_full));
+        seg_end = tw.next(p, u0, u1);
+        more = tw.valid(p);
+        seg_end = seg_end || !more;
+      }
+
+      // ---- segment end: row sums over the CTA; O / (sum of the weights applied), log2-sum-exp
+      // of the fp32 sum
+      mbar_wait(smem_u32(o_bar), (uint32_t)((k - 1) & 1), ab);
+      tc_fence_after_sync();
+      float* sL = sRed + 64;  // [4][16]: per warp, fp32 and rounded sums of the 8 rows
+#pragma unroll
+      for (int i = 0; i < kDecTcRows; ++i) {
+        float a = l_part[i], r = lr_part[i];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          a += __shfl_xor_sync(0xffffffffu, a, off);
+          r += __shfl_xor_sync(0xffffffffu, r, off);
+        }
+        if (lane == 0) {
+          sL[warp * 16 + i] = a;
+          sL[warp * 16 + 8 + i] = r;
+        }
+      }
+      uint32_t o[8];
+      tmem_ld8(tO, o);
+      tmem_wait_ld(o);
+      if (D == 64 && warp >= 2) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sEpi[(tid - 64) * 8 + i] = __uint_as_float(o[i]);
+      }
+      named_bar_sync(2, kDecThreads);
+      const int pf = dec_piece_of(T, Pe, seg_start_unit), pl = dec_piece_of(T, Pe, seg_start_unit + seg_cnt - 1);
+      const size_t slot = (size_t)b + piece;  // partial slot of (b, this piece)
+      if (D == 128 || warp < 2) {
+        const int col = tid;  // column of O
+#pragma unroll
+        for (int i = 0; i < kDecTcRows; ++i) {
+          if (i >= Sq) break;
+          const float lr = sL[i + 8] + sL[16 + i + 8] + sL[32 + i + 8] + sL[48 + i + 8];
+          float v = __uint_as_float(o[i]);
+          if (D == 64) v += sEpi[tid * 8 + i];
+          v = lr > 0.0f ? v / lr : 0.0f;
+          if (pf == pl) {
+            const long long oi = (((long long)b * Sq + i) * p.H + h) * D + col;
+            if (dbg_range(ab, oi, 1, o_size)) p.o[oi] = __float2bfloat16_rn(v);
+          } else {
+            const long long pi = (((long long)slot * p.H + h) * Sq + i) * D + col;
+            if (dbg_range(ab, pi, 1, part_rows * D)) p.o_part[pi] = v;
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kDecTcRows; ++i) {  // thread i writes row i's statistic
+        if (i != tid || i >= Sq) continue;
+        const float l = sL[i] + sL[16 + i] + sL[32 + i] + sL[48 + i];
+        const float l2 = l > 0.0f ? m_used[i] + __log2f(l) : -INFINITY;
+        if (pf == pl) {
+          const long long li = ((long long)b * p.H + h) * Sq + i;
+          if (dbg_range(ab, li, 1, lse_size)) p.lse[li] = l2 == -INFINITY ? -INFINITY : l2 * kDecLn2;
+        } else {
+          const long long pi = ((long long)slot * p.H + h) * Sq + i;
+          if (dbg_range(ab, pi, 1, part_rows)) p.lse_part[pi] = l2;
+        }
+      }
+      tc_fence_before_sync();
+      if (pf != pl) dec_arrive_merge<D>(p, b, h, pf, pl, ab, sInt);
+      named_bar_sync(1, kDecThreads);  // the next segment rewrites the sums, the exchange and the last flag
+    }
+  }
+
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, Cfg::kTmemCols);
   }
 }
 

@@ -1,12 +1,14 @@
 """GPU parity of the paged-KV decode (fa_decode_paged, through the C ABI) against the fp64 oracle.
 
-The kernel computes scores, the online softmax and P·V in fp32 on the CUDA cores from the
-exact bf16 inputs (P is not rounded), so the forward's tolerances apply: per row
-max |ΔO| / max(1, |O_ref|) <= 1e-2 and max |ΔLSE| <= 1e-3. Cases cover ragged lengths (empty,
-shorter than Sq, one key, page and tile boundaries), causal / window / full masks, Sq = 1..8,
-page sizes 64..512, piece counts 1, automatic and more pieces than tiles, pieces that span
-several sequences and sequences spread over several pieces, and the full decode workload
-compared row by row.
+Up to three new rows the kernel computes scores, the online softmax and P·V in fp32 on the CUDA
+cores from the exact bf16 inputs (P is not rounded). From four rows on the tensor-core kernel
+computes Q K^T and P V with tcgen05 (fp32 accumulation), P rounded to bf16 and O divided by the
+sum of the rounded weights, as the training forward does. The forward's tolerances apply to
+both: per element |ΔO| <= 1e-2 + half a bf16 ulp of O and max |ΔLSE| <= 1e-3. Cases cover
+ragged lengths (empty, shorter than Sq, one key, page and tile boundaries), causal / window /
+full masks, Sq = 1..8, page sizes 64..512, piece counts 1, automatic and more pieces than tiles,
+pieces that span several sequences and sequences spread over several pieces, and the full
+decode workloads compared row by row.
 """
 
 from __future__ import annotations
@@ -72,6 +74,54 @@ def test_decode_masks(causal, win, d):
 def test_decode_rows_and_page_sizes(Sq, page):
     cfg = DecodeConfig("pages", 4, Sq, 4, 128, 1, 1500, page, True, seed=63 + Sq)
     check(cfg, splits=0, what=f"Sq={Sq} page={page}")
+
+
+@pytest.mark.parametrize("splits", [1, 0, 3])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Sq", [4, 5, 6, 7, 8])
+def test_decode_tensor_core_rows(Sq, d, splits):
+    # every row count of the tensor-core kernel: empty, shorter than Sq, one key, one tile, a
+    # tile and a key, several pages
+    cfg = DecodeConfig("tc_rows", 6, Sq, 2, d, 1, 700, 64, True, seed=70 + Sq + d)
+    check(cfg, lens=[0, Sq - 2, 1, 64, 65, 700], splits=splits, what=f"Sq={Sq} d={d} splits={splits}")
+
+
+@pytest.mark.parametrize("Sq", [4, 8])
+def test_decode_tensor_core_large_logits(Sq):
+    # q scaled by 24: scores spread over tens of units, so a few keys dominate each row and the
+    # bf16 rounding of their weights moves O unless O is divided by the rounded weights
+    cfg = DecodeConfig("tc_big", 3, Sq, 2, 128, 1, 500, 128, False, seed=80 + Sq)
+    q, kc, vc, table, seqlens = make_decode_inputs(cfg)
+    q = (q.float() * 24.0).to(torch.bfloat16)
+    o, lse = run(q, kc, vc, table, seqlens, cfg.scale, False, (-1, -1), 0)
+    o_ref, lse_ref = oracle_dec.decode_forward(q.double().numpy(), kc.double().numpy(), vc.double().numpy(),
+                                               table.numpy(), seqlens.numpy(), cfg.scale, False, -1, -1)
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            assert_fwd_close(o[b, :, h], lse[b, h], o_ref[b, :, h], lse_ref[b, h], f"large logits b={b} h={h}")
+
+
+@pytest.mark.parametrize("Sq,d", [(1, 128), (3, 64), (4, 128), (8, 64)])
+def test_decode_cache_rows_past_the_end_are_not_used(Sq, d):
+    # a cache from an uninitialised allocation: NaN in every row past each sequence's end, in the
+    # sequences' own last pages and in the pages no sequence uses
+    cfg = DecodeConfig("nan_tail", 4, Sq, 2, d, 1, 600, 128, True, seed=90 + Sq)
+    q, kc, vc, table, seqlens = make_decode_inputs(cfg)
+    lens = torch.tensor([600, 65, 130, Sq + 7], dtype=torch.int32)
+    used = torch.zeros(kc.shape[:2], dtype=torch.bool)
+    for b in range(cfg.B):
+        for j in range(int(lens[b])):
+            used[int(table[b, j // cfg.page_size]), j % cfg.page_size] = True
+    kc, vc = kc.clone(), vc.clone()
+    kc[~used] = float("nan")
+    vc[~used] = float("nan")
+    o, lse = run(q, kc, vc, table, lens, cfg.scale, True, (-1, -1), 0)
+    o_ref, lse_ref = oracle_dec.decode_forward(q.double().numpy(), kc.double().numpy(), vc.double().numpy(),
+                                               table.numpy(), lens.numpy(), cfg.scale, True, -1, -1)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            assert_fwd_close(o[b, :, h], lse[b, h], o_ref[b, :, h], lse_ref[b, h], f"b={b} h={h}")
 
 
 @pytest.mark.parametrize("splits", [1, 2, 7, 0])
@@ -214,12 +264,14 @@ def test_decode_workspace_contents_do_not_matter():
 
 def test_decode_auto_pieces_fill_the_gpu_once():
     """fa_decode_splits: the automatic piece count lets all H x P CTAs run at once (no second
-    wave) and uses at least one CTA per SM; it never exceeds the batch's possible tiles."""
+    wave) and leaves fewer than H SMs without a CTA (the tensor-core kernel for 4 or more rows
+    takes a whole SM; H x P then falls short of the SM count by less than H); it never exceeds
+    the batch's possible tiles."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     for B, Sq, H, d, keys in [(8, 1, 16, 128, 8192), (8, 8, 16, 128, 8192), (4, 2, 8, 64, 4096), (1, 1, 2, 128, 65536)]:
         pieces = fa.decode_splits(B, Sq, H, d, keys)
         assert 1 <= pieces <= 65535
         assert pieces <= B * -(-keys // 64)
-        assert H * pieces >= sms, (B, Sq, H, d, pieces)  # at least one CTA per SM
+        assert H * pieces > sms - H, (B, Sq, H, d, pieces)  # all but fewer than H SMs busy
         assert H * pieces <= 8 * sms, (B, Sq, H, d, pieces)  # bounded by CTAs that fit per SM
     assert fa.decode_splits(1, 1, 2, 128, 64) == 1  # one tile: one piece
