@@ -87,7 +87,8 @@ bool decode_attributes() {
   return decode_kernel_attributes(fa::fa_decode_split_kernel<D, 1>, fa::DecCfg<D, 1>::kSmemBytes) &&
          decode_kernel_attributes(fa::fa_decode_split_kernel<D, 2>, fa::DecCfg<D, 2>::kSmemBytes) &&
          decode_kernel_attributes(fa::fa_decode_split_kernel<D, 4>, fa::DecCfg<D, 4>::kSmemBytes) &&
-         decode_kernel_attributes(fa::fa_decode_mma_kernel<D>, fa::DecTcCfg<D>::kSmemBytes);
+         decode_kernel_attributes(fa::fa_decode_mma_kernel<D, 4>, fa::DecTcCfg<D>::kSmemBytes) &&
+         decode_kernel_attributes(fa::fa_decode_mma_kernel<D, 8>, fa::DecTcCfg<D>::kSmemBytes);
 }
 
 int device_setup(int* dev_out, int* sm_count) {
@@ -690,7 +691,10 @@ int launch_decode(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const
   if (p.Sq < kDecMmaMinSq)
     return launch_decode_kernel(fa::fa_decode_split_kernel<D, 4>, kT, fa::DecCfg<D, 4>::kSmemBytes, grid, mk, mv, p,
                                 cs);
-  return launch_decode_kernel(fa::fa_decode_mma_kernel<D>, kTm, fa::DecTcCfg<D>::kSmemBytes, grid, mk, mv, p, cs);
+  if (p.Sq <= 4)
+    return launch_decode_kernel(fa::fa_decode_mma_kernel<D, 4>, kTm, fa::DecTcCfg<D>::kSmemBytes, grid, mk, mv, p,
+                                cs);
+  return launch_decode_kernel(fa::fa_decode_mma_kernel<D, 8>, kTm, fa::DecTcCfg<D>::kSmemBytes, grid, mk, mv, p, cs);
 }
 
 // Workspace of a call with P > 1 pieces per head: partial O (fp32) and partial LSE for the
@@ -716,7 +720,7 @@ int decode_ctas_per_sm(int Sq) {
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 4>, fa::kDecThreads,
                                                       fa::DecCfg<D, 4>::kSmemBytes);
   else
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_mma_kernel<D>, fa::kDecMmaThreads,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_mma_kernel<D, 4>, fa::kDecMmaThreads,
                                                       fa::DecTcCfg<D>::kSmemBytes);
   if (e != cudaSuccess) {
     cudaGetLastError();

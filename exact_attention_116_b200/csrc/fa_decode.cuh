@@ -47,7 +47,7 @@ namespace fa {
 constexpr int kDecMaxSq = 8;  // new query rows per call
 constexpr int kDecTile = 64;  // keys per tile
 constexpr int kDecThreads = 128;
-constexpr int kDecMmaThreads = 192;  // tensor-core kernel: four softmax warps, a producer and an MMA warp
+constexpr int kDecMmaThreads = 224;  // tensor-core kernel: four softmax warps, a producer, two MMA issuers
 constexpr float kDecLn2 = 0.69314718055994530942f;
 
 // Generic-proxy writes to global memory by this thread are ordered before later async-proxy
@@ -625,7 +625,6 @@ __global__ void __launch_bounds__(kDecThreads)
 // the log-sum-exp taken from the fp32 sum, as in the training forward. Work split, appends and
 // merge are those of the kernel above (pieces are counted in 64-key units).
 constexpr float kDecRescale = 8.0f;  // log2 units
-constexpr int kDecTcRows = 8;        // new rows a thread handles (Sq <= 8), padded to N = 16
 
 template <int D>
 struct DecTcCfg {
@@ -644,13 +643,13 @@ struct DecTcCfg {
   static constexpr int kOffRed = kOffP + 2 * kPBytes;        // [2][4][8] row maxima of the warps, then [4][16] sums
   static constexpr int kOffEpi = kOffRed + 512;              // d = 64: [64][8] second-half columns of O
   static constexpr int kOffMisc = kOffEpi + (D == 64 ? 64 * 8 * 4 : 0);  // scan sums, first segment, flags
-  static constexpr int kOffBar = kOffMisc + 128;             // full, empty [kStages]; s_bar[2], o_bar, p_full, q_full, done
+  static constexpr int kOffBar = kOffMisc + 128;  // full, empty [kStages]; s_bar, o_bar, p_full [2]; q_full, done
   static constexpr int kBarBytes = 256;                      // TMEM slot and abort flag in the last 64 bytes
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
   static constexpr uint32_t kColS = 0;                       // S^T buffers at columns 0 and 16
   static constexpr uint32_t kColO = 32;                      // O^T (kNO columns)
   static constexpr uint32_t kTmemCols = 64;
-  static_assert((2 * kStages + 6) * 8 <= kBarBytes - 64, "barrier area");
+  static_assert((2 * kStages + 8) * 8 <= kBarBytes - 64, "barrier area");
   static_assert(kOffQ % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands sit on 1024-byte boundaries");
 };
 
@@ -675,62 +674,78 @@ struct DecTcWalk {
   }
 };
 
+// Pages and first rows of the (one or two) units of the walk's current tile. The loads are
+// issued here and consumed by dec_tc_issue, so that their latency overlaps the producer's wait
+// for a free slot.
+struct DecTcPages {
+  int page[2], row[2], units;
+};
+__device__ __forceinline__ DecTcPages dec_tc_pages(const DecParams& p, const DecTcWalk& tw, Abort ab) {
+  DecTcPages pg;
+  pg.units = tw.units();
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int key = (tw.ta + min(u, pg.units - 1)) * kDecTile;
+    const long long ti = (long long)tw.w.b * p.max_pages + key / p.page_size;
+    pg.page[u] = dbg_range(ab, ti, 1, (long long)p.B * p.max_pages) ? p.block_table[ti] : 0;
+    pg.row[u] = key % p.page_size;
+  }
+  return pg;
+}
+
 // The producer's loads of one tile into its ring slot: one TMA box per 64-column box and unit,
 // for K and for V; a missing second unit is left as it is (its keys are masked, its V rows
 // zeroed by the softmax warps).
 template <int D>
 __device__ __forceinline__ bool dec_tc_issue(const DecParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                                             uint32_t dst, uint64_t* full_bar, int h, const DecTcWalk& tw, Abort ab,
+                                             uint32_t dst, uint64_t* full_bar, int h, DecTcPages pg, Abort ab,
                                              uint32_t smem_lo, uint32_t smem_end) {
   using Cfg = DecTcCfg<D>;
-  const int nu = tw.units();
-  int page[2] = {0, 0}, row[2] = {0, 0};
-  for (int u = 0; u < nu; ++u) {
-    const int key = (tw.ta + u) * kDecTile;
-    const long long ti = (long long)tw.w.b * p.max_pages + key / p.page_size;
-    if (!dbg_range(ab, ti, 1, (long long)p.B * p.max_pages)) return false;
-    int pg = p.block_table[ti];
-    if (pg < 0 || pg >= p.num_pages) {  // the TMA would read zeros there; report it
+  const int nu = pg.units;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    if (u >= nu) break;
+    if (pg.page[u] < 0 || pg.page[u] >= p.num_pages) {  // the TMA would read zeros there; report it
       atomicOr(&g_fa_error, kErrBadInput);
-      pg = 0;
+      pg.page[u] = 0;
     }
-    page[u] = pg;
-    row[u] = key % p.page_size;
     for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-      if (!dbg_tma(ab, bx * 64, h, row[u], pg, Cfg::kBoxes * 64, p.H, p.page_size, p.num_pages, 2,
+      if (!dbg_tma(ab, bx * 64, h, pg.row[u], pg.page[u], Cfg::kBoxes * 64, p.H, p.page_size, p.num_pages, 2,
                    dst + bx * Cfg::kBoxBytes + u * 8192, Cfg::kStageBytes - bx * Cfg::kBoxBytes - u * 8192, smem_lo,
                    smem_end))
         return false;
   }
   mbar_arrive_expect_tx(smem_u32(full_bar), (uint32_t)(nu * 2 * Cfg::kBoxes * 8192));
-  for (int u = 0; u < nu; ++u)
 #pragma unroll
-    for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int bx = 0; bx < Cfg::kBoxes && u < nu; ++bx) {
       const uint32_t off = bx * Cfg::kBoxBytes + u * 8192;
-      tma_load_4d(dst + off, tmK, smem_u32(full_bar), bx * 64, h, row[u], page[u]);
-      tma_load_4d(dst + Cfg::kTileBytes + off, tmV, smem_u32(full_bar), bx * 64, h, row[u], page[u]);
+      tma_load_4d(dst + off, tmK, smem_u32(full_bar), bx * 64, h, pg.row[u], pg.page[u]);
+      tma_load_4d(dst + Cfg::kTileBytes + off, tmV, smem_u32(full_bar), bx * 64, h, pg.row[u], pg.page[u]);
     }
   return true;
 }
 
-template <int D>
+template <int D, int kRows>
 __global__ void __launch_bounds__(kDecMmaThreads, 1)
     fa_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const DecParams p) {
   using Cfg = DecTcCfg<D>;
   constexpr int kStages = Cfg::kStages;
-  static_assert(kDecThreads == 128 && kDecMmaThreads == kDecThreads + 64, "four softmax warps, producer, MMA");
-  static_assert(kDecMaxSq <= kDecTcRows, "rows per thread");
+  static_assert(kDecThreads == 128 && kDecMmaThreads == kDecThreads + 96, "softmax warps, producer, two issuers");
+  static_assert(kRows == 4 || kRows == 8, "new rows a thread handles (padded to N = 16)");
+  static_assert(kDecMaxSq <= 8, "at most 8 new rows");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t* sm = smem_raw + (smem_base - smem_u32(smem_raw));
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + Cfg::kOffBar);
   uint64_t* empty = full + kStages;       // slot free again (P V of its tile completed)
   uint64_t* s_bar = full + 2 * kStages;   // [2] S(k) done, by k & 1
-  uint64_t* o_bar = s_bar + 2;            // P V(k) done
-  uint64_t* p_full = s_bar + 3;           // P^T(k) written, O rescaled (one arrival per softmax warp)
-  uint64_t* q_full = s_bar + 4;           // Q^T of a segment written (one arrival per softmax warp)
-  uint64_t* done_bar = s_bar + 5;
+  uint64_t* o_bar = s_bar + 2;            // [2] P V(k) done, by k & 1
+  uint64_t* p_full = s_bar + 4;           // [2] P^T(k) written, O rescaled, by k & 1 (one arrival per softmax warp)
+  uint64_t* q_full = s_bar + 6;           // Q^T of a segment written (one arrival per softmax warp)
+  uint64_t* done_bar = s_bar + 7;         // every product of both issuers has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + Cfg::kOffBar + Cfg::kBarBytes - 64);
   int* abort_flag = reinterpret_cast<int*>(sm + Cfg::kOffBar + Cfg::kBarBytes - 60);
   float* sRed = reinterpret_cast<float*>(sm + Cfg::kOffRed);
@@ -749,13 +764,11 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
   if (tid == 0) {
     *abort_flag = 0;
     sInt[0] = p.B;
-    for (int i = 0; i < 2 * kStages; ++i) mbar_init(smem_u32(&full[i]), 1);
-    mbar_init(smem_u32(&s_bar[0]), 1);
-    mbar_init(smem_u32(&s_bar[1]), 1);
-    mbar_init(smem_u32(o_bar), 1);
-    mbar_init(smem_u32(p_full), 4);
+    for (int i = 0; i < 2 * kStages + 4; ++i) mbar_init(smem_u32(&full[i]), 1);  // full, empty, s_bar, o_bar
+    mbar_init(smem_u32(&p_full[0]), 4);
+    mbar_init(smem_u32(&p_full[1]), 4);
     mbar_init(smem_u32(q_full), 4);
-    mbar_init(smem_u32(done_bar), 1);
+    mbar_init(smem_u32(done_bar), 2);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -783,51 +796,54 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
       DecTcWalk tw;
       tw.begin(p, b_first, start_first, u0, u1);
       long long j = 0;
+      DecTcPages pg = dec_tc_pages(p, tw, ab);
       for (bool more = tw.valid(p); more && !ab.raised(); ++j) {
         if (j >= kStages) mbar_wait(smem_u32(&empty[j % kStages]), (uint32_t)(((j / kStages) - 1) & 1), ab);
-        if (ab.raised() ||
-            !dec_tc_issue<D>(p, &tmK, &tmV, kv_smem(j), &full[j % kStages], h, tw, ab, smem_base, smem_end))
+        if (ab.raised() || !dec_tc_issue<D>(p, &tmK, &tmV, kv_smem(j), &full[j % kStages], h, pg, ab, smem_base,
+                                            smem_end))
           break;
         tw.next(p, u0, u1);
         more = tw.valid(p);
+        if (more) pg = dec_tc_pages(p, tw, ab);  // the next tile's pages, read while this slot waits
       }
       if (ab.raised())  // loads issued past a wait that gave up land before the CTA exits
         for (long long i = max(0LL, j - kStages); i < j; ++i)
           mbar_drain(smem_u32(&full[i % kStages]), (uint32_t)((i / kStages) & 1));
     }
   } else if (warp == 5) {
-    // ---- MMA issuer: S(k + 1) before P V(k), so that the softmax of tile k + 1 can start as
-    // soon as P(k) is handed over
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16_f32(128, 16, false, false);      // S^T: A (K) and B (Q) K-major
-      constexpr uint32_t idO = idesc_bf16_f32(128, Cfg::kNO, true, false);  // O^T: A (V^T) MN-major, B (P^T) K-major
-      auto issue_s = [&](long long j) {
-        mbar_wait(smem_u32(&full[j % kStages]), (uint32_t)((j / kStages) & 1), ab);
-        tc_fence_after_sync();
-        const uint32_t kt = kv_smem(j);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)  // 16 columns of d per step, 4 steps per box
-          mma_ss(tmem + Cfg::kColS + (uint32_t)(j & 1) * 16,
-                 sdesc_kmajor(kt + (kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32),
-                 sdesc_kmajor(sQ + (kk >> 2) * 2048 + (kk & 3) * 32), idS, kk > 0);
-        mma_commit(smem_u32(&s_bar[j & 1]));
-      };
+    // ---- S issuer: S(k) into buffer k & 1 once the softmax of tile k - 2 has read it
+    if (elect_one()) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 16, false, false);  // S^T: A (K) and B (Q) K-major
       long long k = 0;
       uint32_t seg = 0;
       DecTcWalk tw;
       tw.begin(p, b_first, start_first, u0, u1);
-      bool more = tw.valid(p), seg_start = true;
-      while (more) {
-        if (seg_start) {
-          mbar_wait(smem_u32(q_full), seg & 1, ab);  // this segment's Q^T
-          ++seg;
-          issue_s(k);
-        }
-        const bool first = seg_start;
+      for (bool more = tw.valid(p), seg_start = true; more; ++k) {
+        if (seg_start) mbar_wait(smem_u32(q_full), (seg++) & 1, ab);  // this segment's Q^T
+        if (k >= 2) mbar_wait(smem_u32(&p_full[k & 1]), (uint32_t)(((k - 2) >> 1) & 1), ab);
+        mbar_wait(smem_u32(&full[k % kStages]), (uint32_t)((k / kStages) & 1), ab);
+        tc_fence_after_sync();
+        const uint32_t kt = kv_smem(k);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)  // 16 columns of d per step, 4 steps per box
+          mma_ss(tmem + Cfg::kColS + (uint32_t)(k & 1) * 16,
+                 sdesc_kmajor(kt + (kk >> 2) * Cfg::kBoxBytes + (kk & 3) * 32),
+                 sdesc_kmajor(sQ + (kk >> 2) * 2048 + (kk & 3) * 32), idS, kk > 0);
+        mma_commit(smem_u32(&s_bar[k & 1]));
         seg_start = tw.next(p, u0, u1);
         more = tw.valid(p);
-        if (more && !seg_start) issue_s(k + 1);  // the next tile is in the same segment
-        mbar_wait(smem_u32(p_full), (uint32_t)(k & 1), ab);
+      }
+      mma_commit(smem_u32(done_bar));
+    }
+  } else if (warp == 6) {
+    // ---- P V issuer: O^T += V^T P^T(k) once P^T(k) is written
+    if (elect_one()) {
+      constexpr uint32_t idO = idesc_bf16_f32(128, Cfg::kNO, true, false);  // O^T: A (V^T) MN-major, B (P^T) K-major
+      long long k = 0;
+      DecTcWalk tw;
+      tw.begin(p, b_first, start_first, u0, u1);
+      for (bool more = tw.valid(p), first = true; more; ++k) {
+        mbar_wait(smem_u32(&p_full[k & 1]), (uint32_t)((k >> 1) & 1), ab);
         tc_fence_after_sync();
         const uint32_t vt = kv_smem(k) + Cfg::kTileBytes;
         const uint32_t pb = smem_base + Cfg::kOffP + (uint32_t)(k & 1) * Cfg::kPBytes;
@@ -842,12 +858,13 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
             mma_ss(tmem + Cfg::kColO, sdesc_mnmajor(vt + kk * 2048, 8192), sdesc_kmajor(pb + kk * 32), idO,
                    !first || kk > 0);
         }
-        mma_commit(smem_u32(o_bar));
-        mma_commit(smem_u32(&empty[k % kStages]));
-        ++k;
+        mma_commit(smem_u32(&o_bar[k & 1]));
+        mma_commit(smem_u32(&empty[k % kStages]));  // (S(k) completed before P^T(k) was written)
+        first = tw.next(p, u0, u1);
+        more = tw.valid(p);
       }
-      mma_commit(smem_u32(done_bar));  // every product has completed before the TMEM is freed
-      mbar_drain(smem_u32(done_bar), 0);
+      mma_commit(smem_u32(done_bar));
+      mbar_drain(smem_u32(done_bar), 0);  // every product has completed before the TMEM is freed
     }
   } else {
     // ---- softmax warps 0-3: thread i owns key i of each tile (TMEM lane i of S^T)
@@ -856,6 +873,7 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
     // sums of column d - 64 in O^T columns 16..23
     const uint32_t tO = tmem + Cfg::kColO + my_lanes + (D == 64 && warp >= 2 ? 16u : 0u);
     const float c = p.scale_log2;
+    const int kk64 = tid & 63, half = tid >> 6;  // this thread's key within its 64-key unit, and the unit
     long long k = 0;
     DecTcWalk tw;
     tw.begin(p, b_first, start_first, u0, u1);
@@ -876,17 +894,17 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(q_full));
       // per new row: the visible keys [kmin, khi] of this segment
-      int kmin[kDecTcRows], khi[kDecTcRows];
+      int kmin[kRows], khi[kRows];
 #pragma unroll
-      for (int i = 0; i < kDecTcRows; ++i) {
+      for (int i = 0; i < kRows; ++i) {
         const int pos = n - Sq + i;
         kmin[i] = p.win_l >= 0 ? pos - p.win_l : 0;
         khi[i] = min(min(n - 1, t_last * kDecTile - 1), p.win_r >= 0 ? pos + p.win_r : n - 1);
         if (i >= Sq) khi[i] = -1;
       }
-      float m_used[kDecTcRows], l_part[kDecTcRows], lr_part[kDecTcRows];
+      float m_used[kRows], l_part[kRows], lr_part[kRows];
 #pragma unroll
-      for (int i = 0; i < kDecTcRows; ++i) {
+      for (int i = 0; i < kRows; ++i) {
         m_used[i] = -INFINITY;
         l_part[i] = 0.0f;
         lr_part[i] = 0.0f;
@@ -894,60 +912,72 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
       bool seg_end = false;
       for (bool first = true; !seg_end; first = false, ++k) {
         const int key0 = tw.ta * kDecTile, nu = tw.units();
-        // ---- scores of key key0 + tid for every new row
+        // ---- scores of key key0 + tid for every new row; the row maxima over the tile
         mbar_wait(smem_u32(&s_bar[k & 1]), (uint32_t)((k >> 1) & 1), ab);
         tc_fence_after_sync();
         uint32_t sr[8];
         tmem_ld8(tmem + Cfg::kColS + (uint32_t)(k & 1) * 16 + my_lanes, sr);
         tmem_wait_ld(sr);
         const int key = key0 + tid;
-        float x[kDecTcRows];
+        float x[kRows], wm[kRows];
 #pragma unroll
-        for (int i = 0; i < kDecTcRows; ++i) {
+        for (int i = 0; i < kRows; ++i) {
           x[i] = (key >= kmin[i] && key <= khi[i]) ? __uint_as_float(sr[i]) * c : -INFINITY;
-          const float wm = warp_max_f32(x[i]);
-          if (lane == 0) sRed[((k & 1) * 4 + warp) * 8 + i] = wm;
+          wm[i] = warp_max_f32(x[i]);
+        }
+        float4* red4 = reinterpret_cast<float4*>(sRed + ((k & 1) * 4 + warp) * 8);
+        if (lane == 0) {
+#pragma unroll
+          for (int i = 0; i < kRows; i += 4) red4[i / 4] = make_float4(wm[i], wm[i + 1], wm[i + 2], wm[i + 3]);
         }
         named_bar_sync(2, kDecThreads);
-        float alpha[kDecTcRows];
+        float m_tile[kRows];
+#pragma unroll
+        for (int i = 0; i < kRows; i += 4) {
+          const float4* r4 = reinterpret_cast<const float4*>(sRed + (k & 1) * 32) + i / 4;
+          const float4 a0 = r4[0], a1 = r4[2], a2 = r4[4], a3 = r4[6];
+          m_tile[i] = fmaxf(fmaxf(a0.x, a1.x), fmaxf(a2.x, a3.x));
+          m_tile[i + 1] = fmaxf(fmaxf(a0.y, a1.y), fmaxf(a2.y, a3.y));
+          m_tile[i + 2] = fmaxf(fmaxf(a0.z, a1.z), fmaxf(a2.z, a3.z));
+          m_tile[i + 3] = fmaxf(fmaxf(a0.w, a1.w), fmaxf(a2.w, a3.w));
+        }
+        // lazy rescale: a row's reference maximum moves only when the tile's exceeds it by more
+        // than 2^8 (from -inf: at its first visible key); alpha = 2^(old - new), 0 from -inf
+        float alpha[kRows];
         bool moved = false;
 #pragma unroll
-        for (int i = 0; i < kDecTcRows; ++i) {
-          const float* rm = sRed + (k & 1) * 32 + i;
-          const float m_tile = fmaxf(fmaxf(rm[0], rm[8]), fmaxf(rm[16], rm[24]));
-          alpha[i] = 1.0f;
-          if (m_tile > m_used[i] + kDecRescale || (m_used[i] == -INFINITY && m_tile != -INFINITY)) {
-            alpha[i] = m_used[i] == -INFINITY ? 0.0f : ex2_approx(m_used[i] - m_tile);
-            m_used[i] = m_tile;
-            moved = true;
-          }
+        for (int i = 0; i < kRows; ++i) {
+          const bool mv = m_tile[i] > m_used[i] + kDecRescale;
+          alpha[i] = ex2_approx(mv ? m_used[i] - m_tile[i] : 0.0f);
+          m_used[i] = mv ? m_tile[i] : m_used[i];
+          moved = moved || mv;
         }
-        // the P^T buffer of this parity and O^T are free: P V of the previous tile has completed
-        // (the segment's first tile: the last segment end waited for all of them)
-        if (!first) mbar_wait(smem_u32(o_bar), (uint32_t)((k - 1) & 1), ab);
-        const uint32_t pb = smem_base + Cfg::kOffP + (uint32_t)(k & 1) * Cfg::kPBytes;
-        // P^T element (row i, key): d = 128: box key / 64, row i; d = 64: row 16 (key / 64) + i
-        const int kk64 = tid & 63, half = tid >> 6;
+        // the P^T buffer of this parity is free once P V(k - 2) has completed
+        if (k >= 2) mbar_wait(smem_u32(&o_bar[k & 1]), (uint32_t)(((k - 2) >> 1) & 1), ab);
+        // P^T element (row i, key): d = 128: box key / 64 (2 KB each), row i; d = 64: row
+        // 16 (key / 64) + i of one box; either way 2048 (key / 64) + 128 i bytes in
+        const uint32_t pb = smem_base + Cfg::kOffP + (uint32_t)(k & 1) * Cfg::kPBytes + (uint32_t)half * 2048u;
 #pragma unroll
-        for (int i = 0; i < kDecTcRows; ++i) {
+        for (int i = 0; i < kRows; ++i) {
           const float m_sub = m_used[i] == -INFINITY ? 0.0f : m_used[i];
           const float pv = ex2_approx(x[i] - m_sub);  // 2^-inf = 0
           const __nv_bfloat16 pr = __float2bfloat16_rn(pv);
-          l_part[i] = l_part[i] * alpha[i] + pv;
-          lr_part[i] = lr_part[i] * alpha[i] + __bfloat162float(pr);
-          const int prow = D == 64 ? half * 16 + i : i;
-          const uint32_t addr = pb + (D == 64 ? 0u : (uint32_t)half * 2048u) + (uint32_t)prow * 128u +
-                                ((((uint32_t)kk64 >> 3) ^ ((uint32_t)prow & 7u)) << 4) + ((uint32_t)kk64 & 7u) * 2u;
+          l_part[i] = fmaf(l_part[i], alpha[i], pv);
+          lr_part[i] = fmaf(lr_part[i], alpha[i], __bfloat162float(pr));
+          const uint32_t addr = pb + (uint32_t)i * 128u + ((((uint32_t)kk64 >> 3) ^ (uint32_t)(i & 7)) << 4) +
+                                ((uint32_t)kk64 & 7u) * 2u;
           asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(__bfloat16_as_ushort(pr)) : "memory");
         }
-        // O^T *= alpha (column i of O^T is new row i) for the rows whose maximum moved
+        // O^T *= alpha (column i of O^T is new row i) for the rows whose maximum moved, once
+        // P V(k - 1) has completed
         if (!first && moved) {
+          mbar_wait(smem_u32(&o_bar[(k - 1) & 1]), (uint32_t)(((k - 1) >> 1) & 1), ab);
           tc_fence_after_sync();
           uint32_t o[8];
           tmem_ld8(tO, o);
           tmem_wait_ld(o);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha[i]);
+          for (int i = 0; i < kRows; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha[i]);
           tmem_st8(tO, o);
         }
         // V rows past the last valid key of the tile (the sequence's end, the piece's last unit,
@@ -966,7 +996,7 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
         tmem_wait_st();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(p_full));
+        if (lane == 0) mbar_arrive(smem_u32(&p_full[k & 1]));
         seg_end = tw.next(p, u0, u1);
         more = tw.valid(p);
         seg_end = seg_end || !more;
@@ -974,11 +1004,11 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
 
       // ---- segment end: row sums over the CTA; O / (sum of the weights applied), log2-sum-exp
       // of the fp32 sum
-      mbar_wait(smem_u32(o_bar), (uint32_t)((k - 1) & 1), ab);
+      mbar_wait(smem_u32(&o_bar[(k - 1) & 1]), (uint32_t)(((k - 1) >> 1) & 1), ab);
       tc_fence_after_sync();
-      float* sL = sRed + 64;  // [4][16]: per warp, fp32 and rounded sums of the 8 rows
+      float* sL = sRed + 64;  // [4][16]: per warp, fp32 and rounded sums of the rows
 #pragma unroll
-      for (int i = 0; i < kDecTcRows; ++i) {
+      for (int i = 0; i < kRows; ++i) {
         float a = l_part[i], r = lr_part[i];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
@@ -995,7 +1025,7 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
       tmem_wait_ld(o);
       if (D == 64 && warp >= 2) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) sEpi[(tid - 64) * 8 + i] = __uint_as_float(o[i]);
+        for (int i = 0; i < kRows; ++i) sEpi[(tid - 64) * 8 + i] = __uint_as_float(o[i]);
       }
       named_bar_sync(2, kDecThreads);
       const int pf = dec_piece_of(T, Pe, seg_start_unit), pl = dec_piece_of(T, Pe, seg_start_unit + seg_cnt - 1);
@@ -1003,7 +1033,7 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
       if (D == 128 || warp < 2) {
         const int col = tid;  // column of O
 #pragma unroll
-        for (int i = 0; i < kDecTcRows; ++i) {
+        for (int i = 0; i < kRows; ++i) {
           if (i >= Sq) break;
           const float lr = sL[i + 8] + sL[16 + i + 8] + sL[32 + i + 8] + sL[48 + i + 8];
           float v = __uint_as_float(o[i]);
@@ -1019,7 +1049,7 @@ __global__ void __launch_bounds__(kDecMmaThreads, 1)
         }
       }
 #pragma unroll
-      for (int i = 0; i < kDecTcRows; ++i) {  // thread i writes row i's statistic
+      for (int i = 0; i < kRows; ++i) {  // thread i writes row i's statistic
         if (i != tid || i >= Sq) continue;
         const float l = sL[i] + sL[16 + i] + sL[32 + i] + sL[48 + i];
         const float l2 = l > 0.0f ? m_used[i] + __log2f(l) : -INFINITY;
