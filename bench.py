@@ -7,7 +7,7 @@ workloads, which fits one GPU). The same run also reports device-timed forward /
 figures of the other workloads (GPT-style forward, training shape, sliding window, tiny) under
 "configs". ``--config train_fwd_fp8`` instead times the E4M3 forward (fa_fwd_fp8) on the training
 shape: one step = one launch. ``--config decode_paged`` times the paged-KV decode
-(fa_decode_paged): one step = one call (append, split kernel and merge in one kernel) over every
+(fa_decode_paged): one step = one call (append, attention and merge in one kernel) over every
 sequence, reported in GB/s of cache read.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
@@ -466,18 +466,18 @@ def run_gpu_decode(args):
                    "l2": "L2 flushed before every timed step (512 MiB written, then 512 MiB read: no dirty lines "
                          "left to write back inside the step); KV cache > L2",
                    "bytes": "K and V rows of every visible key + q, O, LSE"},
-        "roofline": {"kernel": "fa_decode_split_kernel<128> (append and merge fused; timed with the counter-"
+        "roofline": {"kernel": "fa_decode_kernel<128> (append and merge fused; timed with the counter-"
                                "zeroing launch before it)", "bound": "hbm", "achieved": round(gbs, 1),
                      "peak": peak["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peak["hbm_gbs"], 4),
                      "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
-                     "traffic": recorded_traffic("fa_decode_split_kernel", cfg.name), "algorithmic_bytes": nbytes},
+                     "traffic": recorded_traffic("fa_decode_kernel", cfg.name), "algorithmic_bytes": nbytes},
         "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": out_h.numel(),
                 "pipelining": "one packed copy up (q, new K/V rows, block table, lengths) and one down (O, LSE) per "
                               "step, on their own streams, overlapping the previous and next steps' compute (two "
                               "device buffer sets)"},
-        "gpu_launches": (2 if splits > 1 else 1) * args.steps,  # counter zeroing, split kernel
+        "gpu_launches": (2 if splits > 1 else 1) * args.steps,  # counter zeroing, decode kernel
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

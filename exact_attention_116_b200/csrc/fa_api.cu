@@ -73,22 +73,17 @@ bool bwd_attributes() {
          variant_attributes<D, false, true>() && variant_attributes<D, true, true>();
 }
 
-// Dynamic shared memory size, and the largest shared-memory carveout (several CTAs of the
-// CUDA-core decode kernel share an SM; the tensor-core kernel takes nearly all of one).
-template <class Kernel>
-bool decode_kernel_attributes(Kernel kernel, int smem_bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) == cudaSuccess &&
-         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                              cudaSharedmemCarveoutMaxShared) == cudaSuccess;
-}
-
+// Dynamic shared memory size of the decode kernel, and the largest shared-memory carveout (one
+// CTA takes nearly all of an SM's).
 template <int D>
 bool decode_attributes() {
-  return decode_kernel_attributes(fa::fa_decode_split_kernel<D, 1>, fa::DecCfg<D, 1>::kSmemBytes) &&
-         decode_kernel_attributes(fa::fa_decode_split_kernel<D, 2>, fa::DecCfg<D, 2>::kSmemBytes) &&
-         decode_kernel_attributes(fa::fa_decode_split_kernel<D, 4>, fa::DecCfg<D, 4>::kSmemBytes) &&
-         decode_kernel_attributes(fa::fa_decode_mma_kernel<D, 4>, fa::DecTcCfg<D>::kSmemBytes) &&
-         decode_kernel_attributes(fa::fa_decode_mma_kernel<D, 8>, fa::DecTcCfg<D>::kSmemBytes);
+  for (const void* k : {(const void*)fa::fa_decode_kernel<D, 4>, (const void*)fa::fa_decode_kernel<D, 8>})
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::DecTcCfg<D>::kSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+            cudaSuccess)
+      return false;
+  return true;
 }
 
 int device_setup(int* dev_out, int* sm_count) {
@@ -652,49 +647,28 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, const float* q_desca
 
 namespace {
 
-// Decode kernel launched as the programmatic dependent of the kernel before it on the stream
-// (the prep kernel, when there are splits).
-template <class Kernel>
-int launch_decode_kernel(Kernel kernel, int threads, int smem_bytes, dim3 grid, const CUtensorMap& mk,
-                         const CUtensorMap& mv, const fa::DecParams& p, cudaStream_t cs) {
+// The decode kernel, compiled for up to 4 or up to 8 new rows, launched as the programmatic
+// dependent of the kernel before it on the stream (the prep kernel, when there are splits).
+template <int D>
+int launch_decode(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
+                  cudaStream_t cs) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.blockDim = dim3(fa::kDecMmaThreads);
+  cfg.dynamicSmemBytes = fa::DecTcCfg<D>::kSmemBytes;
   cfg.stream = cs;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kernel, mk, mv, p) != cudaSuccess) {
+  const cudaError_t e = p.Sq <= 4 ? cudaLaunchKernelEx(&cfg, fa::fa_decode_kernel<D, 4>, mk, mv, p)
+                                  : cudaLaunchKernelEx(&cfg, fa::fa_decode_kernel<D, 8>, mk, mv, p);
+  if (e != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_CUDA;
   }
   return launch_status();
-}
-
-// Up to 3 new rows: the CUDA-core kernel compiled for Sq rounded up to 1, 2 or 4; from 4 rows
-// on: the tensor-core kernel.
-constexpr int kDecMmaMinSq = 4;
-
-template <int D>
-int launch_decode(dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
-                  cudaStream_t cs) {
-  constexpr int kT = fa::kDecThreads, kTm = fa::kDecMmaThreads;
-  if (p.Sq == 1)
-    return launch_decode_kernel(fa::fa_decode_split_kernel<D, 1>, kT, fa::DecCfg<D, 1>::kSmemBytes, grid, mk, mv, p,
-                                cs);
-  if (p.Sq == 2)
-    return launch_decode_kernel(fa::fa_decode_split_kernel<D, 2>, kT, fa::DecCfg<D, 2>::kSmemBytes, grid, mk, mv, p,
-                                cs);
-  if (p.Sq < kDecMmaMinSq)
-    return launch_decode_kernel(fa::fa_decode_split_kernel<D, 4>, kT, fa::DecCfg<D, 4>::kSmemBytes, grid, mk, mv, p,
-                                cs);
-  if (p.Sq <= 4)
-    return launch_decode_kernel(fa::fa_decode_mma_kernel<D, 4>, kTm, fa::DecTcCfg<D>::kSmemBytes, grid, mk, mv, p,
-                                cs);
-  return launch_decode_kernel(fa::fa_decode_mma_kernel<D, 8>, kTm, fa::DecTcCfg<D>::kSmemBytes, grid, mk, mv, p, cs);
 }
 
 // Workspace of a call with P > 1 pieces per head: partial O (fp32) and partial LSE for the
@@ -705,24 +679,12 @@ size_t decode_workspace_bytes(int B, int Sq, int H, int d, int pieces) {
   return align256(rows * d * 4) + align256(rows * 4) + align256((size_t)B * H * 4);
 }
 
-// CTAs of the decode kernel for (d, Sq) that fit on one SM at a time (0 on error).
+// CTAs of the decode kernel that fit on one SM at a time (0 on error).
 template <int D>
-int decode_ctas_per_sm(int Sq) {
+int decode_ctas_per_sm() {
   int n = 0;
-  cudaError_t e;
-  if (Sq == 1)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 1>, fa::kDecThreads,
-                                                      fa::DecCfg<D, 1>::kSmemBytes);
-  else if (Sq == 2)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 2>, fa::kDecThreads,
-                                                      fa::DecCfg<D, 2>::kSmemBytes);
-  else if (Sq < kDecMmaMinSq)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_split_kernel<D, 4>, fa::kDecThreads,
-                                                      fa::DecCfg<D, 4>::kSmemBytes);
-  else
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_mma_kernel<D, 4>, fa::kDecMmaThreads,
-                                                      fa::DecTcCfg<D>::kSmemBytes);
-  if (e != cudaSuccess) {
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fa::fa_decode_kernel<D, 8>, fa::kDecMmaThreads,
+                                                    fa::DecTcCfg<D>::kSmemBytes) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -732,7 +694,7 @@ int decode_ctas_per_sm(int Sq) {
 // Pieces per head when the caller passes 0: as many as fill every CTA slot of the GPU once
 // (H x P <= resident CTAs), at least 1, no more than the batch can have tiles, at most 65535.
 int decode_auto_pieces(int B, int Sq, int H, int d, int max_keys, int sm_count) {
-  const int per_sm = d == 64 ? decode_ctas_per_sm<64>(Sq) : decode_ctas_per_sm<128>(Sq);
+  const int per_sm = d == 64 ? decode_ctas_per_sm<64>() : decode_ctas_per_sm<128>();
   long long pieces = (long long)std::max(per_sm, 1) * sm_count / H;
   const long long tiles = (long long)B * ((max_keys + fa::kDecTile - 1) / fa::kDecTile);
   pieces = std::min(pieces, std::min(tiles, 65535LL));

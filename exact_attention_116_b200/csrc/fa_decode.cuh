@@ -7,8 +7,9 @@
 // and LSE = ln sum_j exp(scale * q . k_j). Key j of sequence b is row j % page_size of page
 // block_table[b][j / page_size] of the (num_pages, page_size, H, d) cache.
 //
-// The work is one pass over the cache: HBM-bound (each K/V element is used by Sq <= 8 rows),
-// so it runs on the CUDA cores, not the tensor cores.
+// The work is one pass over the cache: HBM-bound (each K/V element is used by Sq <= 8 rows).
+// Both products still run on the tensor core (see the kernel below): on the CUDA cores the dot
+// products and P V of even one to four rows kept the kernel from the cache read.
 //
 // Work split (split-KV, balanced over the whole batch): for each head, the 64-key tiles that
 // the new rows can see are listed sequence after sequence, and that list is cut into P equal
@@ -21,18 +22,12 @@
 // (O / l, log2 l + m) to slot b + piece (unique: a piece after another one on the list never
 // holds an earlier sequence), counts itself on the (b, h) arrival counter, and the piece that
 // arrives last merges the partials by their log-sum-exp, in piece order. The counters are
-// zeroed by fa_decode_prep_kernel, launched just before on the same stream; the split kernel
+// zeroed by fa_decode_prep_kernel, launched just before on the same stream; the decode kernel
 // is launched as its programmatic dependent and waits for it only before its first arrival.
 //
-// CTA (128 threads), per tile of 64 keys:
-//   A: thread (key t = tid % 64, half = tid / 64) forms half of q_i . k_t for every row i
-//   B: warp w owns rows w and w + 4: mask, tile max, exponentials, running max / sum, rescale
-//      factor alpha_i; P goes to shared memory
-//   C: thread (column pair, key group) accumulates O_i += P_i,t v_t over its keys
-// The kernel is compiled for kSq = 1, 2, 4, 8 rows (the call's Sq rounded up; the extra rows
-// have q = 0 and are not written). CTAs of the same piece for consecutive heads are launched
-// next to each other (head is the fastest grid index) and walk the same tiles, so the 128-byte
-// head slices of one cache row (H x d bf16, contiguous) are read at about the same time.
+// CTAs of the same piece for consecutive heads are launched next to each other (head is the
+// fastest grid index) and walk the same tiles, so the 128-byte head slices of one cache row
+// (H x d bf16, contiguous) are read at about the same time.
 //
 // With new K/V rows given (flash_attn_with_kvcache's in-place update of the cache), the CTA
 // whose piece holds a new row's tile writes that row's d columns of its head into the cache
@@ -49,6 +44,26 @@ constexpr int kDecTile = 64;  // keys per tile
 constexpr int kDecThreads = 128;
 constexpr int kDecMmaThreads = 224;  // tensor-core kernel: four softmax warps, a producer, two MMA issuers
 constexpr float kDecLn2 = 0.69314718055994530942f;
+
+// Warp-collective TMEM load of 8 consecutive 32-bit columns: thread t of the warp reads lane
+// (lane field of taddr) + t; and the wait for it (the registers pass through so that no use is
+// hoisted above the wait).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])::"memory");
+}
+
+// Maximum of x over the 32 lanes of the warp (all lanes active), one instruction on sm_100a.
+__device__ __forceinline__ float warp_max_f32(float x) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
+}
 
 // Generic-proxy writes to global memory by this thread are ordered before later async-proxy
 // (TMA) accesses that a barrier orders after this fence.
@@ -75,28 +90,6 @@ struct DecParams {
   const __nv_bfloat16* v_new;
   __nv_bfloat16* k_cache;  // (num_pages, page_size, H, d)
   __nv_bfloat16* v_cache;
-};
-
-// Shared memory of a CTA compiled for kSq rows: a 2-stage K/V ring (64 KB at d = 128) and
-// small per-row buffers, so that three CTAs share an SM for up to 4 rows (two for 8) and hide
-// each other's per-tile latency.
-template <int D, int kSq>
-struct DecCfg {
-  static constexpr int kStages = 2;
-  static constexpr int kBoxes = D / 64;                        // 64-column (128-byte) boxes per row
-  static constexpr int kTileBytes = kDecTile * D * 2;          // one K or V tile
-  static constexpr int kStageBytes = 2 * kTileBytes;           // K and V
-  static constexpr int kOffKV = 0;
-  static constexpr int kOffQ = kStages * kStageBytes;           // q rows, fp32 (kSq x D)
-  static constexpr int kOffS = kOffQ + kSq * D * 4;             // half-dot products (2 x kSq x 64)
-  static constexpr int kOffP = kOffS + 2 * kSq * kDecTile * 4;  // P (kSq x 64)
-  static constexpr int kPairs = D / 2;                          // column pairs
-  static constexpr int kKeyGroups = kDecThreads / kPairs;       // 2 (D=128) or 4 (D=64)
-  static constexpr int kOffRed = kOffP + kSq * kDecTile * 4;    // key groups x kSq x D partial sums
-  static constexpr int kOffAlpha = kOffRed + kKeyGroups * kSq * D * 4;  // per row: alpha, then 1 / l
-  static constexpr int kOffMisc = (kOffAlpha + kSq * 4 + 15) & ~15;     // scan sums, first segment
-  static constexpr int kOffBar = (kOffMisc + 64 + 63) & ~63;
-  static constexpr int kSmemBytes = kOffBar + 128 + 1024;  // barriers + alignment slack
 };
 
 // Length of sequence b; an out-of-range length counts as 0 (reported when `report`).
@@ -174,41 +167,6 @@ struct DecWalk {
   __device__ __forceinline__ bool valid(const DecParams& p) const { return b < p.B; }
 };
 
-// TMA loads of the piece's next tile (stream index `issued`, at the walk's position) into its
-// ring slot; advances the walk and the count.
-// FA_DEBUG: a tile whose table index, coordinates or ring slot fail the bounds check is neither
-// armed nor loaded (the CTA's abort flag is then raised, so its waits return).
-template <class Cfg>
-__device__ __forceinline__ void dec_issue_tile(const DecParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                                               uint32_t smem_base, uint64_t* full, int h, long long u0, long long u1,
-                                               DecWalk& ld, long long& issued, Abort ab, uint32_t smem_end) {
-  const int st = (int)(issued % Cfg::kStages);
-  const int key = ld.t * kDecTile;
-  const long long ti = (long long)ld.b * p.max_pages + key / p.page_size;
-  if (!dbg_range(ab, ti, 1, (long long)p.B * p.max_pages)) return;
-  int page = p.block_table[ti];
-  if (page < 0 || page >= p.num_pages) {  // the TMA would read zeros there; report it
-    atomicOr(&g_fa_error, kErrBadInput);
-    page = 0;
-  }
-  const int row = key % p.page_size;
-  const uint32_t dst = smem_base + Cfg::kOffKV + st * Cfg::kStageBytes;
-  bool ok = true;
-#pragma unroll
-  for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-    ok = ok && dbg_tma(ab, bx * 64, h, row, page, Cfg::kBoxes * 64, p.H, p.page_size, p.num_pages, 2,
-                       dst + bx * (kDecTile * 128), 2 * Cfg::kTileBytes - bx * (kDecTile * 128), smem_base, smem_end);
-  if (!ok) return;
-  mbar_arrive_expect_tx(smem_u32(&full[st]), Cfg::kStageBytes);
-#pragma unroll
-  for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
-    tma_load_4d(dst + bx * (kDecTile * 128), tmK, smem_u32(&full[st]), bx * 64, h, row, page);
-    tma_load_4d(dst + Cfg::kTileBytes + bx * (kDecTile * 128), tmV, smem_u32(&full[st]), bx * 64, h, row, page);
-  }
-  ++issued;
-  if (++ld.t == ld.t1) ld.next_seg(p, u0, u1);
-}
-
 // A CTA's piece of a head's tile list: the list's length T, the pieces in use Pe, this piece's
 // units [u0, u1) and its first segment (sequence b_first, whose tiles start at unit start_first).
 struct DecPiece {
@@ -216,8 +174,8 @@ struct DecPiece {
   int Pe, b_first;
 };
 
-// Set-up shared by the decode kernels (all threads of the CTA; threads 0 .. kDecThreads - 1 do the
-// work, any others only meet the barriers): the piece from the lengths (a
+// Set-up of the decode kernel (all threads of the CTA; threads 0 .. kDecThreads - 1 do the work,
+// the others only meet the barriers): the piece from the lengths (a
 // block-wide prefix sum of tile counts, each thread summing a contiguous run of sequences); O = 0,
 // LSE = -inf for the sequences without a visible tile (written by piece b % P); with new K/V rows
 // given, this piece's new rows of head h written into the cache before any tile load. sSum holds
@@ -377,238 +335,10 @@ __device__ __forceinline__ void dec_arrive_merge(const DecParams& p, int b, int 
     }
 }
 
-template <int D, int kSq>
-__global__ void __launch_bounds__(kDecThreads)
-    fa_decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                           const DecParams p) {
-  using Cfg = DecCfg<D, kSq>;
-  constexpr int kStages = Cfg::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t smem_base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  uint8_t* sm = smem_raw + (smem_base - smem_u32(smem_raw));
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Cfg::kOffBar);
-  int* abort_flag = reinterpret_cast<int*>(sm + Cfg::kOffBar + 64);
-  float* sQ = reinterpret_cast<float*>(sm + Cfg::kOffQ);
-  float* sS = reinterpret_cast<float*>(sm + Cfg::kOffS);
-  float* sP = reinterpret_cast<float*>(sm + Cfg::kOffP);
-  float* sAlpha = reinterpret_cast<float*>(sm + Cfg::kOffAlpha);
-  float* sRed = reinterpret_cast<float*>(sm + Cfg::kOffRed);
-  long long* sSum = reinterpret_cast<long long*>(sm + Cfg::kOffMisc);  // [0, 4) warp sums, [4] first start
-  int* sInt = reinterpret_cast<int*>(sm + Cfg::kOffMisc + 48);          // [0] first sequence, [1] last flag
-  const Abort ab{abort_flag};
-  const uint32_t smem_end = smem_u32(smem_raw) + Cfg::kSmemBytes;  // for the FA_DEBUG bounds checks
-  // FA_DEBUG: index ranges of the outputs and the partial slots
-  const long long o_size = (long long)p.B * p.Sq * p.H * D, lse_size = (long long)p.B * p.H * p.Sq;
-  const long long part_rows = ((long long)p.B + p.pieces - 1) * p.H * p.Sq;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  static_assert(kSq >= 1 && kSq <= kDecMaxSq, "rows per CTA");
-  static_assert(kDecThreads == 128, "the scan below assumes four warps");
-  const int h = blockIdx.x, piece = blockIdx.y;
-  const int Sq = p.Sq;
-
-  if (tid == 0) {
-    *abort_flag = 0;
-    sInt[0] = p.B;
-    for (int st = 0; st < kStages; ++st) mbar_init(smem_u32(&full[st]), 1);
-    fence_barrier_init();
-  }
-
-  const DecPiece pc = dec_prologue<D>(p, h, piece, ab, sSum, sInt);
-  const long long T = pc.T, u0 = pc.u0, u1 = pc.u1, start_first = pc.start_first;
-  const int Pe = pc.Pe, b_first = pc.b_first;
-
-  // ---- the piece's tiles, streamed through the ring in list order (stream index k)
-  const long long n_tiles = u1 - u0;
-  DecWalk ld;  // the producer's position (thread 0)
-  ld.begin(p, p.B, 0, u0, u1);
-  long long issued = 0;
-  if (tid == 0 && n_tiles > 0) {
-    prefetch_tmap(&tmK);
-    prefetch_tmap(&tmV);
-    ld.begin(p, b_first, start_first, u0, u1);
-    while (issued < kStages && issued < n_tiles)
-      dec_issue_tile<Cfg>(p, &tmK, &tmV, smem_base, full, h, u0, u1, ld, issued, ab, smem_end);
-  }
-
-  const float c = p.scale_log2;
-  const int cp = tid % Cfg::kPairs, kg = tid / Cfg::kPairs;
-  long long k = 0;  // stream index of the next tile to consume
-  DecWalk w;
-  w.begin(p, b_first, start_first, u0, u1);
-  for (bool more = w.valid(p); more; more = w.next_seg(p, u0, u1)) {
-    const int b = w.b, n = w.n;
-    // q rows of (b, h) -> shared memory (fp32); rows >= Sq are zero
-    for (int e = tid; e < kSq * D; e += kDecThreads) {
-      const int i = e / D, col = e - i * D;
-      const long long qi = (((long long)b * Sq + i) * p.H + h) * D + col;
-      sQ[e] = (i < Sq && dbg_range(ab, qi, 1, o_size)) ? __bfloat162float(p.q[qi]) : 0.0f;
-    }
-    if (tid < kSq) sAlpha[tid] = 0.0f;  // rows past Sq keep alpha = 0 (their O stays 0)
-    __syncthreads();
-
-    // running state: warp w owns rows w and w + 4 (warp-uniform values)
-    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
-    // O accumulators of this thread: rows 0..kSq-1, columns 2 cp and 2 cp + 1, keys of group kg
-    float2 acc[kSq];
-#pragma unroll
-    for (int i = 0; i < kSq; ++i) acc[i] = make_float2(0.0f, 0.0f);
-
-    for (int t = w.t0; t < w.t1; ++t, ++k) {
-      const int st = (int)(k % kStages);
-      mbar_wait(smem_u32(&full[st]), (uint32_t)((k / kStages) & 1), ab);
-      const uint8_t* kgen = sm + Cfg::kOffKV + st * Cfg::kStageBytes;
-      const uint8_t* vgen = kgen + Cfg::kTileBytes;
-      // ---- A: half dot products, key kt = tid % 64, dims [half * D/2, half * D/2 + D/2)
-      {
-        const int kt = tid % kDecTile, half = tid / kDecTile;
-        float2 part[kSq];  // even / odd columns, packed f32x2 arithmetic
-#pragma unroll
-        for (int i = 0; i < kSq; ++i) part[i] = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int ch = 0; ch < D / 16; ++ch) {  // 16-byte chunks of this thread's half row
-          const int col0 = half * (D / 2) + ch * 8;
-          const int bx = col0 / 64, chunk = (col0 % 64) / 8;
-          const uint4 raw =
-              *reinterpret_cast<const uint4*>(kgen + bx * (kDecTile * 128) + sw128_offset(kt, chunk));
-          const uint32_t wv[4] = {raw.x, raw.y, raw.z, raw.w};
-          float2 kv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) kv[e] = make_float2(bf16lo_to_f32(wv[e]), bf16hi_to_f32(wv[e]));
-#pragma unroll
-          for (int i = 0; i < kSq; ++i) {  // rows past Sq have q = 0
-            const float4 qa = *reinterpret_cast<const float4*>(&sQ[i * D + col0]);
-            const float4 qb = *reinterpret_cast<const float4*>(&sQ[i * D + col0 + 4]);
-            part[i] = fma2(make_float2(qa.x, qa.y), kv[0], part[i]);
-            part[i] = fma2(make_float2(qa.z, qa.w), kv[1], part[i]);
-            part[i] = fma2(make_float2(qb.x, qb.y), kv[2], part[i]);
-            part[i] = fma2(make_float2(qb.z, qb.w), kv[3], part[i]);
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < kSq; ++i) sS[(half * kSq + i) * kDecTile + kt] = part[i].x + part[i].y;
-      }
-      __syncthreads();
-      // every thread has finished with the previous tile's slot: refill it (not after a wait
-      // gave up: that slot's barrier may still be waiting for bytes, and must not be armed twice)
-      if (tid == 0 && k > 0 && issued < n_tiles && !ab.raised())
-        dec_issue_tile<Cfg>(p, &tmK, &tmV, smem_base, full, h, u0, u1, ld, issued, ab, smem_end);
-      // ---- B: softmax bookkeeping, warp w -> rows w, w + 4
-#pragma unroll
-      for (int r = 0; r < (kSq + 3) / 4; ++r) {
-        const int i = warp + 4 * r;
-        if (i < Sq) {
-          const int pos = n - Sq + i;
-          const int kmin = p.win_l >= 0 ? pos - p.win_l : 0;
-          const int kmax = p.win_r >= 0 ? min(n - 1, pos + p.win_r) : n - 1;
-          float x[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int kt = lane + 32 * u, key = t * kDecTile + kt;
-            const float sc = (sS[i * kDecTile + kt] + sS[(kSq + i) * kDecTile + kt]) * c;
-            x[u] = (key >= kmin && key <= kmax) ? sc : -INFINITY;
-          }
-          float tmax = fmaxf(x[0], x[1]);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
-          const float m_new = fmaxf(m_run[r], tmax);
-          const float m_use = m_new == -INFINITY ? 0.0f : m_new;
-          const float alpha = m_run[r] == -INFINITY ? 0.0f : ex2_approx(m_run[r] - m_use);
-          float psum = 0.0f;
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const float pv = ex2_approx(x[u] - m_use);  // exp2(-inf) = 0
-            sP[i * kDecTile + lane + 32 * u] = pv;
-            psum += pv;
-          }
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
-          l_run[r] = l_run[r] * alpha + psum;
-          m_run[r] = m_new;
-          if (lane == 0) sAlpha[i] = alpha;
-        }
-      }
-      __syncthreads();
-      // ---- C: O_i = alpha_i O_i + sum_t P_i,t v_t over this thread's keys t = kg, kg + kKeyGroups, ...
-      {
-        const int col = 2 * cp, bx = col / 64, chunk = (col % 64) / 8, within = (col % 8) * 2;
-#pragma unroll
-        for (int i = 0; i < kSq; ++i) {  // rows past Sq stay 0
-          const float a = sAlpha[i];
-          acc[i] = mul2(acc[i], make_float2(a, a));
-        }
-        // keys past the sequence's end are skipped, not weighted by 0: the cache may hold a NaN there
-        const int kv_end = min(kDecTile, n - t * kDecTile);
-#pragma unroll 4
-        for (int kt = kg; kt < kv_end; kt += Cfg::kKeyGroups) {
-          const uint32_t wv = *reinterpret_cast<const uint32_t*>(vgen + bx * (kDecTile * 128) +
-                                                                 sw128_offset(kt, chunk) + within);
-          const float2 v = make_float2(bf16lo_to_f32(wv), bf16hi_to_f32(wv));
-#pragma unroll
-          for (int i = 0; i < kSq; ++i) {
-            const float pv = sP[i * kDecTile + kt];
-            acc[i] = fma2(make_float2(pv, pv), v, acc[i]);
-          }
-        }
-      }
-    }
-
-    // ---- segment end: combine the key groups' partial sums, normalise, write
-    __syncthreads();  // every thread is past phase C (sAlpha, sS are reused below)
-#pragma unroll
-    for (int i = 0; i < kSq; ++i) {
-      sRed[(kg * kSq + i) * D + 2 * cp] = acc[i].x;
-      sRed[(kg * kSq + i) * D + 2 * cp + 1] = acc[i].y;
-    }
-#pragma unroll
-    for (int r = 0; r < (kSq + 3) / 4; ++r) {  // row statistics: alpha slots -> 1 / l, S -> log2 l + m
-      const int i = warp + 4 * r;
-      if (i < Sq && lane == 0) {
-        sAlpha[i] = l_run[r] > 0.0f ? 1.0f / l_run[r] : 0.0f;
-        sS[i] = l_run[r] > 0.0f ? m_run[r] + __log2f(l_run[r]) : -INFINITY;
-      }
-    }
-    __syncthreads();
-    const int pf = dec_piece_of(T, Pe, w.start), pl = dec_piece_of(T, Pe, w.start + w.cnt - 1);
-    const size_t slot = (size_t)b + piece;  // partial slot of (b, this piece)
-    for (int e = tid; e < Sq * D; e += kDecThreads) {
-      const int i = e / D, col = e - i * D;
-      float v = 0.0f;
-#pragma unroll
-      for (int g = 0; g < Cfg::kKeyGroups; ++g) v += sRed[(g * kSq + i) * D + col];
-      v *= sAlpha[i];
-      const long long oi = (((long long)b * Sq + i) * p.H + h) * D + col;
-      const long long pi = (((long long)slot * p.H + h) * Sq + i) * D + col;
-      if (pf == pl) {
-        if (dbg_range(ab, oi, 1, o_size)) p.o[oi] = __float2bfloat16_rn(v);
-      } else if (dbg_range(ab, pi, 1, part_rows * D)) {
-        p.o_part[pi] = v;
-      }
-    }
-    if (tid < Sq) {
-      const float l2 = sS[tid];
-      const long long li = ((long long)b * p.H + h) * Sq + tid, pi = ((long long)slot * p.H + h) * Sq + tid;
-      if (pf == pl) {
-        if (dbg_range(ab, li, 1, lse_size)) p.lse[li] = l2 == -INFINITY ? -INFINITY : l2 * kDecLn2;
-      } else if (dbg_range(ab, pi, 1, part_rows)) {
-        p.lse_part[pi] = l2;
-      }
-    }
-    if (pf != pl) dec_arrive_merge<D>(p, b, h, pf, pl, ab, sInt);
-    __syncthreads();  // the next segment rewrites sQ, sAlpha and the last flag
-  }
-
-  // drain: loads issued past a wait that gave up must land before the CTA exits
-  if (tid == 0 && ab.raised()) {
-    for (long long j = max(0LL, issued - kStages); j < issued; ++j)
-      mbar_drain(smem_u32(&full[j % kStages]), (uint32_t)((j / kStages) & 1));
-  }
-}
-
-// ------------------------------------------------------------------ tensor-core variant (4 to 8 rows)
+// ------------------------------------------------------------------ the decode kernel
 //
-// With four or more new rows per sequence the CUDA-core dot products of the kernel above bound
-// it, not the cache read. This variant computes both products on the tensor core, transposed so
-// that the keys, not the few new rows, fill the 128 rows of a tcgen05 tile. Per tile of 128 keys
+// Both products run on the tensor core, transposed so that the keys, not the few new rows, fill
+// the 128 rows of a tcgen05 tile. Per tile of 128 keys
 // (two 64-key units of one sequence, each from its own page):
 //   S^T = K Q^T    M = 128 keys, N = 16 (the Sq <= 8 new rows, zero-padded), K = d
 //   O^T += V^T P^T M = d, N = 16, K = 128 keys          (d = 128)
@@ -622,8 +352,8 @@ __global__ void __launch_bounds__(kDecThreads)
 // tiles (a ring of 3 stages at d = 128, 6 at d = 64: one CTA per SM), warp 5 issues the products,
 // S(k + 1) ahead of P V(k). O is rescaled only when a row's maximum has grown by more than 2^8.
 // P is rounded to bf16 for the product, so O is divided by the sum of the rounded weights and
-// the log-sum-exp taken from the fp32 sum, as in the training forward. Work split, appends and
-// merge are those of the kernel above (pieces are counted in 64-key units).
+// the log-sum-exp taken from the fp32 sum, as in the training forward. Pieces are counted in
+// 64-key units (see the work split above).
 constexpr float kDecRescale = 8.0f;  // log2 units
 
 template <int D>
@@ -729,7 +459,7 @@ __device__ __forceinline__ bool dec_tc_issue(const DecParams& p, const CUtensorM
 
 template <int D, int kRows>
 __global__ void __launch_bounds__(kDecMmaThreads, 1)
-    fa_decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+    fa_decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const DecParams p) {
   using Cfg = DecTcCfg<D>;
   constexpr int kStages = Cfg::kStages;

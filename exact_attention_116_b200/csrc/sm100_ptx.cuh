@@ -272,14 +272,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
-// Same, 8 consecutive columns.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];" : FA_R8(0) : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[8]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" : FA_P8(0)::"memory");
-}
-
 // Wait for this thread's TMEM loads; the registers pass through so no use is hoisted above it.
 __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" : FA_P8(0), FA_P8(8), FA_P8(16), FA_P8(24)::"memory");
@@ -444,13 +436,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
   return bits_f2(d);
 }
-// Maximum of x over the 32 lanes of the warp (all lanes active), one instruction on sm_100a.
-__device__ __forceinline__ float warp_max_f32(float x) {
-  float r;
-  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
-  return r;
-}
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));

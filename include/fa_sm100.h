@@ -152,9 +152,12 @@ size_t fa_decode_workspace_bytes(int B, int Sq, int H, int d, int splits);
  * fa_decode_splits(B,Sq,H,d,max_pages*page_size). With splits > 1 a workspace of
  * fa_decode_workspace_bytes(B,Sq,H,d,splits) bytes (256-byte aligned, any contents) is used;
  * if `workspace` is NULL the call allocates it with cudaMallocAsync/cudaFreeAsync on `stream`.
- * One launch on `stream` with one piece per head; with more, a small kernel that zeroes the
- * arrival counters and the split kernel, launched as its programmatic dependent: each CTA
- * writes the new rows that fall in its piece, streams its piece, and the last piece of a
+ * Q K^T and P V run on the tensor cores (bf16 operands, fp32 accumulation; the weights P are
+ * rounded to bf16 for the product and O is divided by the sum of the rounded weights; LSE uses
+ * the fp32 sum). One launch on `stream` with one piece per head; with more, a small kernel
+ * that zeroes the arrival counters and the decode kernel, launched as its programmatic
+ * dependent: each CTA writes the new rows that fall in its piece, streams its piece, and the
+ * last piece of a
  * sequence to finish merges that sequence's partials. Sequence lengths or page indices that
  * are out of range are not read: the sequence counts as empty (or the page as zeros) and
  * fa_check() returns FA_ERR_DEVICE. Host-visible errors as fa_fwd (splits above 65535 is

@@ -1,10 +1,8 @@
 """GPU parity of the paged-KV decode (fa_decode_paged, through the C ABI) against the fp64 oracle.
 
-Up to three new rows the kernel computes scores, the online softmax and P·V in fp32 on the CUDA
-cores from the exact bf16 inputs (P is not rounded). From four rows on the tensor-core kernel
-computes Q K^T and P V with tcgen05 (fp32 accumulation), P rounded to bf16 and O divided by the
-sum of the rounded weights, as the training forward does. The forward's tolerances apply to
-both: per element |ΔO| <= 1e-2 + half a bf16 ulp of O and max |ΔLSE| <= 1e-3. Cases cover
+The kernel computes Q K^T and P V with tcgen05 (fp32 accumulation), P rounded to bf16 and O
+divided by the sum of the rounded weights, as the training forward does, so the forward's
+tolerances apply: per element |ΔO| <= 1e-2 + half a bf16 ulp of O and max |ΔLSE| <= 1e-3. Cases cover
 ragged lengths (empty, shorter than Sq, one key, page and tile boundaries), causal / window /
 full masks, Sq = 1..8, page sizes 64..512, piece counts 1, automatic and more pieces than tiles,
 pieces that span several sequences and sequences spread over several pieces, and the full
@@ -78,12 +76,12 @@ def test_decode_rows_and_page_sizes(Sq, page):
 
 @pytest.mark.parametrize("splits", [1, 0, 3])
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("Sq", [4, 5, 6, 7, 8])
+@pytest.mark.parametrize("Sq", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_decode_tensor_core_rows(Sq, d, splits):
-    # every row count of the tensor-core kernel: empty, shorter than Sq, one key, one tile, a
-    # tile and a key, several pages
+    # the rows of the 8-row build: empty, shorter than Sq, one key, one unit, a unit and a key,
+    # several pages
     cfg = DecodeConfig("tc_rows", 6, Sq, 2, d, 1, 700, 64, True, seed=70 + Sq + d)
-    check(cfg, lens=[0, Sq - 2, 1, 64, 65, 700], splits=splits, what=f"Sq={Sq} d={d} splits={splits}")
+    check(cfg, lens=[0, max(Sq - 2, 0), 1, 64, 65, 700], splits=splits, what=f"Sq={Sq} d={d} splits={splits}")
 
 
 @pytest.mark.parametrize("Sq", [4, 8])
