@@ -273,10 +273,12 @@ __device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[32], const uint32
       } else {
         pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
       }
-      if (kMasked) {
-        const int q0 = qbase + f;
-        pv.x = (q0 >= qlo && q0 <= qhi) ? pv.x : 0.0f;
-        pv.y = (q0 + 1 >= qlo && q0 + 1 <= qhi) ? pv.y : 0.0f;
+      if (kMasked) {  // query qbase + f is visible iff 0 <= qbase + f - qlo <= qhi - qlo
+        const bool any = qhi >= qlo;
+        const unsigned span = any ? (unsigned)(qhi - qlo) : 0u;
+        const int off = any ? qbase - qlo : -(1 << 30);
+        pv.x = ((unsigned)(off + f) <= span) ? pv.x : 0.0f;
+        pv.y = ((unsigned)(off + f + 1) <= span) ? pv.y : 0.0f;
       }
       pk[f >> 1] = pack_bf16x2(pv.x, pv.y);
     }

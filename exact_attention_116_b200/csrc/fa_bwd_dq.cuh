@@ -296,6 +296,10 @@ __global__ void __launch_bounds__(256, 1)
       if (kVarlen) seg_bounds(p.cu_seqlens, p.nseg, p.N, i * 128, seg_first, seg_last);
       for (int j = lo; j <= hi; ++j, ++n) {
         const bool masked = !fwd_tile_unmasked<kVarlen>(fp, i * 128, j, seg_first, seg_last) || (i * 128 + 127 >= p.N);
+        // key j * 128 + c is visible iff 0 <= j * 128 + c - kmin <= kmax - kmin (one unsigned
+        // compare per score; an empty range masks every key)
+        const unsigned span = kmax >= kmin ? (unsigned)(kmax - kmin) : 0u;
+        const int off = kmax >= kmin ? j * 128 - kmin : -(1 << 30);
         mbar_wait(bar(bars->s_full), n & 1, ab);
         tc_fence_after_sync();
         uint32_t pk[64];  // P(q, keys) as bf16 pairs
@@ -315,9 +319,8 @@ __global__ void __launch_bounds__(256, 1)
             }
             float2 pv = make_float2(ex2_approx(xv.x), ex2_approx(xv.y));
             if (masked) {
-              const int key = j * 128 + q4 * 32 + e;
-              pv.x = (key >= kmin && key <= kmax) ? pv.x : 0.0f;
-              pv.y = (key + 1 >= kmin && key + 1 <= kmax) ? pv.y : 0.0f;
+              pv.x = ((unsigned)(off + q4 * 32 + e) <= span) ? pv.x : 0.0f;
+              pv.y = ((unsigned)(off + q4 * 32 + e + 1) <= span) ? pv.y : 0.0f;
             }
             pk[q4 * 16 + (e >> 1)] = pack_bf16x2(pv.x, pv.y);
           }

@@ -251,11 +251,13 @@ __device__ __forceinline__ void fwd_row_max(float (&x)[128], bool masked, int kb
     }
   }
   if (masked) {
+    // key kbase + cc is visible iff 0 <= kbase + cc - kmin <= kmax - kmin: one unsigned compare
+    // per score (an empty range masks every key)
+    const bool any = kmax >= kmin;
+    const unsigned span = any ? (unsigned)(kmax - kmin) : 0u;
+    const int off = any ? kbase - kmin : -(1 << 30);
 #pragma unroll
-    for (int cc = 0; cc < 128; ++cc) {
-      const int key = kbase + cc;
-      x[cc] = ((key >= kmin) & (key <= kmax)) ? x[cc] : -INFINITY;
-    }
+    for (int cc = 0; cc < 128; ++cc) x[cc] = ((unsigned)(off + cc) <= span) ? x[cc] : -INFINITY;
   }
   float mx[8];
 #pragma unroll
