@@ -17,9 +17,11 @@
 //   warp 0       work fetch (atomic counter, head-grouped order: bwd_decode) and TMA producer: K_j, V_j
 //                per item; Q_i with LSE2_i, D_i in two slots; dO_i in one slot
 //   warp 1       MMA issuer, TMEM owner
-//   warps 4-7    dQ: TMEM -> registers -> shared staging -> TMA reduce-add into the accumulator
-//   warps 8-11   P/dS for query columns [0, 64) of each tile; dK epilogue
-//   warps 12-15  P/dS for query columns [64, 128); dV epilogue
+//   warps 4-7    dQ: TMEM -> registers -> shared staging -> TMA reduce-add into the accumulator;
+//                at d = 64 also the dK and dV epilogue of each item (dK / dV have two TMEM buffers
+//                there, so the P/dS warps go on to the next item meanwhile)
+//   warps 8-11   P/dS for query columns [0, 64) of each tile; dK epilogue (d = 128)
+//   warps 12-15  P/dS for query columns [64, 128); dV epilogue (d = 128)
 // TMEM: dK [0,D), dV [D,2D), dP^T / dQ [2D, 2D+128), S^T / P^T [2D+128, 2D+256).
 // Per Q tile i the MMA warp issues dP^T = V dO_i^T, dV += P^T dO_i (P^T from TMEM), then
 // S^T for tile i+1 (= K Q_{i+1}^T), dQ_i = dS K_j and dK += dS^T Q_i (dS^T in shared memory,
@@ -294,6 +296,7 @@ __global__ void __launch_bounds__(512, 1)
   using Cfg = BwdCfg<D>;
   static_assert(sizeof(BwdBars) <= 256, "barrier block");
   constexpr bool kDqFirst = D == 128;  // MMA order per Q tile: see the issuer
+  constexpr bool kEpiInDq = Cfg::kKVSlots == 2;  // d = 64: the dQ warps store dK and dV
   extern __shared__ uint8_t smem_raw[];
   const uint32_t smem_base = smem_u32(smem_raw);
   BwdBars* bars = reinterpret_cast<BwdBars*>(smem_raw + Cfg::kOffBar);
@@ -320,9 +323,9 @@ __global__ void __launch_bounds__(512, 1)
     bars->abort_flag = 0;
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(bars->kv_full[s]), 1);
-      mbar_init(bar(bars->kv_empty[s]), 2);
+      mbar_init(bar(bars->kv_empty[s]), kEpiInDq ? 1 : 2);
       mbar_init(bar(bars->dkv_full[s]), 1);
-      mbar_init(bar(bars->dkv_empty[s]), 256);
+      mbar_init(bar(bars->dkv_empty[s]), kEpiInDq ? 128 : 256);
       mbar_init(bar(bars->q_full[s]), 1);
       mbar_init(bar(bars->q_empty[s]), 1);
       mbar_init(bar(bars->item_full[s]), 1);
@@ -526,7 +529,7 @@ __global__ void __launch_bounds__(512, 1)
     // memory, and the TMA unit adds it into the accumulator in global memory, 64 columns per round.
     const int row = threadIdx.x - 128;
     const uint32_t tDQ = tmem + ((uint32_t)(row & ~31) << 16) + Cfg::kColDP;
-    uint32_t n = 0;
+    uint32_t n = 0, items = 0;
     for (uint32_t it = 0;; ++it) {
       const int w = bwd_take_item(bars, it, lane_id() == 0, ab);
       if (w >= p.num_items) break;
@@ -573,6 +576,54 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
       }
+      if constexpr (kEpiInDq) {
+        // dK (times scale) and dV -> bf16 -> this item's K_j / V_j buffers -> TMA store
+        const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
+        mbar_wait(bar(bars->dkv_full[kvs]), kvphase, ab);
+        tc_fence_after_sync();
+        const uint32_t lane_field = (uint32_t)((row & ~31) << 16);
+#pragma unroll 1
+        for (int g = 0; g < 2; ++g) {
+          const uint32_t src =
+              tmem + lane_field + (g ? (kvs ? Cfg::kColDV1 : Cfg::kColDV) : (kvs ? Cfg::kColDK1 : Cfg::kColDK));
+          const uint32_t stage_buf = g ? sVs(items) : sKs(items);
+          const float mult = g ? 1.0f : p.scale;
+#pragma unroll
+          for (int cc = 0; cc < D; cc += 32) {
+            uint32_t v[32];
+            tmem_ld32(src + cc, v);
+            tmem_wait_ld(v);
+            const uint32_t bx = stage_buf + (cc >> 6) * 16384;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                w4[e] = pack_bf16x2(__uint_as_float(v[ch * 8 + 2 * e]) * mult,
+                                    __uint_as_float(v[ch * 8 + 2 * e + 1]) * mult);
+              st_shared_v4(bx + sw128_offset(row, ((cc & 63) >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
+            }
+          }
+        }
+        tc_fence_before_sync();
+        mbar_arrive(bar(bars->dkv_empty[kvs]));
+        fence_proxy_async_smem();
+        named_bar_sync(3, 128);
+        if (row == 0) {
+#pragma unroll
+          for (int g = 0; g < 2; ++g)
+#pragma unroll
+            for (int bx = 0; bx < Cfg::kBoxes; ++bx) {
+              const uint32_t sb = (g ? sVs(items) : sKs(items)) + bx * 16384;
+              if (dbg_tma(ab, bx * 64, j * 128, h, b, D, p.N, p.H, p.B, 2, sb, 16384, smem_base, smem_end))
+                tma_store_4d(g ? &tmdV : &tmdK, sb, bx * 64, j * 128, h, b);
+            }
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(bar(bars->kv_empty[kvs]));
+        }
+      }
+      ++items;
     }
     if (row == 0) bulk_wait_group0();
   } else if (warp >= 8) {
@@ -666,42 +717,45 @@ __global__ void __launch_bounds__(512, 1)
         if (++qs == 2) { qs = 0; qphase ^= 1; }
       }
 
-      // Epilogue: dK (group 0, times scale) or dV (group 1) -> bf16 -> the K_j / V_j buffer -> TMA store.
-      const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
-      mbar_wait(bar(bars->dkv_full[kvs]), kvphase, ab);
-      tc_fence_after_sync();
-      const uint32_t src =
-          tmem + lane_field + (grp ? (kvs ? Cfg::kColDV1 : Cfg::kColDV) : (kvs ? Cfg::kColDK1 : Cfg::kColDK));
-      const uint32_t stage_buf = grp ? sVs(items) : sKs(items);  // this item's K/V slot: its MMAs are done
-      const float mult = grp ? 1.0f : p.scale;
+      // Epilogue (d = 128; at d = 64 the dQ warps do it): dK (group 0, times scale) or dV
+      // (group 1) -> bf16 -> the K_j / V_j buffer -> TMA store.
+      if constexpr (!kEpiInDq) {
+        const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
+        mbar_wait(bar(bars->dkv_full[kvs]), kvphase, ab);
+        tc_fence_after_sync();
+        const uint32_t src =
+            tmem + lane_field + (grp ? (kvs ? Cfg::kColDV1 : Cfg::kColDV) : (kvs ? Cfg::kColDK1 : Cfg::kColDK));
+        const uint32_t stage_buf = grp ? sVs(items) : sKs(items);  // this item's K/V slot: its MMAs are done
+        const float mult = grp ? 1.0f : p.scale;
 #pragma unroll 1
-      for (int cc = 0; cc < D; cc += 32) {
-        uint32_t v[32];
-        tmem_ld32(src + cc, v);
-        tmem_wait_ld(v);
-        const uint32_t bx = stage_buf + (cc >> 6) * 16384;
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32(src + cc, v);
+          tmem_wait_ld(v);
+          const uint32_t bx = stage_buf + (cc >> 6) * 16384;
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          uint32_t w4[4];
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t w4[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            w4[e] = pack_bf16x2(__uint_as_float(v[ch * 8 + 2 * e]) * mult, __uint_as_float(v[ch * 8 + 2 * e + 1]) * mult);
-          st_shared_v4(bx + sw128_offset(row, ((cc & 63) >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
+            for (int e = 0; e < 4; ++e)
+              w4[e] = pack_bf16x2(__uint_as_float(v[ch * 8 + 2 * e]) * mult, __uint_as_float(v[ch * 8 + 2 * e + 1]) * mult);
+            st_shared_v4(bx + sw128_offset(row, ((cc & 63) >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
+          }
         }
-      }
-      tc_fence_before_sync();
-      mbar_arrive(bar(bars->dkv_empty[kvs]));
-      fence_proxy_async_smem();
-      named_bar_sync(1 + grp, 128);
-      if (row == 0) {
+        tc_fence_before_sync();
+        mbar_arrive(bar(bars->dkv_empty[kvs]));
+        fence_proxy_async_smem();
+        named_bar_sync(1 + grp, 128);
+        if (row == 0) {
 #pragma unroll
-        for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-          if (dbg_tma(ab, bx * 64, j * 128, h, b, D, p.N, p.H, p.B, 2, stage_buf + bx * 16384, 16384, smem_base,
-                      smem_end))
-            tma_store_4d(grp ? &tmdV : &tmdK, stage_buf + bx * 16384, bx * 64, j * 128, h, b);
-        bulk_commit_group();
-        bulk_wait_group_read0();
-        mbar_arrive(bar(bars->kv_empty[kvs]));
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+            if (dbg_tma(ab, bx * 64, j * 128, h, b, D, p.N, p.H, p.B, 2, stage_buf + bx * 16384, 16384, smem_base,
+                        smem_end))
+              tma_store_4d(grp ? &tmdV : &tmdK, stage_buf + bx * 16384, bx * 64, j * 128, h, b);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(bar(bars->kv_empty[kvs]));
+        }
       }
       ++items;
     }
