@@ -11,10 +11,10 @@
 // Both products still run on the tensor core (see the kernel below): on the CUDA cores the dot
 // products and P V of even one to four rows kept the kernel from the cache read.
 //
-// Work split (split-KV, balanced over the whole batch): for each head, the 64-key tiles that
+// Work split (split-KV, balanced over the whole batch): for each head, the 64-key units that
 // the new rows can see are listed sequence after sequence, and that list is cut into P equal
 // contiguous pieces, one CTA each (grid (H, P), P chosen so that the grid fills the GPU once).
-// Every CTA therefore streams the same number of tiles (within one), whatever the mix of
+// Every CTA therefore streams the same number of units (within one), whatever the mix of
 // lengths, and no CTA waits in a second wave. A piece may cover the end of one sequence, some
 // whole sequences and the start of another: the CTA keeps one running state per sequence
 // part ("segment") and its TMA ring runs on across segment boundaries. A sequence that lies
@@ -26,11 +26,11 @@
 // is launched as its programmatic dependent and waits for it only before its first arrival.
 //
 // CTAs of the same piece for consecutive heads are launched next to each other (head is the
-// fastest grid index) and walk the same tiles, so the 128-byte head slices of one cache row
+// fastest grid index) and walk the same units, so the 128-byte head slices of one cache row
 // (H x d bf16, contiguous) are read at about the same time.
 //
 // With new K/V rows given (flash_attn_with_kvcache's in-place update of the cache), the CTA
-// whose piece holds a new row's tile writes that row's d columns of its head into the cache
+// whose piece holds a new row's unit writes that row's d columns of its head into the cache
 // before it loads any tile: every new row is visible to the newest query row, so exactly one
 // piece of each head holds it, and no other CTA reads those bytes.
 #pragma once
@@ -39,10 +39,10 @@
 
 namespace fa {
 
-constexpr int kDecMaxSq = 8;  // new query rows per call
-constexpr int kDecTile = 64;  // keys per tile
-constexpr int kDecThreads = 128;
-constexpr int kDecMmaThreads = 224;  // tensor-core kernel: four softmax warps, a producer, two MMA issuers
+constexpr int kDecMaxSq = 8;         // new query rows per call
+constexpr int kDecTile = 64;         // keys per unit of the work split (one TMA box; a kernel tile is two)
+constexpr int kDecThreads = 128;     // the four softmax warps, which also run the set-up and the merge
+constexpr int kDecMmaThreads = 224;  // the decode kernel's CTA: softmax warps, a producer, two MMA issuers
 constexpr float kDecLn2 = 0.69314718055994530942f;
 
 // Warp-collective TMEM load of 8 consecutive 32-bit columns: thread t of the warp reads lane
@@ -70,8 +70,6 @@ __device__ __forceinline__ float warp_max_f32(float x) {
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
-
-
 
 struct DecParams {
   int B, Sq, H, page_size, max_pages, num_pages;
@@ -102,9 +100,9 @@ __device__ __forceinline__ int dec_len(const DecParams& p, int b, bool report) {
   return n;
 }
 
-// Number of 64-key tiles, from tile vt0 on, that the rows of a sequence of n keys can see
+// Number of 64-key units, from unit vt0 on, that the rows of a sequence of n keys can see
 // (0 for an empty sequence; at least 1 otherwise: each row sees its own key).
-__device__ __forceinline__ int dec_vis_tiles(const DecParams& p, int n, int& vt0) {
+__device__ __forceinline__ int dec_vis_units(const DecParams& p, int n, int& vt0) {
   vt0 = 0;
   if (n <= 0) return 0;
   const int pos0 = n - p.Sq, pos1 = n - 1;
@@ -114,42 +112,41 @@ __device__ __forceinline__ int dec_vis_tiles(const DecParams& p, int n, int& vt0
   return vis_hi / kDecTile + 1 - vt0;
 }
 
-// The next sequence after b with a visible tile (p.B when there is none), its length, first
-// visible tile and tile count.
+// The next sequence after b with a visible unit (p.B when there is none), its length, first
+// visible unit and unit count.
 __device__ __forceinline__ int dec_next_seq(const DecParams& p, int b, int& n, int& vt0, int& cnt) {
   for (++b; b < p.B; ++b) {
     n = dec_len(p, b, false);
-    cnt = dec_vis_tiles(p, n, vt0);
+    cnt = dec_vis_units(p, n, vt0);
     if (cnt > 0) return b;
   }
   return p.B;
 }
 
-// Pieces: piece r of P <= T covers units [T r / P, T (r + 1) / P) of a head's T tiles (at least
+// Pieces: piece r of P <= T covers units [T r / P, T (r + 1) / P) of a head's T units (at least
 // one); the piece that holds unit u (0 <= u < T) is the largest r with T r / P <= u.
 __device__ __forceinline__ long long dec_piece_lo(long long T, int P, int r) { return T * r / P; }
 __device__ __forceinline__ int dec_piece_of(long long T, int P, long long u) {
   return (int)(((u + 1) * P - 1) / T);
 }
 
-// A walk over the tiles of one piece, segment by segment: sequence b (n keys), whose visible
-// tiles start at unit `start` of the list, contributes its tiles [t0, t1).
+// A walk over the 64-key units of one piece, segment by segment: sequence b (n keys), whose
+// visible units start at position `start` of the list, contributes its units [t0, t1).
 struct DecWalk {
-  int b, n, vt0, cnt, t0, t1, t;
+  int b, n, vt0, cnt, t0, t1;
   long long start;
   __device__ __forceinline__ void clip(long long u0, long long u1) {
     t0 = vt0 + (int)max(0LL, u0 - start);
     t1 = vt0 + (int)min((long long)cnt, u1 - start);
-    t = t0;
   }
   // first segment: sequence b0 starting at unit s0 (b0 == p.B: the piece is empty)
   __device__ __forceinline__ void begin(const DecParams& p, int b0, long long s0, long long u0, long long u1) {
     b = b0;
     start = s0;
-    n = vt0 = cnt = t0 = t1 = t = 0;
+    n = vt0 = cnt = t0 = t1 = 0;
     if (b < p.B) {
       n = dec_len(p, b, false);
-      cnt = dec_vis_tiles(p, n, vt0);
+      cnt = dec_vis_units(p, n, vt0);
       clip(u0, u1);
     }
   }
@@ -167,8 +164,9 @@ struct DecWalk {
   __device__ __forceinline__ bool valid(const DecParams& p) const { return b < p.B; }
 };
 
-// A CTA's piece of a head's tile list: the list's length T, the pieces in use Pe, this piece's
-// units [u0, u1) and its first segment (sequence b_first, whose tiles start at unit start_first).
+// A CTA's piece of a head's unit list: the list's length T, the pieces in use Pe, this piece's
+// units [u0, u1) and its first segment (sequence b_first, whose units start at position
+// start_first).
 struct DecPiece {
   long long T, u0, u1, start_first;
   int Pe, b_first;
@@ -176,8 +174,8 @@ struct DecPiece {
 
 // Set-up of the decode kernel (all threads of the CTA; threads 0 .. kDecThreads - 1 do the work,
 // the others only meet the barriers): the piece from the lengths (a
-// block-wide prefix sum of tile counts, each thread summing a contiguous run of sequences); O = 0,
-// LSE = -inf for the sequences without a visible tile (written by piece b % P); with new K/V rows
+// block-wide prefix sum of unit counts, each thread summing a contiguous run of sequences); O = 0,
+// LSE = -inf for the sequences without a visible unit (written by piece b % P); with new K/V rows
 // given, this piece's new rows of head h written into the cache before any tile load. sSum holds
 // 5 and sInt 1 values of scratch in shared memory.
 template <int D>
@@ -187,14 +185,14 @@ __device__ __forceinline__ DecPiece dec_prologue(const DecParams& p, int h, int 
   const int Sq = p.Sq, P = p.pieces;
   const long long o_size = (long long)p.B * p.Sq * p.H * D, lse_size = (long long)p.B * p.H * p.Sq;
   const long long cache_size = (long long)p.num_pages * p.page_size * p.H * D;
-  // ---- tile counts of all sequences, prefix sums (each thread a contiguous run of sequences)
+  // ---- unit counts of all sequences, prefix sums (each thread a contiguous run of sequences)
   const int run = (p.B + kDecThreads - 1) / kDecThreads;
   const int rb0 = min(p.B, tid * run), rb1 = min(p.B, rb0 + run);
   const bool report = h == 0 && piece == 0;
   long long mine = 0;
   for (int b = rb0; b < rb1; ++b) {
     int vt0;
-    mine += dec_vis_tiles(p, dec_len(p, b, report), vt0);
+    mine += dec_vis_units(p, dec_len(p, b, report), vt0);
   }
   long long incl = mine;
 #pragma unroll
@@ -211,16 +209,16 @@ __device__ __forceinline__ DecPiece dec_prologue(const DecParams& p, int h, int 
     T += sw;
     if (w < warp) excl += sw;
   }
-  // With fewer tiles than CTAs only the first T pieces get one each (every piece in use then
-  // holds at least one tile, which the arrival count and the merge rely on).
+  // With fewer units than CTAs only the first T pieces get one each (every piece in use then
+  // holds at least one unit, which the arrival count and the merge rely on).
   const int Pe = (int)min((long long)P, T);
   const long long u0 = piece < Pe ? dec_piece_lo(T, Pe, piece) : T;
   const long long u1 = piece < Pe ? dec_piece_lo(T, Pe, piece + 1) : T;
-  if (u0 < u1 && excl <= u0 && u0 < excl + mine) {  // this thread's run holds the piece's first tile
+  if (u0 < u1 && excl <= u0 && u0 < excl + mine) {  // this thread's run holds the piece's first unit
     long long s = excl;
     for (int b = rb0; b < rb1; ++b) {
       int vt0;
-      const int c = dec_vis_tiles(p, dec_len(p, b, false), vt0);
+      const int c = dec_vis_units(p, dec_len(p, b, false), vt0);
       if (u0 < s + c) {
         sInt[0] = b;
         sSum[4] = s;
@@ -233,10 +231,10 @@ __device__ __forceinline__ DecPiece dec_prologue(const DecParams& p, int h, int 
   const int b_first = sInt[0];
   const long long start_first = b_first < p.B ? sSum[4] : 0;
 
-  // ---- sequences without a visible tile (empty): O = 0, LSE = -inf, written by piece b % P
+  // ---- sequences without a visible unit (empty): O = 0, LSE = -inf, written by piece b % P
   for (int b = piece; b < p.B && tid < kDecThreads; b += P) {
     int vt0;
-    if (dec_vis_tiles(p, dec_len(p, b, false), vt0) != 0) continue;
+    if (dec_vis_units(p, dec_len(p, b, false), vt0) != 0) continue;
     for (int e = tid; e < Sq * D; e += kDecThreads) {
       const int i = e / D, col = e - i * D;
       const long long oi = (((long long)b * Sq + i) * p.H + h) * D + col;
@@ -246,7 +244,7 @@ __device__ __forceinline__ DecPiece dec_prologue(const DecParams& p, int h, int 
     if (tid < Sq && dbg_range(ab, li, 1, lse_size)) p.lse[li] = -INFINITY;
   }
 
-  // ---- new rows in this piece's tiles: head h's columns go into the cache before any tile load
+  // ---- new rows in this piece's units: head h's columns go into the cache before any tile load
   if (p.k_new != nullptr) {
     constexpr int kChunks = D / 8;  // 16-byte chunks of one head's row
     bool wrote = false;
