@@ -577,7 +577,7 @@ def run_gpu_fp8(args):
                 "d2h_bytes_per_step": B * N * H * d * 2 + B * H * N * 4,
                 "pipelining": "copy-in, fa_fwd_fp8 and copy-out of consecutive steps on three streams with two "
                               "device buffer sets (every step copies its own inputs and outputs)"},
-        "gpu_launches": args.steps,
+        "gpu_launches": 2 * args.steps,  # the forward's work-counter reset and the forward
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -802,7 +802,9 @@ def run_gpu(args):
                 "d2h_bytes_per_step": 4 * t_bytes + B * H * N * 4,
                 "pipelining": "copy-in, fa_fwd + fa_bwd and copy-out of consecutive steps on three streams with two "
                               "device buffer sets (every step copies its own inputs and outputs)"},
-        "gpu_launches": 4 * args.steps,
+        # per step: the forward's work-counter reset and the forward; the backward's
+        # preprocess, main kernel and dQ conversion
+        "gpu_launches": 5 * args.steps,
         "clocks": clocks,
     }
     if not args.no_extras:
