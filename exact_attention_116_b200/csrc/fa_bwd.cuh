@@ -19,9 +19,14 @@
 //   warp 1       MMA issuer, TMEM owner
 //   warps 4-7    dQ: TMEM -> registers -> shared staging -> TMA reduce-add into the accumulator;
 //                at d = 64 also the dK and dV epilogue of each item (dK / dV have two TMEM buffers
-//                there, so the P/dS warps go on to the next item meanwhile)
-//   warps 8-11   P/dS for query columns [0, 64) of each tile; dK epilogue (d = 128)
-//   warps 12-15  P/dS for query columns [64, 128); dV epilogue (d = 128)
+//                there, so the P/dS warps go on to the next item meanwhile), staged in the
+//                item's K/V buffers; at d = 128 the dV epilogue, staged in the dQ buffer
+//   warps 8-11   P/dS for query columns [0, 64) of each tile; at d = 128 the dK epilogue of
+//                columns [0, 64), staged in the dS buffer
+//   warps 12-15  P/dS for query columns [64, 128); at d = 128 dK columns [64, 128)
+// At d = 128 the epilogue thus leaves K_j and V_j alone: their single slot is released by the
+// MMA warp's commit after the item's last product, and the next item's K/V load overlaps the
+// epilogue.
 // TMEM: dK [0,D), dV [D,2D), dP^T / dQ [2D, 2D+128), S^T / P^T [2D+128, 2D+256).
 // Per Q tile i the MMA warp issues dP^T = V dO_i^T, dV += P^T dO_i (P^T from TMEM), then
 // S^T for tile i+1 (= K Q_{i+1}^T), dQ_i = dS K_j and dK += dS^T Q_i (dS^T in shared memory,
@@ -323,9 +328,9 @@ __global__ void __launch_bounds__(512, 1)
     bars->abort_flag = 0;
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(bars->kv_full[s]), 1);
-      mbar_init(bar(bars->kv_empty[s]), kEpiInDq ? 1 : 2);
+      mbar_init(bar(bars->kv_empty[s]), 1);
       mbar_init(bar(bars->dkv_full[s]), 1);
-      mbar_init(bar(bars->dkv_empty[s]), kEpiInDq ? 128 : 256);
+      mbar_init(bar(bars->dkv_empty[s]), kEpiInDq ? 128 : 384);
       mbar_init(bar(bars->q_full[s]), 1);
       mbar_init(bar(bars->q_empty[s]), 1);
       mbar_init(bar(bars->item_full[s]), 1);
@@ -518,6 +523,9 @@ __global__ void __launch_bounds__(512, 1)
           qphase = nqphase;
         }
         mma_commit(bar(bars->dkv_full[kvs]));
+        // d = 128: the epilogue stages through the dS and dQ buffers, so K_j and V_j are free
+        // once the item's products are done (d = 64 stages through them: the dQ warps release)
+        if constexpr (!kEpiInDq) mma_commit(bar(bars->kv_empty[kvs]));
         ++items;
       }
       mma_commit(bar(bars->mma_done));
@@ -622,6 +630,42 @@ __global__ void __launch_bounds__(512, 1)
           bulk_wait_group_read0();
           mbar_arrive(bar(bars->kv_empty[kvs]));
         }
+      } else {
+        // d = 128: dV -> bf16 -> the dQ staging buffer (two 64-column boxes) -> TMA store, once
+        // the item's last dQ reduction has read that buffer; the next item's first staging
+        // round waits for this store to read it in turn (the same bulk-group wait)
+        const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
+        mbar_wait(bar(bars->dkv_full[kvs]), kvphase, ab);
+        tc_fence_after_sync();
+        if (row == 0) bulk_wait_group_read0();
+        named_bar_sync(3, 128);
+        const uint32_t src = tmem + ((uint32_t)(row & ~31) << 16) + Cfg::kColDV;
+#pragma unroll 1
+        for (int cc = 0; cc < D; cc += 32) {
+          uint32_t v[32];
+          tmem_ld32(src + cc, v);
+          tmem_wait_ld(v);
+          const uint32_t bx = sDQ + (cc >> 6) * 16384;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w4[e] = pack_bf16x2(__uint_as_float(v[ch * 8 + 2 * e]), __uint_as_float(v[ch * 8 + 2 * e + 1]));
+            st_shared_v4(bx + sw128_offset(row, ((cc & 63) >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+        tc_fence_before_sync();
+        mbar_arrive(bar(bars->dkv_empty[kvs]));
+        fence_proxy_async_smem();
+        named_bar_sync(3, 128);
+        if (row == 0) {
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+            if (dbg_tma(ab, bx * 64, j * 128, h, b, D, p.N, p.H, p.B, 2, sDQ + bx * 16384, 16384, smem_base, smem_end))
+              tma_store_4d(&tmdV, sDQ + bx * 16384, bx * 64, j * 128, h, b);
+          bulk_commit_group();
+        }
       }
       ++items;
     }
@@ -717,29 +761,28 @@ __global__ void __launch_bounds__(512, 1)
         if (++qs == 2) { qs = 0; qphase ^= 1; }
       }
 
-      // Epilogue (d = 128; at d = 64 the dQ warps do it): dK (group 0, times scale) or dV
-      // (group 1) -> bf16 -> the K_j / V_j buffer -> TMA store.
+      // Epilogue (d = 128; at d = 64 the dQ warps do it): dK times scale, columns [64 grp,
+      // 64 grp + 64) -> bf16 -> box grp of the dS buffer (free: the item's last dQ and dK have
+      // read it) -> TMA store. The group's next dS waits for the store to read the box.
       if constexpr (!kEpiInDq) {
         const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
         mbar_wait(bar(bars->dkv_full[kvs]), kvphase, ab);
         tc_fence_after_sync();
-        const uint32_t src =
-            tmem + lane_field + (grp ? (kvs ? Cfg::kColDV1 : Cfg::kColDV) : (kvs ? Cfg::kColDK1 : Cfg::kColDK));
-        const uint32_t stage_buf = grp ? sVs(items) : sKs(items);  // this item's K/V slot: its MMAs are done
-        const float mult = grp ? 1.0f : p.scale;
+        const uint32_t src = tmem + lane_field + Cfg::kColDK + 64 * grp;
+        const uint32_t bx = sDS + grp * 16384;
 #pragma unroll 1
-        for (int cc = 0; cc < D; cc += 32) {
+        for (int cc = 0; cc < 64; cc += 32) {
           uint32_t v[32];
           tmem_ld32(src + cc, v);
           tmem_wait_ld(v);
-          const uint32_t bx = stage_buf + (cc >> 6) * 16384;
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t w4[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              w4[e] = pack_bf16x2(__uint_as_float(v[ch * 8 + 2 * e]) * mult, __uint_as_float(v[ch * 8 + 2 * e + 1]) * mult);
-            st_shared_v4(bx + sw128_offset(row, ((cc & 63) >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
+              w4[e] = pack_bf16x2(__uint_as_float(v[ch * 8 + 2 * e]) * p.scale,
+                                  __uint_as_float(v[ch * 8 + 2 * e + 1]) * p.scale);
+            st_shared_v4(bx + sw128_offset(row, (cc >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
           }
         }
         tc_fence_before_sync();
@@ -747,15 +790,12 @@ __global__ void __launch_bounds__(512, 1)
         fence_proxy_async_smem();
         named_bar_sync(1 + grp, 128);
         if (row == 0) {
-#pragma unroll
-          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            if (dbg_tma(ab, bx * 64, j * 128, h, b, D, p.N, p.H, p.B, 2, stage_buf + bx * 16384, 16384, smem_base,
-                        smem_end))
-              tma_store_4d(grp ? &tmdV : &tmdK, stage_buf + bx * 16384, bx * 64, j * 128, h, b);
+          if (dbg_tma(ab, 64 * grp, j * 128, h, b, D, p.N, p.H, p.B, 2, bx, 16384, smem_base, smem_end))
+            tma_store_4d(&tmdK, bx, 64 * grp, j * 128, h, b);
           bulk_commit_group();
           bulk_wait_group_read0();
-          mbar_arrive(bar(bars->kv_empty[kvs]));
         }
+        named_bar_sync(1 + grp, 128);
       }
       ++items;
     }
