@@ -13,7 +13,7 @@
 //                       dQ_i partial products are added into the fp32 accumulator in global memory
 //   fa_dq_convert_kernel  dQ = bf16(accumulator)
 //
-// fa_bwd_kernel roles (512 threads):
+// fa_bwd_kernel roles (512 or 768 threads):
 //   warp 0       work fetch (atomic counter, head-grouped order: bwd_decode) and TMA producer: K_j, V_j
 //                per item; Q_i with LSE2_i, D_i in two slots; dO_i in one slot
 //   warp 1       MMA issuer, TMEM owner
@@ -21,9 +21,9 @@
 //                at d = 64 also the dK and dV epilogue of each item (dK / dV have two TMEM buffers
 //                there, so the P/dS warps go on to the next item meanwhile), staged in the
 //                item's K/V buffers; at d = 128 the dV epilogue, staged in the dQ buffer
-//   warps 8-11   P/dS for query columns [0, 64) of each tile; at d = 128 the dK epilogue of
-//                columns [0, 64), staged in the dS buffer
-//   warps 12-15  P/dS for query columns [64, 128); at d = 128 dK columns [64, 128)
+//   warps 8-      P/dS in groups of four warps, each for W query columns of every tile: four
+//                groups (W = 32, 768 threads) at d = 64, two (W = 64, 512 threads) at d = 128; at
+//                d = 128 each group also stores dK columns [W g, W g + W), staged in the dS buffer
 // At d = 128 the epilogue thus leaves K_j and V_j alone: their single slot is released by the
 // MMA warp's commit after the item's last product, and the next item's K/V load overlaps the
 // epilogue.
@@ -145,7 +145,13 @@ __global__ void __launch_bounds__(256) fa_dq_convert_kernel(const float* __restr
 
 template <int D>
 struct BwdCfg {
-  static constexpr int kThreads = 512;
+  // P/dS groups of four warps, kGroupCols query columns each: four at d = 64, where their
+  // exponentials and dS bound the kernel, two at d = 128, where the dQ reduction does and the
+  // smaller register budget of a 768-thread CTA measured slower
+  static constexpr int kGroups = (D == 64) ? 4 : 2;
+  static constexpr int kGroupCols = 128 / kGroups;
+  static constexpr int kThreads = 256 + 128 * kGroups;
+  static constexpr uint32_t kItemConsumers = 1 + 4 + 4 * kGroups;  // MMA thread, dQ and P/dS warps
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBoxes = D / 64;
   // d = 64: two K/V slots and two dK/dV TMEM buffers, alternating per work item, so that the
@@ -180,9 +186,6 @@ struct BwdBars {
   uint32_t tmem_base;
   int abort_flag;
 };
-
-// Consumers of a fetched item: the MMA thread, 4 dQ warps and 8 P/dS warps (one arrival each).
-constexpr uint32_t kBwdItemConsumers = 13;
 
 // Item w -> (b, h, j), in two phases:
 //   1. KV tiles [0, num_kv_tiles - tail_tiles): groups of head_group heads in order, inside a
@@ -252,23 +255,21 @@ __device__ __forceinline__ bool bwd_tile_unmasked(const BwdParams& p, int j, int
   return true;
 }
 
-// P^T for 64 query columns of this thread's key row: exp2(S^T * c - LSE_q * log2(e)), zero
+// P^T for W query columns of this thread's key row: exp2(S^T * c - LSE_q * log2(e)), zero
 // where masked (kMasked), packed to bf16 pairs (even column low). nlse2 holds -LSE * log2(e)
-// of the same 64 queries.
-template <bool kMasked, bool kAlibi = false>
-__device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[32], const uint32_t (&s1)[32], float c,
-                                          const float* nlse2, int qbase, int qlo, int qhi, uint32_t (&pk)[32],
-                                          float d0 = 0.0f, float nslope2 = 0.0f) {
+// of the same W queries.
+template <int W, bool kMasked, bool kAlibi = false>
+__device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[W], float c, const float* nlse2, int qbase, int qlo,
+                                          int qhi, uint32_t (&pk)[W / 2], float d0 = 0.0f, float nslope2 = 0.0f) {
   // ALiBi: d0 = qbase - key; the bias of column f is nslope2 * |d0 + f| (nslope2 = -m log2(e)).
   const float2 c2 = make_float2(c, c);
 #pragma unroll
-  for (int e = 0; e < 64; e += 4) {
+  for (int e = 0; e < W; e += 4) {
     const float4 nl = *reinterpret_cast<const float4*>(nlse2 + e);
 #pragma unroll
     for (int h2 = 0; h2 < 4; h2 += 2) {
       const int f = e + h2;
-      const float2 sv = make_float2(__uint_as_float(f < 32 ? s0[f] : s1[f - 32]),
-                                    __uint_as_float(f < 32 ? s0[f + 1] : s1[f - 31]));
+      const float2 sv = make_float2(__uint_as_float(s0[f]), __uint_as_float(s0[f + 1]));
       float2 xv = fma2(sv, c2, h2 ? make_float2(nl.z, nl.w) : make_float2(nl.x, nl.y));
       if (kAlibi) {
         xv.x = fmaf(fabsf(d0 + (float)f), nslope2, xv.x);
@@ -293,7 +294,7 @@ __device__ __forceinline__ void bwd_probs(const uint32_t (&s0)[32], const uint32
 }
 
 template <int D, bool kDQ, bool kAlibi = false, bool kVarlen = false>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
@@ -330,11 +331,11 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(bar(bars->kv_full[s]), 1);
       mbar_init(bar(bars->kv_empty[s]), 1);
       mbar_init(bar(bars->dkv_full[s]), 1);
-      mbar_init(bar(bars->dkv_empty[s]), kEpiInDq ? 128 : 384);
+      mbar_init(bar(bars->dkv_empty[s]), kEpiInDq ? 128 : 128 + 128 * Cfg::kGroups);
       mbar_init(bar(bars->q_full[s]), 1);
       mbar_init(bar(bars->q_empty[s]), 1);
       mbar_init(bar(bars->item_full[s]), 1);
-      mbar_init(bar(bars->item_empty[s]), kBwdItemConsumers);
+      mbar_init(bar(bars->item_empty[s]), Cfg::kItemConsumers);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(bars->do_full[s]), 1);
@@ -342,8 +343,8 @@ __global__ void __launch_bounds__(512, 1)
     }
     mbar_init(bar(bars->s_full), 1);
     mbar_init(bar(bars->dp_full), 1);
-    mbar_init(bar(bars->p_full), 256);
-    mbar_init(bar(bars->ds_full), 256);
+    mbar_init(bar(bars->p_full), 128 * Cfg::kGroups);
+    mbar_init(bar(bars->ds_full), 128 * Cfg::kGroups);
     mbar_init(bar(bars->ds_empty), 1);
     mbar_init(bar(bars->dq_full), 1);
     mbar_init(bar(bars->dq_empty), 128);
@@ -487,13 +488,15 @@ __global__ void __launch_bounds__(512, 1)
             mma_ss(tDP, sdesc_kmajor(sV + off), sdesc_kmajor(sDO + off), idSP, kk > 0);
           }
           mma_commit(bar(bars->dp_full));
-          // dV += P^T dO_i (P^T packed in TMEM: queries [0,64) in S columns [0,32), [64,128) in [64,96))
+          // dV += P^T dO_i (P^T packed in TMEM: the W = kGroupCols queries [W g, W g + W) of P/dS
+          // group g in S columns [W g, W g + W / 2))
           mbar_wait(bar(bars->p_full), n & 1, ab);
           if (first) mbar_wait(bar(bars->dkv_empty[kvs]), kvphase ^ 1, ab);
           tc_fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t acol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
+            constexpr int W = Cfg::kGroupCols;
+            const uint32_t acol = (16 * kk / W) * W + (16 * kk % W) / 2;
             mma_ts(tDV, tS + acol, sdesc_mnmajor(sDO + kk * 2048, 16384), idKV, !first || kk > 0);
           }
           mma_commit(bar(bars->do_empty[dos]));
@@ -671,12 +674,18 @@ __global__ void __launch_bounds__(512, 1)
     }
     if (row == 0) bulk_wait_group0();
   } else if (warp >= 8) {
-    // ---------------------------------------------------------------- P, dS and the dK / dV epilogue
-    const int grp = (warp - 8) >> 2;                // 0: query columns [0,64) and dK; 1: [64,128) and dV
-    const int row = threadIdx.x - 256 - 128 * grp;  // key row within the tile == TMEM lane
+    // ---------------------------------------------------------------- P, dS and the dK epilogue
+    // kGroups groups of four warps; group g takes the W query columns [W g, W g + W) of every
+    // tile (and, at d = 128, dK columns [W g, W g + W) of the epilogue).
+    constexpr int W = Cfg::kGroupCols;
+    const int grp = (warp - 8) >> 2;
+    const int row = (threadIdx.x - 256) & 127;  // key row within the tile == TMEM lane
     const uint32_t lane_field = (uint32_t)((row & ~31) << 16);
-    const uint32_t tS = tmem + lane_field + Cfg::kColS + 64 * grp;
-    const uint32_t tDP = tmem + lane_field + Cfg::kColDP + 64 * grp;
+    const uint32_t tS = tmem + lane_field + Cfg::kColS + W * grp;
+    const uint32_t tDP = tmem + lane_field + Cfg::kColDP + W * grp;
+    // this group's queries in the dS tile: box (W grp) / 64, 16-byte chunks from (W grp % 64) / 8
+    const uint32_t ds_box = sDS + (W * grp / 64) * 16384;
+    const int ds_chunk0 = (W * grp % 64) / 8;
     const float c = p.scale_log2;
     uint32_t items = 0, n = 0, qs = 0, qphase = 0;
     for (uint32_t it = 0;; ++it) {
@@ -700,52 +709,46 @@ __global__ void __launch_bounds__(512, 1)
         const float* nlse2 = reinterpret_cast<const float*>(smem_raw + Cfg::kOffStat + qs * 1024);  // -LSE*log2(e)
         const float* nd = nlse2 + 128;                                                              // -D
         const bool masked = !bwd_tile_unmasked<kVarlen>(p, j, i, seg_first, seg_last);
-        const int qbase = i * 128 + 64 * grp;
+        const int qbase = i * 128 + W * grp;
 
         mbar_wait(bar(bars->s_full), n & 1, ab);
         tc_fence_after_sync();
-        uint32_t s0[32], s1[32];
-        tmem_ld32(tS, s0);
-        tmem_ld32(tS + 32, s1);
-        tmem_wait_ld(s0);
-        tmem_wait_ld(s1);
-        uint32_t pk[32];
+        uint32_t s0[W];
+#pragma unroll
+        for (int q = 0; q < W / 32; ++q) tmem_ld32(tS + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&s0[32 * q]));
+#pragma unroll
+        for (int q = 0; q < W / 32; ++q) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&s0[32 * q]));
+        uint32_t pk[W / 2];  // packed P over the first W / 2 of this group's S columns, read above
         const float dist0 = (float)(qbase - k);
         if (masked)
-          bwd_probs<true, kAlibi>(s0, s1, c, nlse2 + 64 * grp, qbase, qlo, qhi, pk, dist0, nslope2);
+          bwd_probs<W, true, kAlibi>(s0, c, nlse2 + W * grp, qbase, qlo, qhi, pk, dist0, nslope2);
         else
-          bwd_probs<false, kAlibi>(s0, s1, c, nlse2 + 64 * grp, qbase, qlo, qhi, pk, dist0, nslope2);
-        {
-          uint32_t lo16[16], hi16[16];
+          bwd_probs<W, false, kAlibi>(s0, c, nlse2 + W * grp, qbase, qlo, qhi, pk, dist0, nslope2);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) { lo16[e] = pk[e]; hi16[e] = pk[16 + e]; }
-          tmem_st16(tS, lo16);
-          tmem_st16(tS + 16, hi16);
-        }
+        for (int q = 0; q < W / 32; ++q) tmem_st16(tS + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(&pk[16 * q]));
         tmem_wait_st();
         tc_fence_before_sync();
         mbar_arrive(bar(bars->p_full));
 
         mbar_wait(bar(bars->dp_full), n & 1, ab);
         tc_fence_after_sync();
-        uint32_t d0[32], d1[32];
-        tmem_ld32(tDP, d0);
-        tmem_ld32(tDP + 32, d1);
-        tmem_wait_ld(d0);
-        tmem_wait_ld(d1);
-        // dS^T(row, q) = P^T(row, q) * (dP^T(row, q) - D_q) -> bf16 -> shared, 128B-swizzled rows of keys
-        mbar_wait(bar(bars->ds_empty), (n & 1) ^ 1, ab);
-        const uint32_t box = sDS + grp * 16384;
+        uint32_t d0[W];
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int q = 0; q < W / 32; ++q) tmem_ld32(tDP + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&d0[32 * q]));
+#pragma unroll
+        for (int q = 0; q < W / 32; ++q) tmem_wait_ld(*reinterpret_cast<uint32_t(*)[32]>(&d0[32 * q]));
+        // dS^T(row, q) = P^T(row, q) * (dP^T(row, q) - D_q) -> bf16 -> shared, 128B-swizzled rows of
+        // keys (the group's queries: chunks ds_chunk0 .. ds_chunk0 + W / 8 - 1 of box ds_box)
+        mbar_wait(bar(bars->ds_empty), (n & 1) ^ 1, ab);
+#pragma unroll
+        for (int ch = 0; ch < W / 8; ++ch) {
           uint32_t w4[4];
-          const float4 nda = *reinterpret_cast<const float4*>(nd + 64 * grp + ch * 8);
-          const float4 ndb = *reinterpret_cast<const float4*>(nd + 64 * grp + ch * 8 + 4);
+          const float4 nda = *reinterpret_cast<const float4*>(nd + W * grp + ch * 8);
+          const float4 ndb = *reinterpret_cast<const float4*>(nd + W * grp + ch * 8 + 4);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int col = ch * 8 + 2 * e;  // 0..63 within the group
-            const float2 g = make_float2(__uint_as_float(col < 32 ? d0[col] : d1[col - 32]),
-                                         __uint_as_float(col < 32 ? d0[col + 1] : d1[col - 31]));
+            const int col = ch * 8 + 2 * e;  // within the group
+            const float2 g = make_float2(__uint_as_float(d0[col]), __uint_as_float(d0[col + 1]));
             const uint32_t pp = pk[col >> 1];
             const float2 ndv = e == 0 ? make_float2(nda.x, nda.y) : e == 1 ? make_float2(nda.z, nda.w)
                              : e == 2 ? make_float2(ndb.x, ndb.y) : make_float2(ndb.z, ndb.w);
@@ -753,7 +756,7 @@ __global__ void __launch_bounds__(512, 1)
             const float2 ds = mul2(make_float2(bf16lo_to_f32(pp), bf16hi_to_f32(pp)), diff);
             w4[e] = pack_bf16x2(ds.x, ds.y);
           }
-          st_shared_v4(box + sw128_offset(row, ch), w4[0], w4[1], w4[2], w4[3]);
+          st_shared_v4(ds_box + sw128_offset(row, ds_chunk0 + ch), w4[0], w4[1], w4[2], w4[3]);
         }
         fence_proxy_async_smem();
         tc_fence_before_sync();
@@ -761,19 +764,19 @@ __global__ void __launch_bounds__(512, 1)
         if (++qs == 2) { qs = 0; qphase ^= 1; }
       }
 
-      // Epilogue (d = 128; at d = 64 the dQ warps do it): dK times scale, columns [64 grp,
-      // 64 grp + 64) -> bf16 -> box grp of the dS buffer (free: the item's last dQ and dK have
-      // read it) -> TMA store. The group's next dS waits for the store to read the box.
+      // Epilogue (d = 128; at d = 64 the dQ warps do it): dK times scale, columns [W grp,
+      // W grp + W) -> bf16 -> the group's chunks of the dS buffer (free: the item's last dQ and
+      // dK have read it) -> TMA store of each 64-column box once the groups that fill it are
+      // done. Their next dS waits for the store to read the box.
       if constexpr (!kEpiInDq) {
+        constexpr int kBoxGroups = 64 / W;  // groups per 64-column box
         const uint32_t kvs = items % Cfg::kKVSlots, kvphase = (items / Cfg::kKVSlots) & 1;
         mbar_wait(bar(bars->dkv_full[kvs]), kvphase, ab);
         tc_fence_after_sync();
-        const uint32_t src = tmem + lane_field + Cfg::kColDK + 64 * grp;
-        const uint32_t bx = sDS + grp * 16384;
 #pragma unroll 1
-        for (int cc = 0; cc < 64; cc += 32) {
+        for (int cc = 0; cc < W; cc += 32) {
           uint32_t v[32];
-          tmem_ld32(src + cc, v);
+          tmem_ld32(tmem + lane_field + Cfg::kColDK + W * grp + cc, v);
           tmem_wait_ld(v);
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
@@ -782,20 +785,21 @@ __global__ void __launch_bounds__(512, 1)
             for (int e = 0; e < 4; ++e)
               w4[e] = pack_bf16x2(__uint_as_float(v[ch * 8 + 2 * e]) * p.scale,
                                   __uint_as_float(v[ch * 8 + 2 * e + 1]) * p.scale);
-            st_shared_v4(bx + sw128_offset(row, (cc >> 3) + ch), w4[0], w4[1], w4[2], w4[3]);
+            st_shared_v4(ds_box + sw128_offset(row, ds_chunk0 + cc / 8 + ch), w4[0], w4[1], w4[2], w4[3]);
           }
         }
         tc_fence_before_sync();
         mbar_arrive(bar(bars->dkv_empty[kvs]));
         fence_proxy_async_smem();
-        named_bar_sync(1 + grp, 128);
-        if (row == 0) {
-          if (dbg_tma(ab, 64 * grp, j * 128, h, b, D, p.N, p.H, p.B, 2, bx, 16384, smem_base, smem_end))
-            tma_store_4d(&tmdK, bx, 64 * grp, j * 128, h, b);
+        const int box = W * grp / 64;
+        named_bar_sync(1 + box, 128 * kBoxGroups);
+        if (row == 0 && grp % kBoxGroups == 0) {
+          if (dbg_tma(ab, 64 * box, j * 128, h, b, D, p.N, p.H, p.B, 2, ds_box, 16384, smem_base, smem_end))
+            tma_store_4d(&tmdK, ds_box, 64 * box, j * 128, h, b);
           bulk_commit_group();
           bulk_wait_group_read0();
         }
-        named_bar_sync(1 + grp, 128);
+        named_bar_sync(1 + box, 128 * kBoxGroups);
       }
       ++items;
     }
