@@ -20,6 +20,9 @@
 //   warps 2-3   : no role
 //   warps 4-7   : softmax + epilogue for Q tile 0 (one thread per query row / TMEM lane)
 //   warps 8-11  : softmax + epilogue for Q tile 1
+//   warps 12-19 : d = 64 only (640 threads): the second 64 scores of every row of tile 0
+//                 (warps 12-15) and tile 1 (warps 16-19); warps 4-11 then take the first 64.
+//                 The two warps of a row exchange partial maxima and sums (see FwdCfg).
 // TMEM (512 columns): O0 [256,256+D), O1 [256+D, 256+2D); S and P as below. P_t (bf16, two
 // per column; E4M3, four) is the A operand of O_t += P_t V_j, read straight from TMEM.
 //
@@ -102,7 +105,15 @@ constexpr float kLn2 = 0.69314718055994530942f;
 // quantised to E4M3 in TMEM (four per column); O is bf16 as for bf16 inputs.
 template <int D, bool kF8 = false>
 struct FwdCfg {
-  static constexpr int kThreads = 384;
+  // d = 64 (bf16): each row's 128 scores of a KV tile are split over two warps (64 each), which
+  // exchange their partial row maxima through shared memory, so that four softmax warps share
+  // each SM sub-partition; d = 128 keeps one warp per row (its TMEM and registers are full).
+  static constexpr bool kSplitRow = (D == 64) && !kF8;
+  static constexpr int kHalves = kSplitRow ? 2 : 1;
+  static constexpr int kCols = 128 / kHalves;              // scores per softmax thread and KV tile
+  static constexpr int kThreads = 128 + 256 * kHalves;     // 384, or 640 with the row split
+  static constexpr uint32_t kItemConsumers = 1 + 8 * kHalves;  // MMA thread and softmax warps
+  static constexpr int kXBytes = kSplitRow ? 8192 : 0;     // row-split exchange: maxima, then sums
   static constexpr int kElem = kF8 ? 1 : 2;        // bytes per Q/K/V element
   static constexpr int kTileBytes = 128 * D * kElem;  // one 128-row tile of Q, K or V
   static constexpr int kOTileBytes = 128 * D * 2;     // one 128-row bf16 tile of O
@@ -118,7 +129,8 @@ struct FwdCfg {
   static constexpr int kOffQ = 0;                     // Q0, Q1 (also O staging unless kSepO)
   static constexpr int kOffO = 2 * kTileBytes;        // O staging 0, 1 (kSepO)
   static constexpr int kOffKV = kSepO ? kOffO + 2 * kOTileBytes : 2 * kTileBytes;
-  static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
+  static constexpr int kOffX = kOffKV + kSlots * kTileBytes;
+  static constexpr int kOffBar = kOffX + kXBytes;
   static constexpr int kSmemBytes = kOffBar + 512 + 1024;  // barriers + alignment slack
   static constexpr int kOffSort = kOffBar + 512;            // packed batches: pair costs and order
   static constexpr uint32_t kColS0 = 0, kColS1 = kShareS ? 0 : 128, kColO0 = 256, kColO1 = 256 + D;
@@ -139,9 +151,6 @@ struct FwdBars {
   uint32_t tmem_base;
   int abort_flag;
 };
-
-// Consumers of a fetched item: the MMA thread and the 8 softmax warps (one arrival each).
-constexpr uint32_t kFwdItemConsumers = 9;
 
 // Next work item of a consumer role (n counts the items this role has taken); values >=
 // num_items mean "no more work".
@@ -230,21 +239,20 @@ __device__ __forceinline__ bool fwd_tile_unmasked(const FwdParams& p, int r0, in
 
 // ------------------------------------------------------------------ softmax role
 
-// Row maximum of a 128-key tile (scaled, log2 units) with masking, and the lazy update of
-// the reference maximum. x is scaled in place when the scale is not positive, and always with
-// ALiBi, whose bias nslope2 * |d0 - cc| (nslope2 = -m log2(e), d0 = row - kbase) is added
-// after the scaling.
-template <bool kPosScale, bool kAlibi = false>
-__device__ __forceinline__ void fwd_row_max(float (&x)[128], bool masked, int kbase, int kmin, int kmax, float c,
-                                            float& m_run, float& alpha, bool& updated, float d0 = 0.0f,
-                                            float nslope2 = 0.0f) {
+// Maximum of this thread's kC scores of a key tile (scaled, log2 units), x[0] being key kbase,
+// with masking. x is scaled in place when the scale is not positive, and always with ALiBi,
+// whose bias nslope2 * |d0 - cc| (nslope2 = -m log2(e), d0 = row - kbase) is added after the
+// scaling.
+template <bool kPosScale, bool kAlibi = false, int kC>
+__device__ __forceinline__ float fwd_tile_max(float (&x)[kC], bool masked, int kbase, int kmin, int kmax, float c,
+                                              float d0 = 0.0f, float nslope2 = 0.0f) {
   static_assert(!(kAlibi && kPosScale), "the ALiBi bias is added to scaled scores");
   if (kAlibi) {
 #pragma unroll
-    for (int cc = 0; cc < 128; ++cc) x[cc] = fmaf(fabsf(d0 - (float)cc), nslope2, x[cc] * c);
+    for (int cc = 0; cc < kC; ++cc) x[cc] = fmaf(fabsf(d0 - (float)cc), nslope2, x[cc] * c);
   } else if (!kPosScale) {  // then masking must follow the scaling
 #pragma unroll
-    for (int cc = 0; cc < 128; cc += 2) {
+    for (int cc = 0; cc < kC; cc += 2) {
       const float2 v = mul2(make_float2(x[cc], x[cc + 1]), make_float2(c, c));
       x[cc] = v.x;
       x[cc + 1] = v.y;
@@ -257,15 +265,22 @@ __device__ __forceinline__ void fwd_row_max(float (&x)[128], bool masked, int kb
     const unsigned span = any ? (unsigned)(kmax - kmin) : 0u;
     const int off = any ? kbase - kmin : -(1 << 30);
 #pragma unroll
-    for (int cc = 0; cc < 128; ++cc) x[cc] = ((unsigned)(off + cc) <= span) ? x[cc] : -INFINITY;
+    for (int cc = 0; cc < kC; ++cc) x[cc] = ((unsigned)(off + cc) <= span) ? x[cc] : -INFINITY;
   }
   float mx[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
 #pragma unroll
-  for (int k = 0; k < 64; ++k) mx[k & 7] = max3(mx[k & 7], x[2 * k], x[2 * k + 1]);
+  for (int k = 0; k < kC / 2; ++k) mx[k & 7] = max3(mx[k & 7], x[2 * k], x[2 * k + 1]);
   float m_tile = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
   if (kPosScale) m_tile *= c;
+  return m_tile;
+}
+
+// Lazy update of the reference maximum from a tile's row maximum: it moves only when the row
+// maximum exceeds it by more than kRescaleThreshold, and alpha (the factor for O and the sums)
+// is then 2^(old - new).
+__device__ __forceinline__ void fwd_update_max(float m_tile, float& m_run, float& alpha, bool& updated) {
   const float m_new = fmaxf(m_run, m_tile);
   updated = m_new > m_run + kRescaleThreshold;
   alpha = 1.0f;
@@ -281,8 +296,8 @@ __device__ __forceinline__ void fwd_row_max(float (&x)[128], bool masked, int kb
 // divisor of O, so that O is a weighted mean of V rows under exactly the weights applied: a
 // row dominated by one key then returns that key's value row, not the row times the
 // relative rounding error of its weight).
-template <bool kPosScale>
-__device__ __forceinline__ void fwd_exp_chunk(const float (&x)[128], int k0, float c, float m_use, uint32_t (&pk)[16],
+template <bool kPosScale, int kC>
+__device__ __forceinline__ void fwd_exp_chunk(const float (&x)[kC], int k0, float c, float m_use, uint32_t (&pk)[16],
                                               float2& sum, float2& rsum) {
   const float2 neg_m = make_float2(-m_use, -m_use);
   const float2 c2 = make_float2(c, c);
@@ -304,8 +319,8 @@ __device__ __forceinline__ void fwd_exp_chunk(const float (&x)[128], int k0, flo
 
 // Same for E4M3 P: 32 columns -> 8 words of four E4M3 values (column 4w + i in byte i). The
 // row sum takes the exponentials before quantisation.
-template <bool kPosScale>
-__device__ __forceinline__ void fwd_exp_chunk_e4m3(const float (&x)[128], int k0, float c, float m_use,
+template <bool kPosScale, int kC>
+__device__ __forceinline__ void fwd_exp_chunk_e4m3(const float (&x)[kC], int k0, float c, float m_use,
                                                    uint32_t (&pk)[8], float2& sum) {
   const float2 neg_m = make_float2(-m_use, -m_use);
   const float2 c2 = make_float2(c, c);
@@ -333,7 +348,7 @@ __device__ __forceinline__ float lg2_approx(float x) {
 }
 
 template <int D, bool kF8 = false, bool kAlibi = false, bool kVarlen = false>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(FwdCfg<D, kF8>::kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams p) {
@@ -360,8 +375,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(bars->q_full[t]), 1);
       mbar_init(bar(bars->q_empty[t]), 1);
       mbar_init(bar(bars->s_full[t]), 1);
-      mbar_init(bar(bars->p_full[t]), 128);
-      mbar_init(bar(bars->s_empty[t]), 128);
+      mbar_init(bar(bars->p_full[t]), 128 * Cfg::kHalves);
+      mbar_init(bar(bars->s_empty[t]), 128 * Cfg::kHalves);
       mbar_init(bar(bars->pv_done[t]), 1);
     }
     for (int s = 0; s < Cfg::kSlots; ++s) {
@@ -371,7 +386,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar(bars->mma_done), 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(bars->item_full[t]), 1);
-      mbar_init(bar(bars->item_empty[t]), kFwdItemConsumers);
+      mbar_init(bar(bars->item_empty[t]), Cfg::kItemConsumers);
     }
     fence_barrier_init();
     prefetch_tmap(&tmQ);
@@ -418,11 +433,15 @@ __global__ void __launch_bounds__(384, 1)
                           Cfg::kSepO ? smem_base + Cfg::kOffO + Cfg::kOTileBytes : sQ[1]};
   const uint32_t sKV = smem_base + Cfg::kOffKV;
 
-  // Registers: the launch gives every thread 168; the producer / MMA warpgroup (warps 0-3) needs
-  // few and hands some back, and the two softmax warpgroups, which hold a row's 128 scores,
-  // take them: 128 x (96 + 200 + 200) = 63488 <= 384 x 168 = 64512 registers of the launch.
+  // Registers: the launch gives every thread 168 (384 threads) or 96 (640, row split); the
+  // producer / MMA warpgroup (warps 0-3) needs few and hands some back, and the softmax
+  // warpgroups take them: 128 x (96 + 2 x 200) = 63488 <= 384 x 168 = 64512, and
+  // 128 x (80 + 4 x 96) = 59392 <= 640 x 96 = 61440 registers of the launch.
   if (warp < 4) {  // ---- producer / MMA warpgroup (warps 0-3)
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
+  if constexpr (Cfg::kSplitRow)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
+  else
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;" ::: "memory");
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane_id() == 0) {
@@ -638,17 +657,30 @@ __global__ void __launch_bounds__(384, 1)
       mbar_drain(bar(bars->mma_done), 0);
     }
   }
-  } else {  // ---- softmax warpgroups (warps 4-11)
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+  } else {  // ---- softmax warpgroups (warps 4-11, or 4-19 with the row split)
+  if constexpr (Cfg::kSplitRow)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 96;" ::: "memory");
+  else
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
   {
     // ---------------------------------------------------------------- softmax + epilogue
-    const int t = (warp - 4) >> 2;           // Q tile of the pair handled by this warpgroup
-    const int row = threadIdx.x - 128 * (1 + t);  // 0..127: TMEM lane and row within the tile
+    constexpr int kC = Cfg::kCols;            // scores of a row per thread and KV tile
+    const int t = ((warp - 4) >> 2) & 1;      // Q tile of the pair handled by this warpgroup
+    const int half = (warp - 4) >> 3;         // row split: columns [kC half, kC half + kC)
+    const int row = (threadIdx.x - 128) & 127;  // 0..127: TMEM lane and row within the tile
     const uint32_t lane_field = (uint32_t)((row & ~31) << 16);
-    const uint32_t tS = tmem + lane_field + (t ? Cfg::kColS1 : Cfg::kColS0);
+    const uint32_t tS = tmem + lane_field + (t ? Cfg::kColS1 : Cfg::kColS0) + kC * half;
     const uint32_t tO = tmem + lane_field + (t ? Cfg::kColO1 : Cfg::kColO0);
-    const uint32_t tP = tmem + lane_field + (t ? Cfg::kColP1 : Cfg::kColP0);
+    const uint32_t tP = tmem + lane_field + (t ? Cfg::kColP1 : Cfg::kColP0) + (kC / 2) * half;
     uint32_t sn = 0, pvn = 0;
+    // Row split: the two warps holding the same 32 rows of tile t (same TMEM lanes, so the same
+    // sub-partition) meet at named barrier 4 + 4 t + row / 32 and exchange their partial maxima
+    // (two parity slots, so a fast partner never overwrites a value not yet read) and, at the
+    // end of an item, their sums.
+    float* xm = reinterpret_cast<float*>(smem_gen + Cfg::kOffX) + t * 512;         // [parity][half][row]
+    float* xl = reinterpret_cast<float*>(smem_gen + Cfg::kOffX) + 1024 + t * 512;  // [sum][half][row]
+    uint32_t xu = 0;
+    auto pair_sync = [&]() { named_bar_sync(4 + 4 * t + (row >> 5), 64); };
 
     for (uint32_t it = 0;; ++it) {
       const int w = fwd_take_item(bars, it, lane_id() == 0, ab);
@@ -685,28 +717,37 @@ __global__ void __launch_bounds__(384, 1)
         mbar_wait(bar(bars->s_full[t]), sn & 1, ab);
         ++sn;
         tc_fence_after_sync();
-        uint32_t r[4][32];
+        uint32_t r[kC / 32][32];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, r[q4]);
+        for (int q4 = 0; q4 < kC / 32; ++q4) tmem_ld32(tS + q4 * 32, r[q4]);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) tmem_wait_ld(r[q4]);
+        for (int q4 = 0; q4 < kC / 32; ++q4) tmem_wait_ld(r[q4]);
         tc_fence_before_sync();  // the S buffer may now take the next scores
         mbar_arrive(bar(bars->s_empty[Cfg::kShareS ? 0 : t]));
-        float x[128];
+        float x[kC];
 #pragma unroll
-        for (int cc = 0; cc < 128; ++cc) x[cc] = __uint_as_float(r[cc >> 5][cc & 31]);
+        for (int cc = 0; cc < kC; ++cc) x[cc] = __uint_as_float(r[cc >> 5][cc & 31]);
 
         const bool masked = !fwd_tile_unmasked<kVarlen>(p, r0, j, seg_first, seg_last);
+        const int kbase = j * 128 + kC * half;  // key of x[0]
+        const bool pos_scale = !kAlibi && c > 0.0f;  // with ALiBi the scores are scaled before the max
+        float m_tile;
+        if constexpr (kAlibi)
+          m_tile = fwd_tile_max<false, true>(x, masked, kbase, kmin, kmax, c, (float)(i - kbase), nslope2);
+        else if (pos_scale)
+          m_tile = fwd_tile_max<true>(x, masked, kbase, kmin, kmax, c);
+        else
+          m_tile = fwd_tile_max<false>(x, masked, kbase, kmin, kmax, c);
+        if constexpr (Cfg::kSplitRow) {
+          float* slot = xm + (xu & 1) * 256;
+          slot[half * 128 + row] = m_tile;
+          pair_sync();
+          m_tile = fmaxf(m_tile, slot[(half ^ 1) * 128 + row]);
+          ++xu;
+        }
         float alpha;
         bool updated;
-        const bool pos_scale = !kAlibi && c > 0.0f;  // with ALiBi the scores are scaled before the max
-        if constexpr (kAlibi)
-          fwd_row_max<false, true>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated, (float)(i - j * 128),
-                                   nslope2);
-        else if (pos_scale)
-          fwd_row_max<true>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated);
-        else
-          fwd_row_max<false>(x, masked, j * 128, kmin, kmax, c, m_run, alpha, updated);
+        fwd_update_max(m_tile, m_run, alpha, updated);
         const float m_use = (m_run == -INFINITY) ? 0.0f : m_run;
         if (j > lo) {  // PV_t(j-1) has read P_t and O_t is quiescent
           mbar_wait(bar(bars->pv_done[t]), pvn & 1, ab);
@@ -717,7 +758,7 @@ __global__ void __launch_bounds__(384, 1)
         float2 sum0 = make_float2(0.0f, 0.0f), sum1 = make_float2(0.0f, 0.0f);
         float2 rs0 = make_float2(0.0f, 0.0f), rs1 = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int q4 = 0; q4 < kC / 32; ++q4) {
           if constexpr (kF8) {
             uint32_t pk[8];
             if (pos_scale)
@@ -745,7 +786,7 @@ __global__ void __launch_bounds__(384, 1)
         // the first PV of an item overwrites O_t).
         if (__any_sync(0xffffffffu, updated && j > lo)) {
 #pragma unroll 1
-          for (int cc = 0; cc < D; cc += 32) {
+          for (int cc = (D / Cfg::kHalves) * half; cc < (D / Cfg::kHalves) * (half + 1); cc += 32) {
             uint32_t o[32];
             tmem_ld32(tO + cc, o);
             tmem_wait_ld(o);
@@ -764,16 +805,24 @@ __global__ void __launch_bounds__(384, 1)
       ++pvn;
       tc_fence_after_sync();
       if constexpr (Cfg::kSepO) {
-        if (row == 0) bulk_wait_group_read0();  // the previous store has read the staging tile
-        named_bar_sync(1 + t, 128);
+        if (row == 0 && half == 0) bulk_wait_group_read0();  // the previous store has read the staging tile
+        named_bar_sync(1 + t, 128 * Cfg::kHalves);
       }
       // bf16 P: O is divided by the sum of the weights it was accumulated with; E4M3 P keeps the
-      // fp32 sum (its tolerance is derived for that divisor)
-      const float l_o = kF8 ? l_run : lr_run;
+      // fp32 sum (its tolerance is derived for that divisor). Row split: each half summed its
+      // own columns against the same reference maximum, so the row's sums add.
+      float l_tot = l_run, l_o = kF8 ? l_run : lr_run;
+      if constexpr (Cfg::kSplitRow) {
+        xl[half * 128 + row] = l_run;
+        xl[256 + half * 128 + row] = lr_run;
+        pair_sync();
+        l_tot = l_run + xl[(half ^ 1) * 128 + row];
+        l_o = lr_run + xl[256 + (half ^ 1) * 128 + row];
+      }
       const float inv_l = l_o > 0.0f ? o_mul / l_o : 0.0f;
       const uint32_t stage = sO[t];
 #pragma unroll 1
-      for (int cc = 0; cc < D; cc += 32) {
+      for (int cc = (D / Cfg::kHalves) * half; cc < (D / Cfg::kHalves) * (half + 1); cc += 32) {
         uint32_t o[32];
         tmem_ld32(tO + cc, o);
         tmem_wait_ld(o);
@@ -788,8 +837,8 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       fence_proxy_async_smem();
-      named_bar_sync(1 + t, 128);
-      if (row == 0) {
+      named_bar_sync(1 + t, 128 * Cfg::kHalves);
+      if (row == 0 && half == 0) {
 #pragma unroll
         for (int bx = 0; bx < Cfg::kOBoxes; ++bx)
           if (dbg_tma(ab, bx * 64, r0, h, b, D, p.N, p.H, p.B, 2, stage + bx * 16384, 16384, smem_base, smem_end))
@@ -800,13 +849,13 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(bar(bars->q_empty[t]));
         }
       }
-      if (i < p.N) {
-        const float lse = l_run > 0.0f ? (m_run + lg2_approx(l_run)) * kLn2 : -INFINITY;
+      if (i < p.N && half == 0) {
+        const float lse = l_tot > 0.0f ? (m_run + lg2_approx(l_tot)) * kLn2 : -INFINITY;
         const long long li = ((long long)b * p.H + h) * (long long)p.N + i;
         if (dbg_range(ab, li, 1, (long long)p.B * p.H * p.N)) p.lse[li] = lse;
       }
     }
-    if (row == 0) bulk_wait_group0();
+    if (row == 0 && half == 0) bulk_wait_group0();
   }
   }
 
