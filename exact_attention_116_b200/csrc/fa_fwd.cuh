@@ -20,9 +20,9 @@
 //   warps 2-3   : no role
 //   warps 4-7   : softmax + epilogue for Q tile 0 (one thread per query row / TMEM lane)
 //   warps 8-11  : softmax + epilogue for Q tile 1
-//   warps 12-19 : d = 64 only (640 threads): the second 64 scores of every row of tile 0
-//                 (warps 12-15) and tile 1 (warps 16-19); warps 4-11 then take the first 64.
-//                 The two warps of a row exchange partial maxima and sums (see FwdCfg).
+//   warps 12-19 : the second 64 scores of every row of tile 0 (warps 12-15) and tile 1
+//                 (warps 16-19); warps 4-11 take the first 64 (640 threads). The two warps of
+//                 a row exchange partial maxima and sums (see FwdCfg).
 // TMEM (512 columns): O0 [256,256+D), O1 [256+D, 256+2D); S and P as below. P_t (bf16, two
 // per column; E4M3, four) is the A operand of O_t += P_t V_j, read straight from TMEM.
 //
@@ -105,10 +105,10 @@ constexpr float kLn2 = 0.69314718055994530942f;
 // quantised to E4M3 in TMEM (four per column); O is bf16 as for bf16 inputs.
 template <int D, bool kF8 = false>
 struct FwdCfg {
-  // d = 64 (bf16): each row's 128 scores of a KV tile are split over two warps (64 each), which
-  // exchange their partial row maxima through shared memory, so that four softmax warps share
-  // each SM sub-partition; d = 128 keeps one warp per row (its TMEM and registers are full).
-  static constexpr bool kSplitRow = (D == 64) && !kF8;
+  // Each row's 128 scores of a KV tile are split over two warps (64 each), which exchange their
+  // partial row maxima through shared memory, so that four softmax warps share each SM
+  // sub-partition (kept as a switch: kSplitRow = false is the one-warp-per-row layout).
+  static constexpr bool kSplitRow = true;
   static constexpr int kHalves = kSplitRow ? 2 : 1;
   static constexpr int kCols = 128 / kHalves;              // scores per softmax thread and KV tile
   static constexpr int kThreads = 128 + 256 * kHalves;     // 384, or 640 with the row split
@@ -120,7 +120,7 @@ struct FwdCfg {
   static constexpr int kBoxes = D * kElem / 128;      // 128-byte-wide TMA boxes per Q/K/V tile
   static constexpr int kBoxElems = 128 / kElem;       // elements per box row
   static constexpr int kOBoxes = D / 64;              // 64-column boxes per O tile
-  static constexpr int kSlots = (kTileBytes == 32768) ? 4 : 8;
+  static constexpr int kSlots = (kTileBytes == 32768) ? 4 : (kF8 && kSplitRow) ? 7 : 8;
   static constexpr bool kShareS = (D == 128);          // one S buffer for both tiles
   static_assert(D == 128 || !kF8, "E4M3 tiles are 128 bytes wide: d = 128");
   static constexpr bool kSepO = (D == 64) || kF8;     // O staging apart from Q; Q freed by the last S
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kF8>::kThreads, 1)
                           Cfg::kSepO ? smem_base + Cfg::kOffO + Cfg::kOTileBytes : sQ[1]};
   const uint32_t sKV = smem_base + Cfg::kOffKV;
 
-  // Registers: the launch gives every thread 168 (384 threads) or 96 (640, row split); the
+  // Registers: the launch gives every thread 168 (384 threads, no row split) or 96 (640); the
   // producer / MMA warpgroup (warps 0-3) needs few and hands some back, and the softmax
   // warpgroups take them: 128 x (96 + 2 x 200) = 63488 <= 384 x 168 = 64512, and
   // 128 x (80 + 4 x 96) = 59392 <= 640 x 96 = 61440 registers of the launch.
@@ -671,7 +671,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kF8>::kThreads, 1)
     const uint32_t lane_field = (uint32_t)((row & ~31) << 16);
     const uint32_t tS = tmem + lane_field + (t ? Cfg::kColS1 : Cfg::kColS0) + kC * half;
     const uint32_t tO = tmem + lane_field + (t ? Cfg::kColO1 : Cfg::kColO0);
-    const uint32_t tP = tmem + lane_field + (t ? Cfg::kColP1 : Cfg::kColP0) + (kC / 2) * half;
+    const uint32_t tP = tmem + lane_field + (t ? Cfg::kColP1 : Cfg::kColP0) + (kC / (kF8 ? 4 : 2)) * half;
     uint32_t sn = 0, pvn = 0;
     // Row split: the two warps holding the same 32 rows of tile t (same TMEM lanes, so the same
     // sub-partition) meet at named barrier 4 + 4 t + row / 32 and exchange their partial maxima
@@ -817,7 +817,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kF8>::kThreads, 1)
         xl[256 + half * 128 + row] = lr_run;
         pair_sync();
         l_tot = l_run + xl[(half ^ 1) * 128 + row];
-        l_o = lr_run + xl[256 + (half ^ 1) * 128 + row];
+        l_o = kF8 ? l_tot : lr_run + xl[256 + (half ^ 1) * 128 + row];
       }
       const float inv_l = l_o > 0.0f ? o_mul / l_o : 0.0f;
       const uint32_t stage = sO[t];
