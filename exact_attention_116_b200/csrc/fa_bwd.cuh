@@ -220,11 +220,11 @@ __device__ __forceinline__ void bwd_decode(const BwdParams& p, int w, int& b, in
 // item index; values >= num_items mean "no more work".
 __device__ __forceinline__ int bwd_take_item(BwdBars* bars, uint32_t n, bool arrive, Abort ab) {
   const uint32_t slot = n & 1;
-  mbar_wait(smem_u32(&bars->item_full[slot]), (n >> 1) & 1, ab);
+  const bool ok = mbar_wait_ring(smem_u32(&bars->item_full[slot]), (n >> 1) & 1, ab);
   const int w = *reinterpret_cast<volatile int*>(&bars->item_w[slot]);
   __syncwarp(__activemask());
   if (arrive) mbar_arrive(smem_u32(&bars->item_empty[slot]));
-  return ab.raised() ? 0x7fffffff : w;
+  return ok ? w : 0x7fffffff;
 }
 
 // Q tiles whose rows see any key of KV tile j.

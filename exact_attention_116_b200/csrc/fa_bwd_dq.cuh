@@ -72,11 +72,11 @@ __device__ __forceinline__ void bwd_dq_decode(const BwdParams& p, int w, int& b,
 
 __device__ __forceinline__ int bwd_dq_take_item(BwdDqBars* bars, uint32_t n, bool arrive, Abort ab) {
   const uint32_t slot = n & 1;
-  mbar_wait(smem_u32(&bars->item_full[slot]), (n >> 1) & 1, ab);
+  const bool ok = mbar_wait_ring(smem_u32(&bars->item_full[slot]), (n >> 1) & 1, ab);
   const int w = *reinterpret_cast<volatile int*>(&bars->item_w[slot]);
   __syncwarp(__activemask());
   if (arrive) mbar_arrive(smem_u32(&bars->item_empty[slot]));
-  return ab.raised() ? 0x7fffffff : w;
+  return ok ? w : 0x7fffffff;
 }
 
 // The ranges and masks of the forward apply: Q tile rows [i*128, i*128+127] see the KV tiles of

@@ -157,11 +157,11 @@ struct FwdBars {
 template <class Bars>
 __device__ __forceinline__ int fwd_take_item(Bars* bars, uint32_t n, bool arrive, Abort ab) {
   const uint32_t slot = n & 1;
-  mbar_wait(smem_u32(&bars->item_full[slot]), (n >> 1) & 1, ab);
+  const bool ok = mbar_wait_ring(smem_u32(&bars->item_full[slot]), (n >> 1) & 1, ab);
   const int w = *reinterpret_cast<volatile int*>(&bars->item_w[slot]);
   __syncwarp(__activemask());
   if (arrive) mbar_arrive(smem_u32(&bars->item_empty[slot]));
-  return ab.raised() ? 0x7fffffff : w;
+  return ok ? w : 0x7fffffff;
 }
 
 // Item w -> (b, h, pair). Pair rank r is pair num_pairs - 1 - r under causal masking (longest

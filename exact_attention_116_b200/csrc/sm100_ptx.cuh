@@ -159,6 +159,24 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Abort a
   return false;
 }
 
+// Wait on the work-item ring: it ignores the abort flag and allows twice the usual time. Every
+// consumer of an item then decides from the same published value whether to stop, whatever the
+// abort flag reads at the moment it looks, so warps that meet at named barriers (which cannot
+// time out) take the same items. Once the flag is raised the producer publishes stop items at
+// once, well within this limit. Returns false (and raises the flag) if the phase did not
+// complete in time: the producer has stopped, and every consumer then stops as well.
+__device__ __forceinline__ bool mbar_wait_ring(uint32_t bar, uint32_t parity, Abort ab) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1; it < (1u << 30); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0 && global_timer_ns() - t0 > 2 * FA_WAIT_TIMEOUT_NS) break;
+  }
+  *ab.flag = 1;
+  atomicOr(&g_fa_error, kErrWaitTimeout);
+  return false;
+}
+
 // Bounded wait that ignores the abort flag: used to drain copies already in flight.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
