@@ -61,10 +61,13 @@ struct BwdParams {
   int tail_tiles;             // the last (shortest under causal masking) KV tiles, dealt over all heads
 };
 
-// Share of the exponentials computed by exp2_poly on the FMA pipes (pair p of a thread's 32
-// pairs uses the polynomial when p % kPolyDen < kPolyNum).
+// Share of the exponentials computed by exp2_poly on the FMA pipes (pair p of a thread's pairs
+// uses the polynomial when p % kPolyDen < kPolyNum). None by default: with the P/dS work spread
+// over four warps per SM sub-partition (d = 64) the MUFU unit has room, and the polynomial's
+// instructions cost more issue slots than they save (window main kernel 0.1987 ms with 1/4,
+// 0.1951 with none, 0.208 with 2/4; train 1.3075 / 1.3005 / 1.2995 ms).
 #ifndef FA_BWD_POLY_NUM
-#define FA_BWD_POLY_NUM 1
+#define FA_BWD_POLY_NUM 0
 #endif
 #ifndef FA_BWD_POLY_DEN
 #define FA_BWD_POLY_DEN 4
