@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::kThreads, 1)
       int last_q_parity[2] = {-1, -1};
       for (uint32_t n = 0;; ++n) {
         const uint32_t slot = n & 1;
-        mbar_wait(bar(bars->item_empty[slot]), ((n >> 1) & 1) ^ 1, ab);
+        mbar_wait_ring(bar(bars->item_empty[slot]), ((n >> 1) & 1) ^ 1, ab);  // slot read by every consumer
         const int w = ab.raised() ? p.num_items : atomicAdd(p.next_item, 1);
         bars->item_w[slot] = w;
         mbar_arrive(bar(bars->item_full[slot]));

@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(256, 1)
       for (int s = 0; s < Cfg::kSlots; ++s) last_slot_parity[s] = -1;
       for (uint32_t n = 0;; ++n) {
         const uint32_t islot = n & 1;
-        mbar_wait(bar(bars->item_empty[islot]), ((n >> 1) & 1) ^ 1, ab);
+        mbar_wait_ring(bar(bars->item_empty[islot]), ((n >> 1) & 1) ^ 1, ab);  // slot read by every consumer
         const int w = ab.raised() ? p.num_items : atomicAdd(p.next_item + 1, 1);
         bars->item_w[islot] = w;
         mbar_arrive(bar(bars->item_full[islot]));

@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kF8>::kThreads, 1)
       if (!dbg_range(ab, p.counter_slot, 1, kFwdCounterSlots)) counter = nullptr;
       for (uint32_t n = 0;; ++n) {
         const uint32_t islot = n & 1;
-        mbar_wait(bar(bars->item_empty[islot]), ((n >> 1) & 1) ^ 1, ab);
+        mbar_wait_ring(bar(bars->item_empty[islot]), ((n >> 1) & 1) ^ 1, ab);  // slot read by every consumer
         const int w = (ab.raised() || !counter) ? p.num_items : atomicAdd(counter, 1);
         bars->item_w[islot] = w;
         mbar_arrive(bar(bars->item_full[islot]));

@@ -162,9 +162,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Abort a
 // Wait on the work-item ring: it ignores the abort flag and allows twice the usual time. Every
 // consumer of an item then decides from the same published value whether to stop, whatever the
 // abort flag reads at the moment it looks, so warps that meet at named barriers (which cannot
-// time out) take the same items. Once the flag is raised the producer publishes stop items at
-// once, well within this limit. Returns false (and raises the flag) if the phase did not
-// complete in time: the producer has stopped, and every consumer then stops as well.
+// time out) take the same items; and the producer overwrites a slot only after every consumer
+// has read it, abort or not (the consumers keep fetching, since their other waits return at
+// once after an abort). Once the flag is raised the producer publishes stop items, well within
+// this limit. Returns false (and raises the flag) if the phase did not complete in time: a
+// role has stopped for good.
 __device__ __forceinline__ bool mbar_wait_ring(uint32_t bar, uint32_t parity, Abort ab) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
